@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Throughput of multi-LoRA delta application on B200.
+
+One step = the whole hot path over one batch: group the batch's rows by
+adapter id (lora_build_segments) and apply every linear layer's LoRA delta
+(lora_add_linear, which runs the fused shrink/expand kernels).  Inputs are
+synthetic, seeded, with the shapes of the workload named in ``config``.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun);
+every rank applies the deltas of its own batch (rows are independent, so the
+path shards with no collective on the data path) and the step time is the
+maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "multi-LoRA delta tokens/s + achieved HBM GB/s (% of B200 peak), SGMV & BGMV"
+UNIT = "tokens/s"
+HEADLINE = "decode_qproj"
+SWEEP = ["prefill", "multislice_8b", "mixed_70b"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+class Dist:
+    def __init__(self):
+        self.rank = int(os.environ.get("RANK", 0))
+        self.world = int(os.environ.get("WORLD_SIZE", 1))
+        self.local = int(os.environ.get("LOCAL_RANK", 0))
+        self.pg = None
+
+    def init(self):
+        if self.world > 1:
+            import datetime
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                                 device_id=torch.device("cuda", self.local))
+            self.pg = torch.distributed.group.WORLD
+
+    def barrier(self):
+        if self.world > 1:
+            torch.distributed.barrier()
+
+    def max(self, x):
+        if self.world == 1:
+            return float(x)
+        t = torch.tensor([float(x)], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x):
+        if self.world == 1:
+            return float(x)
+        t = torch.tensor([float(x)], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            torch.distributed.destroy_process_group()
+
+
+class ClockSampler(threading.Thread):
+    """NVML clock / clock-event-reason samples of this process's GPU (read only)."""
+
+    def __init__(self, cuda_index, period=0.02):
+        super().__init__(daemon=True)
+        self.samples = []
+        self.period = period
+        self.ok = False
+        self.stop_flag = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = None
+            try:
+                props = torch.cuda.get_device_properties(cuda_index)
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                idx = int(vis.split(",")[cuda_index]) if vis else cuda_index
+                handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv, self.h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = str(e)
+
+    def reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def run(self):
+        while self.ok and not self.stop_flag.is_set():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self.reasons(),
+                                     self.nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self.stop_flag.set()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if len(win) < 3:   # a short timed region: widen to the neighbouring samples
+            mid = 0.5 * (t0 + t1)
+            win = sorted(self.samples, key=lambda s: abs(s[0] - mid))[:5]
+            window = "nearest to timed region"
+        if not win:
+            return {"error": "no samples"}
+        bits = 0
+        for s in win:
+            bits |= int(s[2])
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in REASON_BITS.items() if bits & b and n != "gpu_idle"],
+                "power_w_max": max(s[3] for s in win), "samples": len(win), "window": window}
+
+
+# ----------------------------------------------------------------------------- device data
+class DeviceSet:
+    """One copy of a batch's inputs on the device: ids, and per layer x, y (base
+    output, updated in place), A, B; plus the batch metadata buffers."""
+
+    def __init__(self, w, device, rows_per_tile, min_run):
+        import lora_adapter_application_b200 as lora
+        self.ids = w.ids.to(device)
+        self.ranks = w.ranks.to(device)
+        self.scales = lora.scales_for(w.alpha, w.ranks).to(device)
+        self.layers = []
+        for l in w.layers:
+            self.layers.append({"x": l.x.to(device), "y": l.y0.to(device),
+                                "A": [a.to(device) for a in l.A], "B": [b.to(device) for b in l.B],
+                                "col_off": list(l.col_off)})
+        self.meta = lora.Meta(w.T, w.N, rows_per_tile, min_run, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def nbytes(self):
+        n = self.ids.numel() * 4
+        for l in self.layers:
+            n += l["x"].numel() * l["x"].element_size() + 2 * l["y"].numel() * l["y"].element_size()
+            n += sum(t.numel() * t.element_size() for t in l["A"] + l["B"])
+        return n
+
+
+def step(ds, ka=None, kb=None):
+    import lora_adapter_application_b200 as lora
+    lora.lora_build_segments(ds.ids, ds.meta, ds.status)
+    if ka is not None:
+        ka.record()
+    for l in ds.layers:
+        lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks, ds.scales,
+                             ds.meta, ds.status)
+    if kb is not None:
+        kb.record()
+
+
+def launches_per_step(w):
+    builder = 1 if w.T <= 2048 else 4
+    return builder + len(w.layers)
+
+
+def make_sets(w, device, l2_bytes, rows_per_tile, min_run, max_sets=32):
+    first = DeviceSet(w, device, rows_per_tile, min_run)
+    per = first.nbytes()
+    n = max(1, min(max_sets, math.ceil(2 * l2_bytes / per)))
+    sets = [first] + [DeviceSet(w, device, rows_per_tile, min_run) for _ in range(n - 1)]
+    return sets, per
+
+
+def time_device(sets, K, W, dist):
+    for i in range(W):
+        step(sets[i % len(sets)])
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ka = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t0 = time.perf_counter()
+    start.record()
+    for i in range(K):
+        step(sets[i % len(sets)], ka[i], kb[i])
+    end.record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist.barrier()
+    step_ms = start.elapsed_time(end) / K
+    kern_ms = sum(a.elapsed_time(b) for a, b in zip(ka, kb)) / K
+    for s in sets:
+        st = int(s.status.item())
+        if st:
+            raise RuntimeError(f"device status {st}")
+    return step_ms, kern_ms, t0, t1
+
+
+def time_e2e(w, device, K, dist):
+    """Same step through host buffers: pinned host -> device copies of the step's
+    inputs (ids, x and base output y of every layer), the path, and the updated y
+    back to pinned host memory, all inside the timed region."""
+    import lora_adapter_application_b200 as lora
+    ds = DeviceSet(w, device, 16, 64)
+    host = {"ids": w.ids.pin_memory(),
+            "layers": [{"x": l.x.pin_memory(), "y": l.y0.pin_memory(),
+                        "out": torch.empty_like(l.y0).pin_memory()} for l in w.layers]}
+    h2d = host["ids"].numel() * 4 + sum(h["x"].numel() * h["x"].element_size() +
+                                        h["y"].numel() * h["y"].element_size() for h in host["layers"])
+    d2h = sum(h["out"].numel() * h["out"].element_size() for h in host["layers"])
+
+    def one():
+        ds.ids.copy_(host["ids"], non_blocking=True)
+        for l, h in zip(ds.layers, host["layers"]):
+            l["x"].copy_(h["x"], non_blocking=True)
+            l["y"].copy_(h["y"], non_blocking=True)
+        lora.lora_build_segments(ds.ids, ds.meta, ds.status)
+        for l in ds.layers:
+            lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks, ds.scales,
+                                 ds.meta, ds.status)
+        for l, h in zip(ds.layers, host["layers"]):
+            h["out"].copy_(l["y"], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = dist.max(s.elapsed_time(e) / K)
+    del ds
+    return ms, h2d, d2h
+
+
+def cpu_oracle_rate(w, budget_s, threads=None):
+    """Rows per second of the fp64 C oracle on a bounded sample of the workload."""
+    import oracle
+    oracle.build()
+    if threads:
+        oracle.set_threads(threads)
+    cores = oracle.max_threads()
+    active = np.nonzero(w.ids.numpy() >= 0)[0]
+    probe = active[: min(8, len(active))]
+
+    def run(rows):
+        t = time.perf_counter()
+        for l in w.layers:
+            oracle.lora_apply(l.x, l.A, l.B, l.col_off, w.ranks, w.alpha, w.ids, l.y0, rows=rows)
+        return time.perf_counter() - t
+
+    t_probe = max(run(probe), 1e-6) / max(len(probe), 1)
+    n = int(min(w.T, max(len(probe), budget_s / t_probe)))
+    rows = np.arange(n, dtype=np.int32)          # the first n rows, -1 rows included as in the batch
+    dt = run(rows)
+    return n / dt, cores, n, dt
+
+
+# ----------------------------------------------------------------------------- arms
+def bench_ours(args, dist):
+    import lora_adapter_application_b200 as lora
+    from lora_adapter_application_b200 import roofline
+    lora.load()
+    device = torch.device("cuda", dist.local)
+    torch.cuda.set_device(device)
+    props = torch.cuda.get_device_properties(device)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    pk = peaks()
+
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+
+    w = workloads.make(args.workload, seed=args.seed + 1000 * dist.rank)
+    sets, per_set = make_sets(w, device, l2, 16, 64)
+    step_ms_local, kern_ms_local, t0, t1 = time_device(sets, args.steps, args.warmup, dist)
+    step_ms = dist.max(step_ms_local)
+    kern_ms = dist.max(kern_ms_local)
+    tokens_total = dist.sum(w.T)
+    value = tokens_total / (step_ms * 1e-3)
+    clocks = sampler.summary(t0, t1)
+
+    alg_bytes = roofline.workload_bytes(w)
+    alg_flops = roofline.workload_flops(w)
+    achieved = alg_bytes / (kern_ms_local * 1e-3) / 1e9
+    n_sets = len(sets)
+    del sets
+    torch.cuda.empty_cache()
+
+    e2e_ms, h2d, d2h = time_e2e(w, device, min(args.steps, args.e2e_steps), dist)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.info.get('desc', '')}", "T": w.T, "N": w.N,
+                   "r_max": w.r_max, "layers": [l.name for l in w.layers],
+                   "active_rows": int((w.ids >= 0).sum()),
+                   "l2": f"{n_sets} rotating input sets of {per_set / 1e6:.1f} MB "
+                         f"(inputs {n_sets * per_set / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
+                   "parallelism": f"dp{dist.world} (independent batch per GPU)",
+                   "seed": args.seed},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(pk["hbm_gbs"]),
+                     "unit": "GB/s", "frac": achieved / float(pk["hbm_gbs"]), "traffic": None,
+                     "kernel": "bgmv_mma_kernel (lora_add_linear)", "kernel_ms": kern_ms_local,
+                     "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
+                     "peak_source": f"{pk.get('source')} hbm_gbs"},
+        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "steps": min(args.steps, args.e2e_steps)},
+        "gpu_launches": args.steps * launches_per_step(w),
+        "clocks": clocks,
+    }
+
+    if dist.world == 1 and not args.no_cpu:
+        rate, cores, n, dt = cpu_oracle_rate(w, args.cpu_budget)
+        result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                  "sample": f"first {n} of {w.T} rows of {w.name}, all layers, "
+                                            f"{dt:.1f} s"}
+
+    if dist.world == 1 and not args.no_sweep:
+        sweep = {}
+        for name in SWEEP:
+            sweep[name] = sweep_one(name, args, device, l2, pk, dist)
+        result["sweep"] = sweep
+    sampler.stop()
+    return result
+
+
+def sweep_one(name, args, device, l2, pk, dist):
+    from lora_adapter_application_b200 import roofline
+    w = workloads.make(name, seed=args.seed)
+    sets, per_set = make_sets(w, device, l2, 16, 64, max_sets=4)
+    probe_ms, _, _, _ = time_device(sets, 3, 2, dist)
+    K = int(min(500, max(10, args.sweep_seconds * 1e3 / probe_ms)))
+    step_ms, kern_ms, _, _ = time_device(sets, K, 3, dist)
+    b, f = roofline.workload_bytes(w), roofline.workload_flops(w)
+    gbs = b / (kern_ms * 1e-3) / 1e9
+    del sets
+    torch.cuda.empty_cache()
+    return {"desc": w.info.get("desc", ""), "T": w.T, "steps": K, "ms_per_step": step_ms,
+            "kernel_ms": kern_ms, "tokens_per_s": w.T / (step_ms * 1e-3),
+            "algorithmic_bytes": b, "gbs": gbs, "frac_hbm": gbs / float(pk["hbm_gbs"]),
+            "tflops": f / (kern_ms * 1e-3) / 1e12, "launches_per_step": launches_per_step(w)}
+
+
+def bench_reference(args, dist):
+    """The fp64 CPU oracle as the reference arm, on the host cores."""
+    if dist.rank != 0:
+        return None
+    w = workloads.make(args.workload, seed=args.seed)
+    per_step_budget = max(0.2, args.ref_seconds / max(1, args.steps + args.warmup))
+    rate, cores, n, dt = cpu_oracle_rate(w, per_step_budget)
+    import oracle
+    rows = np.arange(n, dtype=np.int32)
+
+    def one():
+        for l in w.layers:
+            oracle.lora_apply(l.x, l.A, l.B, l.col_off, w.ranks, w.alpha, w.ids, l.y0, rows=rows)
+
+    for _ in range(args.warmup):
+        one()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    total = time.perf_counter() - t
+    ms = total / args.steps * 1e3
+    value = n / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.info.get('desc', '')}", "T": w.T, "N": w.N,
+                   "r_max": w.r_max, "parallelism": "host cores (OpenMP over rows)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: first {n} of {w.T} rows of {w.name}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(workloads.NAMES))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle work")
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--sweep-seconds", type=float, default=0.5)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    dist = Dist()
+    if args.impl == "reference":
+        res = bench_reference(args, dist)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    dist.init()
+    try:
+        res = bench_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,272 @@
+"""Python binding of the B200 multi-LoRA delta library (``liblora_delta.so``).
+
+Argument marshalling only: every function below turns torch tensors into the
+plain pointers, strides and sizes of the C ABI declared in
+``include/lora_delta.h`` and calls the entry point of the same name.  All
+arithmetic runs in the library's CUDA kernels; PyTorch only owns device memory
+and streams.  There is no fallback: if the library is not built, or a call is
+made with CPU tensors, these functions raise.
+
+What is computed (page "Multi-LoRA Serving: one base, many adapters", section
+3.1 and 3.4; page "LoRA service: multi-adapter dynamic loading", section 2):
+for every row i with adapter n = ids[i] != -1,
+
+    y_i[col_off_s : col_off_s + d_out_s] += scales[n] * B_s[n] (A_s[n] x_i)
+
+with scales[n] = alpha / r_n and only the first r_n rank rows/columns used.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "load", "LoraError", "Meta", "LORA_BF16", "LORA_FP32", "DEV_BAD_ID", "DEV_TILE_OVERFLOW",
+    "DEV_BAD_RANK", "lora_version", "lora_meta_capacity", "lora_segments_scratch_bytes",
+    "lora_build_segments", "lora_shrink_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand",
+    "lora_bgmv_fused", "lora_add_linear", "scales_for",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora_delta.so")
+
+LORA_BF16, LORA_FP32 = 0, 1
+DEV_BAD_ID, DEV_TILE_OVERFLOW, DEV_BAD_RANK = 1, 2, 4
+MAX_ROWS, MAX_ADAPTERS, MAX_RANK, MAX_SLICES, LONG_TILE = 131072, 4096, 128, 8, 128
+
+_P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+class lora_meta(ctypes.Structure):
+    _fields_ = [("T", _I32), ("N", _I32), ("rows_per_tile", _I32), ("min_run", _I32),
+                ("long_tile", _I32), ("max_gather_tiles", _I32), ("max_contig_tiles", _I32),
+                ("perm", _P), ("seg_start", _P), ("seg_adapter", _P), ("counts", _P),
+                ("grow", _P), ("gather_tiles", _P), ("contig_tiles", _P)]
+
+
+class lora_slice(ctypes.Structure):
+    _fields_ = [("A", _P), ("B", _P), ("d_out", _I32), ("col_off", _I32)]
+
+
+class LoraError(RuntimeError):
+    pass
+
+
+_lib = None
+
+_SIGS = {
+    "lora_version": (ctypes.c_int, []),
+    "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "lora_meta_capacity": (ctypes.c_int, [_I32, _I32, _I32, _I32, _I32, ctypes.POINTER(_I32),
+                                          ctypes.POINTER(_I32)]),
+    "lora_segments_scratch_bytes": (_SZ, [_I32, _I32]),
+    "lora_build_segments": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _SZ, _P, _P]),
+    "lora_shrink_workspace_bytes": (_SZ, [_I32, _I32, _I32]),
+    "lora_sgmv_shrink": (ctypes.c_int, [_P, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32, _I32,
+                                        _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
+    "lora_sgmv_expand": (ctypes.c_int, [_P, _I64, _P, ctypes.POINTER(lora_slice), _I32, _I32, _P, _P,
+                                        ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
+    "lora_bgmv_fused": (ctypes.c_int, [_P, _I64, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32,
+                                       _I32, _P, _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
+    "lora_add_linear": (ctypes.c_int, [_P, _I64, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32,
+                                       _I32, _P, _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
+}
+
+
+def load():
+    """Load the CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise LoraError(f"{LIB_PATH} is missing: build it with "
+                            "`python -m lora_adapter_application_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(rc):
+    if rc != 0:
+        raise LoraError(load().lora_status_string(rc).decode())
+
+
+def _dev(t: torch.Tensor, what: str):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise LoraError(f"{what} must be a CUDA tensor")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return LORA_BF16
+    if t.dtype == torch.float32:
+        return LORA_FP32
+    raise LoraError(f"unsupported dtype {t.dtype}: bf16 or fp32")
+
+
+def _rows(t, what):
+    _dev(t, what)
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise LoraError(f"{what} must be 2-D with unit column stride")
+    return t.stride(0)
+
+
+def lora_version():
+    return int(load().lora_version())
+
+
+def lora_meta_capacity(T, N, rows_per_tile=16, min_run=64, long_tile=LONG_TILE):
+    mg, mc = _I32(), _I32()
+    _check(load().lora_meta_capacity(T, N, rows_per_tile, min_run, long_tile, ctypes.byref(mg),
+                                     ctypes.byref(mc)))
+    return mg.value, mc.value
+
+
+def lora_segments_scratch_bytes(T, N):
+    return int(load().lora_segments_scratch_bytes(T, N))
+
+
+def lora_shrink_workspace_bytes(T, r_max, n_slices):
+    return int(load().lora_shrink_workspace_bytes(T, r_max, n_slices))
+
+
+class Meta:
+    """Device buffers of a batch's lora_meta, allocated with torch, plus the
+    builder's scratch.  ``rows_per_tile`` caps a gathered tile; ``min_run``
+    (0 = off) is the shortest run of one id that becomes contiguous tiles."""
+
+    def __init__(self, T, N, rows_per_tile=16, min_run=64, long_tile=LONG_TILE, device="cuda"):
+        mg, mc = lora_meta_capacity(T, N, rows_per_tile, min_run, long_tile)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.T, self.N = T, N
+        self.perm = torch.zeros(max(T, 1), **i32)
+        self.seg_start = torch.zeros(N + 1, **i32)
+        self.seg_adapter = torch.zeros(N, **i32)
+        self.counts = torch.zeros(4, **i32)
+        self.grow = torch.zeros(max(T, 1), **i32)
+        self.gather_tiles = torch.zeros(max(mg, 1), 4, **i32)
+        self.contig_tiles = torch.zeros(max(mc, 1), 4, **i32)
+        nbytes = lora_segments_scratch_bytes(T, N)
+        self.scratch = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+        self.scratch_bytes = nbytes
+        self.c = lora_meta(T, N, rows_per_tile, min_run, long_tile, mg, mc,
+                           self.perm.data_ptr(), self.seg_start.data_ptr(),
+                           self.seg_adapter.data_ptr(), self.counts.data_ptr(),
+                           self.grow.data_ptr(), self.gather_tiles.data_ptr(),
+                           self.contig_tiles.data_ptr())
+
+    def host(self):
+        """Copy the metadata to the host (synchronises)."""
+        counts = self.counts.cpu().tolist()
+        n_seg, n_gather, n_contig, n_short = counts
+        return {
+            "perm": self.perm[:self.T].cpu().numpy(),
+            "seg_start": self.seg_start.cpu().numpy(),
+            "seg_adapter": self.seg_adapter[:n_seg].cpu().numpy(),
+            "n_seg": n_seg, "n_gather": n_gather, "n_contig": n_contig, "n_short": n_short,
+            "grow": self.grow[:n_short].cpu().numpy(),
+            "gather_tiles": self.gather_tiles[:n_gather].cpu().numpy(),
+            "contig_tiles": self.contig_tiles[:n_contig].cpu().numpy(),
+        }
+
+
+def lora_build_segments(ids, meta: Meta, status, stream=None):
+    _dev(ids, "ids")
+    _dev(status, "status")
+    if ids.dtype != torch.int32 or ids.numel() != meta.T or not ids.is_contiguous():
+        raise LoraError("ids must be a contiguous int32 tensor of T entries")
+    _check(load().lora_build_segments(_ptr(ids), ctypes.byref(meta.c), _ptr(meta.scratch),
+                                      meta.scratch_bytes, _ptr(status), _stream(stream)))
+
+
+def _slices(A, B, d_out, col_off):
+    n = len(A) if A is not None else len(B)
+    if not 1 <= n <= MAX_SLICES:
+        raise LoraError("1 to 8 slices")
+    arr = (lora_slice * n)()
+    for s in range(n):
+        arr[s].A = A[s].data_ptr() if A is not None else None
+        arr[s].B = B[s].data_ptr() if B is not None else None
+        arr[s].d_out = int(d_out[s]) if d_out is not None else 0
+        arr[s].col_off = int(col_off[s]) if col_off is not None else 0
+    return arr, n
+
+
+def _adapters(A, B):
+    ref = A[0] if A is not None else B[0]
+    N = ref.shape[0]
+    r_max = ref.shape[1] if A is not None else ref.shape[2]
+    for t in (A or []) + (B or []):
+        _dev(t, "adapter tensor")
+        if not t.is_contiguous() or t.dtype != ref.dtype or t.shape[0] != N:
+            raise LoraError("stacked adapters must be contiguous, one dtype, N slots each")
+    return N, r_max
+
+
+def scales_for(alpha, ranks):
+    """alpha / r_n per adapter slot (page "Multi-LoRA Serving", section 3.1), fp32."""
+    return (float(alpha) / ranks.to(torch.float64)).to(torch.float32)
+
+
+def lora_sgmv_shrink(v, x, A, ranks, meta: Meta, status, stream=None):
+    """v[s, i, k] = sum_j A[s][n, k, j] x[i, j] for rows with an adapter, k < r_n."""
+    ld_x = _rows(x, "x")
+    N, r_max = _adapters(A, None)
+    sl, n = _slices(A, None, None, None)
+    _dev(v, "v")
+    if v.dtype != torch.float32 or not v.is_contiguous() or v.numel() < n * meta.T * r_max:
+        raise LoraError("v must be contiguous fp32 [n_slices, T, r_max]")
+    _check(load().lora_sgmv_shrink(_ptr(v), _ptr(x), ld_x, A[0].shape[2], sl, n, r_max,
+                                   _ptr(_dev(ranks, "ranks")), ctypes.byref(meta.c), _dtype_code(x),
+                                   _ptr(status), _stream(stream)))
+
+
+def lora_sgmv_expand(y, v, B, col_off, ranks, scales, meta: Meta, status, stream=None):
+    """y[i, col_off_s + c] += scales[n] sum_k B[s][n, c, k] v[s, i, k]."""
+    ld_y = _rows(y, "y")
+    N, r_max = _adapters(None, B)
+    sl, n = _slices(None, B, [b.shape[1] for b in B], col_off)
+    _dev(v, "v")
+    _check(load().lora_sgmv_expand(_ptr(y), ld_y, _ptr(v), sl, n, r_max, _ptr(_dev(ranks, "ranks")),
+                                   _ptr(_dev(scales, "scales")), ctypes.byref(meta.c),
+                                   _dtype_code(y), _ptr(status), _stream(stream)))
+
+
+def _fused(fn, y, x, A, B, col_off, ranks, scales, meta, status, stream):
+    ld_y = _rows(y, "y")
+    ld_x = _rows(x, "x")
+    N, r_max = _adapters(A, B)
+    if len(A) != len(B):
+        raise LoraError("one A and one B per slice")
+    sl, n = _slices(A, B, [b.shape[1] for b in B], col_off)
+    if x.dtype != y.dtype or A[0].dtype != x.dtype:
+        raise LoraError("x, y, A and B share one dtype")
+    _check(fn(_ptr(y), ld_y, _ptr(x), ld_x, A[0].shape[2], sl, n, r_max, _ptr(_dev(ranks, "ranks")),
+              _ptr(_dev(scales, "scales")), ctypes.byref(meta.c), _dtype_code(x), _ptr(status),
+              _stream(stream)))
+
+
+def lora_bgmv_fused(y, x, A, B, col_off, ranks, scales, meta: Meta, status, stream=None):
+    """Fused shrink + expand of every tile (rank-r intermediate kept on chip)."""
+    _fused(load().lora_bgmv_fused, y, x, A, B, col_off, ranks, scales, meta, status, stream)
+
+
+def lora_add_linear(y, x, A, B, col_off, ranks, scales, meta: Meta, status, stream=None):
+    """All slices of one linear layer applied to y in place (add_lora_linear)."""
+    _fused(load().lora_add_linear, y, x, A, B, col_off, ranks, scales, meta, status, stream)

@@ -1,0 +1,253 @@
+// C ABI of the multi-LoRA delta library: argument checks and the choice of
+// kernel for each unit of work.  Declarations and contracts: lora_delta.h.
+#include "kernels.cuh"
+
+#include <cstdint>
+
+using namespace lora;
+
+namespace {
+
+constexpr int BGMV_CLUSTER = 8;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_meta(const lora_meta *m) {
+    if (!m) return LORA_ERR_NULL;
+    if (m->T < 0 || m->T > LORA_MAX_ROWS || m->N < 1 || m->N > LORA_MAX_ADAPTERS)
+        return LORA_ERR_SHAPE;
+    if (m->rows_per_tile < 1 || m->rows_per_tile > 16 || m->min_run < 0 || m->long_tile < 1 ||
+        m->long_tile > LORA_LONG_TILE)
+        return LORA_ERR_SHAPE;
+    int32_t mg = 0, mc = 0;
+    lora_meta_capacity(m->T, m->N, m->rows_per_tile, m->min_run, m->long_tile, &mg, &mc);
+    if (m->max_gather_tiles < mg || m->max_contig_tiles < mc) return LORA_ERR_CAPACITY;
+    if (!m->perm || !m->seg_start || !m->seg_adapter || !m->counts || !m->grow ||
+        !m->gather_tiles || (mc > 0 && !m->contig_tiles))
+        return LORA_ERR_NULL;
+    return LORA_OK;
+}
+
+struct Call {
+    void *y;
+    int64_t ld_y;
+    const void *x;
+    int64_t ld_x;
+    int32_t d_in;
+    const lora_slice *slices;
+    int32_t n_slices;
+    int32_t r_max;
+    const int32_t *ranks;
+    const float *scales;
+    const float *v_in;
+    float *v_out;
+    const lora_meta *meta;
+    lora_dtype dtype;
+    int32_t *status;
+    cudaStream_t stream;
+};
+
+// need_x / need_y / need_scales: which operands the mode reads
+int check_call(const Call &c, bool need_x, bool need_y, bool need_scales, bool need_v) {
+    if (!c.slices || !c.ranks || !c.status) return LORA_ERR_NULL;
+    if (need_x && !c.x) return LORA_ERR_NULL;
+    if (need_y && !c.y) return LORA_ERR_NULL;
+    if (need_scales && !c.scales) return LORA_ERR_NULL;
+    if (need_v && !(c.v_in || c.v_out)) return LORA_ERR_NULL;
+    if (c.dtype != LORA_BF16 && c.dtype != LORA_FP32) return LORA_ERR_DTYPE;
+    int rc = check_meta(c.meta);
+    if (rc != LORA_OK) return rc;
+    if (c.n_slices < 1 || c.n_slices > LORA_MAX_SLICES) return LORA_ERR_SHAPE;
+    if (c.r_max < 1 || c.r_max > LORA_MAX_RANK) return LORA_ERR_RANK;
+    if (need_x && (c.d_in < 1 || c.ld_x < c.d_in)) return LORA_ERR_SHAPE;
+    for (int s = 0; s < c.n_slices; ++s) {
+        const lora_slice &sl = c.slices[s];
+        if ((need_x && !sl.A) || (need_y && !sl.B)) return LORA_ERR_NULL;
+        if (need_y && (sl.d_out < 1 || sl.col_off < 0 || (int64_t)sl.col_off + sl.d_out > c.ld_y))
+            return LORA_ERR_SHAPE;
+    }
+    return LORA_OK;
+}
+
+Slices make_slices(const Call &c) {
+    Slices s{};
+    s.n = c.n_slices;
+    s.cat_off[0] = 0;
+    for (int i = 0; i < c.n_slices; ++i) {
+        s.A[i] = c.slices[i].A;
+        s.B[i] = c.slices[i].B;
+        s.d_out[i] = c.slices[i].d_out;
+        s.col_off[i] = c.slices[i].col_off;
+        s.cat_off[i + 1] = s.cat_off[i] + c.slices[i].d_out;
+    }
+    return s;
+}
+
+Tiles make_tiles(const lora_meta *m, bool gather, bool contig) {
+    Tiles t{};
+    t.counts = m->counts;
+    t.grow = m->grow;
+    t.gather = reinterpret_cast<const int4 *>(m->gather_tiles);
+    t.contig = reinterpret_cast<const int4 *>(m->contig_tiles);
+    t.max_gather = m->max_gather_tiles;
+    t.max_contig = m->max_contig_tiles;
+    t.rows_per_unit = m->rows_per_tile;
+    t.subs = contig ? (m->long_tile + m->rows_per_tile - 1) / m->rows_per_tile : 0;
+    t.use_gather = gather ? 1 : 0;
+    return t;
+}
+
+int n_units(const Tiles &t) { return t.max_gather + (t.subs ? t.max_contig * t.subs : 0); }
+
+// The vectorised bf16 tensor-pipe kernel takes the call?
+bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
+    if (c.dtype != LORA_BF16 || c.r_max > 64 || (c.r_max & 3)) return false;
+    if (need_x) {
+        if ((c.d_in & 7) || (c.ld_x & 7) || !aligned(c.x, 16)) return false;
+        for (int s = 0; s < c.n_slices; ++s)
+            if (!aligned(c.slices[s].A, 16)) return false;
+    }
+    if (need_y) {
+        if ((c.ld_y & 1) || !aligned(c.y, 4)) return false;
+        for (int s = 0; s < c.n_slices; ++s)
+            if ((c.slices[s].d_out & 1) || (c.slices[s].col_off & 1) || !aligned(c.slices[s].B, 8))
+                return false;
+    }
+    return true;
+}
+
+int run(int mode, const Call &c, bool gather, bool contig) {
+    const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
+    Tiles tiles = make_tiles(c.meta, gather, contig);
+    const int units = n_units(tiles);
+    if (c.meta->T == 0 || units == 0) return LORA_OK;
+    if (units <= 65535 && bgmv_ok(c, need_x, need_y)) {
+        BgArgs a{};
+        a.x = static_cast<const __nv_bfloat16 *>(c.x);
+        a.ld_x = c.ld_x;
+        a.d_in = c.d_in;
+        a.y = static_cast<__nv_bfloat16 *>(c.y);
+        a.ld_y = c.ld_y;
+        a.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
+        a.T = c.meta->T;
+        a.sl = make_slices(c);
+        a.r_max = c.r_max;
+        a.ranks = c.ranks;
+        a.scales = c.scales;
+        a.tiles = tiles;
+        a.status = c.status;
+        return launch_bgmv(mode, a, units, BGMV_CLUSTER, c.stream);
+    }
+    SimtArgs a{};
+    a.x = c.x;
+    a.ld_x = c.ld_x;
+    a.d_in = c.d_in;
+    a.y = c.y;
+    a.ld_y = c.ld_y;
+    a.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
+    a.T = c.meta->T;
+    a.sl = make_slices(c);
+    a.r_max = c.r_max;
+    a.ranks = c.ranks;
+    a.scales = c.scales;
+    a.tiles = tiles;
+    a.status = c.status;
+    return launch_simt(mode, c.dtype == LORA_BF16, a, units, c.stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lora_version(void) { return 100; }
+
+const char *lora_status_string(int status) {
+    switch (status) {
+        case LORA_OK: return "LORA_OK";
+        case LORA_ERR_NULL: return "LORA_ERR_NULL";
+        case LORA_ERR_DTYPE: return "LORA_ERR_DTYPE";
+        case LORA_ERR_SHAPE: return "LORA_ERR_SHAPE";
+        case LORA_ERR_RANK: return "LORA_ERR_RANK";
+        case LORA_ERR_ALIGN: return "LORA_ERR_ALIGN";
+        case LORA_ERR_WORKSPACE: return "LORA_ERR_WORKSPACE";
+        case LORA_ERR_CAPACITY: return "LORA_ERR_CAPACITY";
+        case LORA_ERR_CUDA: return "LORA_ERR_CUDA";
+        default: return "unknown lora_status";
+    }
+}
+
+int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int32_t min_run,
+                       int32_t long_tile, int32_t *max_gather, int32_t *max_contig) {
+    if (!max_gather || !max_contig) return LORA_ERR_NULL;
+    if (T < 0 || T > LORA_MAX_ROWS || N < 1 || N > LORA_MAX_ADAPTERS || rows_per_tile < 1 ||
+        rows_per_tile > 16 || min_run < 0 || long_tile < 1 || long_tile > LORA_LONG_TILE)
+        return LORA_ERR_SHAPE;
+    *max_gather = (T + rows_per_tile - 1) / rows_per_tile + (N < T ? N : T);
+    *max_contig = min_run > 0 ? (T + long_tile - 1) / long_tile + T / min_run : 0;
+    return LORA_OK;
+}
+
+size_t lora_segments_scratch_bytes(int32_t T, int32_t N) {
+    if (T < 0 || N < 1) return 0;
+    return segments_scratch_bytes(T, N);
+}
+
+int lora_build_segments(const int32_t *ids, const lora_meta *meta, void *scratch,
+                        size_t scratch_bytes, int32_t *status, void *stream) {
+    int rc = check_meta(meta);
+    if (rc != LORA_OK) return rc;
+    if (!status || (meta->T > 0 && !ids)) return LORA_ERR_NULL;
+    return launch_build_segments(ids, meta, scratch, scratch_bytes, status,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+size_t lora_shrink_workspace_bytes(int32_t T, int32_t r_max, int32_t n_slices) {
+    if (T < 0 || r_max < 1 || n_slices < 1) return 0;
+    return (size_t)n_slices * (size_t)T * (size_t)r_max * sizeof(float);
+}
+
+int lora_sgmv_shrink(float *v, const void *x, int64_t ld_x, int32_t d_in,
+                     const lora_slice *slices, int32_t n_slices, int32_t r_max,
+                     const int32_t *ranks, const lora_meta *meta, lora_dtype dtype,
+                     int32_t *status, void *stream) {
+    Call c{nullptr, 0, x, ld_x, d_in, slices, n_slices, r_max, ranks, nullptr, nullptr, v,
+           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+    int rc = check_call(c, true, false, false, true);
+    if (rc != LORA_OK) return rc;
+    return run(MODE_SHRINK, c, true, true);
+}
+
+int lora_sgmv_expand(void *y, int64_t ld_y, const float *v, const lora_slice *slices,
+                     int32_t n_slices, int32_t r_max, const int32_t *ranks,
+                     const float *scales, const lora_meta *meta, lora_dtype dtype,
+                     int32_t *status, void *stream) {
+    Call c{y, ld_y, nullptr, 0, 0, slices, n_slices, r_max, ranks, scales, v, nullptr,
+           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+    int rc = check_call(c, false, true, true, true);
+    if (rc != LORA_OK) return rc;
+    return run(MODE_EXPAND, c, true, true);
+}
+
+int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
+                    const lora_slice *slices, int32_t n_slices, int32_t r_max,
+                    const int32_t *ranks, const float *scales, const lora_meta *meta,
+                    lora_dtype dtype, int32_t *status, void *stream) {
+    Call c{y, ld_y, x, ld_x, d_in, slices, n_slices, r_max, ranks, scales, nullptr, nullptr,
+           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+    int rc = check_call(c, true, true, true, false);
+    if (rc != LORA_OK) return rc;
+    return run(MODE_FUSED, c, true, true);
+}
+
+int lora_add_linear(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
+                    const lora_slice *slices, int32_t n_slices, int32_t r_max,
+                    const int32_t *ranks, const float *scales, const lora_meta *meta,
+                    lora_dtype dtype, int32_t *status, void *stream) {
+    Call c{y, ld_y, x, ld_x, d_in, slices, n_slices, r_max, ranks, scales, nullptr, nullptr,
+           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+    int rc = check_call(c, true, true, true, false);
+    if (rc != LORA_OK) return rc;
+    return run(MODE_FUSED, c, true, true);
+}
+
+}  // extern "C"

@@ -45,6 +45,8 @@ def _load():
         lib.oracle_lora_apply.restype = ctypes.c_int
         lib.oracle_lora_apply.argtypes = [ctypes.c_int, P, I64, I32, I32, P, P, P, P, I32, I32, P,
                                           D, P, I32, P, I32, P, I64, P]
+        lib.oracle_lora_shrink.restype = ctypes.c_int
+        lib.oracle_lora_shrink.argtypes = [ctypes.c_int, P, I64, I32, I32, P, I32, I32, P, P, P, I32, P]
         lib.oracle_build_segments.restype = ctypes.c_int
         lib.oracle_build_segments.argtypes = [P, I32, I32, I32, I32, I32, I32, I32,
                                               P, P, P, P, P, P, P]
@@ -119,6 +121,30 @@ def lora_apply(x, A, B, col_off, ranks, alpha, ids, y0, rows=None):
                                y0.data_ptr(), ld_y, out.ctypes.data)
     if rc != 0:
         raise ValueError("oracle_lora_apply rejected its arguments")
+    return out
+
+
+def lora_shrink(x, A, ranks, ids, rows=None):
+    """v = A_n x_i per listed row and slice, fp64, shape [n_rows, n_slices, r_max]
+    (zeros for rows without an adapter and for k >= r_n)."""
+    lib = _load()
+    x = _cpu(x)
+    A = [_cpu(a) for a in A]
+    code = _dtype_code(x)
+    T, ld_x = x.shape
+    N, r_max, d_in = A[0].shape
+    n_slices = len(A)
+    ranks_np = np.ascontiguousarray(np.asarray(ranks, dtype=np.int32))
+    ids_np = np.ascontiguousarray(np.asarray(ids, dtype=np.int32))
+    rows_np = np.arange(T, dtype=np.int32) if rows is None else \
+        np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    A_ptrs = (ctypes.c_void_p * n_slices)(*[a.data_ptr() for a in A])
+    out = np.empty((rows_np.shape[0], n_slices, r_max), dtype=np.float64)
+    rc = lib.oracle_lora_shrink(code, x.data_ptr(), ld_x, d_in, n_slices, A_ptrs, N, r_max,
+                                ranks_np.ctypes.data, ids_np.ctypes.data, rows_np.ctypes.data,
+                                rows_np.shape[0], out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_lora_shrink rejected its arguments")
     return out
 
 

@@ -114,6 +114,45 @@ int oracle_lora_apply(int dtype, const void *x, int64_t ld_x, int32_t d_in,
 }
 
 /*
+ * The shrink alone (page "Multi-LoRA Serving", section 3.4: add_shrink, the
+ * rank-r v = A x): v_out[q][s][k] = sum_j A_s[n][k][j] * x_i[j] for the listed
+ * rows, k < r_n, in fp64; entries of rows without a valid adapter, and k >= r_n,
+ * are set to 0.  v_out is [n_rows][n_slices][r_max].
+ */
+int oracle_lora_shrink(int dtype, const void *x, int64_t ld_x, int32_t d_in,
+                       int32_t n_slices, const void *const *A, int32_t N, int32_t r_max,
+                       const int32_t *ranks, const int32_t *ids, const int32_t *rows,
+                       int32_t n_rows, double *v_out)
+{
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32)
+        return -1;
+    if (n_rows < 0 || d_in <= 0 || n_slices <= 0 || N <= 0 || r_max <= 0)
+        return -1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int32_t q = 0; q < n_rows; ++q) {
+        int32_t i = rows[q];
+        double *vo = v_out + (int64_t)q * n_slices * r_max;
+        for (int64_t e = 0; e < (int64_t)n_slices * r_max; ++e)
+            vo[e] = 0.0;
+        int32_t n = ids[i];
+        if (n < 0 || n >= N)
+            continue;
+        int32_t r = ranks[n];
+        if (r <= 0 || r > r_max)
+            continue;
+        for (int32_t s = 0; s < n_slices; ++s)
+            for (int32_t k = 0; k < r; ++k) {
+                double acc = 0.0;
+                for (int32_t j = 0; j < d_in; ++j)
+                    acc += widen(dtype, A[s], ((int64_t)n * r_max + k) * d_in + j) *
+                           widen(dtype, x, (int64_t)i * ld_x + j);
+                vo[s * r_max + k] = acc;
+            }
+    }
+    return 0;
+}
+
+/*
  * Grouping of rows by adapter id, and the work lists.
  *
  *   valid(i)      = 0 <= ids[i] < N

@@ -1,0 +1,106 @@
+"""The C-ABI library loads and exports every entry point its header declares,
+and the host-side checks reject bad arguments before anything reaches a GPU.
+Runs without a GPU: nothing here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import lora_adapter_application_b200 as lora
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_delta.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    return re.findall(r"LORA_API\s+[A-Za-z_][A-Za-z0-9_\s\*]*?\b(lora_[a-z0-9_]+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lora_adapter_application_b200 import build
+    build.build()
+    return lora.load()
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_entry_points())
+    for required in ["lora_build_segments", "lora_sgmv_shrink", "lora_sgmv_expand",
+                     "lora_bgmv_fused", "lora_add_linear"]:
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_entry_points():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_binding_names_match_the_abi():
+    for name in declared_entry_points():
+        if name != "lora_status_string":
+            assert hasattr(lora, name), name
+
+
+def test_capacity_bounds(lib):
+    mg, mc = lora.lora_meta_capacity(1024, 100, 16, 64, 128)
+    assert mg == 64 + 100 and mc == 8 + 16
+    assert lora.lora_meta_capacity(10, 100, 16, 0, 128) == (1 + 10, 0)
+    with pytest.raises(lora.LoraError):
+        lora.lora_meta_capacity(-1, 4, 16, 0, 128)
+    with pytest.raises(lora.LoraError):
+        lora.lora_meta_capacity(10, 4, 17, 0, 128)
+
+
+def test_scratch_and_workspace_sizes(lib):
+    assert lora.lora_segments_scratch_bytes(2048, 100) == 0
+    assert lora.lora_segments_scratch_bytes(2049, 100) == 2 * 101 * 4
+    assert lora.lora_shrink_workspace_bytes(1024, 64, 3) == 3 * 1024 * 64 * 4
+
+
+def _meta(T=8, N=4, R=4, min_run=0):
+    mg, mc = lora.lora_meta_capacity(T, N, R, min_run, 128)
+    fake = 0x1000   # never dereferenced: every call below fails its host check first
+    return lora.lora_meta(T, N, R, min_run, 128, mg, mc, fake, fake, fake, fake, fake, fake, fake)
+
+
+def _codes(lib):
+    return {n: v for n, v in [("NULL", -1), ("DTYPE", -2), ("SHAPE", -3), ("RANK", -4),
+                              ("WORKSPACE", -6), ("CAPACITY", -7)]}
+
+
+def test_host_checks(lib):
+    c = _codes(lib)
+    fake = ctypes.c_void_p(0x1000)
+    m = _meta()
+    assert lib.lora_build_segments(fake, None, None, 0, fake, None) == c["NULL"]
+    assert lib.lora_build_segments(fake, ctypes.byref(m), None, 0, None, None) == c["NULL"]
+    small = _meta()
+    small.max_gather_tiles = 1
+    assert lib.lora_build_segments(fake, ctypes.byref(small), None, 0, fake, None) == c["CAPACITY"]
+    bad = _meta()
+    bad.rows_per_tile = 0
+    assert lib.lora_build_segments(fake, ctypes.byref(bad), None, 0, fake, None) == c["SHAPE"]
+    sl = (lora.lora_slice * 1)()
+    sl[0].A, sl[0].B, sl[0].d_out, sl[0].col_off = 0x1000, 0x1000, 16, 0
+    args = lambda dtype=0, r_max=16, n=1, ld_y=16, sl=sl: (
+        fake, ld_y, fake, 16, 16, sl, n, r_max, fake, fake, ctypes.byref(m), dtype, fake, None)
+    assert lib.lora_add_linear(*args(dtype=7)) == c["DTYPE"]
+    assert lib.lora_add_linear(*args(r_max=0)) == c["RANK"]
+    assert lib.lora_add_linear(*args(r_max=129)) == c["RANK"]
+    assert lib.lora_add_linear(*args(n=0)) == c["SHAPE"]
+    assert lib.lora_add_linear(*args(n=9)) == c["SHAPE"]
+    assert lib.lora_add_linear(*args(ld_y=8)) == c["SHAPE"]   # slice runs past the row
+    assert lib.lora_bgmv_fused(*args(ld_y=8)) == c["SHAPE"]
+    nul = (lora.lora_slice * 1)()
+    nul[0].A, nul[0].B, nul[0].d_out = None, 0x1000, 16
+    assert lib.lora_add_linear(*args(sl=nul)) == c["NULL"]
+    big = _meta()
+    big.T = lora.MAX_ROWS + 1
+    assert lib.lora_sgmv_shrink(fake, fake, 16, 16, sl, 1, 16, fake, ctypes.byref(big), 0, fake,
+                                None) == c["SHAPE"]
+    assert lib.lora_sgmv_expand(fake, 16, None, sl, 1, 16, fake, fake, ctypes.byref(m), 0, fake,
+                                None) == c["NULL"]
+    assert lib.lora_status_string(-7) == b"LORA_ERR_CAPACITY"

@@ -330,3 +330,22 @@ def test_segments_workload_shapes():
     rq = np.array(w.info["req_ids"])
     assert got["n_short"] <= int(lens[(lens < 64) & (rq >= 0)].sum())
     assert got["n_contig"] >= int(((lens >= 64) & (rq >= 0)).sum() > 0)
+
+
+def test_shrink_equals_library_matmul():
+    """v = A_n x_i (page 'Multi-LoRA Serving', section 3.4: add_shrink computes the
+    rank-r v = A x) against torch's fp64 matmul, per adapter."""
+    w = workloads.random_case(15, 29, 3, 40, [8, 8], 6, ranks=[6, 2, 4], none_frac=0.2,
+                              dtype=torch.bfloat16)
+    lay = w.layers[0]
+    v = oracle.lora_shrink(lay.x, lay.A, w.ranks, w.ids)
+    for i in range(w.T):
+        n = int(w.ids[i])
+        for s in range(2):
+            if n < 0:
+                assert (v[i, s] == 0).all()
+                continue
+            r = int(w.ranks[n])
+            ref = (_f64(lay.A[s][n, :r]) @ _f64(lay.x[i])).numpy()
+            np.testing.assert_allclose(v[i, s, :r], ref, rtol=1e-12, atol=1e-12)
+            assert (v[i, s, r:] == 0).all()
