@@ -46,6 +46,23 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 # ----------------------------------------------------------------------------- helpers
+def measured_traffic(workload):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    or None when the kernel source has changed since that capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "lora_adapter_application_b200", "csrc", "bgmv.cu")
+    try:
+        with open(p) as f:
+            rec = json.load(f)["bgmv_kernel"]
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return rec[workload]["dram_bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -62,13 +79,15 @@ class Dist:
         self.world = int(os.environ.get("WORLD_SIZE", 1))
         self.local = int(os.environ.get("LOCAL_RANK", 0))
         self.pg = None
+        self.device = "cuda"
 
-    def init(self):
+    def init(self, backend="nccl"):
         if self.world > 1:
             import datetime
-            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                                 device_id=torch.device("cuda", self.local))
+            kw = {"device_id": torch.device("cuda", self.local)} if backend == "nccl" else {}
+            torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
             self.pg = torch.distributed.group.WORLD
+        self.device = "cuda" if backend == "nccl" else "cpu"
 
     def barrier(self):
         if self.world > 1:
@@ -77,14 +96,14 @@ class Dist:
     def max(self, x):
         if self.world == 1:
             return float(x)
-        t = torch.tensor([float(x)], dtype=torch.float64, device="cuda")
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
 
     def sum(self, x):
         if self.world == 1:
             return float(x)
-        t = torch.tensor([float(x)], dtype=torch.float64, device="cuda")
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
         return float(t.item())
 
@@ -210,30 +229,63 @@ def make_sets(w, device, l2_bytes, rows_per_tile, min_run, max_sets=32):
     return sets, per
 
 
-def time_device(sets, K, W, dist):
+def _event(external):
+    try:
+        return torch.cuda.Event(enable_timing=True, external=external)
+    except TypeError:
+        return torch.cuda.Event(enable_timing=True)
+
+
+def time_device(sets, K, W, dist, graph=True):
+    """Time exactly K steps on the device.  The K steps (with a CUDA-event pair
+    around each step's layer calls) are captured into one CUDA graph and replayed
+    once, so host launch overhead does not enter the timed region; without a
+    graph the steps are launched one by one."""
     for i in range(W):
         step(sets[i % len(sets)])
     torch.cuda.synchronize()
+    ka = kb = g = None
+    if graph:
+        try:
+            ka = [_event(True) for _ in range(K)]
+            kb = [_event(True) for _ in range(K)]
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for i in range(K):
+                    step(sets[i % len(sets)], ka[i], kb[i])
+            torch.cuda.synchronize()
+        except Exception as e:  # capture not available: launch eagerly
+            print(f"graph capture failed ({e}); timing eager launches", file=sys.stderr)
+            g = None
+            torch.cuda.synchronize()
+    if g is None:
+        ka = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     dist.barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ka = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     t0 = time.perf_counter()
     start.record()
-    for i in range(K):
-        step(sets[i % len(sets)], ka[i], kb[i])
+    if g is not None:
+        g.replay()
+    else:
+        for i in range(K):
+            step(sets[i % len(sets)], ka[i], kb[i])
     end.record()
     torch.cuda.synchronize()
     t1 = time.perf_counter()
     dist.barrier()
     step_ms = start.elapsed_time(end) / K
     kern_ms = sum(a.elapsed_time(b) for a, b in zip(ka, kb)) / K
-    for s in sets:
-        st = int(s.status.item())
-        if st:
-            raise RuntimeError(f"device status {st}")
-    return step_ms, kern_ms, t0, t1
+    for st in sets:
+        code = int(st.status.item())
+        if code:
+            raise RuntimeError(f"device status {code}")
+    graphed = g is not None
+    del g
+    return step_ms, kern_ms, t0, t1, graphed
 
 
 def time_e2e(w, device, K, dist):
@@ -315,7 +367,8 @@ def bench_ours(args, dist):
 
     w = workloads.make(args.workload, seed=args.seed + 1000 * dist.rank)
     sets, per_set = make_sets(w, device, l2, 16, 64)
-    step_ms_local, kern_ms_local, t0, t1 = time_device(sets, args.steps, args.warmup, dist)
+    step_ms_local, kern_ms_local, t0, t1, graphed = time_device(sets, args.steps, args.warmup, dist,
+                                                                   not args.no_graph)
     step_ms = dist.max(step_ms_local)
     kern_ms = dist.max(kern_ms_local)
     tokens_total = dist.sum(w.T)
@@ -342,9 +395,11 @@ def bench_ours(args, dist):
                    "l2": f"{n_sets} rotating input sets of {per_set / 1e6:.1f} MB "
                          f"(inputs {n_sets * per_set / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
                    "parallelism": f"dp{dist.world} (independent batch per GPU)",
+                   "launch": "CUDA graph of the K timed steps" if graphed else "eager",
                    "seed": args.seed},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(pk["hbm_gbs"]),
-                     "unit": "GB/s", "frac": achieved / float(pk["hbm_gbs"]), "traffic": None,
+                     "unit": "GB/s", "frac": achieved / float(pk["hbm_gbs"]),
+                     "traffic": measured_traffic(w.name) if len(w.layers) == 1 else None,
                      "kernel": "bgmv_mma_kernel (lora_add_linear)", "kernel_ms": kern_ms_local,
                      "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
                      "peak_source": f"{pk.get('source')} hbm_gbs"},
@@ -374,9 +429,9 @@ def sweep_one(name, args, device, l2, pk, dist):
     from lora_adapter_application_b200 import roofline
     w = workloads.make(name, seed=args.seed)
     sets, per_set = make_sets(w, device, l2, 16, 64, max_sets=4)
-    probe_ms, _, _, _ = time_device(sets, 3, 2, dist)
+    probe_ms, _, _, _, _ = time_device(sets, 3, 3, dist, graph=False)
     K = int(min(500, max(10, args.sweep_seconds * 1e3 / probe_ms)))
-    step_ms, kern_ms, _, _ = time_device(sets, K, 3, dist)
+    step_ms, kern_ms, _, _, _ = time_device(sets, K, 3, dist, graph=not args.no_graph)
     b, f = roofline.workload_bytes(w), roofline.workload_flops(w)
     gbs = b / (kern_ms * 1e-3) / 1e9
     del sets
@@ -435,6 +490,7 @@ def main():
     ap.add_argument("--sweep-seconds", type=float, default=0.5)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch timed steps one by one")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

@@ -71,6 +71,7 @@ typedef enum {
 #define LORA_DEV_BAD_ID        1  /* id outside [-1, N): that row is treated as -1 */
 #define LORA_DEV_TILE_OVERFLOW 2  /* tile list full: the rows of dropped tiles are untouched */
 #define LORA_DEV_BAD_RANK      4  /* ranks[n] outside [1, r_max]: rows of adapter n untouched */
+#define LORA_DEV_TIMEOUT       8  /* a bounded on-chip wait ran out: the block's rows are unreliable */
 
 typedef enum { LORA_BF16 = 0, LORA_FP32 = 1 } lora_dtype;
 
@@ -142,8 +143,9 @@ LORA_API const char *lora_status_string(int status);
 LORA_API int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int32_t min_run,
                        int32_t long_tile, int32_t *max_gather, int32_t *max_contig);
 
-/* Device scratch bytes lora_build_segments needs for T rows over N slots
- * (0 when T <= 2048: the grouping then runs in one thread block). */
+/* Device scratch bytes lora_build_segments needs for T rows over N slots:
+ * per-chunk id counts plus one byte per row (0 when T <= 2048: the grouping
+ * then runs in one thread block, in shared memory). */
 LORA_API size_t lora_segments_scratch_bytes(int32_t T, int32_t N);
 
 /*

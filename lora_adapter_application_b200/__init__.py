@@ -33,7 +33,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblora_delta.so")
 
 LORA_BF16, LORA_FP32 = 0, 1
-DEV_BAD_ID, DEV_TILE_OVERFLOW, DEV_BAD_RANK = 1, 2, 4
+DEV_BAD_ID, DEV_TILE_OVERFLOW, DEV_BAD_RANK, DEV_TIMEOUT = 1, 2, 4, 8
 MAX_ROWS, MAX_ADAPTERS, MAX_RANK, MAX_SLICES, LONG_TILE = 131072, 4096, 128, 8, 128
 
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t

@@ -3,27 +3,45 @@
 // adapter) for bf16, ranks up to 64.
 //
 // One unit of work = up to 16 rows that share an adapter (a gathered tile, or
-// 16 rows of a contiguous tile).  A cluster of C thread blocks takes a unit:
+// 16 rows of a contiguous tile).  A cluster of C thread blocks takes a unit;
+// block c owns 1/C of the input columns (shrink) and 1/C of the output
+// columns (expand).  Each block is warp-specialised:
 //
-//   shrink   block c reduces its 1/C share of d_in:  v_c[row][k] = sum_j x A^T
-//            (warp-level bf16 tensor-core mma m16n8k16: M = 16 rows,
-//            N = 8 ranks, K = 16 inputs; fp32 accumulation)
-//   reduce   each block sums the C partials through distributed shared memory
-//            (fixed order, so results are run-to-run identical)
-//   expand   block c writes its 1/C share of the output columns: delta =
-//            (s v) B^T with M = 16 rows, N = 8 columns, K = 16 ranks; s v is
-//            split into bf16 hi + lo parts so the product keeps ~16 mantissa
-//            bits; y is read, added in fp32 and rounded once.
+//   producer warp   walks the block's chunk stream and fills a 3-stage
+//                   shared-memory ring through the TMA engine: one 1-D bulk
+//                   copy per x, A or y row and one for a B block whose rows are
+//                   dense; B rows with rank padding take 16-byte cp.async
+//                   pieces.  (Measured on B200: TMA copies keep the load path
+//                   free for the consumers' shared-memory traffic, where a
+//                   cp.async producer competes with it; their cost is per copy,
+//                   so rows should be long.)  Completion is counted on a
+//                   full/empty mbarrier pair per stage.
+//   8 consumer warps
+//     shrink chunks  x rows [cnt][JC] and A rows [r_n][JC] -> partial v
+//                    (tensor-core mma m16n8k16, bf16 in, fp32 accumulate)
+//     exchange       through distributed shared memory, stores only: every
+//                    block sends each partial element to the block that owns
+//                    it; the owner adds the C partials in a fixed order
+//                    (run-to-run identical), scales by alpha/r_n and stores the
+//                    result into every block's copy of v; remote mbarrier
+//                    arrivals say when the stores have landed
+//     expand chunks  B rows [CC][r_n] and y rows [cnt][CC] -> y += (s v) B^T in
+//                    fp32, rounded once, written back with 16-byte stores
 //
-// x, A, B and y cross HBM once; the rank-r intermediate never leaves the chip.
-// The arithmetic intensity (about 4 multiply-adds per byte) would keep the
-// fp32 pipe busier than HBM at the power-capped clock, so the multiply-adds
+// The producer runs up to 3 chunks ahead, across the exchange, so HBM stays
+// busy; every byte of x, A, B and y crosses HBM once and v never leaves the
+// chip.  s v enters the expand products as a bf16 hi + lo pair (about 16
+// mantissa bits): a single bf16 copy (2^-9 relative) is not enough when the
+// delta is large and cancels against y.  The multiply-adds (about 4 per byte)
 // run on the tensor pipe; the kernel is bounded by HBM bandwidth.
 //
-// Inside one 16-wide K step every thread loads 4 consecutive elements of each
-// operand row and assigns them to its four k-slots of the mma fragment; the
-// same assignment is used for both operands, so the sum is unchanged and all
-// loads are plain contiguous vectors.
+// Inside one 16-wide K step each thread assigns 4 consecutive elements of each
+// operand row to its four k-slots of the mma fragment; both operands use the
+// same assignment, so the sum is unchanged and shared-memory reads are vectors.
+//
+// Every wait is bounded (a suspend-time hint per try, and a try limit): a wait
+// that runs out sets LORA_DEV_TIMEOUT in the status word and the block skips
+// its remaining work instead of hanging.
 #include "kernels.cuh"
 
 #include <cooperative_groups.h>
@@ -32,17 +50,16 @@ namespace cg = cooperative_groups;
 
 namespace lora {
 
-constexpr int BG_THREADS = 256;
-constexpr int BG_WARPS = 8;
+constexpr int BG_CONSUMERS = 8;                      // consumer warps
+constexpr int BG_THREADS = (BG_CONSUMERS + 1) * 32;  // + 1 producer warp
 constexpr int BG_ROWS = 16;
 constexpr int BG_RMAX = 64;
-constexpr int BG_PART_STRIDE = 72;    // floats per row of the per-warp partial / staging tile
-constexpr int BG_VF_STRIDE = 80;      // floats per row of the reduced v
-constexpr int BG_COLS = 64;           // output columns per warp block
+constexpr int BG_STAGES = 3;
+constexpr int BG_STAGE_BYTES = 24576;
+constexpr int BG_VF_STRIDE = 80;   // floats per row of the reduced v (bank spread)
+constexpr unsigned BG_WAIT_LIMIT = 1u << 16;
 
-
-
-
+// ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
     asm volatile(
@@ -52,44 +69,177 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg16(const void *p) {
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+// arrival on the mbarrier at the same offset in block `rank` of the cluster
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, unsigned rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}\n" ::"r"(bar),
+        "r"(rank)
+        : "memory");
+}
+// the executing thread's earlier cp.async copies arrive on bar when they land
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+template <bool CLUSTER_ACQUIRE>
+__device__ __forceinline__ bool mbar_try(uint32_t bar, unsigned parity) {
+    uint32_t ok;
+    if (CLUSTER_ACQUIRE)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, 20000;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    return ok != 0;
+}
+// Bounded wait; false (and the status bit) once the limit is reached.
+template <bool CLUSTER_ACQUIRE = false>
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, int32_t *status,
+                                          bool &failed) {
+    if (failed) return false;
+    for (unsigned it = 0; it < BG_WAIT_LIMIT; ++it)
+        if (mbar_try<CLUSTER_ACQUIRE>(bar, parity)) return true;
+    atomicOr(status, LORA_DEV_TIMEOUT);
+    failed = true;
+    return false;
+}
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void *src, int src_bytes = 16) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+// rows x (ppr 16-byte pieces) from global (row stride src_ld elements) to shared
+// (row stride dst_ld bytes), spread over the 32 lanes of a warp.  Pieces at or
+// beyond `live` in a row are zero-filled without reading global memory.  When
+// ppr is a power of two each lane keeps one piece column and walks rows by
+// pointer increments (about four instructions per 16-byte piece).
+__device__ __forceinline__ void copy_rows(uint32_t dst, int dst_ld, const __nv_bfloat16 *src,
+                                          int64_t src_ld, int rows, int ppr, int live, int lane) {
+    if ((ppr & (ppr - 1)) == 0) {
+        if (ppr >= 32) {
+            for (int r = 0; r < rows; ++r, dst += dst_ld, src += src_ld)
+                for (int pc = lane; pc < ppr; pc += 32) {
+                    const bool in = pc < live;
+                    cp16(dst + pc * 16, in ? src + pc * 8 : src, in ? 16 : 0);
+                }
+        } else {
+            const int sh = __ffs(ppr) - 1, step = 32 >> sh;
+            const int pc = lane & (ppr - 1);
+            const bool in = pc < live;
+            const int nb = in ? 16 : 0;
+            uint32_t d = dst + (lane >> sh) * dst_ld + pc * 16;
+            const __nv_bfloat16 *q = src + (lane >> sh) * src_ld + (in ? pc * 8 : 0);
+            const uint32_t dstep = step * dst_ld;
+            const int64_t sstep = step * src_ld;
+            for (int r = lane >> sh; r < rows; r += step, d += dstep, q += sstep) cp16(d, q, nb);
+        }
+        return;
+    }
+    for (int r = 0; r < rows; ++r, dst += dst_ld, src += src_ld)
+        for (int pc = lane; pc < ppr; pc += 32) {
+            const bool in = pc < live;
+            cp16(dst + pc * 16, in ? src + pc * 8 : src, in ? 16 : 0);
+        }
+}
+
+// 1-D bulk copy global -> shared through the TMA engine, completing on bar.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;\n" ::"n"(BG_CONSUMERS * 32) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+                 : "r"(a));
     return r;
 }
-
-__device__ __forceinline__ uint2 ldg8(const void *p) {
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
     uint2 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];\n"
-                 : "=r"(r.x), "=r"(r.y)
-                 : "l"(p));
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(r.x), "=r"(r.y) : "r"(a));
     return r;
 }
-
-__device__ __forceinline__ uint32_t u4_get(const uint4 &v, int i) {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t r;
+    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(r) : "r"(a));
+    return r;
 }
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint4 zero_if(bool z, uint4 v) { return z ? make_uint4(0, 0, 0, 0) : v; }
 
-// Dynamic shared memory:
-//   part   [8 warps][16][72] fp32   shrink partials, later the expand staging tiles
-//   vcta   [S][16][64]       fp32   this block's partial v, read by the peers
-//   vfull  [S][16][80]       fp32   reduced (and scaled) v
+// Shared memory: ring | recv [S*16*64] | vfull [S][16][80] | part [16][64] | barriers
+//   recv[c*(S*1024/C) + e/C] holds block c's partial of element e = (s*16+row)*64+k,
+//   for the elements e with e % C == this block's rank.
 size_t bgmv_smem_bytes(int n_slices) {
-    return (size_t)BG_WARPS * BG_ROWS * BG_PART_STRIDE * 4 +
-           (size_t)n_slices * BG_ROWS * BG_RMAX * 4 + (size_t)n_slices * BG_ROWS * BG_VF_STRIDE * 4;
+    return (size_t)BG_STAGES * BG_STAGE_BYTES + (size_t)n_slices * BG_ROWS * BG_RMAX * 4 +
+           (size_t)n_slices * BG_ROWS * BG_VF_STRIDE * 4 + (size_t)BG_ROWS * BG_RMAX * 4 + 128;
 }
+
+struct Geo {          // chunk geometry of one block for one unit
+    int r8, nb8, nkb16;
+    int j_lo, j_hi, JC, RS, n_sc;        // shrink: columns, chunk width, row stride (bytes), chunks per slice
+    int c_lo, c_hi, CC, YS, BS, ybytes;  // expand: concatenated column range, chunk width, strides
+    bool b_dense;                        // B rows hold exactly r8 = r_max elements: one copy
+    int n_shrink, n_chunks;
+};
+
+// Position in a block's chunk stream, advanced without divisions: shrink
+// chunks slice by slice, then expand chunks slice by slice.
+struct ChunkIt {
+    int i;                 // chunk index
+    int s, q;              // shrink: slice, chunk in slice
+    int es, c0, w;         // expand: slice, first slice-local column, width
+};
 
 template <int MODE>
-__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_mma_kernel(BgArgs a) {
-    extern __shared__ __align__(16) float bg_sm[];
+__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
+    extern __shared__ __align__(128) unsigned char bg_sm[];
     __shared__ int rows_sm[BG_ROWS];
 
     const int S = a.sl.n;
-    float *part = bg_sm;
-    float *vcta = part + BG_WARPS * BG_ROWS * BG_PART_STRIDE;
-    float *vfull = vcta + S * BG_ROWS * BG_RMAX;
+    unsigned char *ring = bg_sm;
+    float *recv = reinterpret_cast<float *>(bg_sm + BG_STAGES * BG_STAGE_BYTES);
+    float *vfull = recv + S * BG_ROWS * BG_RMAX;
+    float *part = vfull + S * BG_ROWS * BG_VF_STRIDE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(part + BG_ROWS * BG_RMAX);
+    const uint32_t ring_s = smem_u32(ring);
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * BG_STAGES;
+    const uint32_t xready = full0 + 16 * BG_STAGES, vready = xready + 8;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -103,155 +253,276 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_mma_kernel(BgArgs a) {
         if (crank == 0 && tid == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
         return;
     }
-    if (tid < BG_ROWS) rows_sm[tid] = tid < u.cnt ? u.row(a.tiles, tid) : -1;
-    __syncthreads();
-
     const int cnt = u.cnt;
-    const int nb8 = (r_n + 7) >> 3;
+    if (tid < BG_ROWS) rows_sm[tid] = tid < cnt ? u.row(a.tiles, tid) : -1;
+    for (int e = tid; e < S * BG_ROWS * BG_VF_STRIDE; e += BG_THREADS) vfull[e] = 0.f;
 
+    // ------------------------------------------------------------ geometry
+    Geo G;
+    G.r8 = (r_n + 7) & ~7;
+    G.nb8 = G.r8 >> 3;
+    G.nkb16 = (r_n + 15) >> 4;
     if (MODE != MODE_EXPAND) {
-        // ------------------------------------------------------------ shrink
-        const int row_g = rows_sm[g], row_h = rows_sm[g + 8];
         const int n64 = (a.d_in + 63) >> 6;
-        const int st_lo = (int)((int64_t)crank * n64 / C), st_hi = (int)((int64_t)(crank + 1) * n64 / C);
-        const __nv_bfloat16 *xg = row_g >= 0 ? a.x + (int64_t)row_g * a.ld_x : nullptr;
-        const __nv_bfloat16 *xh = row_h >= 0 ? a.x + (int64_t)row_h * a.ld_x : nullptr;
-        float *mypart = part + warp * BG_ROWS * BG_PART_STRIDE;
-
+        G.j_lo = (int)((int64_t)crank * n64 / C) * 64;
+        G.j_hi = min((int)((int64_t)(crank + 1) * n64 / C) * 64, a.d_in);
+        // widest power-of-two chunk (>= 64 columns) whose rows fit a stage
+        const int lim = ((BG_STAGE_BYTES / (BG_ROWS + G.r8)) - 16) / 2;
+        int jc = 64;
+        while (jc * 2 <= lim) jc *= 2;
+        const int span = max(0, G.j_hi - G.j_lo);
+        while (jc > 64 && jc / 2 >= span) jc /= 2;
+        G.JC = jc;
+        G.RS = G.JC * 2 + 16;
+        G.n_sc = (span + G.JC - 1) / G.JC;
+    } else {
+        G.j_lo = G.j_hi = 0;
+        G.JC = 64;
+        G.RS = 144;
+        G.n_sc = 0;
+    }
+    G.n_shrink = S * G.n_sc;
+    G.n_chunks = G.n_shrink;
+    G.b_dense = G.r8 == a.r_max;
+    if (MODE != MODE_SHRINK) {
+        const int n8 = a.sl.cat_off[S] >> 3;
+        G.c_lo = (int)((int64_t)crank * n8 / C) * 8;
+        G.c_hi = (int)((int64_t)(crank + 1) * n8 / C) * 8;
+        G.BS = G.b_dense ? G.r8 * 2 : G.r8 * 2 + (G.r8 >= 32 ? 32 : 0);
+        // y rows: stride = 16 (mod 128) bytes, so the 8 rows of an mma tile hit 8 bank groups
+        const int lim = (BG_STAGE_BYTES - 144 * BG_ROWS) / (2 * BG_ROWS + G.BS);
+        int cc = 8;   // widest power-of-two chunk whose y rows and B rows fit a stage
+        while (cc * 2 <= lim) cc *= 2;
+        G.CC = cc;
+        G.YS = ((G.CC * 2 + 127) & ~127) + 16;
+        G.ybytes = BG_ROWS * G.YS;
         for (int s = 0; s < S; ++s) {
-            const __nv_bfloat16 *An =
-                static_cast<const __nv_bfloat16 *>(a.sl.A[s]) + (int64_t)n * a.r_max * a.d_in;
-            float acc[8][4];
-#pragma unroll
-            for (int kb = 0; kb < 8; ++kb)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[kb][e] = 0.f;
-
-            for (int st = st_lo + warp; st < st_hi; st += BG_WARPS) {
-                const int j = st * 64 + 16 * t;
-                const bool in0 = j + 8 <= a.d_in, in1 = j + 16 <= a.d_in;
-                const uint4 z = make_uint4(0, 0, 0, 0);
-                const uint4 xg0 = (xg && in0) ? ldg16(xg + j) : z;
-                const uint4 xg1 = (xg && in1) ? ldg16(xg + j + 8) : z;
-                const uint4 xh0 = (xh && in0) ? ldg16(xh + j) : z;
-                const uint4 xh1 = (xh && in1) ? ldg16(xh + j + 8) : z;
-                uint4 av0[8], av1[8];
-#pragma unroll
-                for (int kb = 0; kb < 8; ++kb) {
-                    const int k = kb * 8 + g;
-                    const bool ok = kb < nb8 && k < r_n;
-                    const __nv_bfloat16 *ap = An + (int64_t)k * a.d_in + j;
-                    av0[kb] = (ok && in0) ? ldg16(ap) : z;
-                    av1[kb] = (ok && in1) ? ldg16(ap + 8) : z;
-                }
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint4 &xa = b < 2 ? xg0 : xg1;
-                    const uint4 &xb = b < 2 ? xh0 : xh1;
-                    const int q = (b & 1) * 2;
-                    const uint32_t fa[4] = {u4_get(xa, q), u4_get(xb, q), u4_get(xa, q + 1),
-                                            u4_get(xb, q + 1)};
-#pragma unroll
-                    for (int kb = 0; kb < 8; ++kb) {
-                        if (kb < nb8) {
-                            const uint4 &av = b < 2 ? av0[kb] : av1[kb];
-                            mma16816(acc[kb], fa, u4_get(av, q), u4_get(av, q + 1));
-                        }
-                    }
-                }
-            }
-            // per-warp partial -> shared, then the block's sum in warp order
-#pragma unroll
-            for (int kb = 0; kb < 8; ++kb) {
-                if (kb < nb8) {
-                    const int k = kb * 8 + 2 * t;
-                    *reinterpret_cast<float2 *>(&mypart[g * BG_PART_STRIDE + k]) =
-                        make_float2(acc[kb][0], acc[kb][1]);
-                    *reinterpret_cast<float2 *>(&mypart[(g + 8) * BG_PART_STRIDE + k]) =
-                        make_float2(acc[kb][2], acc[kb][3]);
-                }
-            }
-            __syncthreads();
-            for (int e = tid; e < BG_ROWS * BG_RMAX; e += BG_THREADS) {
-                const int row = e >> 6, k = e & 63;
-                float sum = 0.f;
-                if (k < nb8 * 8) {
-#pragma unroll
-                    for (int w = 0; w < BG_WARPS; ++w)
-                        sum += part[(w * BG_ROWS + row) * BG_PART_STRIDE + k];
-                }
-                vcta[(s * BG_ROWS + row) * BG_RMAX + k] = sum;
-            }
-            __syncthreads();
+            const int lo = max(G.c_lo, a.sl.cat_off[s]), hi = min(G.c_hi, a.sl.cat_off[s + 1]);
+            if (hi > lo) G.n_chunks += (hi - lo + G.CC - 1) / G.CC;
         }
+    } else {
+        G.c_lo = G.c_hi = 0;
+        G.CC = 8;
+        G.YS = 32;
+        G.BS = 16;
+        G.ybytes = 0;
+    }
 
-        // ------------------------------------------------------------ cluster reduce
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();
-        const float scale = MODE == MODE_FUSED ? a.scales[n] : 1.f;
-        for (int e = tid; e < S * BG_ROWS * BG_RMAX; e += BG_THREADS) {
-            const int s = e / (BG_ROWS * BG_RMAX);
-            const int rem = e - s * BG_ROWS * BG_RMAX;
-            const int row = rem >> 6, k = rem & 63;
-            float sum = 0.f;
-            if (row < cnt && k < r_n) {
-                for (int c = 0; c < C; ++c) {
-                    const float *peer = cluster.map_shared_rank(vcta, c);
-                    sum += peer[e];
-                }
-            }
-            vfull[(s * BG_ROWS + row) * BG_VF_STRIDE + k] = scale * sum;
-        }
-        cluster.sync();
-
-        if (MODE == MODE_SHRINK) {
-            if (crank == 0) {
-                for (int e = tid; e < S * BG_ROWS * BG_RMAX; e += BG_THREADS) {
-                    const int s = e / (BG_ROWS * BG_RMAX);
-                    const int rem = e - s * BG_ROWS * BG_RMAX;
-                    const int row = rem >> 6, k = rem & 63;
-                    if (row < cnt && k < r_n)
-                        a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] =
-                            vfull[(s * BG_ROWS + row) * BG_VF_STRIDE + k];
-                }
+    // next position of the chunk stream
+    auto advance = [&](ChunkIt &it) {
+        ++it.i;
+        if (it.i < G.n_shrink) {
+            if (++it.q == G.n_sc) {
+                it.q = 0;
+                ++it.s;
             }
             return;
         }
-    } else {
-        const float scale = a.scales[n];
-        for (int e = tid; e < S * BG_ROWS * BG_RMAX; e += BG_THREADS) {
-            const int s = e / (BG_ROWS * BG_RMAX);
-            const int rem = e - s * BG_ROWS * BG_RMAX;
-            const int row = rem >> 6, k = rem & 63;
-            float val = 0.f;
-            if (row < cnt && k < r_n)
-                val = scale * a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k];
-            vfull[(s * BG_ROWS + row) * BG_VF_STRIDE + k] = val;
+        if (it.i >= G.n_chunks) return;
+        if (it.es >= 0) {   // next block of columns in this slice?
+            const int hi = min(G.c_hi, a.sl.cat_off[it.es + 1]) - a.sl.cat_off[it.es];
+            if (it.c0 + G.CC < hi) {
+                it.c0 += G.CC;
+                it.w = min(G.CC, hi - it.c0);
+                return;
+            }
         }
+        for (int s = it.es + 1; s < S; ++s) {   // first later slice with columns in this block
+            const int lo = max(G.c_lo, a.sl.cat_off[s]), hi = min(G.c_hi, a.sl.cat_off[s + 1]);
+            if (hi > lo) {
+                it.es = s;
+                it.c0 = lo - a.sl.cat_off[s];
+                it.w = min(G.CC, hi - lo);
+                return;
+            }
+        }
+    };
+    auto first = [&](ChunkIt &it) {
+        it.i = 0;
+        it.s = it.q = 0;
+        it.es = -1;
+        it.c0 = it.w = 0;
+        if (G.n_shrink == 0 && G.n_chunks > 0) {   // the stream starts with expand chunks
+            it.i = -1;
+            advance(it);
+        }
+    };
+
+    // barriers
+    if (tid == 0) {
+        for (int st = 0; st < BG_STAGES; ++st) {
+            mbar_init(full0 + 8 * st, 33);
+            mbar_init(empty0 + 8 * st, BG_CONSUMERS);
+        }
+        mbar_init(xready, C);
+        mbar_init(vready, C);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    __syncthreads();
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();   // barriers initialised in every block; rows_sm and vfull ready
 
-    // ---------------------------------------------------------------- expand
-    int nbt = 0;
-    for (int s = 0; s < S; ++s) nbt += (a.sl.d_out[s] + BG_COLS - 1) / BG_COLS;
-    const int b_lo = (int)((int64_t)crank * nbt / C), b_hi = (int)((int64_t)(crank + 1) * nbt / C);
-    const int nkb = (r_n + 15) >> 4;
-    float *stage = part + warp * BG_ROWS * BG_PART_STRIDE;
+    bool failed = false;
 
-    int cur_s = -1, s_first = 0;
-    uint32_t ahi[4][4], alo[4][4];
-    for (int blk = b_lo + warp; blk < b_hi; blk += BG_WARPS) {
-        // which slice, which block inside it
-        int s = 0, first = 0;
-        while (true) {
-            const int nb_s = (a.sl.d_out[s] + BG_COLS - 1) / BG_COLS;
-            if (blk < first + nb_s) break;
-            first += nb_s;
-            ++s;
+    if (warp == BG_CONSUMERS) {
+        // ============================================================ producer
+        ChunkIt it;
+        first(it);
+        for (; it.i < G.n_chunks; advance(it)) {
+            const int st = it.i % BG_STAGES;
+            const uint32_t full = full0 + 8 * st, dst = ring_s + st * BG_STAGE_BYTES;
+            if (it.i >= BG_STAGES)
+                mbar_wait(empty0 + 8 * st, ((it.i / BG_STAGES) - 1) & 1, a.status, failed);
+            if (failed) break;
+            if (it.i < G.n_shrink) {
+                const int jc0 = G.j_lo + it.q * G.JC;
+                const unsigned bytes = (unsigned)min(G.JC, G.j_hi - jc0) * 2;
+                if (lane == 0) mbar_expect_tx(full, bytes * (cnt + r_n));
+                __syncwarp();
+                const __nv_bfloat16 *An = static_cast<const __nv_bfloat16 *>(a.sl.A[it.s]) + (int64_t)n * a.r_max * a.d_in + jc0;
+                for (int r = lane; r < cnt + r_n; r += 32) {
+                    if (r < cnt) bulk_g2s(dst + r * G.RS, a.x + (int64_t)rows_sm[r] * a.ld_x + jc0, bytes, full);
+                    else bulk_g2s(dst + (BG_ROWS + r - cnt) * G.RS, An + (int64_t)(r - cnt) * a.d_in, bytes, full);
+                }
+            } else {
+                const int s = it.es, d_out = a.sl.d_out[s];
+                const unsigned ybytes = (unsigned)it.w * 2;
+                const __nv_bfloat16 *Bn = static_cast<const __nv_bfloat16 *>(a.sl.B[s]) + ((int64_t)n * d_out + it.c0) * a.r_max;
+                const unsigned bbytes = G.b_dense ? (unsigned)it.w * a.r_max * 2 : 0u;
+                if (lane == 0) mbar_expect_tx(full, ybytes * cnt + bbytes);
+                __syncwarp();
+                for (int r = lane; r < cnt; r += 32)
+                    bulk_g2s(dst + r * G.YS, a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0, ybytes, full);
+                if (G.b_dense) { if (lane == 0) bulk_g2s(dst + G.ybytes, Bn, bbytes, full); }
+                else copy_rows(dst + G.ybytes, G.BS, Bn, a.r_max, it.w, G.r8 >> 3, G.r8 >> 3, lane);
+            }
+            cp_async_arrive(full);
         }
-        if (s != cur_s) {   // fragments of s*v for this slice
+        return;
+    }
+
+    // ================================================================ consumers
+    const int jg = max(1, BG_CONSUMERS / G.nb8);   // warps per 8-rank block
+    const bool shrink_warp = warp < G.nb8 * jg;
+    const int nbw = warp / jg, jgi = warp - (warp / jg) * jg;
+    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ctid = tid;   // 0 .. 255
+    const int per_src = (S * BG_ROWS * BG_RMAX) / C;
+
+    // block partial of slice s (from part, or zeros) -> recv of the owning block
+    auto send_partials = [&](int s, bool from_part) {
+        for (int idx = ctid; idx < cnt * G.r8; idx += BG_CONSUMERS * 32) {
+            const int row = idx / G.r8, k = idx - row * G.r8;
+            float sum = 0.f;
+            if (from_part)
+                for (int j = 0; j < jg; ++j) sum += part[(j * BG_ROWS + row) * G.r8 + k];
+            const int e = (s * BG_ROWS + row) * BG_RMAX + k;
+            float *dst = cluster.map_shared_rank(recv, e % C);
+            dst[crank * per_src + e / C] = sum;
+        }
+    };
+
+    auto shrink_chunk = [&](const ChunkIt &it, uint32_t st) {
+        if (shrink_warp) {
+            const int jc0 = G.j_lo + it.q * G.JC;
+            const int width = min(G.JC, G.j_hi - jc0);
+            const int nsteps = (width + 63) >> 6;
+            const uint32_t xg = st + g * G.RS, xh = st + (g + 8) * G.RS;
+            const uint32_t ak = st + (BG_ROWS + nbw * 8 + g) * G.RS;
+            for (int sp = jgi; sp < nsteps; sp += jg) {
+                const int col = sp * 64 + t * 16;
+                const bool z0 = col >= width, z1 = col + 8 >= width;   // beyond the chunk: zero
+                const uint32_t off = (uint32_t)(col * 2);
+                const uint4 xa0 = zero_if(z0, lds128(xg + off)), xa1 = zero_if(z1, lds128(xg + off + 16));
+                const uint4 xb0 = zero_if(z0, lds128(xh + off)), xb1 = zero_if(z1, lds128(xh + off + 16));
+                const uint4 a0 = zero_if(z0, lds128(ak + off)), a1 = zero_if(z1, lds128(ak + off + 16));
+                {
+                    const uint32_t f[4] = {xa0.x, xb0.x, xa0.y, xb0.y};
+                    mma16816(acc0, f, a0.x, a0.y);
+                }
+                {
+                    const uint32_t f[4] = {xa0.z, xb0.z, xa0.w, xb0.w};
+                    mma16816(acc1, f, a0.z, a0.w);
+                }
+                {
+                    const uint32_t f[4] = {xa1.x, xb1.x, xa1.y, xb1.y};
+                    mma16816(acc0, f, a1.x, a1.y);
+                }
+                {
+                    const uint32_t f[4] = {xa1.z, xb1.z, xa1.w, xb1.w};
+                    mma16816(acc1, f, a1.z, a1.w);
+                }
+            }
+        }
+        if (it.q == G.n_sc - 1) {   // slice done: block partial -> owners
+            consumer_sync();        // every warp is past its reads of part from the last slice
+            if (shrink_warp) {
+                const int k = nbw * 8 + 2 * t;
+                part[(jgi * BG_ROWS + g) * G.r8 + k] = acc0[0] + acc1[0];
+                part[(jgi * BG_ROWS + g) * G.r8 + k + 1] = acc0[1] + acc1[1];
+                part[(jgi * BG_ROWS + g + 8) * G.r8 + k] = acc0[2] + acc1[2];
+                part[(jgi * BG_ROWS + g + 8) * G.r8 + k + 1] = acc0[3] + acc1[3];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc0[e] = acc1[e] = 0.f;
+            }
+            consumer_sync();
+            send_partials(it.s, true);
+        }
+    };
+
+    auto exchange = [&]() {
+        if (MODE == MODE_EXPAND) {
+            const float scale = a.scales[n];
+            for (int e = ctid; e < S * BG_ROWS * BG_RMAX; e += BG_CONSUMERS * 32) {
+                const int s = e >> 10, rem = e & 1023;
+                const int row = rem >> 6, k = rem & 63;
+                if (row < cnt && k < G.r8)
+                    vfull[(s * BG_ROWS + row) * BG_VF_STRIDE + k] =
+                        k < r_n ? scale * a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] : 0.f;
+            }
+            consumer_sync();
+            return;
+        }
+        if (G.n_sc == 0)   // no input columns here: the partials are zero
+            for (int s = 0; s < S; ++s) send_partials(s, false);
+        consumer_sync();
+        if (ctid == 0) {
+            asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
+            for (int c = 0; c < C; ++c) mbar_arrive_remote(xready, c);
+        }
+        mbar_wait<true>(xready, 0, a.status, failed);   // every partial has reached its owner
+        const float scale = MODE == MODE_FUSED ? a.scales[n] : 1.f;
+        const int mine = (S * BG_ROWS * BG_RMAX - crank + C - 1) / C;   // elements e = crank + C*j
+        for (int j = ctid; j < mine; j += BG_CONSUMERS * 32) {
+            const int e = crank + C * j;
+            const int s = e >> 10, rem = e & 1023;
+            const int row = rem >> 6, k = rem & 63;
+            if (row >= cnt || k >= G.r8) continue;
+            float sum = 0.f;
+            for (int c = 0; c < C; ++c) sum += recv[c * per_src + j];
+            const float val = k < r_n ? scale * sum : 0.f;
+            if (MODE == MODE_SHRINK) {
+                if (k < r_n) a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] = val;
+            } else {
+                const int f = (s * BG_ROWS + row) * BG_VF_STRIDE + k;
+                for (int c = 0; c < C; ++c) cluster.map_shared_rank(vfull, c)[f] = val;
+            }
+        }
+        if (MODE == MODE_FUSED) {
+            consumer_sync();
+            if (ctid == 0) {
+                asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
+                for (int c = 0; c < C; ++c) mbar_arrive_remote(vready, c);
+            }
+            mbar_wait<true>(vready, 0, a.status, failed);   // every block holds the full s*v
+        }
+    };
+
+    int cur_s = -1;
+    uint32_t ahi[4][4], alo[4][4];
+    auto expand_chunk = [&](const ChunkIt &it, uint32_t st) {
+        const int s = it.es;
+        if (s != cur_s) {   // mma fragments of s*v (bf16 hi + lo) for this slice
             cur_s = s;
-            s_first = first;
             const float *vf = vfull + s * BG_ROWS * BG_VF_STRIDE;
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
@@ -268,82 +539,99 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_mma_kernel(BgArgs a) {
                 alo[kb][3] = pack_bf16x2(q.z - bf16_lo(ahi[kb][3]), q.w - bf16_hi(ahi[kb][3]));
             }
         }
-        const int d_out = a.sl.d_out[s];
-        const int c0 = (blk - s_first) * BG_COLS;
-        const __nv_bfloat16 *Bn =
-            static_cast<const __nv_bfloat16 *>(a.sl.B[s]) + (int64_t)n * d_out * a.r_max;
-
-        // y of this block: lane owns columns c0 + 2*lane, +1 of every row
-        const int ycol = c0 + 2 * lane;
-        const bool ycol_ok = ycol < d_out;
-        uint32_t yv[BG_ROWS];
+        const int nblk = it.w >> 3;
+        const uint32_t bbase = st + G.ybytes + g * G.BS;
+        for (int nb0 = warp * 2; nb0 < nblk; nb0 += BG_CONSUMERS * 2) {
+            float d[2][4];
 #pragma unroll
-        for (int r = 0; r < BG_ROWS; ++r) {
-            yv[r] = 0;
-            if (r < cnt && ycol_ok)
-                yv[r] = *reinterpret_cast<const uint32_t *>(
-                    a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + ycol);
-        }
-
-        float acc[8][4];
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
-        for (int nb = 0; nb < 8; ++nb)
+                for (int e = 0; e < 4; ++e) d[j][e] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nb][e] = 0.f;
+            for (int kb = 0; kb < 4; ++kb) {
+                if (kb < G.nkb16) {
+                    const int k = kb * 16 + 4 * t;
+                    uint2 bv[2];
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-            if (kb < nkb) {
-                const int k = kb * 16 + 4 * t;
-                uint2 bv[8];
-#pragma unroll
-                for (int nb = 0; nb < 8; ++nb) {
-                    const int col = c0 + nb * 8 + g;
-                    bv[nb] = make_uint2(0, 0);
-                    if (col < d_out && k < r_n) {
-                        bv[nb] = ldg8(Bn + (int64_t)col * a.r_max + k);
-                        if (k + 4 > r_n) {   // rank ends inside this group of 4
-                            const int keep = r_n - k;
-                            if (keep < 2) bv[nb].x &= 0xffffu;
-                            if (keep < 3) bv[nb].y = 0;
-                            else bv[nb].y &= 0xffffu;
+                    for (int j = 0; j < 2; ++j) {
+                        bv[j] = make_uint2(0, 0);
+                        if (k < r_n && nb0 + j < nblk) {
+                            bv[j] = lds64(bbase + (nb0 + j) * 8 * G.BS + k * 2);
+                            if (k + 4 > r_n) {   // the rank ends inside this group of 4
+                                const int keep = r_n - k;
+                                if (keep < 2) bv[j].x &= 0xffffu;
+                                if (keep < 3) bv[j].y = 0;
+                                else bv[j].y &= 0xffffu;
+                            }
                         }
                     }
-                }
 #pragma unroll
-                for (int nb = 0; nb < 8; ++nb) {
-                    mma16816(acc[nb], ahi[kb], bv[nb].x, bv[nb].y);
-                    mma16816(acc[nb], alo[kb], bv[nb].x, bv[nb].y);
+                    for (int j = 0; j < 2; ++j) mma16816(d[j], ahi[kb], bv[j].x, bv[j].y);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) mma16816(d[j], alo[kb], bv[j].x, bv[j].y);
+                }
+            }
+            // y += delta in shared memory (rows g and g+8, columns 2t, 2t+1 of each 8-column block)
+            const uint32_t yg = st + g * G.YS + (nb0 * 8 + 2 * t) * 2;
+            const uint32_t yh = yg + 8 * G.YS;
+            uint32_t y0[2], y1[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const bool ok = nb0 + j < nblk;
+                y0[j] = (ok && g < cnt) ? lds32(yg + j * 16) : 0u;
+                y1[j] = (ok && g + 8 < cnt) ? lds32(yh + j * 16) : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (nb0 + j < nblk) {
+                    if (g < cnt)
+                        sts32(yg + j * 16, pack_bf16x2(bf16_lo(y0[j]) + d[j][0], bf16_hi(y0[j]) + d[j][1]));
+                    if (g + 8 < cnt)
+                        sts32(yh + j * 16, pack_bf16x2(bf16_lo(y1[j]) + d[j][2], bf16_hi(y1[j]) + d[j][3]));
                 }
             }
         }
-        // stage the 16 x 64 fp32 delta, then add it to y row by row
-#pragma unroll
-        for (int nb = 0; nb < 8; ++nb) {
-            *reinterpret_cast<float2 *>(&stage[g * BG_PART_STRIDE + nb * 8 + 2 * t]) =
-                make_float2(acc[nb][0], acc[nb][1]);
-            *reinterpret_cast<float2 *>(&stage[(g + 8) * BG_PART_STRIDE + nb * 8 + 2 * t]) =
-                make_float2(acc[nb][2], acc[nb][3]);
+        consumer_sync();
+        const int ypc = it.w >> 3;
+        const unsigned char *stp = ring + (st - ring_s);
+        for (int r = warp; r < cnt; r += BG_CONSUMERS) {
+            __nv_bfloat16 *dst = a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0;
+            for (int pc = lane; pc < ypc; pc += 32)
+                *reinterpret_cast<uint4 *>(dst + pc * 8) =
+                    *reinterpret_cast<const uint4 *>(stp + r * G.YS + pc * 16);
         }
-        __syncwarp();
-#pragma unroll
-        for (int r = 0; r < BG_ROWS; ++r) {
-            if (r < cnt && ycol_ok) {
-                const float2 d = *reinterpret_cast<const float2 *>(&stage[r * BG_PART_STRIDE + 2 * lane]);
-                const uint32_t out = pack_bf16x2(bf16_lo(yv[r]) + d.x, bf16_hi(yv[r]) + d.y);
-                *reinterpret_cast<uint32_t *>(a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] +
-                                              ycol) = out;
-            }
+    };
+
+    ChunkIt it;
+    first(it);
+    bool exchanged = false;
+    for (; it.i < G.n_chunks; advance(it)) {
+        const int st = it.i % BG_STAGES;
+        const uint32_t sta = ring_s + st * BG_STAGE_BYTES;
+        if (!exchanged && it.i >= G.n_shrink) {
+            exchange();
+            exchanged = true;
         }
+        const bool ready = mbar_wait(full0 + 8 * st, (it.i / BG_STAGES) & 1, a.status, failed);
+        if (ready) {
+            if (it.i < G.n_shrink)
+                shrink_chunk(it, sta);
+            else
+                expand_chunk(it, sta);
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * st);
     }
+    if (!exchanged) exchange();
 }
 
 int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_t st) {
     const size_t smem = bgmv_smem_bytes(a.sl.n);
     static bool attr_done[3] = {false, false, false};
-    const void *fn = mode == MODE_FUSED    ? (const void *)bgmv_mma_kernel<MODE_FUSED>
-                     : mode == MODE_SHRINK ? (const void *)bgmv_mma_kernel<MODE_SHRINK>
-                                           : (const void *)bgmv_mma_kernel<MODE_EXPAND>;
+    const void *fn = mode == MODE_FUSED    ? (const void *)bgmv_kernel<MODE_FUSED>
+                     : mode == MODE_SHRINK ? (const void *)bgmv_kernel<MODE_SHRINK>
+                                           : (const void *)bgmv_kernel<MODE_EXPAND>;
     if (!attr_done[mode]) {
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bgmv_smem_bytes(LORA_MAX_SLICES));
@@ -361,14 +649,14 @@ int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = mode == MODE_EXPAND ? 0 : 1;
+    cfg.numAttrs = 1;
     cudaError_t err;
     if (mode == MODE_FUSED)
-        err = cudaLaunchKernelEx(&cfg, bgmv_mma_kernel<MODE_FUSED>, a);
+        err = cudaLaunchKernelEx(&cfg, bgmv_kernel<MODE_FUSED>, a);
     else if (mode == MODE_SHRINK)
-        err = cudaLaunchKernelEx(&cfg, bgmv_mma_kernel<MODE_SHRINK>, a);
+        err = cudaLaunchKernelEx(&cfg, bgmv_kernel<MODE_SHRINK>, a);
     else
-        err = cudaLaunchKernelEx(&cfg, bgmv_mma_kernel<MODE_EXPAND>, a);
+        err = cudaLaunchKernelEx(&cfg, bgmv_kernel<MODE_EXPAND>, a);
     return err == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 

@@ -8,7 +8,17 @@ using namespace lora;
 
 namespace {
 
-constexpr int BGMV_CLUSTER = 8;
+// Blocks per unit of the fused kernel: the smallest power of two (up to 8)
+// that gives about three blocks per SM, so a unit is split only as far as
+// needed to fill the GPU (fewer, larger blocks hide their start-up latency).
+int bgmv_cluster(int units) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int c = 1;
+    while (c < 8 && (int64_t)units * c < 3LL * sms) c <<= 1;
+    return c;
+}
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -99,18 +109,19 @@ Tiles make_tiles(const lora_meta *m, bool gather, bool contig) {
 
 int n_units(const Tiles &t) { return t.max_gather + (t.subs ? t.max_contig * t.subs : 0); }
 
-// The vectorised bf16 tensor-pipe kernel takes the call?
+// The vectorised bf16 tensor-pipe kernel takes the call?  It moves 16-byte
+// pieces, so every row start and width must be a multiple of 8 elements.
 bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
-    if (c.dtype != LORA_BF16 || c.r_max > 64 || (c.r_max & 3)) return false;
+    if (c.dtype != LORA_BF16 || c.r_max > 64 || (c.r_max & 7)) return false;
     if (need_x) {
         if ((c.d_in & 7) || (c.ld_x & 7) || !aligned(c.x, 16)) return false;
         for (int s = 0; s < c.n_slices; ++s)
             if (!aligned(c.slices[s].A, 16)) return false;
     }
     if (need_y) {
-        if ((c.ld_y & 1) || !aligned(c.y, 4)) return false;
+        if ((c.ld_y & 7) || !aligned(c.y, 16)) return false;
         for (int s = 0; s < c.n_slices; ++s)
-            if ((c.slices[s].d_out & 1) || (c.slices[s].col_off & 1) || !aligned(c.slices[s].B, 8))
+            if ((c.slices[s].d_out & 7) || (c.slices[s].col_off & 7) || !aligned(c.slices[s].B, 16))
                 return false;
     }
     return true;
@@ -136,7 +147,7 @@ int run(int mode, const Call &c, bool gather, bool contig) {
         a.scales = c.scales;
         a.tiles = tiles;
         a.status = c.status;
-        return launch_bgmv(mode, a, units, BGMV_CLUSTER, c.stream);
+        return launch_bgmv(mode, a, units, bgmv_cluster(units), c.stream);
     }
     SimtArgs a{};
     a.x = c.x;

@@ -7,7 +7,7 @@
 // all in a single launch (decode batches).  Above that:
 //   seg_hist     one block per chunk of SEG_CHUNK rows: per-chunk id histogram
 //   seg_scan     one block: totals -> seg_start, seg_adapter, per-chunk bases
-//   seg_scatter  one warp per chunk: stable ranks with __match_any_sync
+//   seg_scatter  one block per chunk: every warp ranks its share of the rows
 //   seg_tiles    one block: runs, contiguous tiles, gathered rows and tiles
 // No block ever waits for another block: the phases are separate launches.
 #include "common.cuh"
@@ -52,34 +52,6 @@ __device__ int block_excl_sum(int v, int *total, int *sm) {
     return res;
 }
 
-// For each thread, the minimum of v over the threads after it (INT_MAX if none).
-__device__ int block_excl_suffix_min(int v, int *sm) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int t = __shfl_down_sync(FULL, incl, o);
-        if (lane + o < 32) incl = min(incl, t);
-    }
-    if (lane == 0) sm[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int wi = sm[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int t = __shfl_down_sync(FULL, wi, o);
-            if (lane + o < 32) wi = min(wi, t);
-        }
-        sm[lane] = wi;
-    }
-    __syncthreads();
-    int within = __shfl_down_sync(FULL, incl, 1);
-    if (lane == 31) within = INT_MAX;
-    int after = warp < 31 ? sm[warp + 1] : INT_MAX;
-    __syncthreads();
-    return min(within, after);
-}
-
 // Turn per-id counts hist[0..N] (bin N = rows without a valid id) into start
 // offsets; write seg_start, seg_adapter and counts[0].  Whole block.
 __device__ void seg_scan_block(int *hist, int N, int32_t *seg_start, int32_t *seg_adapter,
@@ -109,28 +81,69 @@ __device__ void seg_scan_block(int *hist, int N, int32_t *seg_start, int32_t *se
     }
 }
 
-// Stable placement of rows [lo, hi) by one warp, starting at base[bin].
-__device__ void scatter_warp(const int32_t *ids, int lo, int hi, int N, int *base, int32_t *perm) {
+// Lanes of the warp whose key equals this lane's key.  One ballot per key bit
+// (keys < 2^nbits); a hardware match instruction is far slower here.
+__device__ __forceinline__ unsigned equal_lanes(int key, int nbits) {
+    unsigned eq = FULL;
+    for (int b = 0; b < nbits; ++b) {
+        const unsigned m = __ballot_sync(FULL, (key >> b) & 1);
+        eq &= ((key >> b) & 1) ? m : ~m;
+    }
+    return eq;
+}
+
+// Stable placement of rows [lo, hi) by one warp, starting at base[bin].  Also
+// records, for every placed row, whether it starts a run: a row starts a run
+// when the row before it (in row order) has another id.  Because the grouping
+// is stable, that is the same as "the previous position holds another id or a
+// row that is not the previous row".
+__device__ void scatter_warp(const int32_t *ids, int lo, int hi, int N, int *base, int32_t *perm,
+                             uint8_t *brkb) {
     const int lane = threadIdx.x & 31;
+    const int nbits = 32 - __clz(N + 1 + 32);
     for (int i0 = lo; i0 < hi; i0 += 32) {
         const int i = i0 + lane;
         const bool v = i < hi;
-        const int key = v ? bin_of(ids[i], N) : N + 1 + lane;
-        const unsigned m = __match_any_sync(FULL, key);
+        const int id = v ? ids[i] : 0;
+        int prev = __shfl_up_sync(FULL, id, 1);
+        if (lane == 0) prev = i > 0 ? ids[i - 1] : INT_MIN;
+        const int key = v ? bin_of(id, N) : N + 1 + lane;
+        const unsigned m = equal_lanes(key, nbits);
         const int rank = __popc(m & ((1u << lane) - 1u));
         const int pos = v ? base[key] + rank : 0;
         __syncwarp();
         if (v) {
             perm[pos] = i;
+            if (key < N) brkb[pos] = (i == 0 || prev != id) ? 1 : 0;
             if (rank == 0) base[key] += __popc(m);
         }
         __syncwarp();
     }
 }
 
-__device__ __forceinline__ uint32_t bit_range(int a, int b) {   // bits [a, b), 0 <= a < b <= 32
-    uint32_t hi = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
-    return hi & ~((1u << a) - 1u);
+// Exclusive prefix over the block's warps of one value per warp (taken from
+// lane 0), and the total.  All threads of the block call it.  wsum: 33 ints.
+__device__ int warp_excl_scan(int v, int *total, int *wsum) {
+    constexpr int NW = SEG_THREADS / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) wsum[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        const int x = lane < NW ? wsum[lane] : 0;
+        int incl = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o) incl += t;
+        }
+        wsum[lane] = incl - x;
+        if (lane == 31) wsum[32] = incl;
+    }
+    __syncthreads();
+    const int r = wsum[warp];
+    *total = wsum[32];
+    __syncthreads();
+    return r;
 }
 
 struct TileOut {
@@ -143,196 +156,326 @@ struct TileOut {
     int R, min_run, LT;
 };
 
+// Shared-memory words used by dev_tiles: 4 arrays of ceil(P/32) words plus 64.
+__host__ __device__ constexpr int tiles_smem_words(int T) { return 64 + 4 * ((T + 31) / 32); }
+
 // Runs, contiguous tiles, gathered rows and gathered tiles (see lora_meta).
-// Whole block.  brkw/lngw/aux: ceil(P/32) words of shared memory each.
-__device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const int32_t *seg_start, int N,
-                          const TileOut &o, uint32_t *brkw, uint32_t *lngw, int *aux, int *sm33) {
-    const int tid = threadIdx.x;
+// Whole block; every loop over positions runs one position per lane and packs
+// flags into 32-bit words with ballots, so no thread walks positions serially.
+//   perm, ids  : global or shared
+//   brkb[p]    : 1 if position p starts a run (p < P)
+//   sm         : tiles_smem_words(T) words of shared memory
+__device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t *brkb,
+                          const int32_t *seg_start, int N, const TileOut &o, int *sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = SEG_THREADS / 32;
     const int P = seg_start[N];
     const int W = (P + 31) >> 5;
+    int *wsum = sm;                                   // 64 ints: per-warp values
+    uint32_t *brkw = reinterpret_cast<uint32_t *>(sm + 64);
+    uint32_t *lngw = brkw + W;
+    int *nxt = reinterpret_cast<int *>(lngw + W);      // first run start at a position >= 32w (P if none)
+    int *prv = nxt + W;                                // last run start at a position < 32w (-1 if none)
+    const uint32_t lt = (1u << lane) - 1u;
 
-    // 1. run starts: a new id, or a row that does not follow the previous one
-    for (int w = tid; w < W; w += SEG_THREADS) {
-        const int p0 = w * 32;
-        int prev_row = -2, prev_id = -2;
-        if (p0 > 0) {
-            prev_row = perm[p0 - 1];
-            prev_id = ids[prev_row];
-        }
-        uint32_t bits = 0;
-        for (int b = 0; b < 32 && p0 + b < P; ++b) {
-            const int row = perm[p0 + b];
-            const int id = ids[row];
-            if (id != prev_id || row != prev_row + 1) bits |= 1u << b;
-            prev_row = row;
-            prev_id = id;
-        }
-        brkw[w] = bits;
-        lngw[w] = 0;
+    // 1. pack run starts
+    for (int w = warp; w < W; w += NW) {
+        const int p = w * 32 + lane;
+        const uint32_t word = __ballot_sync(FULL, p < P && brkb[p]);
+        if (lane == 0) brkw[w] = word;
     }
     __syncthreads();
 
-    // aux[w] = first run start at a position >= 32*w (P if none)
-    const int wpt = (W + SEG_THREADS - 1) / SEG_THREADS;
-    const int w_lo = min(tid * wpt, W), w_hi = min(w_lo + wpt, W);
-    int first = INT_MAX;
-    for (int w = w_lo; w < w_hi; ++w)
-        if (brkw[w]) {
-            first = w * 32 + __ffs(brkw[w]) - 1;
-            break;
-        }
-    int nxt = min(block_excl_suffix_min(first, sm33), P);
-    for (int w = w_hi - 1; w >= w_lo; --w) {
-        if (brkw[w]) nxt = w * 32 + __ffs(brkw[w]) - 1;
-        aux[w] = nxt;
-    }
-    __syncthreads();
+    // word ranges per warp, contiguous so that per-warp order is position order
+    const int wpw = (W + NW - 1) / NW;
+    const int wl = min(warp * wpw, W), wh = min(wl + wpw, W);
 
-    auto run_end = [&](int p) -> int {
-        const int w = p >> 5, b = p & 31;
-        const uint32_t rest = b == 31 ? 0u : (brkw[w] & (0xffffffffu << (b + 1)));
-        if (rest) return min(w * 32 + __ffs(rest) - 1, P);
-        return (w + 1 < W) ? aux[w + 1] : P;
-    };
-
-    // 2. long runs
-    if (o.min_run > 0) {
-        for (int w = tid; w < W; w += SEG_THREADS) {
-            uint32_t bits = brkw[w];
-            while (bits) {
-                const int b = __ffs(bits) - 1;
-                bits &= bits - 1;
-                const int p = w * 32 + b, e = run_end(p);
-                if (e - p >= o.min_run) {
-                    for (int ww = p >> 5; ww <= (e - 1) >> 5; ++ww) {
-                        const int a = max(p, ww * 32) - ww * 32, z = min(e, ww * 32 + 32) - ww * 32;
-                        atomicOr(&lngw[ww], bit_range(a, z));
-                    }
-                }
+    // 2. nxt[] (suffix) and prv[] (prefix) over words
+    {
+        int first = INT_MAX, last = -1;
+        for (int w = wl + lane; w < wh; w += 32) {
+            const uint32_t b = brkw[w];
+            if (b) {
+                first = min(first, w * 32 + __ffs(b) - 1);
+                last = max(last, w * 32 + 31 - __clz(b));
             }
         }
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) {
+            first = min(first, __shfl_xor_sync(FULL, first, o2));
+            last = max(last, __shfl_xor_sync(FULL, last, o2));
+        }
+        if (lane == 0) {
+            wsum[warp] = first;
+            wsum[32 + warp] = last;
+        }
+        __syncthreads();
+        if (warp == 0) {   // exclusive suffix-min of firsts, exclusive prefix-max of lasts
+            const int f = wsum[lane], l = wsum[32 + lane];
+            int sf = f, pl = l;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const int tf = __shfl_down_sync(FULL, sf, o2);
+                if (lane + o2 < 32) sf = min(sf, tf);
+                const int tl = __shfl_up_sync(FULL, pl, o2);
+                if (lane >= o2) pl = max(pl, tl);
+            }
+            int after = __shfl_down_sync(FULL, sf, 1);
+            if (lane == 31) after = INT_MAX;
+            int before = __shfl_up_sync(FULL, pl, 1);
+            if (lane == 0) before = -1;
+            __syncwarp();
+            wsum[lane] = min(after, P);
+            wsum[32 + lane] = before;
+        }
+        __syncthreads();
+        const int after = wsum[warp], before = wsum[32 + warp];
+        // backward over my words, 32 at a time: suffix minimum of first starts
+        int carry = after;
+        const int nchunk = (wh - wl + 31) / 32;
+        for (int c = nchunk - 1; c >= 0; --c) {
+            const int w = wl + c * 32 + lane;
+            int f = INT_MAX;
+            if (w < wh && brkw[w]) f = w * 32 + __ffs(brkw[w]) - 1;
+            int incl = f;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const int t = __shfl_down_sync(FULL, incl, o2);
+                if (lane + o2 < 32) incl = min(incl, t);
+            }
+            if (w < wh) nxt[w] = min(incl, carry);
+            carry = min(carry, __shfl_sync(FULL, incl, 0));
+        }
+        // forward: prefix maximum of last starts (strictly before the word)
+        carry = before;
+        for (int c = 0; c < nchunk; ++c) {
+            const int w = wl + c * 32 + lane;
+            int l = -1;
+            if (w < wh && brkw[w]) l = w * 32 + 31 - __clz(brkw[w]);
+            int incl = l;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const int t = __shfl_up_sync(FULL, incl, o2);
+                if (lane >= o2) incl = max(incl, t);
+            }
+            int excl = __shfl_up_sync(FULL, incl, 1);
+            if (lane == 0) excl = -1;
+            if (w < wh) prv[w] = max(carry, excl);
+            carry = max(carry, __shfl_sync(FULL, incl, 31));
+        }
+    }
+    __syncthreads();
+
+    auto run_end = [&](int p) -> int {   // first run start after p, or P
+        const int w = p >> 5, b = p & 31;
+        const uint32_t rest = b == 31 ? 0u : (brkw[w] & (0xffffffffu << (b + 1)));
+        if (rest) return w * 32 + __ffs(rest) - 1;
+        return (w + 1 < W) ? nxt[w + 1] : P;
+    };
+    auto run_start = [&](int p) -> int {   // last run start at or before p
+        const int w = p >> 5, b = p & 31;
+        const uint32_t upto = brkw[w] & (b == 31 ? 0xffffffffu : ((2u << b) - 1u));
+        if (upto) return w * 32 + 31 - __clz(upto);
+        return prv[w];
+    };
+
+    // 3. long positions: the run through the position has at least min_run rows
+    for (int w = warp; w < W; w += NW) {
+        const int p = w * 32 + lane;
+        bool lg = false;
+        if (o.min_run > 0 && p < P) lg = run_end(p) - run_start(p) >= o.min_run;
+        const uint32_t word = __ballot_sync(FULL, lg);
+        if (lane == 0) lngw[w] = word;
     }
     __syncthreads();
 
     bool overflow = false;
 
-    // 3. contiguous tiles, in position order
-    int my_ct = 0;
-    for (int w = w_lo; w < w_hi; ++w) {
-        uint32_t bits = brkw[w] & lngw[w];
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1;
-            const int p = w * 32 + b;
-            my_ct += (run_end(p) - p + o.LT - 1) / o.LT;
+    // 4. contiguous tiles: long runs in position order, cut every LT rows
+    {
+        int cnt = 0;
+        for (int w = wl; w < wh; ++w) {
+            const int p = w * 32 + lane;
+            int k = 0;
+            if (((brkw[w] & lngw[w]) >> lane) & 1u) k = (run_end(p) - p + o.LT - 1) / o.LT;
+            cnt += k;
         }
-    }
-    int n_contig;
-    int cbase = block_excl_sum(my_ct, &n_contig, sm33);
-    for (int w = w_lo; w < w_hi; ++w) {
-        uint32_t bits = brkw[w] & lngw[w];
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1;
-            const int p = w * 32 + b, len = run_end(p) - p;
-            const int row0 = perm[p], id = ids[row0];
-            for (int off = 0; off < len; off += o.LT, ++cbase) {
-                if (cbase < o.max_contig)
-                    o.contig[cbase] = make_int4(id, row0 + off, min(o.LT, len - off), 0);
-                else
-                    overflow = true;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o2);
+        int n_contig;
+        int base = warp_excl_scan(cnt, &n_contig, wsum);
+        for (int w = wl; w < wh; ++w) {
+            const int p = w * 32 + lane;
+            int len = 0, k = 0;
+            if (((brkw[w] & lngw[w]) >> lane) & 1u) {
+                len = run_end(p) - p;
+                k = (len + o.LT - 1) / o.LT;
             }
+            int incl = k;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const int t = __shfl_up_sync(FULL, incl, o2);
+                if (lane >= o2) incl += t;
+            }
+            int idx = base + incl - k;
+            if (k) {
+                const int row0 = perm[p], id = ids[row0];
+                for (int off = 0; off < len; off += o.LT, ++idx) {
+                    if (idx < o.max_contig)
+                        o.contig[idx] = make_int4(id, row0 + off, min(o.LT, len - off), 0);
+                    else
+                        overflow = true;
+                }
+            }
+            base += __shfl_sync(FULL, incl, 31);
         }
+        if (tid == 0) o.counts[2] = min(n_contig, o.max_contig);
     }
+    __syncthreads();
 
-    // 4. gathered rows (positions outside long runs), in position order
+    // 5. gathered rows: positions outside long runs, in position order
+    int *gpre = prv;   // reused: gathered rows before word w
     auto short_bits = [&](int w) -> uint32_t {
         const int rem = P - w * 32;
         const uint32_t valid = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
         return ~lngw[w] & valid;
     };
-    int my_sh = 0;
-    for (int w = w_lo; w < w_hi; ++w) my_sh += __popc(short_bits(w));
     int n_short;
-    int sbase = block_excl_sum(my_sh, &n_short, sm33);
-    for (int w = w_lo; w < w_hi; ++w) {
-        aux[w] = sbase;
-        uint32_t bits = short_bits(w);
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1;
-            o.grow[sbase++] = perm[w * 32 + b];
+    {
+        int cnt = 0;
+        for (int w = wl + lane; w < wh; w += 32) cnt += __popc(short_bits(w));
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o2);
+        int base = warp_excl_scan(cnt, &n_short, wsum);
+        for (int w = wl; w < wh; ++w) {
+            const uint32_t bits = short_bits(w);
+            if ((bits >> lane) & 1u) o.grow[base + __popc(bits & lt)] = perm[w * 32 + lane];
+            if (lane == 0) gpre[w] = base;
+            base += __popc(bits);
         }
     }
     __syncthreads();
 
-    // 5. gathered tiles: each id's gathered rows cut every R rows
+    // 6. gathered tiles: each id's gathered rows cut every R rows
     auto short_before = [&](int q) -> int {
         if (q >= P) return n_short;
         const int w = q >> 5, b = q & 31;
-        return aux[w] + __popc(short_bits(w) & ((1u << b) - 1u));
+        return gpre[w] + __popc(short_bits(w) & ((1u << b) - 1u));
     };
-    const int spt = (N + SEG_THREADS - 1) / SEG_THREADS;
-    const int n_lo = min(tid * spt, N), n_hi = min(n_lo + spt, N);
-    int my_gt = 0;
-    for (int n = n_lo; n < n_hi; ++n) {
-        const int cnt = short_before(seg_start[n + 1]) - short_before(seg_start[n]);
-        my_gt += (cnt + o.R - 1) / o.R;
-    }
-    int n_gather;
-    int gbase = block_excl_sum(my_gt, &n_gather, sm33);
-    for (int n = n_lo; n < n_hi; ++n) {
-        const int g0 = short_before(seg_start[n]);
-        const int cnt = short_before(seg_start[n + 1]) - g0;
-        for (int off = 0; off < cnt; off += o.R, ++gbase) {
-            if (gbase < o.max_gather)
-                o.gather[gbase] = make_int4(n, g0 + off, min(o.R, cnt - off), 0);
-            else
-                overflow = true;
+    {
+        const int spt = (N + SEG_THREADS - 1) / SEG_THREADS;
+        const int n_lo = min(tid * spt, N), n_hi = min(n_lo + spt, N);
+        int my_gt = 0;
+        for (int n = n_lo; n < n_hi; ++n) {
+            const int c = short_before(seg_start[n + 1]) - short_before(seg_start[n]);
+            my_gt += (c + o.R - 1) / o.R;
+        }
+        int n_gather;
+        int gbase = block_excl_sum(my_gt, &n_gather, wsum);
+        for (int n = n_lo; n < n_hi; ++n) {
+            const int g0 = short_before(seg_start[n]);
+            const int c = short_before(seg_start[n + 1]) - g0;
+            for (int off = 0; off < c; off += o.R, ++gbase) {
+                if (gbase < o.max_gather)
+                    o.gather[gbase] = make_int4(n, g0 + off, min(o.R, c - off), 0);
+                else
+                    overflow = true;
+            }
+        }
+        if (tid == 0) {
+            o.counts[1] = min(n_gather, o.max_gather);
+            o.counts[3] = n_short;
         }
     }
     if (overflow) atomicOr(o.status, LORA_DEV_TILE_OVERFLOW);
-    if (tid == 0) {
-        o.counts[1] = min(n_gather, o.max_gather);
-        o.counts[2] = min(n_contig, o.max_contig);
-        o.counts[3] = n_short;
-    }
 }
 
 struct SegArgs {
     const int32_t *ids;
     int T, N;
     int32_t *perm, *seg_start, *seg_adapter;
-    int *ws;   // [n_chunks][N+1] (multi-block path)
+    int *ws;          // [n_chunks][N+1] (multi-block path)
+    uint8_t *brkb;    // [T]            (multi-block path)
     TileOut out;
 };
 
-// Everything in one block (T <= SEG_SMALL_T).
+// Warps that rank rows in parallel: each keeps a private count per id, so the
+// counts must fit the shared-memory budget.
+__host__ __device__ constexpr int rank_warps(int N) {
+    return (8192 / (N + 1)) >= 32 ? 32 : ((8192 / (N + 1)) < 1 ? 1 : 8192 / (N + 1));
+}
+
+// Stable placement of rows [lo, hi) by up to 32 warps.  Warp w ranks the rows
+// [lo + w*rpw, lo + (w+1)*rpw); hw[w][b] holds its private count of id b on
+// entry, and is turned into its first position (base[b] plus the counts of
+// warps before it).  Whole block.
+__device__ void scatter_block(const int32_t *ids, int lo, int hi, int N, const int *base, int *hw,
+                              int nwr, int32_t *perm, uint8_t *brkb) {
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int rpw = (hi - lo + nwr - 1) / nwr;
+    for (int b = tid; b <= N; b += blockDim.x) {
+        int run = base[b];
+        for (int w = 0; w < nwr; ++w) {
+            const int c = hw[w * (N + 1) + b];
+            hw[w * (N + 1) + b] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    if (warp < nwr) {
+        const int wl = lo + warp * rpw, wh = min(wl + rpw, hi);
+        if (wl < wh) scatter_warp(ids, wl, wh, N, hw + warp * (N + 1), perm, brkb);
+    }
+}
+
+// Per-warp id counts of rows [lo, hi) into hw[w][*] (zeroed here).  Whole block.
+__device__ bool count_block(const int32_t *ids, int lo, int hi, int N, int *hw, int nwr) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < nwr * (N + 1); e += blockDim.x) hw[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    if (warp < nwr) {
+        const int rpw = (hi - lo + nwr - 1) / nwr;
+        const int wl = lo + warp * rpw, wh = min(wl + rpw, hi);
+        for (int i = wl + lane; i < wh; i += 32) {
+            const int id = ids[i];
+            bad |= (id < -1 || id >= N);
+            atomicAdd(&hw[warp * (N + 1) + bin_of(id, N)], 1);
+        }
+    }
+    __syncthreads();
+    return bad;
+}
+
+// Everything in one block (T <= SEG_SMALL_T); ids, perm and the run starts
+// stay in shared memory.
 __global__ void __launch_bounds__(SEG_THREADS) seg_small_kernel(SegArgs a) {
     extern __shared__ int sm[];
     int *sm33 = sm;
-    int *hist = sm + 64;
-    const int W = (a.T + 31) >> 5;
-    uint32_t *brkw = reinterpret_cast<uint32_t *>(hist + a.N + 1);
-    uint32_t *lngw = brkw + W;
-    int *aux = reinterpret_cast<int *>(lngw + W);
+    const int nwr = rank_warps(a.N);
+    int *hist = sm + 64;                                  // N+1
+    int *hw = hist + ((a.N + 1 + 3) & ~3);                // nwr * (N+1)
+    int *ids_s = hw + ((nwr * (a.N + 1) + 3) & ~3);       // T
+    int *perm_s = ids_s + a.T;                            // T
+    int *tsm = perm_s + a.T;                              // tiles_smem_words(T)
+    uint8_t *brk_s = reinterpret_cast<uint8_t *>(tsm + tiles_smem_words(a.T));   // T bytes
     const int tid = threadIdx.x;
 
-    for (int b = tid; b <= a.N; b += SEG_THREADS) hist[b] = 0;
+    for (int i = tid; i < a.T; i += SEG_THREADS) ids_s[i] = a.ids[i];
     __syncthreads();
-    bool bad = false;
-    for (int i = tid; i < a.T; i += SEG_THREADS) {
-        const int id = a.ids[i];
-        bad |= (id < -1 || id >= a.N);
-        atomicAdd(&hist[bin_of(id, a.N)], 1);
+    if (count_block(ids_s, 0, a.T, a.N, hw, nwr)) atomicOr(a.out.status, LORA_DEV_BAD_ID);
+    for (int b = tid; b <= a.N; b += SEG_THREADS) {
+        int t = 0;
+        for (int w = 0; w < nwr; ++w) t += hw[w * (a.N + 1) + b];
+        hist[b] = t;
     }
-    if (bad) atomicOr(a.out.status, LORA_DEV_BAD_ID);
     __syncthreads();
     seg_scan_block(hist, a.N, a.seg_start, a.seg_adapter, a.out.counts, sm33);
     __syncthreads();
-    if (tid < 32) scatter_warp(a.ids, 0, a.T, a.N, hist, a.perm);
+    scatter_block(ids_s, 0, a.T, a.N, hist, hw, nwr, perm_s, brk_s);
     __syncthreads();
-    dev_tiles(a.ids, a.perm, a.seg_start, a.N, a.out, brkw, lngw, aux, sm33);
+    for (int i = tid; i < a.T; i += SEG_THREADS) a.perm[i] = perm_s[i];
+    dev_tiles(ids_s, perm_s, brk_s, a.seg_start, a.N, a.out, tsm);
 }
 
 __global__ void __launch_bounds__(SEG_HIST_THREADS) seg_hist_kernel(SegArgs a) {
@@ -374,28 +517,30 @@ __global__ void __launch_bounds__(SEG_THREADS) seg_scan_kernel(SegArgs a, int n_
     }
 }
 
-__global__ void __launch_bounds__(32) seg_scatter_kernel(SegArgs a) {
-    extern __shared__ int base[];
+__global__ void __launch_bounds__(SEG_THREADS) seg_scatter_kernel(SegArgs a) {
+    extern __shared__ int sm[];
+    const int nwr = rank_warps(a.N);
+    int *base = sm;                                   // N+1
+    int *hw = sm + ((a.N + 1 + 3) & ~3);              // nwr * (N+1)
     const int c = blockIdx.x, lo = c * SEG_CHUNK, hi = min(lo + SEG_CHUNK, a.T);
-    for (int b = threadIdx.x; b <= a.N; b += 32) base[b] = a.ws[(size_t)c * (a.N + 1) + b];
-    __syncwarp();
-    scatter_warp(a.ids, lo, hi, a.N, base, a.perm);
+    for (int b = threadIdx.x; b <= a.N; b += SEG_THREADS) base[b] = a.ws[(size_t)c * (a.N + 1) + b];
+    count_block(a.ids, lo, hi, a.N, hw, nwr);
+    scatter_block(a.ids, lo, hi, a.N, base, hw, nwr, a.perm, a.brkb);
 }
 
 __global__ void __launch_bounds__(SEG_THREADS) seg_tiles_kernel(SegArgs a) {
     extern __shared__ int sm[];
-    int *sm33 = sm;
-    const int W = (a.T + 31) >> 5;
-    uint32_t *brkw = reinterpret_cast<uint32_t *>(sm + 64);
-    uint32_t *lngw = brkw + W;
-    int *aux = reinterpret_cast<int *>(lngw + W);
-    dev_tiles(a.ids, a.perm, a.seg_start, a.N, a.out, brkw, lngw, aux, sm33);
+    dev_tiles(a.ids, a.perm, a.brkb, a.seg_start, a.N, a.out, sm);
+}
+
+static size_t ws_bytes(int T, int N) {
+    const size_t n_chunks = (T + SEG_CHUNK - 1) / SEG_CHUNK;
+    return (n_chunks * (size_t)(N + 1) * sizeof(int) + 255) & ~(size_t)255;
 }
 
 size_t segments_scratch_bytes(int T, int N) {
     if (T <= SEG_SMALL_T) return 0;
-    const size_t n_chunks = (T + SEG_CHUNK - 1) / SEG_CHUNK;
-    return n_chunks * (size_t)(N + 1) * sizeof(int);
+    return ws_bytes(T, N) + (size_t)T;
 }
 
 int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
@@ -408,6 +553,7 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
     a.seg_start = m->seg_start;
     a.seg_adapter = m->seg_adapter;
     a.ws = static_cast<int *>(scratch);
+    a.brkb = scratch ? static_cast<uint8_t *>(scratch) + ws_bytes(m->T, m->N) : nullptr;
     a.out.grow = m->grow;
     a.out.gather = reinterpret_cast<int4 *>(m->gather_tiles);
     a.out.contig = reinterpret_cast<int4 *>(m->contig_tiles);
@@ -419,9 +565,11 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
     a.out.min_run = m->min_run;
     a.out.LT = m->long_tile;
 
-    const int W = (a.T + 31) / 32;
     if (a.T <= SEG_SMALL_T) {
-        const size_t smem = (64 + (size_t)a.N + 1 + 3 * (size_t)W) * sizeof(int);
+        const size_t nwr = rank_warps(a.N);
+        const size_t smem = (64 + (((size_t)a.N + 1 + 3) & ~(size_t)3) +
+                             ((nwr * (a.N + 1) + 3) & ~(size_t)3) + 2 * (size_t)a.T +
+                             tiles_smem_words(a.T)) * sizeof(int) + (size_t)a.T;
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(seg_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
@@ -434,8 +582,13 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
         seg_hist_kernel<<<n_chunks, SEG_HIST_THREADS, bins * sizeof(int), st>>>(a);
         const size_t scan_smem = (64 + bins) * sizeof(int);
         seg_scan_kernel<<<1, SEG_THREADS, scan_smem, st>>>(a, n_chunks);
-        seg_scatter_kernel<<<n_chunks, 32, bins * sizeof(int), st>>>(a);
-        const size_t tile_smem = (64 + 3 * (size_t)W) * sizeof(int);
+        const size_t scat_smem =
+            ((((size_t)a.N + 1 + 3) & ~(size_t)3) + (size_t)rank_warps(a.N) * bins) * sizeof(int);
+        if (scat_smem > 48 * 1024)
+            cudaFuncSetAttribute(seg_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)scat_smem);
+        seg_scatter_kernel<<<n_chunks, SEG_THREADS, scat_smem, st>>>(a);
+        const size_t tile_smem = (size_t)tiles_smem_words(a.T) * sizeof(int);
         if (tile_smem > 48 * 1024)
             cudaFuncSetAttribute(seg_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tile_smem);
