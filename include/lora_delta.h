@@ -159,6 +159,30 @@ LORA_API size_t lora_segments_scratch_bytes(int32_t T, int32_t N);
 LORA_API int lora_build_segments(const int32_t *ids, const lora_meta *meta, void *scratch,
                         size_t scratch_bytes, int32_t *status, void *stream);
 
+/*
+ * Bytes of the scratch array compiled into the library for
+ * lora_build_segments_static (1 MiB per device that loads the library).
+ */
+#define LORA_STATIC_SCRATCH_BYTES (1 << 20)
+
+/*
+ * lora_build_segments without caller-provided scratch memory.  The pages have
+ * no counterpart: this exists for callers that cannot allocate device memory
+ * when they group a batch (a pool that owns all device memory, callbacks and
+ * hooks that must not call cudaMalloc, runtimes that only hand over input and
+ * output buffers).  Same ids, meta and status as lora_build_segments, same
+ * results; the scratch is one library-owned array of
+ * LORA_STATIC_SCRATCH_BYTES bytes per device, so nothing is allocated.
+ *   - Returns LORA_ERR_WORKSPACE when lora_segments_scratch_bytes(T, N)
+ *     exceeds LORA_STATIC_SCRATCH_BYTES (use lora_build_segments then).
+ *   - The first call on a device (that device current) looks up the array's
+ *     device address; make it before any stream capture.
+ *   - Every call uses the same array; calls that overlap on the GPU race and
+ *     corrupt each other: keep them ordered (one stream).
+ */
+LORA_API int lora_build_segments_static(const int32_t *ids, const lora_meta *meta,
+                                        int32_t *status, void *stream);
+
 /* Bytes of the fp32 intermediate v = A x that lora_sgmv_shrink writes and
  * lora_sgmv_expand reads: n_slices * T * r_max * 4. */
 LORA_API size_t lora_shrink_workspace_bytes(int32_t T, int32_t r_max, int32_t n_slices);

@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "load", "LoraError", "Meta", "LORA_BF16", "LORA_FP32", "DEV_BAD_ID", "DEV_TILE_OVERFLOW",
     "DEV_BAD_RANK", "lora_version", "lora_meta_capacity", "lora_segments_scratch_bytes",
-    "lora_build_segments", "lora_shrink_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand",
+    "lora_build_segments", "lora_build_segments_static", "lora_shrink_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand",
     "lora_bgmv_fused", "lora_add_linear", "scales_for",
 ]
 
@@ -63,6 +63,7 @@ _SIGS = {
                                           ctypes.POINTER(_I32)]),
     "lora_segments_scratch_bytes": (_SZ, [_I32, _I32]),
     "lora_build_segments": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _SZ, _P, _P]),
+    "lora_build_segments_static": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _P]),
     "lora_shrink_workspace_bytes": (_SZ, [_I32, _I32, _I32]),
     "lora_sgmv_shrink": (ctypes.c_int, [_P, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32, _I32,
                                         _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
@@ -140,6 +141,19 @@ def lora_meta_capacity(T, N, rows_per_tile=16, min_run=64, long_tile=LONG_TILE):
 
 def lora_segments_scratch_bytes(T, N):
     return int(load().lora_segments_scratch_bytes(T, N))
+
+
+def lora_build_segments_static(ids, meta: Meta, status, stream=None):
+    """lora_build_segments with the library's own fixed scratch array instead of
+    meta.scratch, for callers that cannot allocate device memory (see
+    include/lora_delta.h: first call per device before any stream capture;
+    calls must not overlap on the GPU)."""
+    _dev(ids, "ids")
+    _dev(status, "status")
+    if ids.dtype != torch.int32 or ids.numel() != meta.T or not ids.is_contiguous():
+        raise LoraError("ids must be a contiguous int32 tensor of T entries")
+    _check(load().lora_build_segments_static(_ptr(ids), ctypes.byref(meta.c), _ptr(status),
+                                             _stream(stream)))
 
 
 def lora_shrink_workspace_bytes(T, r_max, n_slices):
