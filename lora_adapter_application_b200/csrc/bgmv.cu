@@ -8,14 +8,15 @@
 // columns (expand).  Each block is warp-specialised:
 //
 //   producer warp   walks the block's chunk stream and fills a 3-stage
-//                   shared-memory ring through the TMA engine: one 1-D bulk
-//                   copy per x, A or y row and one for a B block whose rows are
-//                   dense; B rows with rank padding take 16-byte cp.async
-//                   pieces.  (Measured on B200: TMA copies keep the load path
-//                   free for the consumers' shared-memory traffic, where a
-//                   cp.async producer competes with it; their cost is per copy,
-//                   so rows should be long.)  Completion is counted on a
-//                   full/empty mbarrier pair per stage.
+//                   shared-memory ring through the TMA engine: 2-D tensor
+//                   copies of 1 KB boxes for the adapters (A: 8 ranks x 64
+//                   columns, 128-byte swizzle; B: 64 output columns x 8 ranks)
+//                   and one 1-D bulk copy per gathered x or y row.  (Measured
+//                   on B200: TMA copies leave the load/store pipe to the
+//                   consumers, where a cp.async producer competes with their
+//                   shared-memory traffic; TMA pays per copy, so copies should
+//                   be 1 KB or more.)  A full/empty mbarrier pair guards each
+//                   stage.
 //   8 consumer warps
 //     shrink chunks  x rows [cnt][JC] and A rows [r_n][JC] -> partial v
 //                    (tensor-core mma m16n8k16, bf16 in, fp32 accumulate)
@@ -92,10 +93,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, unsigned rank) 
         "r"(rank)
         : "memory");
 }
-// the executing thread's earlier cp.async copies arrive on bar when they land
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
-}
 template <bool CLUSTER_ACQUIRE>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, unsigned parity) {
     uint32_t ok;
@@ -129,44 +126,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, int32_t
     return false;
 }
 
-__device__ __forceinline__ void cp16(uint32_t dst, const void *src, int src_bytes = 16) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-// rows x (ppr 16-byte pieces) from global (row stride src_ld elements) to shared
-// (row stride dst_ld bytes), spread over the 32 lanes of a warp.  Pieces at or
-// beyond `live` in a row are zero-filled without reading global memory.  When
-// ppr is a power of two each lane keeps one piece column and walks rows by
-// pointer increments (about four instructions per 16-byte piece).
-__device__ __forceinline__ void copy_rows(uint32_t dst, int dst_ld, const __nv_bfloat16 *src,
-                                          int64_t src_ld, int rows, int ppr, int live, int lane) {
-    if ((ppr & (ppr - 1)) == 0) {
-        if (ppr >= 32) {
-            for (int r = 0; r < rows; ++r, dst += dst_ld, src += src_ld)
-                for (int pc = lane; pc < ppr; pc += 32) {
-                    const bool in = pc < live;
-                    cp16(dst + pc * 16, in ? src + pc * 8 : src, in ? 16 : 0);
-                }
-        } else {
-            const int sh = __ffs(ppr) - 1, step = 32 >> sh;
-            const int pc = lane & (ppr - 1);
-            const bool in = pc < live;
-            const int nb = in ? 16 : 0;
-            uint32_t d = dst + (lane >> sh) * dst_ld + pc * 16;
-            const __nv_bfloat16 *q = src + (lane >> sh) * src_ld + (in ? pc * 8 : 0);
-            const uint32_t dstep = step * dst_ld;
-            const int64_t sstep = step * src_ld;
-            for (int r = lane >> sh; r < rows; r += step, d += dstep, q += sstep) cp16(d, q, nb);
-        }
-        return;
-    }
-    for (int r = 0; r < rows; ++r, dst += dst_ld, src += src_ld)
-        for (int pc = lane; pc < ppr; pc += 32) {
-            const bool in = pc < live;
-            cp16(dst + pc * 16, in ? src + pc * 8 : src, in ? 16 : 0);
-        }
-}
-
 // 1-D bulk copy global -> shared through the TMA engine, completing on bar.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned bytes,
                                          uint32_t bar) {
@@ -176,6 +135,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// 2-D tensor copy (one box) global -> shared through the TMA engine.
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                       uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;\n" ::"n"(BG_CONSUMERS * 32) : "memory");
 }
@@ -206,17 +175,22 @@ __device__ __forceinline__ uint4 zero_if(bool z, uint4 v) { return z ? make_uint
 //   recv[c*(S*1024/C) + e/C] holds block c's partial of element e = (s*16+row)*64+k,
 //   for the elements e with e % C == this block's rank.
 size_t bgmv_smem_bytes(int n_slices) {
-    return (size_t)BG_STAGES * BG_STAGE_BYTES + (size_t)n_slices * BG_ROWS * BG_RMAX * 4 +
+    return 1024 /* alignment of the ring to the 128-byte swizzle atom */ +
+           (size_t)BG_STAGES * BG_STAGE_BYTES + (size_t)n_slices * BG_ROWS * BG_RMAX * 4 +
            (size_t)n_slices * BG_ROWS * BG_VF_STRIDE * 4 + (size_t)BG_ROWS * BG_RMAX * 4 + 128;
 }
 
 struct Geo {          // chunk geometry of one block for one unit
     int r8, nb8, nkb16;
-    int j_lo, j_hi, JC, RS, n_sc;        // shrink: columns, chunk width, row stride (bytes), chunks per slice
-    int c_lo, c_hi, CC, YS, BS, ybytes;  // expand: concatenated column range, chunk width, strides
-    bool b_dense;                        // B rows hold exactly r8 = r_max elements: one copy
+    int j_lo, j_hi, JC, RS, A0, n_sc;    // shrink: columns, chunk width, x row stride, A boxes offset, chunks/slice
+    int c_lo, c_hi, CC, YS, B0;          // expand: concatenated column range, chunk width, y row stride, B boxes offset
     int n_shrink, n_chunks;
 };
+
+// Shared-memory bytes of a chunk: 16 padded rows, then 1 KB TMA boxes (1 KB aligned).
+__device__ __forceinline__ int chunk_bytes(int row_stride, int boxes) {
+    return ((BG_ROWS * row_stride + 1023) & ~1023) + boxes * 1024;
+}
 
 // Position in a block's chunk stream, advanced without divisions: shrink
 // chunks slice by slice, then expand chunks slice by slice.
@@ -227,13 +201,14 @@ struct ChunkIt {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
+__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_constant__ BgArgs a) {
     extern __shared__ __align__(128) unsigned char bg_sm[];
     __shared__ int rows_sm[BG_ROWS];
 
     const int S = a.sl.n;
-    unsigned char *ring = bg_sm;
-    float *recv = reinterpret_cast<float *>(bg_sm + BG_STAGES * BG_STAGE_BYTES);
+    // ring on a 1 KB boundary: swizzled TMA boxes need their 1 KB atom aligned
+    unsigned char *ring = bg_sm + ((1024u - (smem_u32(bg_sm) & 1023u)) & 1023u);
+    float *recv = reinterpret_cast<float *>(ring + BG_STAGES * BG_STAGE_BYTES);
     float *vfull = recv + S * BG_ROWS * BG_RMAX;
     float *part = vfull + S * BG_ROWS * BG_VF_STRIDE;
     uint64_t *bars = reinterpret_cast<uint64_t *>(part + BG_ROWS * BG_RMAX);
@@ -266,46 +241,43 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
         const int n64 = (a.d_in + 63) >> 6;
         G.j_lo = (int)((int64_t)crank * n64 / C) * 64;
         G.j_hi = min((int)((int64_t)(crank + 1) * n64 / C) * 64, a.d_in);
-        // widest power-of-two chunk (>= 64 columns) whose rows fit a stage
-        const int lim = ((BG_STAGE_BYTES / (BG_ROWS + G.r8)) - 16) / 2;
+        // widest power-of-two chunk (>= 64 columns) whose x rows and A boxes fit a stage
         int jc = 64;
-        while (jc * 2 <= lim) jc *= 2;
+        while (chunk_bytes(jc * 4 + 16, G.nb8 * (jc / 32)) <= BG_STAGE_BYTES) jc *= 2;
         const int span = max(0, G.j_hi - G.j_lo);
         while (jc > 64 && jc / 2 >= span) jc /= 2;
         G.JC = jc;
         G.RS = G.JC * 2 + 16;
+        G.A0 = (BG_ROWS * G.RS + 1023) & ~1023;
         G.n_sc = (span + G.JC - 1) / G.JC;
     } else {
         G.j_lo = G.j_hi = 0;
         G.JC = 64;
         G.RS = 144;
+        G.A0 = 0;
         G.n_sc = 0;
     }
     G.n_shrink = S * G.n_sc;
     G.n_chunks = G.n_shrink;
-    G.b_dense = G.r8 == a.r_max;
     if (MODE != MODE_SHRINK) {
         const int n8 = a.sl.cat_off[S] >> 3;
         G.c_lo = (int)((int64_t)crank * n8 / C) * 8;
         G.c_hi = (int)((int64_t)(crank + 1) * n8 / C) * 8;
-        G.BS = G.b_dense ? G.r8 * 2 : G.r8 * 2 + (G.r8 >= 32 ? 32 : 0);
-        // y rows: stride = 16 (mod 128) bytes, so the 8 rows of an mma tile hit 8 bank groups
-        const int lim = (BG_STAGE_BYTES - 144 * BG_ROWS) / (2 * BG_ROWS + G.BS);
-        int cc = 8;   // widest power-of-two chunk whose y rows and B rows fit a stage
-        while (cc * 2 <= lim) cc *= 2;
+        // widest power-of-two chunk (>= 64 columns) whose y rows and B boxes fit a stage
+        int cc = 64;
+        while (chunk_bytes(cc * 4 + 16, G.nb8 * (cc / 32)) <= BG_STAGE_BYTES) cc *= 2;
         G.CC = cc;
-        G.YS = ((G.CC * 2 + 127) & ~127) + 16;
-        G.ybytes = BG_ROWS * G.YS;
+        G.YS = G.CC * 2 + 16;   // 16 (mod 128) bytes: the 8 rows of an mma tile hit 8 bank groups
+        G.B0 = (BG_ROWS * G.YS + 1023) & ~1023;
         for (int s = 0; s < S; ++s) {
             const int lo = max(G.c_lo, a.sl.cat_off[s]), hi = min(G.c_hi, a.sl.cat_off[s + 1]);
             if (hi > lo) G.n_chunks += (hi - lo + G.CC - 1) / G.CC;
         }
     } else {
         G.c_lo = G.c_hi = 0;
-        G.CC = 8;
-        G.YS = 32;
-        G.BS = 16;
-        G.ybytes = 0;
+        G.CC = 64;
+        G.YS = 144;
+        G.B0 = 0;
     }
 
     // next position of the chunk stream
@@ -351,7 +323,7 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
     // barriers
     if (tid == 0) {
         for (int st = 0; st < BG_STAGES; ++st) {
-            mbar_init(full0 + 8 * st, 33);
+            mbar_init(full0 + 8 * st, 1);
             mbar_init(empty0 + 8 * st, BG_CONSUMERS);
         }
         mbar_init(xready, C);
@@ -375,27 +347,33 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
             if (failed) break;
             if (it.i < G.n_shrink) {
                 const int jc0 = G.j_lo + it.q * G.JC;
-                const unsigned bytes = (unsigned)min(G.JC, G.j_hi - jc0) * 2;
-                if (lane == 0) mbar_expect_tx(full, bytes * (cnt + r_n));
+                const int width = min(G.JC, G.j_hi - jc0), nbox = (width + 63) >> 6;
+                const int ncb = G.JC >> 6;
+                const unsigned xbytes = (unsigned)width * 2;
+                if (lane == 0) mbar_expect_tx(full, xbytes * cnt + (unsigned)(G.nb8 * nbox) * 1024u);
                 __syncwarp();
-                const __nv_bfloat16 *An = static_cast<const __nv_bfloat16 *>(a.sl.A[it.s]) + (int64_t)n * a.r_max * a.d_in + jc0;
-                for (int r = lane; r < cnt + r_n; r += 32) {
-                    if (r < cnt) bulk_g2s(dst + r * G.RS, a.x + (int64_t)rows_sm[r] * a.ld_x + jc0, bytes, full);
-                    else bulk_g2s(dst + (BG_ROWS + r - cnt) * G.RS, An + (int64_t)(r - cnt) * a.d_in, bytes, full);
+                for (int r = lane; r < cnt; r += 32)   // gathered x rows
+                    bulk_g2s(dst + r * G.RS, a.x + (int64_t)rows_sm[r] * a.ld_x + jc0, xbytes, full);
+                for (int e = lane; e < G.nb8 * nbox; e += 32) {   // A: 8 ranks x 64 columns per box
+                    const int kg = e / nbox, cb = e - kg * nbox;
+                    tma_2d(dst + G.A0 + (kg * ncb + cb) * 1024, &a.tmA[it.s], jc0 + 64 * cb,
+                           n * a.r_max + 8 * kg, full);
                 }
             } else {
                 const int s = it.es, d_out = a.sl.d_out[s];
+                const int nbox = (it.w + 63) >> 6, nbx = G.CC >> 6;
                 const unsigned ybytes = (unsigned)it.w * 2;
-                const __nv_bfloat16 *Bn = static_cast<const __nv_bfloat16 *>(a.sl.B[s]) + ((int64_t)n * d_out + it.c0) * a.r_max;
-                const unsigned bbytes = G.b_dense ? (unsigned)it.w * a.r_max * 2 : 0u;
-                if (lane == 0) mbar_expect_tx(full, ybytes * cnt + bbytes);
+                if (lane == 0) mbar_expect_tx(full, ybytes * cnt + (unsigned)(G.nb8 * nbox) * 1024u);
                 __syncwarp();
-                for (int r = lane; r < cnt; r += 32)
-                    bulk_g2s(dst + r * G.YS, a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0, ybytes, full);
-                if (G.b_dense) { if (lane == 0) bulk_g2s(dst + G.ybytes, Bn, bbytes, full); }
-                else copy_rows(dst + G.ybytes, G.BS, Bn, a.r_max, it.w, G.r8 >> 3, G.r8 >> 3, lane);
+                for (int r = lane; r < cnt; r += 32)   // gathered y rows
+                    bulk_g2s(dst + r * G.YS,
+                             a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0, ybytes, full);
+                for (int e = lane; e < G.nb8 * nbox; e += 32) {   // B: 64 columns x 8 ranks per box
+                    const int kg = e / nbox, cb = e - kg * nbox;
+                    tma_2d(dst + G.B0 + (kg * nbx + cb) * 1024, &a.tmB[s], 8 * kg,
+                           n * d_out + it.c0 + 64 * cb, full);
+                }
             }
-            cp_async_arrive(full);
         }
         return;
     }
@@ -427,14 +405,17 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
             const int width = min(G.JC, G.j_hi - jc0);
             const int nsteps = (width + 63) >> 6;
             const uint32_t xg = st + g * G.RS, xh = st + (g + 8) * G.RS;
-            const uint32_t ak = st + (BG_ROWS + nbw * 8 + g) * G.RS;
+            // A box (8 ranks x 64 columns, 128-byte swizzle): row g, 16-byte chunks 2t and 2t+1
+            const uint32_t ak = st + G.A0 + nbw * (G.JC >> 6) * 1024 + g * 128;
+            const uint32_t c0 = (uint32_t)(((2 * t) ^ g) << 4), c1 = (uint32_t)(((2 * t + 1) ^ g) << 4);
             for (int sp = jgi; sp < nsteps; sp += jg) {
                 const int col = sp * 64 + t * 16;
                 const bool z0 = col >= width, z1 = col + 8 >= width;   // beyond the chunk: zero
                 const uint32_t off = (uint32_t)(col * 2);
                 const uint4 xa0 = zero_if(z0, lds128(xg + off)), xa1 = zero_if(z1, lds128(xg + off + 16));
                 const uint4 xb0 = zero_if(z0, lds128(xh + off)), xb1 = zero_if(z1, lds128(xh + off + 16));
-                const uint4 a0 = zero_if(z0, lds128(ak + off)), a1 = zero_if(z1, lds128(ak + off + 16));
+                const uint32_t box = ak + sp * 1024;
+                const uint4 a0 = zero_if(z0, lds128(box + c0)), a1 = zero_if(z1, lds128(box + c1));
                 {
                     const uint32_t f[4] = {xa0.x, xb0.x, xa0.y, xb0.y};
                     mma16816(acc0, f, a0.x, a0.y);
@@ -540,7 +521,7 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
             }
         }
         const int nblk = it.w >> 3;
-        const uint32_t bbase = st + G.ybytes + g * G.BS;
+        const uint32_t bbase = st + G.B0, nbx = G.CC >> 6;
         for (int nb0 = warp * 2; nb0 < nblk; nb0 += BG_CONSUMERS * 2) {
             float d[2][4];
 #pragma unroll
@@ -556,7 +537,9 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(BgArgs a) {
                     for (int j = 0; j < 2; ++j) {
                         bv[j] = make_uint2(0, 0);
                         if (k < r_n && nb0 + j < nblk) {
-                            bv[j] = lds64(bbase + (nb0 + j) * 8 * G.BS + k * 2);
+                            const int col = (nb0 + j) * 8 + g;   // B box: 64 columns x 8 ranks, 16 B per column
+                            bv[j] = lds64(bbase + ((k >> 3) * nbx + (col >> 6)) * 1024 + (col & 63) * 16 +
+                                          (k & 7) * 2);
                             if (k + 4 > r_n) {   // the rank ends inside this group of 4
                                 const int keep = r_n - k;
                                 if (keep < 2) bv[j].x &= 0xffffu;

@@ -3,11 +3,23 @@
 
 #include "common.cuh"
 
+#include <cuda.h>
+
 namespace lora {
 
 enum { MODE_FUSED = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 
+// Tensor maps of the fused kernel (bf16 2-D views of the stacked adapters):
+//   A_s as [N*r_max rows][d_in], boxes of 8 rows x 64 columns, 128-byte swizzle
+//   B_s as [N*d_out rows][r_max], boxes of 64 rows x 8 ranks
+constexpr int BG_ABOX_COLS = 64, BG_ABOX_ROWS = 8;
+constexpr int BG_BBOX_RANKS = 8, BG_BBOX_ROWS = 64;
+int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
+                  uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
 struct BgArgs {
+    CUtensorMap tmA[LORA_MAX_SLICES];
+    CUtensorMap tmB[LORA_MAX_SLICES];
     const __nv_bfloat16 *x;
     int64_t ld_x;
     int d_in;

@@ -132,22 +132,36 @@ int run(int mode, const Call &c, bool gather, bool contig) {
     Tiles tiles = make_tiles(c.meta, gather, contig);
     const int units = n_units(tiles);
     if (c.meta->T == 0 || units == 0) return LORA_OK;
-    if (units <= 65535 && bgmv_ok(c, need_x, need_y)) {
-        BgArgs a{};
-        a.x = static_cast<const __nv_bfloat16 *>(c.x);
-        a.ld_x = c.ld_x;
-        a.d_in = c.d_in;
-        a.y = static_cast<__nv_bfloat16 *>(c.y);
-        a.ld_y = c.ld_y;
-        a.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
-        a.T = c.meta->T;
-        a.sl = make_slices(c);
-        a.r_max = c.r_max;
-        a.ranks = c.ranks;
-        a.scales = c.scales;
-        a.tiles = tiles;
-        a.status = c.status;
-        return launch_bgmv(mode, a, units, bgmv_cluster(units), c.stream);
+    bool maps_ok = units <= 65535 && bgmv_ok(c, need_x, need_y);
+    if (maps_ok) {
+        BgArgs bg{};
+        for (int s = 0; s < c.n_slices && maps_ok; ++s) {
+            const int N = c.meta->N;
+            if (need_x)
+                maps_ok = tensor_map_2d(&bg.tmA[s], c.slices[s].A, (uint64_t)c.d_in,
+                                        (uint64_t)N * c.r_max, BG_ABOX_COLS, BG_ABOX_ROWS,
+                                        true) == LORA_OK;
+            if (need_y && maps_ok)
+                maps_ok = tensor_map_2d(&bg.tmB[s], c.slices[s].B, (uint64_t)c.r_max,
+                                        (uint64_t)N * c.slices[s].d_out, BG_BBOX_RANKS,
+                                        BG_BBOX_ROWS, false) == LORA_OK;
+        }
+        if (maps_ok) {
+            bg.x = static_cast<const __nv_bfloat16 *>(c.x);
+            bg.ld_x = c.ld_x;
+            bg.d_in = c.d_in;
+            bg.y = static_cast<__nv_bfloat16 *>(c.y);
+            bg.ld_y = c.ld_y;
+            bg.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
+            bg.T = c.meta->T;
+            bg.sl = make_slices(c);
+            bg.r_max = c.r_max;
+            bg.ranks = c.ranks;
+            bg.scales = c.scales;
+            bg.tiles = tiles;
+            bg.status = c.status;
+            return launch_bgmv(mode, bg, units, bgmv_cluster(units), c.stream);
+        }
     }
     SimtArgs a{};
     a.x = c.x;

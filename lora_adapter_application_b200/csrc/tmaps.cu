@@ -1,0 +1,82 @@
+// 2-D TMA tensor maps for the stacked adapter tensors, encoded on the host
+// through the driver entry point the CUDA runtime exposes, and cached: a
+// serving loop calls with the same adapter tensors over and over.
+#include "kernels.cuh"
+
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+namespace lora {
+namespace {
+
+struct Entry {
+    const void *base;
+    uint64_t inner, outer;
+    uint32_t box_inner, box_outer;
+    int swizzle;
+    int dev;
+    CUtensorMap map;
+};
+
+constexpr int kCache = 256;
+std::mutex g_mu;
+Entry g_cache[kCache];
+int g_used = 0, g_next = 0;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
+                  uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_used; ++i) {
+        const Entry &e = g_cache[i];
+        if (e.base == base && e.inner == inner && e.outer == outer && e.box_inner == box_inner &&
+            e.box_outer == box_outer && e.swizzle == (int)swizzle128 && e.dev == dev) {
+            *out = e.map;
+            return LORA_OK;
+        }
+    }
+    auto fn = encoder();
+    if (!fn) return LORA_ERR_CUDA;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};   // bf16 rows
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUtensorMap m;
+    const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return LORA_ERR_CUDA;
+    Entry &e = g_cache[g_used < kCache ? g_used++ : (g_next++ % kCache)];
+    e.base = base;
+    e.inner = inner;
+    e.outer = outer;
+    e.box_inner = box_inner;
+    e.box_outer = box_outer;
+    e.swizzle = (int)swizzle128;
+    e.dev = dev;
+    e.map = m;
+    *out = m;
+    return LORA_OK;
+}
+
+}  // namespace lora
