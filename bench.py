@@ -38,6 +38,10 @@ METRIC = "multi-LoRA delta tokens/s + achieved HBM GB/s (% of B200 peak), SGMV &
 UNIT = "tokens/s"
 HEADLINE = "decode_qproj"
 SWEEP = ["prefill", "multislice_8b", "mixed_70b"]
+# Runs of at least this many rows become contiguous tiles (the tensor-core SGMV
+# kernel); 0 = gathered tiles only.  A serving engine knows whether a batch
+# holds prompts: decode-only batches are grouped without contiguous tiles.
+MIN_RUN = {"tiny": 0, "decode_qproj": 0, "multislice_8b": 0, "prefill": 64, "mixed_70b": 64}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -216,9 +220,23 @@ def step(ds, ka=None, kb=None):
         kb.record()
 
 
+def min_run_of(w):
+    return MIN_RUN.get(w.name, 64)
+
+
 def launches_per_step(w):
+    """Kernels one step launches: the grouping (one block when T <= 2048, else
+    four passes), then per layer the gathered-tile kernel, plus the tensor-core
+    SGMV kernel when contiguous tiles are enabled and the layer qualifies (bf16,
+    r_max a multiple of 16, n_slices * r_max <= 128)."""
     builder = 1 if w.T <= 2048 else 4
-    return builder + len(w.layers)
+    n = builder
+    for l in w.layers:
+        n += 1
+        if (min_run_of(w) > 0 and w.dtype == torch.bfloat16 and w.r_max % 16 == 0 and
+                len(l.d_out) * w.r_max <= 128):
+            n += 1
+    return n
 
 
 def make_sets(w, device, l2_bytes, rows_per_tile, min_run, max_sets=32):
@@ -293,7 +311,7 @@ def time_e2e(w, device, K, dist):
     inputs (ids, x and base output y of every layer), the path, and the updated y
     back to pinned host memory, all inside the timed region."""
     import lora_adapter_application_b200 as lora
-    ds = DeviceSet(w, device, 16, 64)
+    ds = DeviceSet(w, device, 16, min_run_of(w))
     host = {"ids": w.ids.pin_memory(),
             "layers": [{"x": l.x.pin_memory(), "y": l.y0.pin_memory(),
                         "out": torch.empty_like(l.y0).pin_memory()} for l in w.layers]}
@@ -366,7 +384,7 @@ def bench_ours(args, dist):
     sampler.start()
 
     w = workloads.make(args.workload, seed=args.seed + 1000 * dist.rank)
-    sets, per_set = make_sets(w, device, l2, 16, 64)
+    sets, per_set = make_sets(w, device, l2, 16, min_run_of(w))
     step_ms_local, kern_ms_local, t0, t1, graphed = time_device(sets, args.steps, args.warmup, dist,
                                                                    not args.no_graph)
     step_ms = dist.max(step_ms_local)
@@ -400,7 +418,7 @@ def bench_ours(args, dist):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(pk["hbm_gbs"]),
                      "unit": "GB/s", "frac": achieved / float(pk["hbm_gbs"]),
                      "traffic": measured_traffic(w.name) if len(w.layers) == 1 else None,
-                     "kernel": "bgmv_mma_kernel (lora_add_linear)", "kernel_ms": kern_ms_local,
+                     "kernel": "bgmv_kernel<MODE_FUSED> (lora_add_linear, gathered tiles)", "kernel_ms": kern_ms_local,
                      "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
                      "peak_source": f"{pk.get('source')} hbm_gbs"},
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -428,7 +446,7 @@ def bench_ours(args, dist):
 def sweep_one(name, args, device, l2, pk, dist):
     from lora_adapter_application_b200 import roofline
     w = workloads.make(name, seed=args.seed)
-    sets, per_set = make_sets(w, device, l2, 16, 64, max_sets=4)
+    sets, per_set = make_sets(w, device, l2, 16, min_run_of(w), max_sets=4)
     probe_ms, _, _, _, _ = time_device(sets, 3, 3, dist, graph=False)
     K = int(min(500, max(10, args.sweep_seconds * 1e3 / probe_ms)))
     step_ms, kern_ms, _, _, _ = time_device(sets, K, 3, dist, graph=not args.no_graph)

@@ -135,6 +135,12 @@ LORA_API int lora_version(void);
 /* Human-readable name of a lora_status value. */
 LORA_API const char *lora_status_string(int status);
 
+/* The CUDA failure behind the last LORA_ERR_CUDA returned on the calling
+ * thread ("cudaErrorName: description", or the failing driver step); an empty
+ * string if there was none.  The text stays valid until the thread's next
+ * failing call.  No counterpart in the pages: a diagnostic of this library. */
+LORA_API const char *lora_last_error(void);
+
 /*
  * Tile-list capacities that always suffice for a batch of T rows over N
  * slots: *max_gather >= T/rows_per_tile + N, *max_contig >= T/long_tile +

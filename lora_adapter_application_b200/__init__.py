@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "load", "LoraError", "Meta", "LORA_BF16", "LORA_FP32", "DEV_BAD_ID", "DEV_TILE_OVERFLOW",
-    "DEV_BAD_RANK", "lora_version", "lora_meta_capacity", "lora_segments_scratch_bytes",
+    "DEV_BAD_RANK", "lora_version", "lora_last_error", "lora_meta_capacity", "lora_segments_scratch_bytes",
     "lora_build_segments", "lora_build_segments_static", "lora_shrink_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand",
     "lora_bgmv_fused", "lora_add_linear", "scales_for",
 ]
@@ -34,6 +34,7 @@ LIB_PATH = os.path.join(_HERE, "liblora_delta.so")
 
 LORA_BF16, LORA_FP32 = 0, 1
 DEV_BAD_ID, DEV_TILE_OVERFLOW, DEV_BAD_RANK, DEV_TIMEOUT = 1, 2, 4, 8
+ERR_CUDA = -8   # LORA_ERR_CUDA
 MAX_ROWS, MAX_ADAPTERS, MAX_RANK, MAX_SLICES, LONG_TILE = 131072, 4096, 128, 8, 128
 
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -59,6 +60,7 @@ _lib = None
 _SIGS = {
     "lora_version": (ctypes.c_int, []),
     "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "lora_last_error": (ctypes.c_char_p, []),
     "lora_meta_capacity": (ctypes.c_int, [_I32, _I32, _I32, _I32, _I32, ctypes.POINTER(_I32),
                                           ctypes.POINTER(_I32)]),
     "lora_segments_scratch_bytes": (_SZ, [_I32, _I32]),
@@ -92,9 +94,17 @@ def load():
     return _lib
 
 
+def lora_last_error() -> str:
+    """The CUDA failure behind the last LORA_ERR_CUDA on this thread ('' if none)."""
+    return load().lora_last_error().decode()
+
+
 def _check(rc):
     if rc != 0:
-        raise LoraError(load().lora_status_string(rc).decode())
+        msg = load().lora_status_string(rc).decode()
+        if rc == ERR_CUDA:
+            msg += f" ({load().lora_last_error().decode()})"
+        raise LoraError(msg)
 
 
 def _dev(t: torch.Tensor, what: str):

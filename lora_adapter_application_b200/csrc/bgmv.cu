@@ -44,6 +44,7 @@
 // that runs out sets LORA_DEV_TIMEOUT in the status word and the block skips
 // its remaining work instead of hanging.
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 #include <cooperative_groups.h>
 
@@ -58,7 +59,7 @@ constexpr int BG_RMAX = 64;
 constexpr int BG_STAGES = 3;
 constexpr int BG_STAGE_BYTES = 24576;
 constexpr int BG_VF_STRIDE = 80;   // floats per row of the reduced v (bank spread)
-constexpr unsigned BG_WAIT_LIMIT = 1u << 16;
+
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -70,105 +71,10 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-// arrival on the mbarrier at the same offset in block `rank` of the cluster
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, unsigned rank) {
-    asm volatile(
-        "{\n\t.reg .b32 ra;\n\t"
-        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}\n" ::"r"(bar),
-        "r"(rank)
-        : "memory");
-}
-template <bool CLUSTER_ACQUIRE>
-__device__ __forceinline__ bool mbar_try(uint32_t bar, unsigned parity) {
-    uint32_t ok;
-    if (CLUSTER_ACQUIRE)
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, 20000;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-    else
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-    return ok != 0;
-}
-// Bounded wait; false (and the status bit) once the limit is reached.
-template <bool CLUSTER_ACQUIRE = false>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, int32_t *status,
-                                          bool &failed) {
-    if (failed) return false;
-    for (unsigned it = 0; it < BG_WAIT_LIMIT; ++it)
-        if (mbar_try<CLUSTER_ACQUIRE>(bar, parity)) return true;
-    atomicOr(status, LORA_DEV_TIMEOUT);
-    failed = true;
-    return false;
-}
-
-// 1-D bulk copy global -> shared through the TMA engine, completing on bar.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned bytes,
-                                         uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-// 2-D tensor copy (one box) global -> shared through the TMA engine.
-__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                       uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
-        "{%2, %3}], [%4];\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;\n" ::"n"(BG_CONSUMERS * 32) : "memory");
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-    uint4 r;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "r"(a));
-    return r;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 r;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(r.x), "=r"(r.y) : "r"(a));
-    return r;
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t r;
-    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(r) : "r"(a));
-    return r;
-}
-__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
-    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(a), "r"(v) : "memory");
-}
 __device__ __forceinline__ uint4 zero_if(bool z, uint4 v) { return z ? make_uint4(0, 0, 0, 0) : v; }
 
 // Shared memory: ring | recv [S*16*64] | vfull [S][16][80] | part [16][64] | barriers
@@ -640,7 +546,7 @@ int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_
         err = cudaLaunchKernelEx(&cfg, bgmv_kernel<MODE_SHRINK>, a);
     else
         err = cudaLaunchKernelEx(&cfg, bgmv_kernel<MODE_EXPAND>, a);
-    return err == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    return cuda_rc(err);
 }
 
 }  // namespace lora

@@ -14,8 +14,10 @@ enum { MODE_FUSED = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 //   B_s as [N*d_out rows][r_max], boxes of 64 rows x 8 ranks
 constexpr int BG_ABOX_COLS = 64, BG_ABOX_ROWS = 8;
 constexpr int BG_BBOX_RANKS = 8, BG_BBOX_ROWS = 64;
+// row_stride: elements between consecutive rows (0 = inner, densely packed)
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
-                  uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+                  uint32_t box_inner, uint32_t box_outer, bool swizzle128,
+                  uint64_t row_stride = 0);
 
 struct BgArgs {
     CUtensorMap tmA[LORA_MAX_SLICES];
@@ -51,6 +53,39 @@ struct SimtArgs {
     int32_t *status;
 };
 
+// Tensor-core SGMV (contiguous tiles): maps over
+//   x      [T][d_in] (row stride ld_x), boxes of 64 columns x 128 rows, 128-byte swizzle
+//   A_s    [N*r_max][d_in], boxes of 64 columns x r_max rows, 128-byte swizzle
+//   B_s    [N*d_out_s][r_max], boxes of 8 ranks x 128 rows, no swizzle
+//   y_s    y + col_off_s as [T][d_out_s] (row stride ld_y), boxes of 64 columns x 128 rows,
+//          128-byte swizzle (loads and stores)
+struct TcArgs {
+    CUtensorMap tmX;
+    CUtensorMap tmA[LORA_MAX_SLICES];
+    CUtensorMap tmB[LORA_MAX_SLICES];
+    CUtensorMap tmY[LORA_MAX_SLICES];
+    __nv_bfloat16 *y;
+    int64_t ld_y;
+    float *v;          // [S][T][r_max] fp32 (shrink / expand modes)
+    int T;
+    int d_in;
+    Slices sl;
+    int r_max;
+    const int32_t *ranks;
+    const float *scales;
+    const int4 *contig;
+    const int32_t *counts;
+    int max_contig;
+    int stages;        // ring slots (set by the launcher)
+    int C;             // blocks per cluster (set by the launcher)
+    int32_t *status;
+};
+
+// lora_api.cu: LORA_OK, or LORA_ERR_CUDA after recording e for lora_last_error()
+int cuda_rc(cudaError_t e);
+// records a failure without a runtime error code (e.g. a driver call) and returns LORA_ERR_CUDA
+int cuda_fail(const char *what);
+
 // segments.cu
 size_t segments_scratch_bytes(int T, int N);
 int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
@@ -59,6 +94,11 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
 // bgmv.cu: bf16, r_max <= 64, vector-aligned data; grid = cluster x n_units
 size_t bgmv_smem_bytes(int n_slices);
 int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_t st);
+
+// sgmv_tc.cu: bf16, r_max % 16 == 0, n_slices * r_max <= 128, 16-byte aligned rows;
+// chooses the cluster size and ring depth, launches persistent clusters
+size_t sgmv_tc_smem_bytes(int mode, int stages, int SR, int C);
+int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st);
 
 // simt.cu: any element type and alignment, r_max <= LORA_MAX_RANK
 size_t simt_smem_bytes(int n_slices, int r_max);

@@ -3,8 +3,30 @@
 #include "kernels.cuh"
 
 #include <cstdint>
+#include <cstdio>
 
 using namespace lora;
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+}  // namespace
+
+namespace lora {
+
+int cuda_rc(cudaError_t e) {
+    if (e == cudaSuccess) return LORA_OK;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return LORA_ERR_CUDA;
+}
+
+int cuda_fail(const char *what) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", what);
+    return LORA_ERR_CUDA;
+}
+
+}  // namespace lora
 
 namespace {
 
@@ -127,8 +149,75 @@ bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
     return true;
 }
 
-int run(int mode, const Call &c, bool gather, bool contig) {
+// The tensor-core SGMV kernel takes the contiguous tiles?  bf16, ranks padded
+// to a multiple of 16, all slices' ranks in one MMA (n_slices * r_max <= 128),
+// 16-byte aligned rows and slices (TMA).
+bool tc_ok(const Call &c, bool need_x, bool need_y) {
+    if (c.dtype != LORA_BF16 || c.meta->min_run <= 0 || c.meta->max_contig_tiles <= 0) return false;
+    if ((c.r_max & 15) || c.n_slices * c.r_max > 128) return false;
+    if (need_x) {
+        if ((c.d_in & 7) || (c.ld_x & 7) || !aligned(c.x, 16)) return false;
+        for (int s = 0; s < c.n_slices; ++s)
+            if (!aligned(c.slices[s].A, 16)) return false;
+    }
+    if (need_y) {
+        if ((c.ld_y & 7) || !aligned(c.y, 16)) return false;
+        for (int s = 0; s < c.n_slices; ++s)
+            if ((c.slices[s].d_out & 7) || (c.slices[s].col_off & 7) || !aligned(c.slices[s].B, 16))
+                return false;
+    }
+    return true;
+}
+
+// Contiguous tiles on the tensor-core SGMV kernel; false if a tensor map
+// cannot be encoded (the caller then keeps those tiles on the other kernels).
+bool run_tc(int mode, const Call &c, int *rc) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
+    const int N = c.meta->N;
+    TcArgs a{};
+    if (need_x &&
+        tensor_map_2d(&a.tmX, c.x, (uint64_t)c.d_in, (uint64_t)c.meta->T, 64, 128, true,
+                      (uint64_t)c.ld_x) != LORA_OK)
+        return false;
+    for (int s = 0; s < c.n_slices; ++s) {
+        const lora_slice &sl = c.slices[s];
+        if (need_x && tensor_map_2d(&a.tmA[s], sl.A, (uint64_t)c.d_in, (uint64_t)N * c.r_max, 64,
+                                    (uint32_t)c.r_max, true) != LORA_OK)
+            return false;
+        if (need_y &&
+            (tensor_map_2d(&a.tmB[s], sl.B, (uint64_t)c.r_max, (uint64_t)N * sl.d_out, 8, 128,
+                           false) != LORA_OK ||
+             tensor_map_2d(&a.tmY[s], static_cast<const __nv_bfloat16 *>(c.y) + sl.col_off,
+                           (uint64_t)sl.d_out, (uint64_t)c.meta->T, 64, 128, true,
+                           (uint64_t)c.ld_y) != LORA_OK))
+            return false;
+    }
+    a.y = static_cast<__nv_bfloat16 *>(c.y);
+    a.ld_y = c.ld_y;
+    a.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
+    a.T = c.meta->T;
+    a.d_in = c.d_in;
+    a.sl = make_slices(c);
+    a.r_max = c.r_max;
+    a.ranks = c.ranks;
+    a.scales = c.scales;
+    a.contig = reinterpret_cast<const int4 *>(c.meta->contig_tiles);
+    a.counts = c.meta->counts;
+    a.max_contig = c.meta->max_contig_tiles;
+    a.status = c.status;
+    *rc = launch_sgmv_tc(mode, a, c.stream);
+    return *rc != LORA_ERR_SHAPE;
+}
+
+int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = true) {
+    const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
+    if (tensor_core && contig && c.meta->T > 0 && tc_ok(c, need_x, need_y)) {
+        int rc = LORA_OK;
+        if (run_tc(mode, c, &rc)) {
+            if (rc != LORA_OK) return rc;
+            contig = false;   // the remaining launch takes the gathered tiles only
+        }
+    }
     Tiles tiles = make_tiles(c.meta, gather, contig);
     const int units = n_units(tiles);
     if (c.meta->T == 0 || units == 0) return LORA_OK;
@@ -185,6 +274,8 @@ int run(int mode, const Call &c, bool gather, bool contig) {
 extern "C" {
 
 int lora_version(void) { return 100; }
+
+const char *lora_last_error(void) { return g_last_error; }
 
 const char *lora_status_string(int status) {
     switch (status) {
@@ -261,7 +352,7 @@ int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t 
            meta, dtype, status, static_cast<cudaStream_t>(stream)};
     int rc = check_call(c, true, true, true, false);
     if (rc != LORA_OK) return rc;
-    return run(MODE_FUSED, c, true, true);
+    return run(MODE_FUSED, c, true, true, false);
 }
 
 int lora_add_linear(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,

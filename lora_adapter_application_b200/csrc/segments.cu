@@ -10,7 +10,7 @@
 //   seg_scatter  one block per chunk: every warp ranks its share of the rows
 //   seg_tiles    one block: runs, contiguous tiles, gathered rows and tiles
 // No block ever waits for another block: the phases are separate launches.
-#include "common.cuh"
+#include "kernels.cuh"
 
 #include <climits>
 
@@ -594,7 +594,7 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
                                  (int)tile_smem);
         seg_tiles_kernel<<<1, SEG_THREADS, tile_smem, st>>>(a);
     }
-    return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    return cuda_rc(cudaGetLastError());
 }
 
 }  // namespace lora

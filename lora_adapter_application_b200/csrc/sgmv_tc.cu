@@ -1,0 +1,815 @@
+// Tensor-core SGMV for contiguous tiles (prompt runs), bf16: page "Multi-LoRA
+// Serving", section 3.2 (SGMV: rows that share an adapter form a segment and
+// the per-segment products are dense) and section 3.4 (add_shrink, then
+// add_expand, in one batched call).
+//
+// A contiguous tile is up to 128 consecutive rows with one adapter n, so both
+// products are dense contractions with M = 128 rows:
+//   shrink  D1[128][S*r_max] = X[128][d_in] . [A_0[n]; ...; A_{S-1}[n]]^T   (K = d_in)
+//   expand  D2[128][128]     = (s_n v)[128][r_max] . B_s[n][cols]^T          (K = r_max)
+// Both run on the 5th-generation tensor cores (tcgen05.mma kind::f16: bf16
+// operands in shared memory, fp32 accumulators in tensor memory); every
+// operand tile reaches shared memory through a TMA tensor copy.
+//
+// A cluster of C thread blocks takes a tile.  Block c reduces 1/C of the input
+// columns and owns 1/C of the 128-column output chunks.  Every block sends its
+// partial D1 to every block of the cluster through distributed shared memory;
+// each block adds the C partials in rank order (run-to-run identical), keeps
+// ranks k < r_n, scales by s_n = alpha/r_n and splits s_n v into a bf16 hi + lo
+// pair (about 16 mantissa bits; one bf16 copy is not enough when the delta is
+// large and cancels against y).  Clusters are persistent: cluster k takes
+// tiles k, k + #clusters, ...; the TMA producer runs ahead across tiles, so
+// HBM keeps streaming while a cluster exchanges its partials.
+//
+// Warp roles (320 threads, one block per SM):
+//   warp 0     TMA producer: x and A boxes (shrink), y and B boxes (expand)
+//              into a ring of `stages` slots; a full/empty mbarrier pair per slot
+//   warp 1     tensor-memory allocator and MMA issuer (one thread issues; when
+//              r_n is not a multiple of 16 the warp first zeroes B's padded
+//              ranks in the slot, so padding never reaches the sum)
+//   warps 2-9  epilogue: D1 -> exchange -> s v in shared memory; D2 + y -> y
+//              (fp32 add, rounded once to bf16) written back by TMA tensor
+//              stores (full tiles) or 16-byte stores of the tile's rows
+//              (partial tiles: a tensor store would write the neighbours' rows)
+//
+// Tensor memory, 512 columns: D2 double buffer at columns 0 and 128, D1 at 256.
+//
+// Every wait is bounded: a wait that runs out sets LORA_DEV_TIMEOUT in the
+// status word; the block then drains its copies and MMAs in flight and leaves.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+#include <cstdlib>
+#include <mutex>
+
+namespace lora {
+
+constexpr int TC_THREADS = 320;
+constexpr int TC_M = 128;                 // rows per tile = MMA M
+constexpr uint32_t TC_XY = 32768;         // x or y part of a slot: two 64-column x 128-row boxes
+constexpr uint32_t TC_BOX = 16384;        // one 64-column x 128-row bf16 box
+constexpr uint32_t TC_D1_COL = 256;       // tensor-memory column of D1
+constexpr uint32_t TC_TMEM_COLS = 512;
+constexpr int TC_MAX_STAGES = 6;
+
+// ------------------------------------------------------------------ descriptors
+// Shared-memory matrix descriptor (tcgen05), K-major, 128-byte swizzle: rows of
+// 128 bytes in 8-row atoms of 1 KB (the layout a TMA box of 64 bf16 columns
+// with 128-byte swizzle leaves behind); the next 8 rows start 1 KB later.
+// Fields: start address >> 4 [0,14), leading offset >> 4 [16,30) (unused
+// here), stride offset >> 4 [32,46), descriptor version 1 [46,48), layout
+// 2 = 128-byte swizzle [61,64).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+// K-major without swizzle: 8-row x 16-byte core matrices stored as 128
+// contiguous bytes; the next 8 rows start 128 B later (stride offset) and the
+// next 8 K elements 2 KB later (leading offset) - a TMA box of 8 bf16 columns
+// x 128 rows, or the s v buffer below.
+__device__ __forceinline__ uint64_t desc_plain(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(2048 >> 4) << 16) |
+           ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator [4,6) = 1, A and B bf16
+// [7,10) = [10,13) = 1, both K-major (bits 15, 16 clear), N >> 3 at [17,23),
+// M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ tcgen05
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// mbarrier arrival once every tcgen05 operation this thread issued has completed
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+// 8 / 16 consecutive fp32 columns of this thread's tensor-memory lane
+__device__ __forceinline__ void tc_ld8(uint32_t taddr, float *v) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------ misc PTX
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n"
+                 "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+    float4 r;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "r"(a));
+    return r;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_cluster() {
+    asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
+}
+// 2-D tensor store (one box) shared -> global, tracked by the bulk-group counter
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(src)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
+
+// Bounded wait taken by a whole warp: every lane sees the same outcome.
+template <bool CLUSTER_ACQUIRE = false>
+__device__ __forceinline__ bool warp_wait(uint32_t bar, unsigned parity, int32_t *status,
+                                          bool &failed) {
+    bool ok = mbar_wait<CLUSTER_ACQUIRE>(bar, parity, status, failed);
+    ok = __all_sync(FULL, ok);
+    if (!ok) failed = true;
+    return ok;
+}
+
+// y += d for 8 bf16 columns (fp32 add, one rounding)
+__device__ __forceinline__ uint4 add8(uint4 y, const float *d) {
+    uint4 o;
+    o.x = pack_bf16x2(bf16_lo(y.x) + d[0], bf16_hi(y.x) + d[1]);
+    o.y = pack_bf16x2(bf16_lo(y.y) + d[2], bf16_hi(y.y) + d[3]);
+    o.z = pack_bf16x2(bf16_lo(y.z) + d[4], bf16_hi(y.z) + d[5]);
+    o.w = pack_bf16x2(bf16_lo(y.w) + d[6], bf16_hi(y.w) + d[7]);
+    return o;
+}
+// keep the first `keep` (0..8) bf16 elements of 8, zero the rest
+__device__ __forceinline__ uint4 keep8(uint4 v, int keep) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (2 * i >= keep) w[i] = 0u;
+        else if (2 * i + 1 >= keep) w[i] &= 0xffffu;
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Shared memory (from a 1 KB boundary):
+//   ring  stages x [x or y boxes: 32 KB | A or B boxes: SR*256 B]
+//   V     SR*512 B   s v as bf16: [slice][hi, lo][rank / 8][128 rows][8]
+//   XCH   C*SR*512 B partials (C > 1, shrink modes): [source block][SR/4][128 rows][4] fp32
+//   mbarriers
+// At least 120 KB, so that one block holds an SM: a block takes all 512
+// tensor-memory columns, and two blocks of different clusters waiting for
+// each other's columns could otherwise stall both clusters.
+size_t sgmv_tc_smem_bytes(int mode, int stages, int SR, int C) {
+    const size_t b = 1024 + (size_t)stages * (TC_XY + (size_t)SR * 256) + (size_t)SR * 512 +
+                     ((mode != MODE_EXPAND && C > 1) ? (size_t)C * SR * 512 : 0) + 512;
+    return b < (size_t)120 * 1024 ? (size_t)120 * 1024 : b;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_constant__ TcArgs a) {
+    extern __shared__ __align__(1024) unsigned char tc_sm[];
+    __shared__ uint32_t tmem_sm;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = a.sl.n, R = a.r_max, SR = S * R, C = a.C, STG = a.stages;
+    const uint32_t crank = cluster_rank();
+    const int cl = blockIdx.x / C, ncl = gridDim.x / C;
+    const bool xchg = MODE != MODE_EXPAND && C > 1;
+    // No tile for this cluster (a batch without prompt runs): leave before
+    // touching tensor memory or the cluster barrier; the same for every block
+    // of the cluster.
+    const int n_tiles = min(a.counts[2], a.max_contig);
+    if (cl >= n_tiles) return;
+
+    const uint32_t ring = (smem_u32(tc_sm) + 1023u) & ~1023u;
+    const uint32_t slot_bytes = TC_XY + (uint32_t)SR * 256u;
+    const uint32_t vbuf = ring + (uint32_t)STG * slot_bytes;
+    const uint32_t xch = vbuf + (uint32_t)SR * 512u;
+    const uint32_t bars = xch + (xchg ? (uint32_t)(C * SR) * 512u : 0u);
+    // per slot: full, empty, and "rows of the y box written" for each half
+    const uint32_t b_full = bars, b_empty = bars + 8u * STG, b_ystage = bars + 16u * STG;   // [2][STG]
+    const uint32_t b_d1full = bars + 32u * STG, b_d1free = b_d1full + 8, b_vfull = b_d1full + 16;
+    const uint32_t b_d2full = b_d1full + 24, b_d2empty = b_d1full + 40;   // [2] each
+    const uint32_t b_xfull = b_d1full + 56, b_xfree = b_d1full + 64, b_mma = b_d1full + 72;
+
+    if (tid == 0) {
+        for (int st = 0; st < STG; ++st) {
+            mbar_init(b_full + 8 * st, 1);
+            mbar_init(b_empty + 8 * st, 2);
+            mbar_init(b_ystage + 8 * st, 4);
+            mbar_init(b_ystage + 8 * (STG + st), 4);
+        }
+        mbar_init(b_d1full, 1);
+        mbar_init(b_d1free, 8);
+        mbar_init(b_vfull, 8);
+        mbar_init(b_d2full, 1);
+        mbar_init(b_d2full + 8, 1);
+        mbar_init(b_d2empty, 8);
+        mbar_init(b_d2empty + 8, 8);
+        mbar_init(b_xfull, 8 * C);
+        mbar_init(b_xfree, 8 * C);
+        mbar_init(b_mma, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_u32(&tmem_sm)),
+                     "r"(TC_TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();   // barriers initialised in every block of the cluster
+    tc_fence_after();
+    const uint32_t tmem = tmem_sm;
+
+    // ------------------------------------------------------------ geometry
+    const int nk = (a.d_in + 127) >> 7;   // 128-column chunks of the input
+    const int k_lo = MODE == MODE_EXPAND ? 0 : (int)(((int64_t)crank * nk) / C);
+    const int k_hi = MODE == MODE_EXPAND ? 0 : (int)(((int64_t)(crank + 1) * nk) / C);
+    int NE = 0;
+    for (int s = 0; s < S; ++s) NE += (a.sl.d_out[s] + 127) >> 7;
+    const int e_lo = MODE == MODE_SHRINK ? 0 : (int)(((int64_t)crank * NE) / C);
+    const int e_hi = MODE == MODE_SHRINK ? 0 : (int)(((int64_t)(crank + 1) * NE) / C);
+    int es0 = 0, ec0 = 0;   // slice and first slice-local column of chunk e_lo
+    {
+        int e = e_lo;
+        while (es0 < S - 1 && e >= ((a.sl.d_out[es0] + 127) >> 7)) {
+            e -= (a.sl.d_out[es0] + 127) >> 7;
+            ++es0;
+        }
+        ec0 = e * 128;
+    }
+    bool failed = false;
+
+    if (warp == 0) {
+        // ============================================================ producer
+        uint32_t fills = 0;
+        int st = 0;
+        uint32_t ph = 0;
+        for (int t = cl; t < n_tiles && !failed; t += ncl) {
+            const int4 tile = a.contig[t];
+            const int id = tile.x, row0 = tile.y;
+            const int r_n = a.ranks[id];
+            if (r_n < 1 || r_n > R) {
+                if (crank == 0 && lane == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
+                continue;
+            }
+            for (int kc = k_lo; kc < k_hi; ++kc) {
+                if (!warp_wait(b_empty + 8 * st, ph ^ 1u, a.status, failed)) break;
+                if (lane == 0) {
+                    const uint32_t slot = ring + (uint32_t)st * slot_bytes, full = b_full + 8 * st;
+                    const int k0 = kc * 128, nb = min(2, (a.d_in - k0 + 63) >> 6);
+                    mbar_expect_tx(full, (uint32_t)nb * (TC_BOX + (uint32_t)SR * 128u));
+                    for (int b = 0; b < nb; ++b) {
+                        tma_2d(slot + b * TC_BOX, &a.tmX, k0 + 64 * b, row0, full);
+                        for (int s = 0; s < S; ++s)
+                            tma_2d(slot + TC_XY + (uint32_t)((b * S + s) * R) * 128u, &a.tmA[s],
+                                   k0 + 64 * b, id * R, full);
+                    }
+                }
+                __syncwarp();
+                ++fills;
+                if (++st == STG) {
+                    st = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (failed) break;
+            int s = es0, c0 = ec0;
+            for (int e = e_lo; e < e_hi; ++e) {
+                if (!warp_wait(b_empty + 8 * st, ph ^ 1u, a.status, failed)) break;
+                const int d_out = a.sl.d_out[s];
+                if (lane == 0) {
+                    const uint32_t slot = ring + (uint32_t)st * slot_bytes, full = b_full + 8 * st;
+                    const int ny = d_out - c0 > 64 ? 2 : 1;
+                    mbar_expect_tx(full, (uint32_t)ny * TC_BOX + (uint32_t)(R >> 3) * 2048u);
+                    for (int h = 0; h < ny; ++h)
+                        tma_2d(slot + h * TC_BOX, &a.tmY[s], c0 + 64 * h, row0, full);
+                    for (int g = 0; g < (R >> 3); ++g)
+                        tma_2d(slot + TC_XY + g * 2048u, &a.tmB[s], 8 * g, id * d_out + c0, full);
+                }
+                __syncwarp();
+                ++fills;
+                if (++st == STG) {
+                    st = 0;
+                    ph ^= 1u;
+                }
+                c0 += 128;
+                if (c0 >= d_out) {
+                    ++s;
+                    c0 = 0;
+                }
+            }
+        }
+        // drain: the copies of the last fill of every slot have landed
+        bool f2 = false;
+        for (int i = 0; i < STG; ++i) {
+            if ((uint32_t)i >= fills) break;
+            const uint32_t f = (uint32_t)i + (uint32_t)STG * ((fills - 1u - (uint32_t)i) / (uint32_t)STG);
+            mbar_wait(b_full + 8 * i, (f / (uint32_t)STG) & 1u, a.status, f2);
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        int st = 0;
+        uint32_t ph = 0, it = 0, ech = 0;
+        const uint32_t id1 = idesc_bf16(TC_M, SR), id2 = idesc_bf16(TC_M, 128);
+        for (int t = cl; t < n_tiles && !failed; t += ncl) {
+            const int4 tile = a.contig[t];
+            const int id = tile.x;
+            const int r_n = a.ranks[id];
+            if (r_n < 1 || r_n > R) continue;
+            if (MODE != MODE_EXPAND) {
+                if (!warp_wait(b_d1free, (it & 1u) ^ 1u, a.status, failed)) break;
+                tc_fence_after();
+                for (int kc = k_lo; kc < k_hi; ++kc) {
+                    if (!warp_wait(b_full + 8 * st, ph, a.status, failed)) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t slot = ring + (uint32_t)st * slot_bytes;
+                        const int nb = min(2, (a.d_in - kc * 128 + 63) >> 6);
+                        for (int b = 0; b < nb; ++b)
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_mma(tmem + TC_D1_COL, desc_sw128(slot + b * TC_BOX + kk * 32),
+                                       desc_sw128(slot + TC_XY + (uint32_t)(b * SR) * 128u + kk * 32),
+                                       id1, (kc > k_lo || b > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(b_empty + 8 * st);   // two arrivals: the slot's count
+                        tc_commit(b_empty + 8 * st);
+                    }
+                    __syncwarp();
+                    if (++st == STG) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (failed) break;
+                if (lane == 0) tc_commit(b_d1full);
+                __syncwarp();
+            }
+            if (MODE != MODE_SHRINK) {
+                if (!warp_wait(b_vfull, it & 1u, a.status, failed)) break;
+                tc_fence_after();
+                const int ksteps = (r_n + 15) >> 4;
+                int s = es0, c0 = ec0;
+                for (int e = e_lo; e < e_hi; ++e) {
+                    const uint32_t buf = ech & 1u;
+                    if (!warp_wait(b_d2empty + 8 * buf, ((ech >> 1) & 1u) ^ 1u, a.status, failed))
+                        break;
+                    if (!warp_wait(b_full + 8 * st, ph, a.status, failed)) break;
+                    tc_fence_after();
+                    const uint32_t slot = ring + (uint32_t)st * slot_bytes;
+                    if (r_n & 15) {   // zero B's ranks r_n .. 16*ksteps-1 (padding)
+                        for (int g = r_n >> 3; g < 2 * ksteps; ++g) {
+                            const int keep = max(0, r_n - 8 * g);
+                            for (int nrow = lane; nrow < 128; nrow += 32) {
+                                const uint32_t ad = slot + TC_XY + g * 2048u + nrow * 16u;
+                                sts128(ad, keep8(lds128(ad), keep));
+                            }
+                        }
+                        fence_proxy_async();
+                        __syncwarp();
+                    }
+                    if (lane == 0) {
+                        const uint32_t vh = vbuf + (uint32_t)(2 * s * R) * 256u, vl = vh + (uint32_t)R * 256u;
+                        const uint32_t d = tmem + buf * 128u;
+                        for (int kk = 0; kk < ksteps; ++kk) {
+                            const uint64_t db = desc_plain(slot + TC_XY + kk * 4096u);
+                            tc_mma(d, desc_plain(vh + kk * 4096u), db, id2, kk > 0 ? 1u : 0u);
+                            tc_mma(d, desc_plain(vl + kk * 4096u), db, id2, 1u);
+                        }
+                        tc_commit(b_d2full + 8 * buf);
+                    }
+                    __syncwarp();
+                    ++ech;
+                    if (++st == STG) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                    c0 += 128;
+                    if (c0 >= a.sl.d_out[s]) {
+                        ++s;
+                        c0 = 0;
+                    }
+                }
+                if (failed) break;
+            }
+            ++it;
+        }
+        // drain: every MMA this warp issued has completed
+        if (lane == 0) tc_commit(b_mma);
+        __syncwarp();
+        bool f2 = false;
+        warp_wait(b_mma, 0, a.status, f2);
+    } else {
+        // ============================================================ epilogue
+        const int q = warp & 3, h = (warp - 2) >> 2, m = 32 * q + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        const bool storer = lane == 0 && (warp == 2 || warp == 6);
+        const int half = SR >> 1, n8 = half >> 3;   // D1 columns of this thread's half
+        int st = 0;
+        uint32_t ph = 0, it = 0, ech = 0;
+        uint32_t yph = 0;   // bit st: phase parity of slot st's y-store barriers (expand uses only)
+        for (int t = cl; t < n_tiles && !failed; t += ncl) {
+            const int4 tile = a.contig[t];
+            const int id = tile.x, row0 = tile.y, cnt = tile.z;
+            const int r_n = a.ranks[id];
+            if (r_n < 1 || r_n > R) continue;
+            float p[64];
+            if (MODE != MODE_EXPAND) {
+                for (int kc = k_lo; kc < k_hi; ++kc)   // slots the MMA warp consumes
+                    if (++st == STG) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                if (!warp_wait(b_d1full, it & 1u, a.status, failed)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j < n8) tc_ld8(lane_base + TC_D1_COL + (uint32_t)(h * half + 8 * j), &p[8 * j]);
+                tc_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_d1free);
+                if (xchg) {
+                    // all-to-all of the partials through distributed shared memory
+                    const int NQ = SR >> 2, qh = half >> 2, q0 = h * qh;
+                    if (!warp_wait<true>(b_xfree, (it & 1u) ^ 1u, a.status, failed)) break;
+                    const uint32_t off = (uint32_t)(((int)crank * NQ + q0) * 128 + m) * 16u;
+                    for (int k = 0; k < C; ++k) {
+                        const uint32_t rb = map_rank(xch, (uint32_t)k) + off;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (j < qh)
+                                st_cluster_f4(rb + j * 2048u, p[4 * j], p[4 * j + 1], p[4 * j + 2],
+                                              p[4 * j + 3]);
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        fence_cluster();
+                        for (int k = 0; k < C; ++k) mbar_arrive_remote(b_xfull, (unsigned)k);
+                    }
+                    if (!warp_wait<true>(b_xfull, it & 1u, a.status, failed)) break;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) p[j] = 0.f;
+                    for (int src = 0; src < C; ++src) {
+                        const uint32_t lb = xch + (uint32_t)((src * NQ + q0) * 128 + m) * 16u;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (j < qh) {
+                                const float4 v = lds128f(lb + j * 2048u);
+                                p[4 * j] += v.x;
+                                p[4 * j + 1] += v.y;
+                                p[4 * j + 2] += v.z;
+                                p[4 * j + 3] += v.w;
+                            }
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        fence_cluster();
+                        for (int k = 0; k < C; ++k) mbar_arrive_remote(b_xfree, (unsigned)k);
+                    }
+                }
+                if (MODE == MODE_SHRINK) {
+                    // v rows of the tile; with a cluster, block c writes the rows m = c (mod C)
+                    if (m < cnt && (m % C) == (int)crank) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (j < n8) {
+                                const int col = h * half + 8 * j, s = col / R, kl = col - s * R;
+                                float *dst = a.v + ((int64_t)s * a.T + row0 + m) * R + kl;
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    if (kl + e < r_n) dst[e] = p[8 * j + e];
+                            }
+                    }
+                    ++it;
+                    continue;
+                }
+            } else {
+                // s v from the caller's v (rows of the tile; zero beyond it)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j < n8) {
+                        const int col = h * half + 8 * j, s = col / R, kl = col - s * R;
+                        const float *src = a.v + ((int64_t)s * a.T + row0 + min(m, cnt - 1)) * R + kl;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            p[8 * j + e] = (m < cnt && kl + e < r_n) ? src[e] : 0.f;
+                    }
+            }
+            if (MODE != MODE_SHRINK) {
+                // s v -> bf16 hi + lo in the no-swizzle K-major layout of the expand MMA
+                const float scale = a.scales[id];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j < n8) {
+                        const int col = h * half + 8 * j, s = col / R, kl = col - s * R;
+                        uint4 hi, lo;
+                        uint32_t *hw = &hi.x, *lw = &lo.x;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const float v0 = kl + 2 * w < r_n ? scale * p[8 * j + 2 * w] : 0.f;
+                            const float v1 = kl + 2 * w + 1 < r_n ? scale * p[8 * j + 2 * w + 1] : 0.f;
+                            hw[w] = pack_bf16x2(v0, v1);
+                            lw[w] = pack_bf16x2(v0 - bf16_lo(hw[w]), v1 - bf16_hi(hw[w]));
+                        }
+                        const uint32_t va =
+                            vbuf + (uint32_t)((2 * s) * (R >> 3) + (kl >> 3)) * 2048u + (uint32_t)m * 16u;
+                        sts128(va, hi);
+                        sts128(va + (uint32_t)R * 256u, lo);
+                    }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_vfull);
+
+                const bool fulltile = cnt == TC_M;
+                int s = es0, c0 = ec0;
+                for (int e = e_lo; e < e_hi; ++e) {
+                    const uint32_t buf = ech & 1u;
+                    if (!warp_wait(b_d2full + 8 * buf, (ech >> 1) & 1u, a.status, failed)) break;
+                    if (!warp_wait(b_full + 8 * st, ph, a.status, failed)) break;
+                    tc_fence_after();
+                    float d[64];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        tc_ld16(lane_base + buf * 128u + (uint32_t)(64 * h + 16 * j), &d[16 * j]);
+                    tc_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_d2empty + 8 * buf);
+
+                    const int d_out = a.sl.d_out[s];
+                    const int cb = c0 + 64 * h;   // first slice-local column of this half's box
+                    const uint32_t ybox = ring + (uint32_t)st * slot_bytes + (uint32_t)h * TC_BOX;
+                    if (cb < d_out) {
+                        const uint32_t rowa = ybox + (uint32_t)(m >> 3) * 1024u + (uint32_t)(m & 7) * 128u;
+                        __nv_bfloat16 *yrow =
+                            a.y + (int64_t)(row0 + min(m, cnt - 1)) * a.ld_y + a.sl.col_off[s] + cb;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (cb + 8 * c < d_out) {
+                                const uint32_t ad = rowa + (uint32_t)((c ^ (m & 7)) << 4);
+                                const uint4 o = add8(lds128(ad), &d[8 * c]);
+                                if (fulltile) sts128(ad, o);
+                                else if (m < cnt) *reinterpret_cast<uint4 *>(yrow + 8 * c) = o;
+                            }
+                    }
+                    if (fulltile) fence_proxy_async();
+                    __syncwarp();
+                    // The slot's own barrier: its next use needs this storer's release
+                    // first, so arrivals of two uses of the slot never mix.
+                    const uint32_t ystage = b_ystage + 8u * (uint32_t)(h * STG + st);
+                    if (lane == 0) mbar_arrive(ystage);
+                    if (storer) {
+                        // the 4 warps of this half have written their rows of the box
+                        bool ok = mbar_wait(ystage, (yph >> st) & 1u, a.status, failed);
+                        if (ok && fulltile && cb < d_out) {
+                            tma_store_2d(&a.tmY[s], cb, row0, ybox);
+                            bulk_wait_read();
+                        }
+                        mbar_arrive(b_empty + 8 * st);
+                    }
+                    __syncwarp();
+                    if (__any_sync(FULL, failed)) failed = true;
+                    yph ^= 1u << st;
+                    ++ech;
+                    if (++st == STG) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                    c0 += 128;
+                    if (c0 >= d_out) {
+                        ++s;
+                        c0 = 0;
+                    }
+                }
+                if (failed) break;
+            }
+            ++it;
+        }
+        if (storer) bulk_wait_all();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                     "r"(TC_TMEM_COLS)
+                     : "memory");
+    }
+    cluster_sync_all();   // no block leaves while a peer may still write to it
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+const void *tc_fn(int mode) {
+    return mode == MODE_FUSED    ? (const void *)sgmv_tc_kernel<MODE_FUSED>
+           : mode == MODE_SHRINK ? (const void *)sgmv_tc_kernel<MODE_SHRINK>
+                                 : (const void *)sgmv_tc_kernel<MODE_EXPAND>;
+}
+
+int env_int(const char *name, int dflt) {
+    const char *s = std::getenv(name);
+    return s && *s ? std::atoi(s) : dflt;
+}
+
+// Largest dynamic shared memory a block of fn may request (the opt-in limit
+// less the kernel's static shared memory), set once as fn's attribute.  A
+// failing runtime call leaves its error as the thread's last error: cleared
+// here so that no later launch check reports it.
+int tc_max_dynamic_smem(const void *fn, int dev) {
+    int optin = 0;
+    cudaFuncAttributes fa{};
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    const int max_dyn = optin - (int)fa.sharedSizeBytes;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return max_dyn;
+}
+
+// Clusters of size C with `smem` bytes per block that fit the device at once.
+int active_clusters(int mode, int C, size_t smem) {
+    struct Key {
+        int dev, mode, C;
+        size_t smem;
+        int n;
+    };
+    static std::mutex mu;
+    static Key cache[64];
+    static int used = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].dev == dev && cache[i].mode == mode && cache[i].C == C && cache[i].smem == smem)
+                return cache[i].n;
+    }
+    const void *fn = tc_fn(mode);
+    const int max_dyn = tc_max_dynamic_smem(fn, dev);
+    if (max_dyn <= 0 || smem > (size_t)max_dyn) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, 1, 1);
+    cfg.blockDim = dim3(TC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < 64) cache[used++] = Key{dev, mode, C, smem, n};
+    return n;
+}
+
+}  // namespace
+
+int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st) {
+    if (a.max_contig <= 0 || a.T <= 0) return LORA_OK;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int optin = tc_max_dynamic_smem(tc_fn(mode), dev);
+    if (optin <= 0) return LORA_ERR_SHAPE;
+    const int SR = a.sl.n * a.r_max;
+    const int nk = (a.d_in + 127) / 128;
+    int NE = 0;
+    for (int s = 0; s < a.sl.n; ++s) NE += (a.sl.d_out[s] + 127) / 128;
+    // Tiles to expect: every row in a full tile (the tile list on the device may be longer).
+    const int est = std::max(1, std::min(a.max_contig, (a.T + TC_M - 1) / TC_M));
+    const int forced_c = env_int("LORA_TC_CLUSTER", 0), forced_s = env_int("LORA_TC_STAGES", 0);
+
+    int best_c = 0, best_stages = 0, best_ncl = 0;
+    double best = -1.0;
+    for (int C = 1; C <= 8; C <<= 1) {
+        if (forced_c && C != forced_c) continue;
+        if (mode != MODE_EXPAND && nk < C) continue;
+        if (mode != MODE_SHRINK && NE < C) continue;
+        int stages = 0;
+        for (int s = TC_MAX_STAGES; s >= 2; --s)
+            if (sgmv_tc_smem_bytes(mode, s, SR, C) <= (size_t)optin) {
+                stages = s;
+                break;
+            }
+        if (forced_s >= 2 && forced_s <= stages) stages = forced_s;
+        if (stages < 2) continue;
+        const size_t smem = sgmv_tc_smem_bytes(mode, stages, SR, C);
+        const int ncl = active_clusters(mode, C, smem);
+        if (ncl < 1) continue;
+        // fraction of the SMs busy over the whole launch, with whole rounds of tiles
+        const int rounds = (est + ncl - 1) / ncl;
+        const double score = (double)est / ((double)rounds * ncl) * ((double)ncl * C / sms);
+        if (score > best * 1.03) {
+            best = score;
+            best_c = C;
+            best_stages = stages;
+            best_ncl = ncl;
+        }
+    }
+    if (best_c == 0) return LORA_ERR_SHAPE;
+    a.C = best_c;
+    a.stages = best_stages;
+    const size_t smem = sgmv_tc_smem_bytes(mode, best_stages, SR, best_c);
+    const int clusters = std::min(best_ncl, a.max_contig);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(best_c * clusters, 1, 1);
+    cfg.blockDim = dim3(TC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = best_c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err;
+    if (mode == MODE_FUSED)
+        err = cudaLaunchKernelEx(&cfg, sgmv_tc_kernel<MODE_FUSED>, a);
+    else if (mode == MODE_SHRINK)
+        err = cudaLaunchKernelEx(&cfg, sgmv_tc_kernel<MODE_SHRINK>, a);
+    else
+        err = cudaLaunchKernelEx(&cfg, sgmv_tc_kernel<MODE_EXPAND>, a);
+    return cuda_rc(err);
+}
+
+}  // namespace lora

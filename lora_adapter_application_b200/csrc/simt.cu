@@ -119,7 +119,7 @@ int launch_simt(int mode, bool bf16, const SimtArgs &a, int n_units, cudaStream_
     if (n_units <= 0) return LORA_OK;
     cudaError_t e = bf16 ? launch_simt_t<__nv_bfloat16>(mode, a, n_units, st)
                          : launch_simt_t<float>(mode, a, n_units, st);
-    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    return cuda_rc(e);
 }
 
 }  // namespace lora

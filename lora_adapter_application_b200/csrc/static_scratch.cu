@@ -39,12 +39,15 @@ void *g_addr[kMaxDevices] = {};
 // Device address of the array on the current device (looked up once).
 int static_scratch_address(void **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_ERR_CUDA;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return lora::cuda_rc(e);
+    if (dev < 0 || dev >= kMaxDevices) return lora::cuda_fail("device index beyond the static scratch table");
     std::lock_guard<std::mutex> lock(g_mutex);
     if (g_addr[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, lora_static_scratch) != cudaSuccess || p == nullptr)
-            return LORA_ERR_CUDA;
+        const cudaError_t e = cudaGetSymbolAddress(&p, lora_static_scratch);
+        if (e != cudaSuccess) return lora::cuda_rc(e);
+        if (p == nullptr) return lora::cuda_fail("cudaGetSymbolAddress returned no address");
         g_addr[dev] = p;
     }
     *out = g_addr[dev];

@@ -13,7 +13,7 @@ namespace {
 
 struct Entry {
     const void *base;
-    uint64_t inner, outer;
+    uint64_t inner, outer, stride;
     uint32_t box_inner, box_outer;
     int swizzle;
     int dev;
@@ -42,22 +42,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 }  // namespace
 
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
-                  uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+                  uint32_t box_inner, uint32_t box_outer, bool swizzle128, uint64_t row_stride) {
+    if (row_stride == 0) row_stride = inner;
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lock(g_mu);
     for (int i = 0; i < g_used; ++i) {
         const Entry &e = g_cache[i];
-        if (e.base == base && e.inner == inner && e.outer == outer && e.box_inner == box_inner &&
+        if (e.base == base && e.inner == inner && e.outer == outer && e.stride == row_stride &&
+            e.box_inner == box_inner &&
             e.box_outer == box_outer && e.swizzle == (int)swizzle128 && e.dev == dev) {
             *out = e.map;
             return LORA_OK;
         }
     }
     auto fn = encoder();
-    if (!fn) return LORA_ERR_CUDA;
+    if (!fn) return cuda_fail("cuTensorMapEncodeTiled: driver entry point not found");
     const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {inner * 2};   // bf16 rows
+    const cuuint64_t strides[1] = {row_stride * 2};   // bf16 rows
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     CUtensorMap m;
@@ -65,11 +67,12 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return LORA_ERR_CUDA;
+    if (r != CUDA_SUCCESS) return cuda_fail("cuTensorMapEncodeTiled failed");
     Entry &e = g_cache[g_used < kCache ? g_used++ : (g_next++ % kCache)];
     e.base = base;
     e.inner = inner;
     e.outer = outer;
+    e.stride = row_stride;
     e.box_inner = box_inner;
     e.box_outer = box_outer;
     e.swizzle = (int)swizzle128;
