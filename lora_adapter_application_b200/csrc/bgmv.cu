@@ -48,6 +48,8 @@
 
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 namespace cg = cooperative_groups;
 
 namespace lora {
@@ -106,37 +108,34 @@ struct ChunkIt {
     int es, c0, w;         // expand: slice, first slice-local column, width
 };
 
-template <int MODE>
-__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_constant__ BgArgs a) {
-    extern __shared__ __align__(128) unsigned char bg_sm[];
-    __shared__ int rows_sm[BG_ROWS];
+// Shared-memory carve-up of a block (the same for every unit it takes).
+struct BgSmem {
+    unsigned char *ring;
+    float *recv, *vfull, *part;
+    int *rows;
+    uint32_t ring_s, full0, empty0, xready, vready;
+};
 
+// One unit on one block of its cluster.  `base`: chunks this block streamed
+// through the ring for earlier units (slot and phase of every chunk follow
+// from base + its index); `uiter`: units this block took before (phase of the
+// exchange barriers).  Returns the unit's chunk count.
+template <int MODE>
+__device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm, const Unit &u,
+                                              int r_n, uint32_t base, uint32_t uiter,
+                                              bool &failed) {
     const int S = a.sl.n;
-    // ring on a 1 KB boundary: swizzled TMA boxes need their 1 KB atom aligned
-    unsigned char *ring = bg_sm + ((1024u - (smem_u32(bg_sm) & 1023u)) & 1023u);
-    float *recv = reinterpret_cast<float *>(ring + BG_STAGES * BG_STAGE_BYTES);
-    float *vfull = recv + S * BG_ROWS * BG_RMAX;
-    float *part = vfull + S * BG_ROWS * BG_VF_STRIDE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(part + BG_ROWS * BG_RMAX);
-    const uint32_t ring_s = smem_u32(ring);
-    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * BG_STAGES;
-    const uint32_t xready = full0 + 16 * BG_STAGES, vready = xready + 8;
+    unsigned char *ring = sm.ring;
+    float *recv = sm.recv, *vfull = sm.vfull, *part = sm.part;
+    const int *rows_sm = sm.rows;
+    const uint32_t ring_s = sm.ring_s, full0 = sm.full0, empty0 = sm.empty0;
+    const uint32_t xready = sm.xready, vready = sm.vready;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int C = gridDim.x, crank = blockIdx.x;
-
-    const Unit u = resolve_unit(a.tiles, blockIdx.y);
-    if (u.cnt == 0) return;                        // uniform over the cluster
     const int n = u.id;
-    const int r_n = a.ranks[n];
-    if (r_n < 1 || r_n > a.r_max) {
-        if (crank == 0 && tid == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
-        return;
-    }
     const int cnt = u.cnt;
-    if (tid < BG_ROWS) rows_sm[tid] = tid < cnt ? u.row(a.tiles, tid) : -1;
-    for (int e = tid; e < S * BG_ROWS * BG_VF_STRIDE; e += BG_THREADS) vfull[e] = 0.f;
 
     // ------------------------------------------------------------ geometry
     Geo G;
@@ -226,30 +225,18 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
         }
     };
 
-    // barriers
-    if (tid == 0) {
-        for (int st = 0; st < BG_STAGES; ++st) {
-            mbar_init(full0 + 8 * st, 1);
-            mbar_init(empty0 + 8 * st, BG_CONSUMERS);
-        }
-        mbar_init(xready, C);
-        mbar_init(vready, C);
-        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    }
     cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();   // barriers initialised in every block; rows_sm and vfull ready
-
-    bool failed = false;
 
     if (warp == BG_CONSUMERS) {
         // ============================================================ producer
         ChunkIt it;
         first(it);
         for (; it.i < G.n_chunks; advance(it)) {
-            const int st = it.i % BG_STAGES;
+            const uint32_t gi = base + (uint32_t)it.i;   // position in the block's ring stream
+            const int st = (int)(gi % BG_STAGES);
             const uint32_t full = full0 + 8 * st, dst = ring_s + st * BG_STAGE_BYTES;
-            if (it.i >= BG_STAGES)
-                mbar_wait(empty0 + 8 * st, ((it.i / BG_STAGES) - 1) & 1, a.status, failed);
+            if (gi >= BG_STAGES)
+                mbar_wait(empty0 + 8 * st, ((gi / BG_STAGES) - 1) & 1, a.status, failed);
             if (failed) break;
             if (it.i < G.n_shrink) {
                 const int jc0 = G.j_lo + it.q * G.JC;
@@ -281,7 +268,7 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
                 }
             }
         }
-        return;
+        return (uint32_t)G.n_chunks;
     }
 
     // ================================================================ consumers
@@ -376,7 +363,7 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
             asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
             for (int c = 0; c < C; ++c) mbar_arrive_remote(xready, c);
         }
-        mbar_wait<true>(xready, 0, a.status, failed);   // every partial has reached its owner
+        mbar_wait<true>(xready, uiter & 1u, a.status, failed);   // every partial has reached its owner
         const float scale = MODE == MODE_FUSED ? a.scales[n] : 1.f;
         const int mine = (S * BG_ROWS * BG_RMAX - crank + C - 1) / C;   // elements e = crank + C*j
         for (int j = ctid; j < mine; j += BG_CONSUMERS * 32) {
@@ -400,7 +387,7 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
                 asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
                 for (int c = 0; c < C; ++c) mbar_arrive_remote(vready, c);
             }
-            mbar_wait<true>(vready, 0, a.status, failed);   // every block holds the full s*v
+            mbar_wait<true>(vready, uiter & 1u, a.status, failed);   // every block holds the full s*v
         }
     };
 
@@ -495,13 +482,14 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
     first(it);
     bool exchanged = false;
     for (; it.i < G.n_chunks; advance(it)) {
-        const int st = it.i % BG_STAGES;
+        const uint32_t gi = base + (uint32_t)it.i;
+        const int st = (int)(gi % BG_STAGES);
         const uint32_t sta = ring_s + st * BG_STAGE_BYTES;
         if (!exchanged && it.i >= G.n_shrink) {
             exchange();
             exchanged = true;
         }
-        const bool ready = mbar_wait(full0 + 8 * st, (it.i / BG_STAGES) & 1, a.status, failed);
+        const bool ready = mbar_wait(full0 + 8 * st, (gi / BG_STAGES) & 1, a.status, failed);
         if (ready) {
             if (it.i < G.n_shrink)
                 shrink_chunk(it, sta);
@@ -513,22 +501,135 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
         if (lane == 0) mbar_arrive(empty0 + 8 * st);
     }
     if (!exchanged) exchange();
+    return (uint32_t)G.n_chunks;
 }
 
-int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_t st) {
-    const size_t smem = bgmv_smem_bytes(a.sl.n);
-    static bool attr_done[3] = {false, false, false};
-    const void *fn = mode == MODE_FUSED    ? (const void *)bgmv_kernel<MODE_FUSED>
-                     : mode == MODE_SHRINK ? (const void *)bgmv_kernel<MODE_SHRINK>
-                                           : (const void *)bgmv_kernel<MODE_EXPAND>;
-    if (!attr_done[mode]) {
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)bgmv_smem_bytes(LORA_MAX_SLICES));
-        attr_done[mode] = true;
+// Persistent clusters: cluster k takes the live units k, k + #clusters, ...
+template <int MODE>
+__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_constant__ BgArgs a) {
+    extern __shared__ __align__(128) unsigned char bg_sm[];
+    __shared__ int rows_sm[BG_ROWS];
+
+    const int S = a.sl.n;
+    BgSmem sm;
+    // ring on a 1 KB boundary: swizzled TMA boxes need their 1 KB atom aligned
+    sm.ring = bg_sm + ((1024u - (smem_u32(bg_sm) & 1023u)) & 1023u);
+    sm.recv = reinterpret_cast<float *>(sm.ring + BG_STAGES * BG_STAGE_BYTES);
+    sm.vfull = sm.recv + S * BG_ROWS * BG_RMAX;
+    sm.part = sm.vfull + S * BG_ROWS * BG_VF_STRIDE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm.part + BG_ROWS * BG_RMAX);
+    sm.rows = rows_sm;
+    sm.ring_s = smem_u32(sm.ring);
+    sm.full0 = smem_u32(bars);
+    sm.empty0 = sm.full0 + 8 * BG_STAGES;
+    sm.xready = sm.full0 + 16 * BG_STAGES;
+    sm.vready = sm.xready + 8;
+
+    const int tid = threadIdx.x;
+    const int C = gridDim.x;
+    if (tid == 0) {
+        for (int st = 0; st < BG_STAGES; ++st) {
+            mbar_init(sm.full0 + 8 * st, 1);
+            mbar_init(sm.empty0 + 8 * st, BG_CONSUMERS);
+        }
+        mbar_init(sm.xready, C);
+        mbar_init(sm.vready, C);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
+    cg::cluster_group cluster = cg::this_cluster();
+
+    // Every block of a cluster walks the same units and takes the same branches,
+    // so the cluster barriers below always pair up; a block whose wait ran out
+    // keeps walking (its waits then return at once) instead of leaving early.
+    bool failed = false;
+    uint32_t base = 0, uiter = 0;
+    const int live = n_live_units(a.tiles);
+    for (int v = blockIdx.y; v < live; v += gridDim.y) {
+        const Unit u = resolve_live_unit(a.tiles, v);
+        if (u.cnt == 0) continue;
+        const int r_n = a.ranks[u.id];
+        if (r_n < 1 || r_n > a.r_max) {
+            if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
+            continue;
+        }
+        if (uiter > 0) cluster.sync();   // the previous unit is done in every block
+        if (tid < BG_ROWS) rows_sm[tid] = tid < u.cnt ? u.row(a.tiles, tid) : -1;
+        for (int e = tid; e < S * BG_ROWS * BG_VF_STRIDE; e += BG_THREADS) sm.vfull[e] = 0.f;
+        cluster.sync();                  // barriers, rows and zeroed s*v ready in every block
+        base += bgmv_unit<MODE>(a, sm, u, r_n, base, uiter, failed);
+        ++uiter;
+    }
+    cluster.sync();   // no block leaves while a peer may still write to it
+}
+
+namespace {
+
+const void *bg_fn(int mode) {
+    return mode == MODE_FUSED    ? (const void *)bgmv_kernel<MODE_FUSED>
+           : mode == MODE_SHRINK ? (const void *)bgmv_kernel<MODE_SHRINK>
+                                 : (const void *)bgmv_kernel<MODE_EXPAND>;
+}
+
+// Clusters of `cluster` blocks with `smem` bytes each that fit the device at once
+// (0 if the query fails).
+int bg_active_clusters(int mode, int cluster, size_t smem) {
+    struct Key {
+        int dev, mode, cluster;
+        size_t smem;
+        int n;
+    };
+    static std::mutex mu;
+    static Key cache[64];
+    static int used = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].dev == dev && cache[i].mode == mode && cache[i].cluster == cluster &&
+                cache[i].smem == smem)
+                return cache[i].n;
+    }
+    const void *fn = bg_fn(mode);
+    int n = 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bgmv_smem_bytes(LORA_MAX_SLICES)) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cluster, 1, 1);
+        cfg.blockDim = dim3(BG_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();   // a failed query must not surface as a later launch error
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < 64) cache[used++] = Key{dev, mode, cluster, smem, n};
+    return n;
+}
+
+}  // namespace
+
+// Persistent launch: as many clusters as fit the device at once (at most one
+// per unit of the tile-list capacity); each walks the live units.
+int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_t st) {
     if (n_units <= 0) return LORA_OK;
+    const size_t smem = bgmv_smem_bytes(a.sl.n);
+    int clusters = bg_active_clusters(mode, cluster, smem);
+    if (clusters < 1) {
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        clusters = sms / cluster > 0 ? sms / cluster : 1;
+    }
+    clusters = clusters < n_units ? clusters : n_units;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cluster, n_units, 1);
+    cfg.gridDim = dim3(cluster, clusters, 1);
     cfg.blockDim = dim3(BG_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;

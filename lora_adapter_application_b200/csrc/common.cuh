@@ -82,4 +82,31 @@ __device__ __forceinline__ Unit resolve_unit(const Tiles &t, int u) {
     return r;
 }
 
+// Units that exist in this batch, numbered without gaps: the gathered tiles
+// first, then rows_per_unit-row slices of the contiguous tiles (a slice past
+// its tile's end resolves to cnt = 0).  Read from the device-side counts, so a
+// persistent grid walks only real work.
+__device__ __forceinline__ int n_live_units(const Tiles &t) {
+    const int ng = t.use_gather ? min(t.counts[1], t.max_gather) : 0;
+    const int nc = t.subs ? min(t.counts[2], t.max_contig) : 0;
+    return ng + nc * t.subs;
+}
+
+__device__ __forceinline__ Unit resolve_live_unit(const Tiles &t, int v) {
+    Unit r{0, 0, 0, true};
+    const int ng = t.use_gather ? min(t.counts[1], t.max_gather) : 0;
+    if (v < ng) {
+        const int4 g = t.gather[v];
+        r.id = g.x; r.base = g.y; r.cnt = g.z; r.gathered = true;
+        return r;
+    }
+    v -= ng;
+    const int tile = v / t.subs, sub = v - tile * t.subs;
+    const int4 c = t.contig[tile];
+    const int first = sub * t.rows_per_unit;
+    if (first >= c.z) return r;
+    r.id = c.x; r.base = c.y + first; r.cnt = min(t.rows_per_unit, c.z - first); r.gathered = false;
+    return r;
+}
+
 }  // namespace lora

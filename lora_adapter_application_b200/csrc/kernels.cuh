@@ -54,16 +54,20 @@ struct SimtArgs {
 };
 
 // Tensor-core SGMV (contiguous tiles): maps over
-//   x      [T][d_in] (row stride ld_x), boxes of 64 columns x 128 rows, 128-byte swizzle
+//   x      [T][d_in] (row stride ld_x), boxes of 64 columns x lbr rows, 128-byte swizzle
 //   A_s    [N*r_max][d_in], boxes of 64 columns x r_max rows, 128-byte swizzle
 //   B_s    [N*d_out_s][r_max], boxes of 8 ranks x 128 rows, no swizzle
-//   y_s    y + col_off_s as [T][d_out_s] (row stride ld_y), boxes of 64 columns x 128 rows,
-//          128-byte swizzle (loads and stores)
+//   y_s    y + col_off_s as [T][d_out_s] (row stride ld_y), 128-byte swizzle: boxes of
+//          64 columns x lbr rows (tmY, loads) and x sbr rows (tmYs, stores)
+// (about 4.6 KB of kernel parameters: within the 32 KB CUDA 12.1+ allows)
 struct TcArgs {
     CUtensorMap tmX;
     CUtensorMap tmA[LORA_MAX_SLICES];
     CUtensorMap tmB[LORA_MAX_SLICES];
     CUtensorMap tmY[LORA_MAX_SLICES];
+    CUtensorMap tmYs[LORA_MAX_SLICES];
+    int lbr;           // rows of an x / y load box (8 .. 128, power of two)
+    int sbr;           // rows of a y store box (8 .. 128, power of two)
     __nv_bfloat16 *y;
     int64_t ld_y;
     float *v;          // [S][T][r_max] fp32 (shrink / expand modes)

@@ -4,6 +4,8 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
+#include <mutex>
 
 using namespace lora;
 
@@ -30,16 +32,60 @@ int cuda_fail(const char *what) {
 
 namespace {
 
-// Blocks per unit of the fused kernel: the smallest power of two (up to 8)
-// that gives about three blocks per SM, so a unit is split only as far as
-// needed to fill the GPU (fewer, larger blocks hide their start-up latency).
-int bgmv_cluster(int units) {
+// Blocks per unit of the fused kernel.  Measured on B200 (persistent grid,
+// about two blocks per SM): 4 suits decode batches from the q_proj shape to
+// the Llama-3-8B layer set; 8 when the units are few - the gathered rows of a
+// batch whose prompt runs went to the tensor-core kernel (est_units = 1), or
+// a tile list of a handful of units.
+int bgmv_cluster(int est_units) {
+    if (const char *e = std::getenv("LORA_BG_CLUSTER")) {   // tuning override: 1, 2, 4 or 8
+        const int c = std::atoi(e);
+        if (c == 1 || c == 2 || c == 4 || c == 8) return c;
+    }
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int c = 1;
-    while (c < 8 && (int64_t)units * c < 3LL * sms) c <<= 1;
-    return c;
+    return (int64_t)est_units * 4 * 2 < sms ? 8 : 4;
+}
+
+// A second stream per device for the gathered-tile launch of a call whose
+// contiguous tiles take the tensor-core kernel: forked from and joined back to
+// the caller's stream with events (also under stream capture), so that its
+// blocks fill the SMs the persistent tensor-core grid leaves free.  The two
+// launches touch disjoint rows.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kSideDevices = 64;
+std::mutex g_side_mu;
+SideStream g_side[kSideDevices];
+
+// fn(side stream) between a fork from and a join into `caller`
+template <class F>
+int on_side_stream(cudaStream_t caller, F &&fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_rc(e);
+    if (dev < 0 || dev >= kSideDevices) return fn(caller);
+    std::lock_guard<std::mutex> lock(g_side_mu);   // one fork/join sequence at a time
+    SideStream &ss = g_side[dev];
+    if (!ss.stream) {
+        if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) {
+            ss = SideStream{};
+            return cuda_rc(e);
+        }
+    }
+    if ((e = cudaEventRecord(ss.fork, caller)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ss.stream, ss.fork, 0)) != cudaSuccess)
+        return cuda_rc(e);
+    const int rc = fn(ss.stream);
+    if ((e = cudaEventRecord(ss.join, ss.stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(caller, ss.join, 0)) != cudaSuccess)
+        return cuda_rc(e);
+    return rc;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -175,8 +221,17 @@ bool run_tc(int mode, const Call &c, int *rc) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
     const int N = c.meta->N;
     TcArgs a{};
+    // rows of the x / y load boxes and of the y store boxes (tuning overrides:
+    // LORA_TC_LOAD_ROWS, LORA_TC_STORE_ROWS; powers of two from 8 to 128)
+    auto box_rows = [](const char *name, int dflt) {
+        const char *e = std::getenv(name);
+        const int v = e ? std::atoi(e) : 0;
+        return (v >= 8 && v <= 128 && (v & (v - 1)) == 0) ? v : dflt;
+    };
+    a.lbr = box_rows("LORA_TC_LOAD_ROWS", 128);
+    a.sbr = box_rows("LORA_TC_STORE_ROWS", 128);
     if (need_x &&
-        tensor_map_2d(&a.tmX, c.x, (uint64_t)c.d_in, (uint64_t)c.meta->T, 64, 128, true,
+        tensor_map_2d(&a.tmX, c.x, (uint64_t)c.d_in, (uint64_t)c.meta->T, 64, (uint32_t)a.lbr, true,
                       (uint64_t)c.ld_x) != LORA_OK)
         return false;
     for (int s = 0; s < c.n_slices; ++s) {
@@ -184,12 +239,14 @@ bool run_tc(int mode, const Call &c, int *rc) {
         if (need_x && tensor_map_2d(&a.tmA[s], sl.A, (uint64_t)c.d_in, (uint64_t)N * c.r_max, 64,
                                     (uint32_t)c.r_max, true) != LORA_OK)
             return false;
+        const __nv_bfloat16 *ys = static_cast<const __nv_bfloat16 *>(c.y) + sl.col_off;
         if (need_y &&
             (tensor_map_2d(&a.tmB[s], sl.B, (uint64_t)c.r_max, (uint64_t)N * sl.d_out, 8, 128,
                            false) != LORA_OK ||
-             tensor_map_2d(&a.tmY[s], static_cast<const __nv_bfloat16 *>(c.y) + sl.col_off,
-                           (uint64_t)sl.d_out, (uint64_t)c.meta->T, 64, 128, true,
-                           (uint64_t)c.ld_y) != LORA_OK))
+             tensor_map_2d(&a.tmY[s], ys, (uint64_t)sl.d_out, (uint64_t)c.meta->T, 64,
+                           (uint32_t)a.lbr, true, (uint64_t)c.ld_y) != LORA_OK ||
+             tensor_map_2d(&a.tmYs[s], ys, (uint64_t)sl.d_out, (uint64_t)c.meta->T, 64,
+                           (uint32_t)a.sbr, true, (uint64_t)c.ld_y) != LORA_OK))
             return false;
     }
     a.y = static_cast<__nv_bfloat16 *>(c.y);
@@ -211,11 +268,13 @@ bool run_tc(int mode, const Call &c, int *rc) {
 
 int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = true) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
+    bool tc_took = false;
     if (tensor_core && contig && c.meta->T > 0 && tc_ok(c, need_x, need_y)) {
         int rc = LORA_OK;
         if (run_tc(mode, c, &rc)) {
             if (rc != LORA_OK) return rc;
             contig = false;   // the remaining launch takes the gathered tiles only
+            tc_took = true;
         }
     }
     Tiles tiles = make_tiles(c.meta, gather, contig);
@@ -249,7 +308,12 @@ int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = tr
             bg.scales = c.scales;
             bg.tiles = tiles;
             bg.status = c.status;
-            return launch_bgmv(mode, bg, units, bgmv_cluster(units), c.stream);
+            const int cl = bgmv_cluster(tc_took ? 1 : units);
+            if (tc_took)
+                return on_side_stream(c.stream, [&](cudaStream_t s) {
+                    return launch_bgmv(mode, bg, units, cl, s);
+                });
+            return launch_bgmv(mode, bg, units, cl, c.stream);
         }
     }
     SimtArgs a{};

@@ -21,16 +21,23 @@
 // tiles k, k + #clusters, ...; the TMA producer runs ahead across tiles, so
 // HBM keeps streaming while a cluster exchanges its partials.
 //
-// Warp roles (320 threads, one block per SM):
+// Warp roles (352 threads, one block per SM):
 //   warp 0     TMA producer: x and A boxes (shrink), y and B boxes (expand)
-//              into a ring of `stages` slots; a full/empty mbarrier pair per slot
+//              into a ring of `stages` slots; a full/empty mbarrier pair per
+//              slot.  x and y move in boxes of lbr rows issued row group by row
+//              group (both 64-column halves of a row group back to back), one
+//              box per lane; a partial tile loads only the row groups it has.
 //   warp 1     tensor-memory allocator and MMA issuer (one thread issues; when
 //              r_n is not a multiple of 16 the warp first zeroes B's padded
 //              ranks in the slot, so padding never reaches the sum)
 //   warps 2-9  epilogue: D1 -> exchange -> s v in shared memory; D2 + y -> y
-//              (fp32 add, rounded once to bf16) written back by TMA tensor
-//              stores (full tiles) or 16-byte stores of the tile's rows
-//              (partial tiles: a tensor store would write the neighbours' rows)
+//              (fp32 add, rounded once to bf16) in place in the slot, or with
+//              16-byte stores straight to the tile's rows for a partial tile
+//              (a tensor store would write the neighbours' rows)
+//   warp 10    store warp: TMA tensor stores of finished y boxes; it frees a
+//              slot once its stores have read it.  (A store waits in the TMA
+//              queue behind the loads issued before it, about 2 us under load;
+//              on its own warp that wait no longer holds up the epilogue.)
 //
 // Tensor memory, 512 columns: D2 double buffer at columns 0 and 128, D1 at 256.
 //
@@ -44,7 +51,7 @@
 
 namespace lora {
 
-constexpr int TC_THREADS = 320;
+constexpr int TC_THREADS = 352;
 constexpr int TC_M = 128;                 // rows per tile = MMA M
 constexpr uint32_t TC_XY = 32768;         // x or y part of a slot: two 64-column x 128-row boxes
 constexpr uint32_t TC_BOX = 16384;        // one 64-column x 128-row bf16 box
@@ -166,17 +173,23 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void fence_cluster() {
     asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
 }
-// 2-D tensor store (one box) shared -> global, tracked by the bulk-group counter
+// 2-D tensor store (one box) shared -> global, tracked by this thread's bulk groups
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src) {
     asm volatile(
         "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
             reinterpret_cast<uint64_t>(map)),
         "r"(x), "r"(y), "r"(src)
         : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+// every bulk group but the most recent one has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_but1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
@@ -247,18 +260,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
     const uint32_t vbuf = ring + (uint32_t)STG * slot_bytes;
     const uint32_t xch = vbuf + (uint32_t)SR * 512u;
     const uint32_t bars = xch + (xchg ? (uint32_t)(C * SR) * 512u : 0u);
-    // per slot: full, empty, and "rows of the y box written" for each half
-    const uint32_t b_full = bars, b_empty = bars + 8u * STG, b_ystage = bars + 16u * STG;   // [2][STG]
-    const uint32_t b_d1full = bars + 32u * STG, b_d1free = b_d1full + 8, b_vfull = b_d1full + 16;
+    // per slot: full, empty, and "the epilogue has written the slot's y"
+    const uint32_t b_full = bars, b_empty = bars + 8u * STG, b_ystage = bars + 16u * STG;
+    const uint32_t b_d1full = bars + 24u * STG, b_d1free = b_d1full + 8, b_vfull = b_d1full + 16;
     const uint32_t b_d2full = b_d1full + 24, b_d2empty = b_d1full + 40;   // [2] each
     const uint32_t b_xfull = b_d1full + 56, b_xfree = b_d1full + 64, b_mma = b_d1full + 72;
 
     if (tid == 0) {
         for (int st = 0; st < STG; ++st) {
             mbar_init(b_full + 8 * st, 1);
-            mbar_init(b_empty + 8 * st, 2);
-            mbar_init(b_ystage + 8 * st, 4);
-            mbar_init(b_ystage + 8 * (STG + st), 4);
+            mbar_init(b_empty + 8 * st, 1);
+            mbar_init(b_ystage + 8 * st, 8);
         }
         mbar_init(b_d1full, 1);
         mbar_init(b_d1free, 8);
@@ -316,18 +328,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
                 if (crank == 0 && lane == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
                 continue;
             }
+            const int lbr = a.lbr, nrg = (tile.z + lbr - 1) / lbr;   // load boxes down the tile
+            const uint32_t lbox = (uint32_t)lbr * 128u;                  // bytes of one load box
             for (int kc = k_lo; kc < k_hi; ++kc) {
                 if (!warp_wait(b_empty + 8 * st, ph ^ 1u, a.status, failed)) break;
-                if (lane == 0) {
-                    const uint32_t slot = ring + (uint32_t)st * slot_bytes, full = b_full + 8 * st;
-                    const int k0 = kc * 128, nb = min(2, (a.d_in - k0 + 63) >> 6);
-                    mbar_expect_tx(full, (uint32_t)nb * (TC_BOX + (uint32_t)SR * 128u));
-                    for (int b = 0; b < nb; ++b) {
-                        tma_2d(slot + b * TC_BOX, &a.tmX, k0 + 64 * b, row0, full);
-                        for (int s = 0; s < S; ++s)
-                            tma_2d(slot + TC_XY + (uint32_t)((b * S + s) * R) * 128u, &a.tmA[s],
-                                   k0 + 64 * b, id * R, full);
-                    }
+                const uint32_t slot = ring + (uint32_t)st * slot_bytes, full = b_full + 8 * st;
+                const int k0 = kc * 128, nb = min(2, (a.d_in - k0 + 63) >> 6);
+                if (lane == 0)
+                    mbar_expect_tx(full, (uint32_t)(nb * nrg) * lbox + (uint32_t)(nb * SR) * 128u);
+                __syncwarp();
+                for (int i = lane; i < nrg * nb; i += 32) {   // x: row group major
+                    const int rg = i / nb, b = i - rg * nb;
+                    tma_2d(slot + b * TC_BOX + rg * lbox, &a.tmX, k0 + 64 * b, row0 + lbr * rg, full);
+                }
+                for (int i = lane; i < nb * S; i += 32) {     // A of every slice
+                    const int b = i / S, s = i - b * S;
+                    tma_2d(slot + TC_XY + (uint32_t)((b * S + s) * R) * 128u, &a.tmA[s], k0 + 64 * b,
+                           id * R, full);
                 }
                 __syncwarp();
                 ++fills;
@@ -341,15 +358,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
             for (int e = e_lo; e < e_hi; ++e) {
                 if (!warp_wait(b_empty + 8 * st, ph ^ 1u, a.status, failed)) break;
                 const int d_out = a.sl.d_out[s];
-                if (lane == 0) {
-                    const uint32_t slot = ring + (uint32_t)st * slot_bytes, full = b_full + 8 * st;
-                    const int ny = d_out - c0 > 64 ? 2 : 1;
-                    mbar_expect_tx(full, (uint32_t)ny * TC_BOX + (uint32_t)(R >> 3) * 2048u);
-                    for (int h = 0; h < ny; ++h)
-                        tma_2d(slot + h * TC_BOX, &a.tmY[s], c0 + 64 * h, row0, full);
-                    for (int g = 0; g < (R >> 3); ++g)
-                        tma_2d(slot + TC_XY + g * 2048u, &a.tmB[s], 8 * g, id * d_out + c0, full);
+                const uint32_t slot = ring + (uint32_t)st * slot_bytes, full = b_full + 8 * st;
+                const int ny = d_out - c0 > 64 ? 2 : 1;
+                if (lane == 0)
+                    mbar_expect_tx(full, (uint32_t)(ny * nrg) * lbox + (uint32_t)(R >> 3) * 2048u);
+                __syncwarp();
+                for (int i = lane; i < nrg * ny; i += 32) {   // y: row group major
+                    const int rg = i / ny, h = i - rg * ny;
+                    tma_2d(slot + h * TC_BOX + rg * lbox, &a.tmY[s], c0 + 64 * h, row0 + lbr * rg, full);
                 }
+                for (int g = lane; g < (R >> 3); g += 32)    // B: 8 ranks x 128 output columns
+                    tma_2d(slot + TC_XY + g * 2048u, &a.tmB[s], 8 * g, id * d_out + c0, full);
                 __syncwarp();
                 ++fills;
                 if (++st == STG) {
@@ -395,7 +414,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
                                 tc_mma(tmem + TC_D1_COL, desc_sw128(slot + b * TC_BOX + kk * 32),
                                        desc_sw128(slot + TC_XY + (uint32_t)(b * SR) * 128u + kk * 32),
                                        id1, (kc > k_lo || b > 0 || kk > 0) ? 1u : 0u);
-                        tc_commit(b_empty + 8 * st);   // two arrivals: the slot's count
                         tc_commit(b_empty + 8 * st);
                     }
                     __syncwarp();
@@ -462,15 +480,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
         __syncwarp();
         bool f2 = false;
         warp_wait(b_mma, 0, a.status, f2);
-    } else {
+    } else if (warp < 10) {
         // ============================================================ epilogue
         const int q = warp & 3, h = (warp - 2) >> 2, m = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-        const bool storer = lane == 0 && (warp == 2 || warp == 6);
         const int half = SR >> 1, n8 = half >> 3;   // D1 columns of this thread's half
         int st = 0;
         uint32_t ph = 0, it = 0, ech = 0;
-        uint32_t yph = 0;   // bit st: phase parity of slot st's y-store barriers (expand uses only)
         for (int t = cl; t < n_tiles && !failed; t += ncl) {
             const int4 tile = a.contig[t];
             const int id = tile.x, row0 = tile.y, cnt = tile.z;
@@ -616,24 +632,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
                                 else if (m < cnt) *reinterpret_cast<uint4 *>(yrow + 8 * c) = o;
                             }
                     }
-                    if (fulltile) fence_proxy_async();
+                    if (fulltile) fence_proxy_async();   // generic writes -> the TMA store
                     __syncwarp();
-                    // The slot's own barrier: its next use needs this storer's release
-                    // first, so arrivals of two uses of the slot never mix.
-                    const uint32_t ystage = b_ystage + 8u * (uint32_t)(h * STG + st);
-                    if (lane == 0) mbar_arrive(ystage);
-                    if (storer) {
-                        // the 4 warps of this half have written their rows of the box
-                        bool ok = mbar_wait(ystage, (yph >> st) & 1u, a.status, failed);
-                        if (ok && fulltile && cb < d_out) {
-                            tma_store_2d(&a.tmY[s], cb, row0, ybox);
-                            bulk_wait_read();
-                        }
-                        mbar_arrive(b_empty + 8 * st);
-                    }
-                    __syncwarp();
-                    if (__any_sync(FULL, failed)) failed = true;
-                    yph ^= 1u << st;
+                    if (lane == 0) mbar_arrive(b_ystage + 8 * st);   // this warp's rows are done
                     ++ech;
                     if (++st == STG) {
                         st = 0;
@@ -649,7 +650,75 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
             }
             ++it;
         }
-        if (storer) bulk_wait_all();
+    } else if (warp == 10) {
+        // ============================================================ store warp
+        // Full tiles: TMA stores of the finished boxes (8-row boxes, one per lane),
+        // the slot freed once they have read it (one chunk later, so that a store
+        // stays in flight meanwhile).  Partial tiles: the epilogue stored the rows
+        // itself; the slot is freed at once.
+        int st = 0;
+        uint32_t ph = 0;
+        uint32_t yph = 0;   // bit st: phase parity of slot st's y barrier (expand uses only)
+        int pend = -1;      // slot whose stores may still be reading it
+        for (int t = cl; t < n_tiles && !failed; t += ncl) {
+            const int4 tile = a.contig[t];
+            const int id = tile.x, row0 = tile.y, cnt = tile.z;
+            const int r_n = a.ranks[id];
+            if (r_n < 1 || r_n > R) continue;
+            if (MODE == MODE_SHRINK) continue;
+            for (int kc = k_lo; kc < k_hi; ++kc)
+                if (++st == STG) {
+                    st = 0;
+                    ph ^= 1u;
+                }
+            const bool fulltile = cnt == TC_M;
+            int s = es0, c0 = ec0;
+            for (int e = e_lo; e < e_hi; ++e) {
+                if (!warp_wait(b_ystage + 8 * st, (yph >> st) & 1u, a.status, failed)) break;
+                const int d_out = a.sl.d_out[s];
+                const int ny = d_out - c0 > 64 ? 2 : 1;
+                const uint32_t slot = ring + (uint32_t)st * slot_bytes;
+                if (fulltile) {
+                    const int sbr = a.sbr, nsg = TC_M / sbr;
+                    for (int i = lane; i < nsg * ny; i += 32) {
+                        const int rg = i / ny, h = i - rg * ny;
+                        tma_store_2d(&a.tmYs[s], c0 + 64 * h, row0 + sbr * rg,
+                                     slot + h * TC_BOX + rg * (uint32_t)sbr * 128u);
+                    }
+                    bulk_commit();
+                }
+                if (pend >= 0) {
+                    if (fulltile) bulk_wait_read_but1();
+                    else bulk_wait_read();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_empty + 8 * pend);
+                    pend = -1;
+                }
+                if (fulltile) {
+                    pend = st;
+                } else {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_empty + 8 * st);
+                }
+                yph ^= 1u << st;
+                if (++st == STG) {
+                    st = 0;
+                    ph ^= 1u;
+                }
+                c0 += 128;
+                if (c0 >= d_out) {
+                    ++s;
+                    c0 = 0;
+                }
+            }
+            if (pend >= 0) {   // no slot stays held into the next tile
+                bulk_wait_read();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_empty + 8 * pend);
+                pend = -1;
+            }
+        }
+        bulk_wait_all();
     }
 
     // ---------------------------------------------------------------- teardown
