@@ -20,6 +20,8 @@ constexpr int SEG_THREADS = 1024;
 constexpr int SEG_CHUNK = 2048;
 constexpr int SEG_SMALL_T = 2048;
 constexpr int SEG_HIST_THREADS = 512;
+// ints of scan scratch in front of a kernel's other shared arrays (33 long longs)
+constexpr int SEG_SCAN_WORDS = 80;
 
 __device__ __forceinline__ int bin_of(int id, int N) { return (id >= 0 && id < N) ? id : N; }
 
@@ -52,6 +54,35 @@ __device__ int block_excl_sum(int v, int *total, int *sm) {
     return res;
 }
 
+// block_excl_sum for 64-bit values.  sm: 33 long longs.
+__device__ long long block_excl_sum64(long long v, long long *total, long long *sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        long long t = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) sm[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        long long w = sm[lane];
+        long long wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            long long t = __shfl_up_sync(FULL, wi, o);
+            if (lane >= o) wi += t;
+        }
+        sm[lane] = wi - w;
+        if (lane == 31) sm[32] = wi;
+    }
+    __syncthreads();
+    long long res = sm[warp] + incl - v;
+    *total = sm[32];
+    __syncthreads();
+    return res;
+}
+
 // Turn per-id counts hist[0..N] (bin N = rows without a valid id) into start
 // offsets; write seg_start, seg_adapter and counts[0].  Whole block.
 __device__ void seg_scan_block(int *hist, int N, int32_t *seg_start, int32_t *seg_adapter,
@@ -64,9 +95,11 @@ __device__ void seg_scan_block(int *hist, int N, int32_t *seg_start, int32_t *se
         s += hist[b];
         nz += hist[b] > 0;
     }
-    int P, nseg;
-    int pre = block_excl_sum(s, &P, sm33);
-    int zpre = block_excl_sum(nz, &nseg, sm33);
+    // one block scan for both prefix sums: rows (high word) and non-empty ids (low word)
+    long long tot2;
+    const long long pre2 = block_excl_sum64(((long long)s << 32) | nz, &tot2, reinterpret_cast<long long *>(sm33));
+    const int P = (int)(tot2 >> 32), nseg = (int)(tot2 & 0xffffffffll);
+    int pre = (int)(pre2 >> 32), zpre = (int)(pre2 & 0xffffffffll);
     for (int b = lo; b < hi; ++b) {
         int c = hist[b];
         seg_start[b] = pre;
@@ -178,6 +211,16 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
     int *prv = nxt + W;                                // last run start at a position < 32w (-1 if none)
     const uint32_t lt = (1u << lane) - 1u;
 
+    // word ranges per warp, contiguous so that per-warp order is position order
+    const int wpw = (W + NW - 1) / NW;
+    const int wl = min(warp * wpw, W), wh = min(wl + wpw, W);
+    bool overflow = false;
+
+    if (o.min_run <= 0) {   // no contiguous tiles: every valid position is gathered
+        for (int w = tid; w < W; w += SEG_THREADS) lngw[w] = 0u;
+        if (tid == 0) o.counts[2] = 0;
+        __syncthreads();
+    } else {
     // 1. pack run starts
     for (int w = warp; w < W; w += NW) {
         const int p = w * 32 + lane;
@@ -185,10 +228,6 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
         if (lane == 0) brkw[w] = word;
     }
     __syncthreads();
-
-    // word ranges per warp, contiguous so that per-warp order is position order
-    const int wpw = (W + NW - 1) / NW;
-    const int wl = min(warp * wpw, W), wh = min(wl + wpw, W);
 
     // 2. nxt[] (suffix) and prv[] (prefix) over words
     {
@@ -289,8 +328,6 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
     }
     __syncthreads();
 
-    bool overflow = false;
-
     // 4. contiguous tiles: long runs in position order, cut every LT rows
     {
         int cnt = 0;
@@ -332,6 +369,7 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
         if (tid == 0) o.counts[2] = min(n_contig, o.max_contig);
     }
     __syncthreads();
+    }   // min_run > 0
 
     // 5. gathered rows: positions outside long runs, in position order
     int *gpre = prv;   // reused: gathered rows before word w
@@ -452,8 +490,9 @@ __device__ bool count_block(const int32_t *ids, int lo, int hi, int N, int *hw, 
 __global__ void __launch_bounds__(SEG_THREADS) seg_small_kernel(SegArgs a) {
     extern __shared__ int sm[];
     int *sm33 = sm;
-    const int nwr = rank_warps(a.N);
-    int *hist = sm + 64;                                  // N+1
+    // ranking warps: at most one per 32 rows (each per-id loop below walks them)
+    const int nwr = min(rank_warps(a.N), max(1, (a.T + 31) / 32));
+    int *hist = sm + SEG_SCAN_WORDS;                      // N+1
     int *hw = hist + ((a.N + 1 + 3) & ~3);                // nwr * (N+1)
     int *ids_s = hw + ((nwr * (a.N + 1) + 3) & ~3);       // T
     int *perm_s = ids_s + a.T;                            // T
@@ -497,7 +536,7 @@ __global__ void __launch_bounds__(SEG_HIST_THREADS) seg_hist_kernel(SegArgs a) {
 __global__ void __launch_bounds__(SEG_THREADS) seg_scan_kernel(SegArgs a, int n_chunks) {
     extern __shared__ int sm[];
     int *sm33 = sm;
-    int *tot = sm + 64;
+    int *tot = sm + SEG_SCAN_WORDS;
     const int stride = a.N + 1;
     for (int b = threadIdx.x; b <= a.N; b += SEG_THREADS) {
         int run = 0;
@@ -567,7 +606,7 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
 
     if (a.T <= SEG_SMALL_T) {
         const size_t nwr = rank_warps(a.N);
-        const size_t smem = (64 + (((size_t)a.N + 1 + 3) & ~(size_t)3) +
+        const size_t smem = (SEG_SCAN_WORDS + (((size_t)a.N + 1 + 3) & ~(size_t)3) +
                              ((nwr * (a.N + 1) + 3) & ~(size_t)3) + 2 * (size_t)a.T +
                              tiles_smem_words(a.T)) * sizeof(int) + (size_t)a.T;
         if (smem > 48 * 1024)
@@ -580,7 +619,7 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
         const int n_chunks = (a.T + SEG_CHUNK - 1) / SEG_CHUNK;
         const size_t bins = (size_t)a.N + 1;
         seg_hist_kernel<<<n_chunks, SEG_HIST_THREADS, bins * sizeof(int), st>>>(a);
-        const size_t scan_smem = (64 + bins) * sizeof(int);
+        const size_t scan_smem = (SEG_SCAN_WORDS + bins) * sizeof(int);
         seg_scan_kernel<<<1, SEG_THREADS, scan_smem, st>>>(a, n_chunks);
         const size_t scat_smem =
             ((((size_t)a.N + 1 + 3) & ~(size_t)3) + (size_t)rank_warps(a.N) * bins) * sizeof(int);

@@ -650,7 +650,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
             }
             ++it;
         }
-    } else if (warp == 10) {
+    } else if (MODE != MODE_SHRINK && warp == 10) {
         // ============================================================ store warp
         // Full tiles: TMA stores of the finished boxes (8-row boxes, one per lane),
         // the slot freed once they have read it (one chunk later, so that a store
@@ -665,7 +665,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
             const int id = tile.x, row0 = tile.y, cnt = tile.z;
             const int r_n = a.ranks[id];
             if (r_n < 1 || r_n > R) continue;
-            if (MODE == MODE_SHRINK) continue;
             for (int kc = k_lo; kc < k_hi; ++kc)
                 if (++st == STG) {
                     st = 0;
