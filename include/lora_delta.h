@@ -149,9 +149,11 @@ LORA_API const char *lora_last_error(void);
 LORA_API int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int32_t min_run,
                        int32_t long_tile, int32_t *max_gather, int32_t *max_contig);
 
-/* Device scratch bytes lora_build_segments needs for T rows over N slots:
- * per-chunk id counts plus one byte per row (0 when T <= 2048: the grouping
- * then runs in one thread block, in shared memory). */
+/* Device scratch bytes lora_build_segments needs for T rows over N slots,
+ * each part rounded up to 256 bytes: per-chunk id counts (4 * (N+1) per 2048
+ * rows), one byte per row, 12 bytes per 32 rows (run bitmaps and offsets) and
+ * 16 bytes per 2048 rows (per-block totals).  0 when T <= 2048: the grouping
+ * then runs in one thread block, in shared memory. */
 LORA_API size_t lora_segments_scratch_bytes(int32_t T, int32_t N);
 
 /*

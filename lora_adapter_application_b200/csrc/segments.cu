@@ -6,9 +6,16 @@
 // A stable counting sort.  Up to SEG_SMALL_T rows one thread block does it
 // all in a single launch (decode batches).  Above that:
 //   seg_hist     one block per chunk of SEG_CHUNK rows: per-chunk id histogram
-//   seg_scan     one block: totals -> seg_start, seg_adapter, per-chunk bases
+//   seg_scan     one block, a warp per id: chunk offsets by warp scans; totals
+//                -> seg_start, seg_adapter
 //   seg_scatter  one block per chunk: every warp ranks its share of the rows
-//   seg_tiles    one block: runs, contiguous tiles, gathered rows and tiles
+//   seg_runs     one block per TW_WORDS x 32 positions: run starts as bits,
+//                the block's first and last run start
+//   seg_long     per block: runs through its positions (neighbours from the
+//                other blocks' first / last starts), long-run bits, counts of
+//                contiguous tiles and gathered rows
+//   seg_emit     per block: contiguous tiles, gathered rows, per-word offsets
+//   seg_gtiles   one block: each id's gathered rows cut into tiles
 // No block ever waits for another block: the phases are separate launches.
 #include "kernels.cuh"
 
@@ -434,8 +441,17 @@ struct SegArgs {
     int32_t *perm, *seg_start, *seg_adapter;
     int *ws;          // [n_chunks][N+1] (multi-block path)
     uint8_t *brkb;    // [T]            (multi-block path)
+    // multi-block tile passes: per word of 32 positions, and per block of TW_WORDS words
+    uint32_t *brkw;   // [W] run-start bits
+    uint32_t *lngw;   // [W] long-run bits
+    int *gpre;        // [W] gathered rows before word w
+    int4 *blk;        // [B] {first run start, last run start, contiguous tiles, gathered rows}
+    int W, B;
     TileOut out;
 };
+
+constexpr int TW_WORDS = 64;      // words per block of the multi-block tile passes
+constexpr int TW_THREADS = 256;   // 8 warps x 8 words
 
 // Warps that rank rows in parallel: each keeps a private count per id, so the
 // counts must fit the shared-memory budget.
@@ -537,23 +553,26 @@ __global__ void __launch_bounds__(SEG_THREADS) seg_scan_kernel(SegArgs a, int n_
     extern __shared__ int sm[];
     int *sm33 = sm;
     int *tot = sm + SEG_SCAN_WORDS;
-    const int stride = a.N + 1;
-    for (int b = threadIdx.x; b <= a.N; b += SEG_THREADS) {
-        int run = 0;
-        for (int c = 0; c < n_chunks; ++c) {
-            const int t = a.ws[(size_t)c * stride + b];
-            a.ws[(size_t)c * stride + b] = run;
-            run += t;
+    const int stride = a.N + 1, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // per id: exclusive offsets of the chunks (chunk order), 32 chunks per warp step
+    for (int b = warp; b <= a.N; b += SEG_THREADS / 32) {
+        int carry = 0;
+        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < n_chunks ? a.ws[(size_t)c * stride + b] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(FULL, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (c < n_chunks) a.ws[(size_t)c * stride + b] = carry + incl - v;
+            carry += __shfl_sync(FULL, incl, 31);
         }
-        tot[b] = run;
+        if (lane == 0) tot[b] = carry;
     }
     __syncthreads();
     seg_scan_block(tot, a.N, a.seg_start, a.seg_adapter, a.out.counts, sm33);
-    __syncthreads();
-    for (int b = threadIdx.x; b <= a.N; b += SEG_THREADS) {
-        const int base = tot[b];
-        for (int c = 0; c < n_chunks; ++c) a.ws[(size_t)c * stride + b] += base;
-    }
 }
 
 __global__ void __launch_bounds__(SEG_THREADS) seg_scatter_kernel(SegArgs a) {
@@ -562,14 +581,257 @@ __global__ void __launch_bounds__(SEG_THREADS) seg_scatter_kernel(SegArgs a) {
     int *base = sm;                                   // N+1
     int *hw = sm + ((a.N + 1 + 3) & ~3);              // nwr * (N+1)
     const int c = blockIdx.x, lo = c * SEG_CHUNK, hi = min(lo + SEG_CHUNK, a.T);
-    for (int b = threadIdx.x; b <= a.N; b += SEG_THREADS) base[b] = a.ws[(size_t)c * (a.N + 1) + b];
+    for (int b = threadIdx.x; b <= a.N; b += SEG_THREADS)   // id start + rows of earlier chunks
+        base[b] = a.seg_start[b] + a.ws[(size_t)c * (a.N + 1) + b];
     count_block(a.ids, lo, hi, a.N, hw, nwr);
     scatter_block(a.ids, lo, hi, a.N, base, hw, nwr, a.perm, a.brkb);
 }
 
-__global__ void __launch_bounds__(SEG_THREADS) seg_tiles_kernel(SegArgs a) {
-    extern __shared__ int sm[];
-    dev_tiles(a.ids, a.perm, a.brkb, a.seg_start, a.N, a.out, sm);
+// ---------------------------------------------------------------- multi-block tile passes
+// Block b covers words [b*TW_WORDS, (b+1)*TW_WORDS) of the P valid positions;
+// warp w of a block takes TW_WORDS/8 consecutive words, one word (32
+// positions, one per lane) at a time, so per-warp order is position order.
+
+// Sum / min / max of one int per thread over a TW_THREADS block.  sm: 8 ints.
+template <class Op>
+__device__ int tw_reduce(int v, int *sm, Op op) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(FULL, v, o));
+    __syncthreads();
+    if (lane == 0) sm[warp] = v;
+    __syncthreads();
+    v = sm[0];
+    for (int w = 1; w < TW_THREADS / 32; ++w) v = op(v, sm[w]);
+    return v;
+}
+
+__global__ void __launch_bounds__(TW_THREADS) seg_runs_kernel(SegArgs a) {
+    __shared__ int red[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = a.seg_start[a.N];
+    int first = INT_MAX, last = -1;
+    for (int i = 0; i < TW_WORDS / 8; ++i) {
+        const int w = blockIdx.x * TW_WORDS + warp * (TW_WORDS / 8) + i;
+        if (w >= a.W) break;
+        const int p = w * 32 + lane;
+        const uint32_t word = __ballot_sync(FULL, p < P && a.brkb[p]);
+        if (lane == 0) a.brkw[w] = word;
+        if (word) {
+            first = min(first, w * 32 + __ffs(word) - 1);
+            last = max(last, w * 32 + 31 - __clz(word));
+        }
+    }
+    first = tw_reduce(first, red, [](int x, int y) { return min(x, y); });
+    last = tw_reduce(last, red, [](int x, int y) { return max(x, y); });
+    if (threadIdx.x == 0) a.blk[blockIdx.x] = make_int4(first, last, 0, 0);
+}
+
+// Run bits of this block's words plus the neighbouring runs outside the block.
+struct RunWords {
+    uint32_t bw[TW_WORDS];
+    int nx[TW_WORDS + 1];    // first run start at a position >= 32 (w0 + i)
+    int pv[TW_WORDS];        // last run start at a position < 32 (w0 + i)
+};
+
+// Fills rw for block blockIdx.x (whole block).  red: 8 ints.
+__device__ void load_run_words(const SegArgs &a, int P, RunWords &rw, int *red) {
+    const int tid = threadIdx.x, w0 = blockIdx.x * TW_WORDS;
+    // first start after this block and last start before it, from the block table
+    int after = INT_MAX, before = -1;
+    for (int b = tid; b < a.B; b += TW_THREADS) {
+        const int4 e = a.blk[b];
+        if (b > (int)blockIdx.x) after = min(after, e.x);
+        if (b < (int)blockIdx.x) before = max(before, e.y);
+    }
+    after = tw_reduce(after, red, [](int x, int y) { return min(x, y); });
+    before = tw_reduce(before, red, [](int x, int y) { return max(x, y); });
+    for (int i = tid; i < TW_WORDS; i += TW_THREADS) rw.bw[i] = (w0 + i < a.W) ? a.brkw[w0 + i] : 0u;
+    __syncthreads();
+    if (tid == 0) {   // suffix minimum of first starts, prefix maximum of last starts (64 steps)
+        int nx = min(after, P);
+        rw.nx[TW_WORDS] = nx;
+        for (int i = TW_WORDS - 1; i >= 0; --i) {
+            if (rw.bw[i]) nx = (w0 + i) * 32 + __ffs(rw.bw[i]) - 1;
+            rw.nx[i] = nx;
+        }
+        int pv = before;
+        for (int i = 0; i < TW_WORDS; ++i) {
+            rw.pv[i] = pv;
+            if (rw.bw[i]) pv = (w0 + i) * 32 + 31 - __clz(rw.bw[i]);
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ int rw_run_end(const RunWords &rw, int w0, int p) {   // first start after p
+    const int i = (p >> 5) - w0, b = p & 31;
+    const uint32_t rest = b == 31 ? 0u : (rw.bw[i] & (0xffffffffu << (b + 1)));
+    return rest ? (p & ~31) + __ffs(rest) - 1 : rw.nx[i + 1];
+}
+__device__ __forceinline__ int rw_run_start(const RunWords &rw, int w0, int p) {   // last start <= p
+    const int i = (p >> 5) - w0, b = p & 31;
+    const uint32_t upto = rw.bw[i] & (b == 31 ? 0xffffffffu : ((2u << b) - 1u));
+    return upto ? (p & ~31) + 31 - __clz(upto) : rw.pv[i];
+}
+
+__global__ void __launch_bounds__(TW_THREADS) seg_long_kernel(SegArgs a) {
+    __shared__ RunWords rw;
+    __shared__ int red[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = a.seg_start[a.N], w0 = blockIdx.x * TW_WORDS;
+    load_run_words(a, P, rw, red);
+    int tiles = 0, shorts = 0;
+    for (int i = 0; i < TW_WORDS / 8; ++i) {
+        const int li = warp * (TW_WORDS / 8) + i, w = w0 + li;
+        if (w >= a.W) break;
+        const int p = w * 32 + lane;
+        bool lg = false;
+        int k = 0;
+        if (p < P) {
+            const int e = rw_run_end(rw, w0, p);
+            lg = a.out.min_run > 0 && e - rw_run_start(rw, w0, p) >= a.out.min_run;
+            if (lg && ((rw.bw[li] >> lane) & 1u)) k = (e - p + a.out.LT - 1) / a.out.LT;
+        }
+        const uint32_t word = __ballot_sync(FULL, lg);
+        if (lane == 0) a.lngw[w] = word;
+        tiles += k;
+        shorts += (p < P && !lg) ? 1 : 0;
+    }
+    tiles = tw_reduce(tiles, red, [](int x, int y) { return x + y; });
+    shorts = tw_reduce(shorts, red, [](int x, int y) { return x + y; });
+    if (threadIdx.x == 0) {
+        a.blk[blockIdx.x].z = tiles;
+        a.blk[blockIdx.x].w = shorts;
+    }
+}
+
+__global__ void __launch_bounds__(TW_THREADS) seg_emit_kernel(SegArgs a) {
+    __shared__ RunWords rw;
+    __shared__ int red[8];
+    __shared__ int wt[8], wsh[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int P = a.seg_start[a.N], w0 = blockIdx.x * TW_WORDS;
+    const uint32_t lt = (1u << lane) - 1u;
+    // tiles and gathered rows of the blocks before this one
+    int tb = 0, sb = 0;
+    for (int b = tid; b < (int)blockIdx.x; b += TW_THREADS) {
+        const int4 e = a.blk[b];
+        tb += e.z;
+        sb += e.w;
+    }
+    tb = tw_reduce(tb, red, [](int x, int y) { return x + y; });
+    sb = tw_reduce(sb, red, [](int x, int y) { return x + y; });
+    load_run_words(a, P, rw, red);
+    // per-warp totals (its words are consecutive), then the warp's base
+    int wtiles = 0, wshort = 0;
+    for (int i = 0; i < TW_WORDS / 8; ++i) {
+        const int li = warp * (TW_WORDS / 8) + i, w = w0 + li;
+        if (w >= a.W) break;
+        const int p = w * 32 + lane;
+        const uint32_t lw = a.lngw[w];
+        if (p < P && ((rw.bw[li] & lw) >> lane) & 1u)
+            wtiles += (rw_run_end(rw, w0, p) - p + a.out.LT - 1) / a.out.LT;
+        if (p < P && !((lw >> lane) & 1u)) ++wshort;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        wtiles += __shfl_xor_sync(FULL, wtiles, o);
+        wshort += __shfl_xor_sync(FULL, wshort, o);
+    }
+    if (lane == 0) {
+        wt[warp] = wtiles;
+        wsh[warp] = wshort;
+    }
+    __syncthreads();
+    int tbase = tb, sbase = sb;
+    for (int v = 0; v < warp; ++v) {
+        tbase += wt[v];
+        sbase += wsh[v];
+    }
+    bool overflow = false;
+    for (int i = 0; i < TW_WORDS / 8; ++i) {
+        const int li = warp * (TW_WORDS / 8) + i, w = w0 + li;
+        if (w >= a.W) break;
+        const int p = w * 32 + lane;
+        const uint32_t lw = a.lngw[w];
+        const uint32_t valid = P - w * 32 >= 32 ? 0xffffffffu : (P > w * 32 ? ((1u << (P - w * 32)) - 1u) : 0u);
+        // contiguous tiles of the long runs starting in this word
+        int len = 0, k = 0;
+        if (((rw.bw[li] & lw & valid) >> lane) & 1u) {
+            len = rw_run_end(rw, w0, p) - p;
+            k = (len + a.out.LT - 1) / a.out.LT;
+        }
+        int incl = k;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int idx = tbase + incl - k;
+        if (k) {
+            const int row0 = a.perm[p], id = a.ids[row0];
+            for (int off = 0; off < len; off += a.out.LT, ++idx) {
+                if (idx < a.out.max_contig)
+                    a.out.contig[idx] = make_int4(id, row0 + off, min(a.out.LT, len - off), 0);
+                else
+                    overflow = true;
+            }
+        }
+        tbase += __shfl_sync(FULL, incl, 31);
+        // gathered rows
+        const uint32_t sbits = ~lw & valid;
+        if ((sbits >> lane) & 1u) a.out.grow[sbase + __popc(sbits & lt)] = a.perm[p];
+        if (lane == 0) a.gpre[w] = sbase;
+        sbase += __popc(sbits);
+    }
+    if (overflow) atomicOr(a.out.status, LORA_DEV_TILE_OVERFLOW);
+}
+
+__global__ void __launch_bounds__(SEG_THREADS) seg_gtiles_kernel(SegArgs a) {
+    __shared__ int sm33[33];
+    const int tid = threadIdx.x;
+    const int P = a.seg_start[a.N];
+    int n_contig = 0, n_short = 0;
+    for (int b = 0; b < a.B; ++b) {   // the block table is small (T / 2048 entries)
+        const int4 e = a.blk[b];
+        n_contig += e.z;
+        n_short += e.w;
+    }
+    auto short_before = [&](int q) -> int {
+        if (q >= P) return n_short;
+        const int w = q >> 5, bit = q & 31;
+        const int rem = P - w * 32;
+        const uint32_t valid = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+        return a.gpre[w] + __popc(~a.lngw[w] & valid & ((1u << bit) - 1u));
+    };
+    const int spt = (a.N + SEG_THREADS - 1) / SEG_THREADS;
+    const int n_lo = min(tid * spt, a.N), n_hi = min(n_lo + spt, a.N);
+    int my_gt = 0;
+    for (int n = n_lo; n < n_hi; ++n) {
+        const int c = short_before(a.seg_start[n + 1]) - short_before(a.seg_start[n]);
+        my_gt += (c + a.out.R - 1) / a.out.R;
+    }
+    int n_gather;
+    int gbase = block_excl_sum(my_gt, &n_gather, sm33);
+    bool overflow = false;
+    for (int n = n_lo; n < n_hi; ++n) {
+        const int g0 = short_before(a.seg_start[n]);
+        const int c = short_before(a.seg_start[n + 1]) - g0;
+        for (int off = 0; off < c; off += a.out.R, ++gbase) {
+            if (gbase < a.out.max_gather)
+                a.out.gather[gbase] = make_int4(n, g0 + off, min(a.out.R, c - off), 0);
+            else
+                overflow = true;
+        }
+    }
+    if (tid == 0) {
+        a.out.counts[1] = min(n_gather, a.out.max_gather);
+        a.out.counts[2] = min(n_contig, a.out.max_contig);
+        a.out.counts[3] = n_short;
+        if (n_contig > a.out.max_contig) overflow = true;
+    }
+    if (overflow) atomicOr(a.out.status, LORA_DEV_TILE_OVERFLOW);
 }
 
 static size_t ws_bytes(int T, int N) {
@@ -577,9 +839,15 @@ static size_t ws_bytes(int T, int N) {
     return (n_chunks * (size_t)(N + 1) * sizeof(int) + 255) & ~(size_t)255;
 }
 
+static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+static int tw_words(int T) { return (T + 31) / 32; }
+static int tw_blocks(int T) { return (tw_words(T) + TW_WORDS - 1) / TW_WORDS; }
+
+// per-chunk id counts | run-start byte per row | 3 words per 32 rows | 4 ints per block
 size_t segments_scratch_bytes(int T, int N) {
     if (T <= SEG_SMALL_T) return 0;
-    return ws_bytes(T, N) + (size_t)T;
+    return ws_bytes(T, N) + round256((size_t)T) + round256((size_t)12 * tw_words(T)) +
+           round256((size_t)16 * tw_blocks(T));
 }
 
 int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
@@ -592,7 +860,22 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
     a.seg_start = m->seg_start;
     a.seg_adapter = m->seg_adapter;
     a.ws = static_cast<int *>(scratch);
-    a.brkb = scratch ? static_cast<uint8_t *>(scratch) + ws_bytes(m->T, m->N) : nullptr;
+    a.brkb = nullptr;
+    a.brkw = a.lngw = nullptr;
+    a.gpre = nullptr;
+    a.blk = nullptr;
+    a.W = tw_words(m->T);
+    a.B = tw_blocks(m->T);
+    if (scratch) {
+        uint8_t *p = static_cast<uint8_t *>(scratch) + ws_bytes(m->T, m->N);
+        a.brkb = p;
+        p += round256((size_t)m->T);
+        a.brkw = reinterpret_cast<uint32_t *>(p);
+        a.lngw = a.brkw + a.W;
+        a.gpre = reinterpret_cast<int *>(a.lngw + a.W);
+        p += round256((size_t)12 * a.W);
+        a.blk = reinterpret_cast<int4 *>(p);
+    }
     a.out.grow = m->grow;
     a.out.gather = reinterpret_cast<int4 *>(m->gather_tiles);
     a.out.contig = reinterpret_cast<int4 *>(m->contig_tiles);
@@ -627,11 +910,10 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
             cudaFuncSetAttribute(seg_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)scat_smem);
         seg_scatter_kernel<<<n_chunks, SEG_THREADS, scat_smem, st>>>(a);
-        const size_t tile_smem = (size_t)tiles_smem_words(a.T) * sizeof(int);
-        if (tile_smem > 48 * 1024)
-            cudaFuncSetAttribute(seg_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tile_smem);
-        seg_tiles_kernel<<<1, SEG_THREADS, tile_smem, st>>>(a);
+        seg_runs_kernel<<<a.B, TW_THREADS, 0, st>>>(a);
+        seg_long_kernel<<<a.B, TW_THREADS, 0, st>>>(a);
+        seg_emit_kernel<<<a.B, TW_THREADS, 0, st>>>(a);
+        seg_gtiles_kernel<<<1, SEG_THREADS, 0, st>>>(a);
     }
     return cuda_rc(cudaGetLastError());
 }

@@ -56,8 +56,16 @@ def test_capacity_bounds(lib):
 
 def test_scratch_and_workspace_sizes(lib):
     assert lora.lora_segments_scratch_bytes(2048, 100) == 0
-    # per-chunk id counts (rounded to 256 bytes) plus one run-start byte per row
-    assert lora.lora_segments_scratch_bytes(2049, 100) == 1024 + 2049
+
+    def r256(b):
+        return (b + 255) // 256 * 256
+
+    # as the header states: per-chunk id counts, one byte per row, 12 bytes per
+    # 32 rows and 16 bytes per 2048 rows, each part rounded up to 256 bytes
+    for T, N in [(2049, 100), (77431, 8), (131072, 4096)]:
+        chunks, words, blocks = -(-T // 2048), -(-T // 32), -(-T // 2048)
+        want = r256(4 * (N + 1) * chunks) + r256(T) + r256(12 * words) + r256(16 * blocks)
+        assert lora.lora_segments_scratch_bytes(T, N) == want, (T, N)
     assert lora.lora_shrink_workspace_bytes(1024, 64, 3) == 3 * 1024 * 64 * 4
 
 

@@ -83,3 +83,18 @@ def test_deterministic(cuda_lib):
     ha, hb = a.host(), b.host()
     for k in ha:
         np.testing.assert_array_equal(np.asarray(ha[k]), np.asarray(hb[k]))
+
+
+@pytest.mark.parametrize("T,N,min_run,seed", [
+    (5000, 3, 64, 1), (20000, 7, 1000, 2), (50000, 40, 64, 3), (131072, 4096, 128, 4),
+    (131072, 9, 1, 5), (70000, 2, 2048, 6)])
+def test_long_runs_across_blocks(cuda_lib, T, N, min_run, seed):
+    """Runs of up to 6000 rows: many straddle or span the 2048-position blocks
+    of the multi-block tile passes; ids -1 and short runs in between."""
+    rng = np.random.default_rng(500 + seed)
+    parts = []
+    while sum(len(p) for p in parts) < T:
+        L = int(rng.choice([1, 3, 40, 129, 700, 2047, 2049, 6000]))
+        parts.append(np.full(L, int(rng.integers(-1, N)), dtype=np.int32))
+    ids = np.concatenate(parts)[:T]
+    _compare(ids, N, int(rng.choice([1, 16])), min_run, 0)
