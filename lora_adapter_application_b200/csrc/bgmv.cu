@@ -9,9 +9,9 @@
 //
 //   producer warp   walks the block's chunk stream and fills a 3-stage
 //                   shared-memory ring through the TMA engine: 2-D tensor
-//                   copies of 1 KB boxes for the adapters (A: 8 ranks x 64
-//                   columns, 128-byte swizzle; B: 64 output columns x 8 ranks)
-//                   and one 1-D bulk copy per gathered x or y row.  (Measured
+//                   copies of 1-2 KB boxes for the adapters (A: 8 or 16 ranks
+//                   x 64 columns, 128-byte swizzle; B: 64 output columns x 8
+//                   or 16 ranks) and one 1-D bulk copy per gathered x or y row.  (Measured
 //                   on B200: TMA copies leave the load/store pipe to the
 //                   consumers, where a cp.async producer competes with their
 //                   shared-memory traffic; TMA pays per copy, so copies should
@@ -243,27 +243,31 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
                 const int width = min(G.JC, G.j_hi - jc0), nbox = (width + 63) >> 6;
                 const int ncb = G.JC >> 6;
                 const unsigned xbytes = (unsigned)width * 2;
-                if (lane == 0) mbar_expect_tx(full, xbytes * cnt + (unsigned)(G.nb8 * nbox) * 1024u);
+                const int nkg = a.ab16 ? (G.nb8 + 1) >> 1 : G.nb8;   // rank boxes
+                const unsigned abox = a.ab16 ? 2048u : 1024u;
+                if (lane == 0) mbar_expect_tx(full, xbytes * cnt + (unsigned)(nkg * nbox) * abox);
                 __syncwarp();
                 for (int r = lane; r < cnt; r += 32)   // gathered x rows
                     bulk_g2s(dst + r * G.RS, a.x + (int64_t)rows_sm[r] * a.ld_x + jc0, xbytes, full);
-                for (int e = lane; e < G.nb8 * nbox; e += 32) {   // A: 8 ranks x 64 columns per box
+                for (int e = lane; e < nkg * nbox; e += 32) {   // A: 8 or 16 ranks x 64 columns per box
                     const int kg = e / nbox, cb = e - kg * nbox;
-                    tma_2d(dst + G.A0 + (kg * ncb + cb) * 1024, &a.tmA[it.s], jc0 + 64 * cb,
-                           n * a.r_max + 8 * kg, full);
+                    tma_2d(dst + G.A0 + (kg * ncb + cb) * abox, &a.tmA[it.s], jc0 + 64 * cb,
+                           n * a.r_max + (a.ab16 ? 16 : 8) * kg, full);
                 }
             } else {
                 const int s = it.es, d_out = a.sl.d_out[s];
                 const int nbox = (it.w + 63) >> 6, nbx = G.CC >> 6;
                 const unsigned ybytes = (unsigned)it.w * 2;
-                if (lane == 0) mbar_expect_tx(full, ybytes * cnt + (unsigned)(G.nb8 * nbox) * 1024u);
+                const int nkg = a.ab16 ? (G.nb8 + 1) >> 1 : G.nb8;
+                const unsigned bbox = a.ab16 ? 2048u : 1024u;
+                if (lane == 0) mbar_expect_tx(full, ybytes * cnt + (unsigned)(nkg * nbox) * bbox);
                 __syncwarp();
                 for (int r = lane; r < cnt; r += 32)   // gathered y rows
                     bulk_g2s(dst + r * G.YS,
                              a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0, ybytes, full);
-                for (int e = lane; e < G.nb8 * nbox; e += 32) {   // B: 64 columns x 8 ranks per box
+                for (int e = lane; e < nkg * nbox; e += 32) {   // B: 64 columns x 8 or 16 ranks per box
                     const int kg = e / nbox, cb = e - kg * nbox;
-                    tma_2d(dst + G.B0 + (kg * nbx + cb) * 1024, &a.tmB[s], 8 * kg,
+                    tma_2d(dst + G.B0 + (kg * nbx + cb) * bbox, &a.tmB[s], (a.ab16 ? 16 : 8) * kg,
                            n * d_out + it.c0 + 64 * cb, full);
                 }
             }
@@ -298,8 +302,11 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
             const int width = min(G.JC, G.j_hi - jc0);
             const int nsteps = (width + 63) >> 6;
             const uint32_t xg = st + g * G.RS, xh = st + (g + 8) * G.RS;
-            // A box (8 ranks x 64 columns, 128-byte swizzle): row g, 16-byte chunks 2t and 2t+1
-            const uint32_t ak = st + G.A0 + nbw * (G.JC >> 6) * 1024 + g * 128;
+            // A box (8 or 16 ranks x 64 columns, 128-byte swizzle): rank 8 nbw + g, 16-byte
+            // chunks 2t and 2t+1 (the swizzle follows address bits 7-9, the same in either box)
+            const uint32_t ak = a.ab16 ? st + G.A0 + (nbw >> 1) * (G.JC >> 6) * 2048 + (nbw & 1) * 1024 + g * 128
+                                       : st + G.A0 + nbw * (G.JC >> 6) * 1024 + g * 128;
+            const uint32_t astep = a.ab16 ? 2048u : 1024u;
             const uint32_t c0 = (uint32_t)(((2 * t) ^ g) << 4), c1 = (uint32_t)(((2 * t + 1) ^ g) << 4);
             for (int sp = jgi; sp < nsteps; sp += jg) {
                 const int col = sp * 64 + t * 16;
@@ -307,7 +314,7 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
                 const uint32_t off = (uint32_t)(col * 2);
                 const uint4 xa0 = zero_if(z0, lds128(xg + off)), xa1 = zero_if(z1, lds128(xg + off + 16));
                 const uint4 xb0 = zero_if(z0, lds128(xh + off)), xb1 = zero_if(z1, lds128(xh + off + 16));
-                const uint32_t box = ak + sp * 1024;
+                const uint32_t box = ak + sp * astep;
                 const uint4 a0 = zero_if(z0, lds128(box + c0)), a1 = zero_if(z1, lds128(box + c1));
                 {
                     const uint32_t f[4] = {xa0.x, xb0.x, xa0.y, xb0.y};
@@ -430,9 +437,11 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
                     for (int j = 0; j < 2; ++j) {
                         bv[j] = make_uint2(0, 0);
                         if (k < r_n && nb0 + j < nblk) {
-                            const int col = (nb0 + j) * 8 + g;   // B box: 64 columns x 8 ranks, 16 B per column
-                            bv[j] = lds64(bbase + ((k >> 3) * nbx + (col >> 6)) * 1024 + (col & 63) * 16 +
-                                          (k & 7) * 2);
+                            const int col = (nb0 + j) * 8 + g;   // B box: 64 columns x 8 (16) ranks
+                            bv[j] = a.ab16 ? lds64(bbase + ((k >> 4) * nbx + (col >> 6)) * 2048 +
+                                                   (col & 63) * 32 + (k & 15) * 2)
+                                           : lds64(bbase + ((k >> 3) * nbx + (col >> 6)) * 1024 +
+                                                   (col & 63) * 16 + (k & 7) * 2);
                             if (k + 4 > r_n) {   // the rank ends inside this group of 4
                                 const int keep = r_n - k;
                                 if (keep < 2) bv[j].x &= 0xffffu;

@@ -9,11 +9,12 @@ namespace lora {
 
 enum { MODE_FUSED = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 
-// Tensor maps of the fused kernel (bf16 2-D views of the stacked adapters):
-//   A_s as [N*r_max rows][d_in], boxes of 8 rows x 64 columns, 128-byte swizzle
-//   B_s as [N*d_out rows][r_max], boxes of 64 rows x 8 ranks
-constexpr int BG_ABOX_COLS = 64, BG_ABOX_ROWS = 8;
-constexpr int BG_BBOX_RANKS = 8, BG_BBOX_ROWS = 64;
+// Tensor maps of the fused kernel (bf16 2-D views of the stacked adapters),
+// K = 16 ranks per box when r_max % 16 == 0, else 8:
+//   A_s as [N*r_max rows][d_in], boxes of K rows x 64 columns, 128-byte swizzle
+//   B_s as [N*d_out rows][r_max], boxes of 64 rows x K ranks
+constexpr int BG_ABOX_COLS = 64;
+constexpr int BG_BBOX_ROWS = 64;
 // row_stride: elements between consecutive rows (0 = inner, densely packed)
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
                   uint32_t box_inner, uint32_t box_outer, bool swizzle128,
@@ -35,6 +36,7 @@ struct BgArgs {
     const float *scales;
     Tiles tiles;
     int32_t *status;
+    int ab16;          // adapters in 16-rank boxes (r_max % 16 == 0): A 64 x 16, B 16 x 64
 };
 
 struct SimtArgs {

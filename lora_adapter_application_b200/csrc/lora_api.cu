@@ -285,14 +285,16 @@ int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = tr
         BgArgs bg{};
         for (int s = 0; s < c.n_slices && maps_ok; ++s) {
             const int N = c.meta->N;
+            // 16-rank boxes when the slot rank allows: half the TMA operations, and B
+            // comes in 32-byte pieces (full sectors) instead of 16-byte ones
+            const uint32_t kbox = (c.r_max & 15) == 0 ? 16 : 8;
             if (need_x)
                 maps_ok = tensor_map_2d(&bg.tmA[s], c.slices[s].A, (uint64_t)c.d_in,
-                                        (uint64_t)N * c.r_max, BG_ABOX_COLS, BG_ABOX_ROWS,
-                                        true) == LORA_OK;
+                                        (uint64_t)N * c.r_max, BG_ABOX_COLS, kbox, true) == LORA_OK;
             if (need_y && maps_ok)
                 maps_ok = tensor_map_2d(&bg.tmB[s], c.slices[s].B, (uint64_t)c.r_max,
-                                        (uint64_t)N * c.slices[s].d_out, BG_BBOX_RANKS,
-                                        BG_BBOX_ROWS, false) == LORA_OK;
+                                        (uint64_t)N * c.slices[s].d_out, kbox, BG_BBOX_ROWS,
+                                        false) == LORA_OK;
         }
         if (maps_ok) {
             bg.x = static_cast<const __nv_bfloat16 *>(c.x);
@@ -308,6 +310,7 @@ int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = tr
             bg.scales = c.scales;
             bg.tiles = tiles;
             bg.status = c.status;
+            bg.ab16 = (c.r_max & 15) == 0 ? 1 : 0;
             const int cl = bgmv_cluster(tc_took ? 1 : units);
             if (tc_took)
                 return on_side_stream(c.stream, [&](cudaStream_t s) {
