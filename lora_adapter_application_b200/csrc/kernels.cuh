@@ -104,7 +104,9 @@ int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_
 // sgmv_tc.cu: bf16, r_max % 16 == 0, n_slices * r_max <= 128, 16-byte aligned rows;
 // chooses the cluster size and ring depth, launches persistent clusters
 size_t sgmv_tc_smem_bytes(int mode, int stages, int SR, int C);
-int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st);
+// idle_sms (may be NULL): SMs the launch is expected to leave free (clusters
+// beyond the estimated tile count)
+int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st, int *idle_sms = nullptr);
 
 // simt.cu: any element type and alignment, r_max <= LORA_MAX_RANK
 size_t simt_smem_bytes(int n_slices, int r_max);

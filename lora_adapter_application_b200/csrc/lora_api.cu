@@ -36,12 +36,15 @@ namespace {
 // about two blocks per SM): 4 suits decode batches from the q_proj shape to
 // the Llama-3-8B layer set; 8 when the units are few - the gathered rows of a
 // batch whose prompt runs went to the tensor-core kernel (est_units = 1), or
-// a tile list of a handful of units.
-int bgmv_cluster(int est_units) {
+// a tile list of a handful of units; 2 when those gathered rows run beside a
+// tensor-core launch that leaves SMs free (idle_sms): 2-block clusters fit
+// there, 8-block ones wait for it to finish.
+int bgmv_cluster(int est_units, int idle_sms = 0) {
     if (const char *e = std::getenv("LORA_BG_CLUSTER")) {   // tuning override: 1, 2, 4 or 8
         const int c = std::atoi(e);
         if (c == 1 || c == 2 || c == 4 || c == 8) return c;
     }
+    if (idle_sms >= 16) return 2;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -61,9 +64,10 @@ constexpr int kSideDevices = 64;
 std::mutex g_side_mu;
 SideStream g_side[kSideDevices];
 
-// fn(side stream) between a fork from and a join into `caller`
+// fn(side stream) between a fork from and a join into `caller`: work fn puts on
+// `caller` after the fork and work it puts on the side stream may overlap.
 template <class F>
-int on_side_stream(cudaStream_t caller, F &&fn) {
+int with_side_stream(cudaStream_t caller, F &&fn) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_rc(e);
@@ -217,7 +221,7 @@ bool tc_ok(const Call &c, bool need_x, bool need_y) {
 
 // Contiguous tiles on the tensor-core SGMV kernel; false if a tensor map
 // cannot be encoded (the caller then keeps those tiles on the other kernels).
-bool run_tc(int mode, const Call &c, int *rc) {
+bool run_tc(int mode, const Call &c, int *rc, int *idle_sms) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
     const int N = c.meta->N;
     TcArgs a{};
@@ -262,21 +266,15 @@ bool run_tc(int mode, const Call &c, int *rc) {
     a.counts = c.meta->counts;
     a.max_contig = c.meta->max_contig_tiles;
     a.status = c.status;
-    *rc = launch_sgmv_tc(mode, a, c.stream);
+    *rc = launch_sgmv_tc(mode, a, c.stream, idle_sms);
     return *rc != LORA_ERR_SHAPE;
 }
 
-int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = true) {
+// The gathered tiles (and the contiguous ones unless tc_took) on the fused
+// kernel, or the general kernel when the data does not suit it, on `stream`.
+int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took, int idle_sms,
+                cudaStream_t stream) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
-    bool tc_took = false;
-    if (tensor_core && contig && c.meta->T > 0 && tc_ok(c, need_x, need_y)) {
-        int rc = LORA_OK;
-        if (run_tc(mode, c, &rc)) {
-            if (rc != LORA_OK) return rc;
-            contig = false;   // the remaining launch takes the gathered tiles only
-            tc_took = true;
-        }
-    }
     Tiles tiles = make_tiles(c.meta, gather, contig);
     const int units = n_units(tiles);
     if (c.meta->T == 0 || units == 0) return LORA_OK;
@@ -311,12 +309,8 @@ int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = tr
             bg.tiles = tiles;
             bg.status = c.status;
             bg.ab16 = (c.r_max & 15) == 0 ? 1 : 0;
-            const int cl = bgmv_cluster(tc_took ? 1 : units);
-            if (tc_took)
-                return on_side_stream(c.stream, [&](cudaStream_t s) {
-                    return launch_bgmv(mode, bg, units, cl, s);
-                });
-            return launch_bgmv(mode, bg, units, cl, c.stream);
+            const int cl = tc_took ? bgmv_cluster(1, idle_sms) : bgmv_cluster(units);
+            return launch_bgmv(mode, bg, units, cl, stream);
         }
     }
     SimtArgs a{};
@@ -333,7 +327,23 @@ int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = tr
     a.scales = c.scales;
     a.tiles = tiles;
     a.status = c.status;
-    return launch_simt(mode, c.dtype == LORA_BF16, a, units, c.stream);
+    return launch_simt(mode, c.dtype == LORA_BF16, a, units, stream);
+}
+
+int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = true) {
+    const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
+    if (tensor_core && contig && c.meta->T > 0 && tc_ok(c, need_x, need_y)) {
+        // contiguous tiles on the tensor-core kernel (caller's stream), gathered tiles on
+        // the side stream: the fork comes first, so the two launches overlap
+        return with_side_stream(c.stream, [&](cudaStream_t side) -> int {
+            int rc = LORA_OK, idle_sms = 0;
+            if (!run_tc(mode, c, &rc, &idle_sms))   // a tensor map could not be encoded
+                return launch_rest(mode, c, gather, true, false, 0, c.stream);
+            if (rc != LORA_OK) return rc;
+            return launch_rest(mode, c, gather, false, true, idle_sms, side);
+        });
+    }
+    return launch_rest(mode, c, gather, contig, false, 0, c.stream);
 }
 
 }  // namespace

@@ -810,7 +810,8 @@ int active_clusters(int mode, int C, size_t smem) {
 
 }  // namespace
 
-int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st) {
+int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st, int *idle_sms) {
+    if (idle_sms) *idle_sms = 0;
     if (a.max_contig <= 0 || a.T <= 0) return LORA_OK;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -857,6 +858,7 @@ int launch_sgmv_tc(int mode, TcArgs &a, cudaStream_t st) {
     a.stages = best_stages;
     const size_t smem = sgmv_tc_smem_bytes(mode, best_stages, SR, best_c);
     const int clusters = std::min(best_ncl, a.max_contig);
+    if (idle_sms) *idle_sms = std::max(0, clusters - est) * best_c;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(best_c * clusters, 1, 1);
