@@ -150,10 +150,18 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
+// 16 bytes into the shared memory of a block of the cluster (address and
+// mbarrier both mapped with map_rank), completing 16 transaction bytes on that
+// mbarrier: its waiters see the data once the phase completes, with no fence
+// on either side (measured on B200: a cluster-scope fence or acquire costs
+// ~1-2 us under this kernel's load, several per tile with plain stores).
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float a, float b, float c, float d,
+                                            uint32_t bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];\n" ::"r"(
+            addr),
+        "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
+        : "memory");
 }
 __device__ __forceinline__ float4 lds128f(uint32_t a) {
     float4 r;
@@ -169,9 +177,6 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 }
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-__device__ __forceinline__ void fence_cluster() {
-    asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
 }
 // 2-D tensor store (one box) shared -> global, tracked by this thread's bulk groups
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src) {
@@ -228,14 +233,15 @@ __device__ __forceinline__ uint4 keep8(uint4 v, int keep) {
 // Shared memory (from a 1 KB boundary):
 //   ring  stages x [x or y boxes: 32 KB | A or B boxes: SR*256 B]
 //   V     SR*512 B   s v as bf16: [slice][hi, lo][rank / 8][128 rows][8]
-//   XCH   C*SR*512 B partials (C > 1, shrink modes): [source block][SR/4][128 rows][4] fp32
+//   XCH   2*C*SR*512 B partials (C > 1, shrink modes), one buffer per tile parity:
+//         [parity][source block][SR/4][128 rows][4] fp32
 //   mbarriers
 // At least 120 KB, so that one block holds an SM: a block takes all 512
 // tensor-memory columns, and two blocks of different clusters waiting for
 // each other's columns could otherwise stall both clusters.
 size_t sgmv_tc_smem_bytes(int mode, int stages, int SR, int C) {
     const size_t b = 1024 + (size_t)stages * (TC_XY + (size_t)SR * 256) + (size_t)SR * 512 +
-                     ((mode != MODE_EXPAND && C > 1) ? (size_t)C * SR * 512 : 0) + 512;
+                     ((mode != MODE_EXPAND && C > 1) ? (size_t)2 * C * SR * 512 : 0) + 512;
     return b < (size_t)120 * 1024 ? (size_t)120 * 1024 : b;
 }
 
@@ -259,12 +265,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
     const uint32_t slot_bytes = TC_XY + (uint32_t)SR * 256u;
     const uint32_t vbuf = ring + (uint32_t)STG * slot_bytes;
     const uint32_t xch = vbuf + (uint32_t)SR * 512u;
-    const uint32_t bars = xch + (xchg ? (uint32_t)(C * SR) * 512u : 0u);
+    const uint32_t xch_bytes = (uint32_t)(C * SR) * 512u;   // one exchange buffer
+    const uint32_t bars = xch + (xchg ? 2u * xch_bytes : 0u);
     // per slot: full, empty, and "the epilogue has written the slot's y"
     const uint32_t b_full = bars, b_empty = bars + 8u * STG, b_ystage = bars + 16u * STG;
     const uint32_t b_d1full = bars + 24u * STG, b_d1free = b_d1full + 8, b_vfull = b_d1full + 16;
     const uint32_t b_d2full = b_d1full + 24, b_d2empty = b_d1full + 40;   // [2] each
-    const uint32_t b_xfull = b_d1full + 56, b_xfree = b_d1full + 64, b_mma = b_d1full + 72;
+    const uint32_t b_xfull = b_d1full + 56, b_mma = b_d1full + 72;   // b_xfull[2]
 
     if (tid == 0) {
         for (int st = 0; st < STG; ++st) {
@@ -279,8 +286,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
         mbar_init(b_d2full + 8, 1);
         mbar_init(b_d2empty, 8);
         mbar_init(b_d2empty + 8, 8);
-        mbar_init(b_xfull, 8 * C);
-        mbar_init(b_xfree, 8 * C);
+        mbar_init(b_xfull, 1);       // per phase: this block's expect_tx, then the partials' bytes
+        mbar_init(b_xfull + 8, 1);
         mbar_init(b_mma, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
@@ -509,28 +516,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(b_d1free);
                 if (xchg) {
-                    // all-to-all of the partials through distributed shared memory
+                    // All-to-all of the partials through distributed shared memory: st.async
+                    // stores that count their bytes on the receiver's barrier.  A buffer per
+                    // tile parity: a block writes tile i+2 into a peer only after it received
+                    // every peer's tile i+1 partials, which each peer sent after reading tile i.
                     const int NQ = SR >> 2, qh = half >> 2, q0 = h * qh;
-                    if (!warp_wait<true>(b_xfree, (it & 1u) ^ 1u, a.status, failed)) break;
+                    const uint32_t xb = it & 1u, xbuf = xch + xb * xch_bytes, xbar = b_xfull + 8u * xb;
+                    if (warp == 2 && lane == 0) mbar_expect_tx(xbar, xch_bytes);
                     const uint32_t off = (uint32_t)(((int)crank * NQ + q0) * 128 + m) * 16u;
                     for (int k = 0; k < C; ++k) {
-                        const uint32_t rb = map_rank(xch, (uint32_t)k) + off;
+                        const uint32_t rb = map_rank(xbuf, (uint32_t)k) + off;
+                        const uint32_t rbar = map_rank(xbar, (uint32_t)k);
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             if (j < qh)
-                                st_cluster_f4(rb + j * 2048u, p[4 * j], p[4 * j + 1], p[4 * j + 2],
-                                              p[4 * j + 3]);
+                                st_async_f4(rb + j * 2048u, p[4 * j], p[4 * j + 1], p[4 * j + 2],
+                                            p[4 * j + 3], rbar);
                     }
-                    __syncwarp();
-                    if (lane == 0) {
-                        fence_cluster();
-                        for (int k = 0; k < C; ++k) mbar_arrive_remote(b_xfull, (unsigned)k);
-                    }
-                    if (!warp_wait<true>(b_xfull, it & 1u, a.status, failed)) break;
+                    if (!warp_wait(xbar, (it >> 1) & 1u, a.status, failed)) break;
 #pragma unroll
                     for (int j = 0; j < 64; ++j) p[j] = 0.f;
                     for (int src = 0; src < C; ++src) {
-                        const uint32_t lb = xch + (uint32_t)((src * NQ + q0) * 128 + m) * 16u;
+                        const uint32_t lb = xbuf + (uint32_t)((src * NQ + q0) * 128 + m) * 16u;
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             if (j < qh) {
@@ -540,11 +547,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
                                 p[4 * j + 2] += v.z;
                                 p[4 * j + 3] += v.w;
                             }
-                    }
-                    __syncwarp();
-                    if (lane == 0) {
-                        fence_cluster();
-                        for (int k = 0; k < C; ++k) mbar_arrive_remote(b_xfree, (unsigned)k);
                     }
                 }
                 if (MODE == MODE_SHRINK) {
