@@ -24,8 +24,9 @@
 //                    block sends each partial element to the block that owns
 //                    it; the owner adds the C partials in a fixed order
 //                    (run-to-run identical), scales by alpha/r_n and stores the
-//                    result into every block's copy of v; remote mbarrier
-//                    arrivals say when the stores have landed
+//                    result into every block's copy of v; the stores are
+//                    st.async, counted in bytes on the receiver's mbarrier, so
+//                    neither side needs a cluster-scope fence
 //     expand chunks  B rows [CC][r_n] and y rows [cnt][CC] -> y += (s v) B^T in
 //                    fp32, rounded once, written back with 16-byte stores
 //
@@ -225,7 +226,6 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         }
     };
 
-    cg::cluster_group cluster = cg::this_cluster();
 
     if (warp == BG_CONSUMERS) {
         // ============================================================ producer
@@ -282,6 +282,16 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
     float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
     const int ctid = tid;   // 0 .. 255
     const int per_src = (S * BG_ROWS * BG_RMAX) / C;
+    const uint32_t recv_s = smem_u32(recv), vfull_s = smem_u32(vfull);
+    // Exchange rounds: st.async stores that count their bytes on the receiver's
+    // barrier (no fence on either side).  With C dividing 64, every block
+    // receives S * cnt * r8 partials (4 bytes each) in either round: the
+    // elements it owns from every block, then every owner's scaled sums.
+    if (MODE != MODE_EXPAND && ctid == 0) {
+        const unsigned bytes = (unsigned)(S * cnt * G.r8) * 4u;
+        mbar_expect_tx(xready, bytes);
+        if (MODE == MODE_FUSED) mbar_expect_tx(vready, bytes);
+    }
 
     // block partial of slice s (from part, or zeros) -> recv of the owning block
     auto send_partials = [&](int s, bool from_part) {
@@ -291,8 +301,9 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
             if (from_part)
                 for (int j = 0; j < jg; ++j) sum += part[(j * BG_ROWS + row) * G.r8 + k];
             const int e = (s * BG_ROWS + row) * BG_RMAX + k;
-            float *dst = cluster.map_shared_rank(recv, e % C);
-            dst[crank * per_src + e / C] = sum;
+            const uint32_t owner = (uint32_t)(e % C);
+            st_async_f32(map_rank(recv_s + (uint32_t)(crank * per_src + e / C) * 4u, owner), sum,
+                         map_rank(xready, owner));
         }
     };
 
@@ -365,12 +376,7 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         }
         if (G.n_sc == 0)   // no input columns here: the partials are zero
             for (int s = 0; s < S; ++s) send_partials(s, false);
-        consumer_sync();
-        if (ctid == 0) {
-            asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
-            for (int c = 0; c < C; ++c) mbar_arrive_remote(xready, c);
-        }
-        mbar_wait<true>(xready, uiter & 1u, a.status, failed);   // every partial has reached its owner
+        mbar_wait(xready, uiter & 1u, a.status, failed);   // every partial has reached its owner
         const float scale = MODE == MODE_FUSED ? a.scales[n] : 1.f;
         const int mine = (S * BG_ROWS * BG_RMAX - crank + C - 1) / C;   // elements e = crank + C*j
         for (int j = ctid; j < mine; j += BG_CONSUMERS * 32) {
@@ -384,18 +390,12 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
             if (MODE == MODE_SHRINK) {
                 if (k < r_n) a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] = val;
             } else {
-                const int f = (s * BG_ROWS + row) * BG_VF_STRIDE + k;
-                for (int c = 0; c < C; ++c) cluster.map_shared_rank(vfull, c)[f] = val;
+                const uint32_t f = vfull_s + (uint32_t)((s * BG_ROWS + row) * BG_VF_STRIDE + k) * 4u;
+                for (int c = 0; c < C; ++c) st_async_f32(map_rank(f, (uint32_t)c), val, map_rank(vready, (uint32_t)c));
             }
         }
-        if (MODE == MODE_FUSED) {
-            consumer_sync();
-            if (ctid == 0) {
-                asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
-                for (int c = 0; c < C; ++c) mbar_arrive_remote(vready, c);
-            }
-            mbar_wait<true>(vready, uiter & 1u, a.status, failed);   // every block holds the full s*v
-        }
+        if (MODE == MODE_FUSED)
+            mbar_wait(vready, uiter & 1u, a.status, failed);   // every block holds the full s*v
     };
 
     int cur_s = -1;
@@ -535,14 +535,13 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
     sm.vready = sm.xready + 8;
 
     const int tid = threadIdx.x;
-    const int C = gridDim.x;
     if (tid == 0) {
         for (int st = 0; st < BG_STAGES; ++st) {
             mbar_init(sm.full0 + 8 * st, 1);
             mbar_init(sm.empty0 + 8 * st, BG_CONSUMERS);
         }
-        mbar_init(sm.xready, C);
-        mbar_init(sm.vready, C);
+        mbar_init(sm.xready, 1);   // per unit: the expect_tx arrival, then C x the owned partials' bytes
+        mbar_init(sm.vready, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     cg::cluster_group cluster = cg::this_cluster();

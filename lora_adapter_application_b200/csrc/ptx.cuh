@@ -106,4 +106,30 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(a), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// 16 bytes into the shared memory of a block of the cluster (address and
+// mbarrier both mapped with map_rank), completing 16 transaction bytes on that
+// mbarrier: its waiters see the data once the phase completes, with no fence
+// on either side (measured on B200: a cluster-scope fence or acquire costs
+// ~1-2 us under this kernel's load, several per tile with plain stores).
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float a, float b, float c, float d,
+                                            uint32_t bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];\n" ::"r"(
+            addr),
+        "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
+        : "memory");
+}
+// 4 bytes into the shared memory of a block of the cluster, completing 4
+// transaction bytes on that block's mbarrier (see st_async_f4)
+__device__ __forceinline__ void st_async_f32(uint32_t addr, float v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];\n" ::"r"(addr),
+                 "f"(v), "r"(bar)
+                 : "memory");
+}
+
 }  // namespace lora

@@ -145,24 +145,6 @@ __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n"
                  "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
-__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-// 16 bytes into the shared memory of a block of the cluster (address and
-// mbarrier both mapped with map_rank), completing 16 transaction bytes on that
-// mbarrier: its waiters see the data once the phase completes, with no fence
-// on either side (measured on B200: a cluster-scope fence or acquire costs
-// ~1-2 us under this kernel's load, several per tile with plain stores).
-__device__ __forceinline__ void st_async_f4(uint32_t addr, float a, float b, float c, float d,
-                                            uint32_t bar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];\n" ::"r"(
-            addr),
-        "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
-        : "memory");
-}
 __device__ __forceinline__ float4 lds128f(uint32_t a) {
     float4 r;
     asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
