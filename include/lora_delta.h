@@ -238,7 +238,10 @@ LORA_API int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x,
  * y in place.  Gathered tiles (decode rows) take the fused BGMV kernel;
  * contiguous tiles (prompt runs) take the tensor-core SGMV kernel when the
  * data is bf16; everything else takes the general kernel.  Same result as
- * lora_bgmv_fused.
+ * lora_bgmv_fused.  When both kinds of tiles are present the gathered ones run
+ * on a library-owned second stream, forked from and joined back into `stream`
+ * with events (also under stream capture); the first such call on a device
+ * creates that stream and its events, so make it before any capture.
  */
 LORA_API int lora_add_linear(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
                     const lora_slice *slices, int32_t n_slices, int32_t r_max,

@@ -535,6 +535,11 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
     sm.vready = sm.xready + 8;
 
     const int tid = threadIdx.x;
+    if (tid >= BG_CONSUMERS * 32 && tid - BG_CONSUMERS * 32 < S) {   // producer lanes: descriptors
+        const int s = tid - BG_CONSUMERS * 32;
+        if (MODE != MODE_EXPAND) prefetch_tmap(&a.tmA[s]);   // only the maps this mode built
+        if (MODE != MODE_SHRINK) prefetch_tmap(&a.tmB[s]);
+    }
     if (tid == 0) {
         for (int st = 0; st < BG_STAGES; ++st) {
             mbar_init(sm.full0 + 8 * st, 1);

@@ -76,6 +76,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// Pull a tensor map (kernel parameter) into the TMA unit's descriptor cache
+// ahead of its first copy.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 // 2-D tensor copy (one box) global -> shared through the TMA engine.
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                        uint32_t bar) {

@@ -273,6 +273,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmv_tc_kernel(const __grid_con
         mbar_init(b_mma, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
+    if (warp == 0) {   // descriptors of every map this block will copy with
+        if (lane < S) {
+            if (MODE != MODE_EXPAND) prefetch_tmap(&a.tmA[lane]);
+            if (MODE != MODE_SHRINK) {
+                prefetch_tmap(&a.tmB[lane]);
+                prefetch_tmap(&a.tmY[lane]);
+                prefetch_tmap(&a.tmYs[lane]);
+            }
+        }
+        if (lane == 0 && MODE != MODE_EXPAND) prefetch_tmap(&a.tmX);
+    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                          smem_u32(&tmem_sm)),

@@ -151,3 +151,29 @@ def test_tensor_core_kernel_runs(cuda_lib):
     meta0, status0 = build_meta(w.ids, w.N, 16, 0)
     _, names = _kernels_of(lambda: run_fused(w, dl, meta0, status0))
     assert not _on_tensor_cores(names), sorted(names)
+
+
+def test_captured_graph_matches_eager(cuda_lib):
+    """lora_add_linear inside a CUDA graph (the side-stream fork and join are captured
+    too) gives bit-identical results to eager calls, replay after replay."""
+    w = _case(CASES[0])          # prompt runs and decode rows: both kernels, both streams
+    dl = DeviceLayer(w.layers[0])
+    meta, status = build_meta(w.ids, w.N, 16, 16)
+    ranks, scales = w.ranks.cuda(), lora.scales_for(w.alpha, w.ranks).cuda()
+    eager = dl.y0.clone()
+    lora.lora_add_linear(eager, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status)
+    torch.cuda.synchronize()
+    y = dl.y0.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status,
+                             stream=s)
+    for _ in range(2):
+        y.copy_(dl.y0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(y, eager)
+    del g
