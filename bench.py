@@ -225,11 +225,11 @@ def min_run_of(w):
 
 
 def launches_per_step(w):
-    """Kernels one step launches: the grouping (one block when T <= 2048, else
-    four passes), then per layer the gathered-tile kernel, plus the tensor-core
+    """Kernels one step launches: the grouping (one block when T <= 2048, or
+    T <= 8192 with N <= 1023; else seven passes), then per layer the gathered-tile kernel, plus the tensor-core
     SGMV kernel when contiguous tiles are enabled and the layer qualifies (bf16,
     r_max a multiple of 16, n_slices * r_max <= 128)."""
-    builder = 1 if w.T <= 2048 else 4
+    builder = 1 if (w.T <= 2048 or (w.T <= 8192 and w.N <= 1023)) else 7
     n = builder
     for l in w.layers:
         n += 1

@@ -152,8 +152,8 @@ LORA_API int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int
 /* Device scratch bytes lora_build_segments needs for T rows over N slots,
  * each part rounded up to 256 bytes: per-chunk id counts (4 * (N+1) per 2048
  * rows), one byte per row, 12 bytes per 32 rows (run bitmaps and offsets) and
- * 16 bytes per 2048 rows (per-block totals).  0 when T <= 2048: the grouping
- * then runs in one thread block, in shared memory. */
+ * 16 bytes per 2048 rows (per-block totals).  0 when T <= 2048, or T <= 8192
+ * and N <= 1023: the grouping then runs in one thread block, in shared memory. */
 LORA_API size_t lora_segments_scratch_bytes(int32_t T, int32_t N);
 
 /*

@@ -3,8 +3,10 @@
 // section 2 flowchart and section 3.2; LoraBatchInfo of page "LoRA hot load
 // and adapter routing").
 //
-// A stable counting sort.  Up to SEG_SMALL_T rows one thread block does it
-// all in a single launch (decode batches).  Above that:
+// A stable counting sort.  One thread block does it all in a single launch
+// up to SEG_SMALL_T rows, or up to SEG_ONE_BLOCK_T rows when N < 1024 (then at
+// least 8 warps rank rows in parallel; measured on B200 at 3000-8192 rows:
+// 15-26 us in one block against 33-40 us in seven launches).  Above that:
 //   seg_hist     one block per chunk of SEG_CHUNK rows: per-chunk id histogram
 //   seg_scan     one block, a warp per id: chunk offsets by warp scans; totals
 //                -> seg_start, seg_adapter
@@ -26,6 +28,12 @@ namespace lora {
 constexpr int SEG_THREADS = 1024;
 constexpr int SEG_CHUNK = 2048;
 constexpr int SEG_SMALL_T = 2048;
+constexpr int SEG_ONE_BLOCK_T = 8192, SEG_ONE_BLOCK_N = 1023;
+
+// The whole grouping in one block (shared memory only, no scratch)?
+__host__ __device__ constexpr bool one_block(int T, int N) {
+    return T <= SEG_SMALL_T || (T <= SEG_ONE_BLOCK_T && N <= SEG_ONE_BLOCK_N);
+}
 constexpr int SEG_HIST_THREADS = 512;
 // ints of scan scratch in front of a kernel's other shared arrays (33 long longs)
 constexpr int SEG_SCAN_WORDS = 80;
@@ -845,7 +853,7 @@ static int tw_blocks(int T) { return (tw_words(T) + TW_WORDS - 1) / TW_WORDS; }
 
 // per-chunk id counts | run-start byte per row | 3 words per 32 rows | 4 ints per block
 size_t segments_scratch_bytes(int T, int N) {
-    if (T <= SEG_SMALL_T) return 0;
+    if (one_block(T, N)) return 0;
     return ws_bytes(T, N) + round256((size_t)T) + round256((size_t)12 * tw_words(T)) +
            round256((size_t)16 * tw_blocks(T));
 }
@@ -887,7 +895,7 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
     a.out.min_run = m->min_run;
     a.out.LT = m->long_tile;
 
-    if (a.T <= SEG_SMALL_T) {
+    if (one_block(a.T, a.N)) {
         const size_t nwr = rank_warps(a.N);
         const size_t smem = (SEG_SCAN_WORDS + (((size_t)a.N + 1 + 3) & ~(size_t)3) +
                              ((nwr * (a.N + 1) + 3) & ~(size_t)3) + 2 * (size_t)a.T +

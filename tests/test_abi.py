@@ -56,13 +56,16 @@ def test_capacity_bounds(lib):
 
 def test_scratch_and_workspace_sizes(lib):
     assert lora.lora_segments_scratch_bytes(2048, 100) == 0
+    # one thread block, no scratch: T <= 2048, or T <= 8192 with N <= 1023
+    assert lora.lora_segments_scratch_bytes(2048, 4096) == 0
+    assert lora.lora_segments_scratch_bytes(8192, 1023) == 0
 
     def r256(b):
         return (b + 255) // 256 * 256
 
     # as the header states: per-chunk id counts, one byte per row, 12 bytes per
     # 32 rows and 16 bytes per 2048 rows, each part rounded up to 256 bytes
-    for T, N in [(2049, 100), (77431, 8), (131072, 4096)]:
+    for T, N in [(2049, 1024), (8192, 1024), (8193, 8), (77431, 8), (131072, 4096)]:
         chunks, words, blocks = -(-T // 2048), -(-T // 32), -(-T // 2048)
         want = r256(4 * (N + 1) * chunks) + r256(T) + r256(12 * words) + r256(16 * blocks)
         assert lora.lora_segments_scratch_bytes(T, N) == want, (T, N)

@@ -98,3 +98,19 @@ def test_long_runs_across_blocks(cuda_lib, T, N, min_run, seed):
         parts.append(np.full(L, int(rng.integers(-1, N)), dtype=np.int32))
     ids = np.concatenate(parts)[:T]
     _compare(ids, N, int(rng.choice([1, 16])), min_run, 0)
+
+
+@pytest.mark.parametrize("T,N", [(2049, 24), (4100, 24), (8192, 24), (8192, 1023),
+                                 (5000, 2000), (8192, 4096)])
+def test_grouping_one_block_and_multi_block_bounds(cuda_lib, T, N):
+    """Around the bounds of the one-block grouping (up to 8192 rows when N <= 1023)
+    and the multi-block passes (more ids): decode-like ids, prompt runs, -1 rows."""
+    rng = np.random.default_rng(T + N)
+    parts, n = [], 0
+    while n < T:
+        L = int(rng.choice([1, 2, 70, 300, 129]))
+        parts.append(np.full(L, int(rng.integers(-1, N)), dtype=np.int32))
+        n += L
+    ids = np.concatenate(parts)[:T]
+    for min_run in (0, 64):
+        _compare(ids, N, 16, min_run, 0)
