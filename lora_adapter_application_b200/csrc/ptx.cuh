@@ -25,15 +25,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
-// arrival on the mbarrier at the same offset in block `rank` of the cluster
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, unsigned rank) {
-    asm volatile(
-        "{\n\t.reg .b32 ra;\n\t"
-        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}\n" ::"r"(bar),
-        "r"(rank)
-        : "memory");
-}
 template <bool CLUSTER_ACQUIRE>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, unsigned parity) {
     uint32_t ok;
