@@ -306,43 +306,59 @@ def time_device(sets, K, W, dist, graph=True):
     return step_ms, kern_ms, t0, t1, graphed
 
 
-def time_e2e(w, device, K, dist):
+def time_e2e(w, device, K, dist, n_streams=2):
     """Same step through host buffers: pinned host -> device copies of the step's
     inputs (ids, x and base output y of every layer), the path, and the updated y
-    back to pinned host memory, all inside the timed region."""
+    back to pinned host memory, all inside the timed region.  Consecutive steps
+    alternate between n_streams streams, each with its own device buffers and
+    pinned output, so that one step's copies overlap another's kernels as in a
+    serving loop; every step still copies its own inputs in and its result out."""
     import lora_adapter_application_b200 as lora
-    ds = DeviceSet(w, device, 16, min_run_of(w))
+    n_streams = max(1, int(n_streams))
+    sets = [DeviceSet(w, device, 16, min_run_of(w)) for _ in range(n_streams)]
+    streams = [torch.cuda.Stream(device) for _ in range(n_streams)]
     host = {"ids": w.ids.pin_memory(),
-            "layers": [{"x": l.x.pin_memory(), "y": l.y0.pin_memory(),
-                        "out": torch.empty_like(l.y0).pin_memory()} for l in w.layers]}
+            "layers": [{"x": l.x.pin_memory(), "y": l.y0.pin_memory()} for l in w.layers]}
+    outs = [[torch.empty_like(l.y0).pin_memory() for l in w.layers] for _ in range(n_streams)]
     h2d = host["ids"].numel() * 4 + sum(h["x"].numel() * h["x"].element_size() +
                                         h["y"].numel() * h["y"].element_size() for h in host["layers"])
-    d2h = sum(h["out"].numel() * h["out"].element_size() for h in host["layers"])
+    d2h = sum(o.numel() * o.element_size() for o in outs[0])
 
-    def one():
-        ds.ids.copy_(host["ids"], non_blocking=True)
-        for l, h in zip(ds.layers, host["layers"]):
-            l["x"].copy_(h["x"], non_blocking=True)
-            l["y"].copy_(h["y"], non_blocking=True)
-        lora.lora_build_segments(ds.ids, ds.meta, ds.status)
-        for l in ds.layers:
-            lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks, ds.scales,
-                                 ds.meta, ds.status)
-        for l, h in zip(ds.layers, host["layers"]):
-            h["out"].copy_(l["y"], non_blocking=True)
+    def one(i):
+        ds, st, out = sets[i % n_streams], streams[i % n_streams], outs[i % n_streams]
+        with torch.cuda.stream(st):
+            ds.ids.copy_(host["ids"], non_blocking=True)
+            for l, h in zip(ds.layers, host["layers"]):
+                l["x"].copy_(h["x"], non_blocking=True)
+                l["y"].copy_(h["y"], non_blocking=True)
+            lora.lora_build_segments(ds.ids, ds.meta, ds.status, stream=st)
+            for l in ds.layers:
+                lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks,
+                                     ds.scales, ds.meta, ds.status, stream=st)
+            for l, o in zip(ds.layers, out):
+                o.copy_(l["y"], non_blocking=True)
 
-    for _ in range(3):
-        one()
+    for i in range(3 * n_streams):
+        one(i)
     torch.cuda.synchronize()
     dist.barrier()
+    cur = torch.cuda.current_stream()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(K):
-        one()
-    e.record()
+    s.record(cur)
+    for st in streams:
+        st.wait_event(s)
+    for i in range(K):
+        one(i)
+    for st in streams:
+        cur.wait_stream(st)
+    e.record(cur)
     torch.cuda.synchronize()
     ms = dist.max(s.elapsed_time(e) / K)
-    del ds
+    for ds in sets:
+        code = int(ds.status.item())
+        if code:
+            raise RuntimeError(f"device status {code}")
+    del sets
     return ms, h2d, d2h
 
 
@@ -403,7 +419,7 @@ def bench_ours(args, dist):
     del sets
     torch.cuda.empty_cache()
 
-    e2e_ms, h2d, d2h = time_e2e(w, device, min(args.steps, args.e2e_steps), dist)
+    e2e_ms, h2d, d2h = time_e2e(w, device, min(args.steps, args.e2e_steps), dist, args.e2e_streams)
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
@@ -426,7 +442,7 @@ def bench_ours(args, dist):
                      "peak_source": f"{pk.get('source')} hbm_gbs"},
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "steps": min(args.steps, args.e2e_steps)},
+                "steps": min(args.steps, args.e2e_steps), "streams": args.e2e_streams},
         "gpu_launches": args.steps * launches_per_step(w),
         "clocks": clocks,
     }
@@ -506,6 +522,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(workloads.NAMES))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--e2e-streams", type=int, default=2,
+                    help="streams the end-to-end steps alternate between (1 = one step at a time)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--sweep-seconds", type=float, default=0.5)
