@@ -33,7 +33,7 @@ def test_static_scratch_matches_caller_scratch_twice(cuda_lib):
     lora = cuda_lib
     lib = lora.load()
     rng = np.random.default_rng(2024)
-    T, N = 5000, 100                      # more than one block: the grouping needs scratch
+    T, N = 20000, 100                     # beyond one block (> 8192 rows): the grouping needs scratch
     assert 0 < lora.lora_segments_scratch_bytes(T, N) <= (1 << 20)
     for call in range(2):
         ids_d = torch.as_tensor(_ids(rng, T, N)).cuda()
