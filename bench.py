@@ -50,18 +50,29 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 # ----------------------------------------------------------------------------- helpers
+def code_digest(path):
+    """sha256 of a C++/CUDA source with comments and blank space removed: edits to
+    comments leave it unchanged, any change to the code does not."""
+    import hashlib
+    import re
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()
+
+
 def measured_traffic(workload):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    or None when the kernel source has changed since that capture."""
-    import hashlib
+    or None when the kernel's code has changed since that capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     src = os.path.join(ROOT, "lora_adapter_application_b200", "csrc", "bgmv.cu")
     try:
         with open(p) as f:
             rec = json.load(f)["bgmv_kernel"]
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
+        if code_digest(src) != rec["code_sha256"]:
+            return None
         return rec[workload]["dram_bytes_per_launch"]
     except (OSError, KeyError, ValueError):
         return None

@@ -5,18 +5,20 @@
 // One unit of work = up to 16 rows that share an adapter (a gathered tile, or
 // 16 rows of a contiguous tile).  A cluster of C thread blocks takes a unit;
 // block c owns 1/C of the input columns (shrink) and 1/C of the output
-// columns (expand).  Each block is warp-specialised:
+// columns (expand).  Clusters are persistent: cluster k walks the units k,
+// k + #clusters, ... of those counted on the device.  Each block is
+// warp-specialised:
 //
 //   producer warp   walks the block's chunk stream and fills a 3-stage
 //                   shared-memory ring through the TMA engine: 2-D tensor
 //                   copies of 1-2 KB boxes for the adapters (A: 8 or 16 ranks
 //                   x 64 columns, 128-byte swizzle; B: 64 output columns x 8
-//                   or 16 ranks) and one 1-D bulk copy per gathered x or y row.  (Measured
-//                   on B200: TMA copies leave the load/store pipe to the
-//                   consumers, where a cp.async producer competes with their
-//                   shared-memory traffic; TMA pays per copy, so copies should
-//                   be 1 KB or more.)  A full/empty mbarrier pair guards each
-//                   stage.
+//                   or 16 ranks) and one 1-D bulk copy per gathered x or y
+//                   row piece.  (Measured on B200: TMA copies leave the
+//                   load/store pipe to the consumers, where a cp.async
+//                   producer competes with their shared-memory traffic; TMA
+//                   pays per copy, so copies should be 1 KB or more.)  A
+//                   full/empty mbarrier pair guards each stage.
 //   8 consumer warps
 //     shrink chunks  x rows [cnt][JC] and A rows [r_n][JC] -> partial v
 //                    (tensor-core mma m16n8k16, bf16 in, fp32 accumulate)
@@ -35,7 +37,9 @@
 // chip.  s v enters the expand products as a bf16 hi + lo pair (about 16
 // mantissa bits): a single bf16 copy (2^-9 relative) is not enough when the
 // delta is large and cancels against y.  The multiply-adds (about 4 per byte)
-// run on the tensor pipe; the kernel is bounded by HBM bandwidth.
+// run on the tensor pipe.  Large batches are bounded by HBM bandwidth; a
+// small decode batch is latency-bound: each unit is a chain of dependent
+// loads, the exchange and the expand, a few microseconds each.
 //
 // Inside one 16-wide K step each thread assigns 4 consecutive elements of each
 // operand row to its four k-slots of the mma fragment; both operands use the
