@@ -1,0 +1,95 @@
+"""Host-side bookkeeping of bench.py: the digest that ties a committed DRAM-traffic
+capture to the kernel source it was taken on, and the kernel count per step that
+the bench reports as its launch figure."""
+import json
+import os
+from types import SimpleNamespace
+
+import torch
+
+import bench
+
+CODE = """// fused kernel
+__global__ void k(float* y) {   /* body */
+    y[threadIdx.x] += 1.0f;     // one add
+}
+"""
+
+
+def _write(path, text):
+    with open(path, "w") as f:
+        f.write(text)
+
+
+def test_code_digest_ignores_comments_and_spacing(tmp_path):
+    a, b = tmp_path / "a.cu", tmp_path / "b.cu"
+    _write(a, CODE)
+    _write(b, "/* a different\n   header */\n__global__ void k(float* y)\n{\n"
+              "  y[threadIdx.x]  +=  1.0f;  // another comment\n}\n")
+    assert bench.code_digest(a) == bench.code_digest(b)
+
+
+def test_code_digest_changes_with_code(tmp_path):
+    a, b = tmp_path / "a.cu", tmp_path / "b.cu"
+    _write(a, CODE)
+    _write(b, CODE.replace("1.0f", "2.0f"))
+    assert bench.code_digest(a) != bench.code_digest(b)
+
+
+def _fake_root(tmp_path, src_text, recorded_text):
+    csrc = tmp_path / "lora_adapter_application_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    _write(csrc / "bgmv.cu", src_text)
+    rec_src = tmp_path / "recorded.cu"
+    _write(rec_src, recorded_text)
+    rec = {"bgmv_kernel": {"code_sha256": bench.code_digest(rec_src),
+                           "decode_qproj": {"dram_bytes_per_launch": 123456.0}}}
+    _write(tmp_path / "profiles" / "traffic.json", json.dumps(rec))
+
+
+def test_traffic_kept_while_code_unchanged(tmp_path, monkeypatch):
+    _fake_root(tmp_path, CODE + "// a note added after the capture\n", CODE)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("decode_qproj") == 123456.0
+    assert bench.measured_traffic("prefill") is None          # no capture for it
+
+
+def test_traffic_dropped_once_code_changes(tmp_path, monkeypatch):
+    _fake_root(tmp_path, CODE.replace("+=", "-="), CODE)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("decode_qproj") is None
+
+
+def test_traffic_missing_record(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("decode_qproj") is None
+
+
+def _w(name, T, N, r_max, slices_per_layer, dtype=torch.bfloat16):
+    layers = [SimpleNamespace(d_out=[64] * s) for s in slices_per_layer]
+    return SimpleNamespace(name=name, T=T, N=N, r_max=r_max, dtype=dtype, layers=layers)
+
+
+def test_launches_per_step_hand_counted():
+    # decode-only batch: one-block grouping + one gathered-tile kernel per layer
+    assert bench.launches_per_step(_w("decode_qproj", 256, 32, 16, [1])) == 2
+    assert bench.launches_per_step(_w("multislice_8b", 1024, 100, 64, [3, 1, 2, 1])) == 5
+    # prompts: the tensor-core kernel joins each layer it can take
+    assert bench.launches_per_step(_w("prefill", 77000, 8, 16, [1])) == 7 + 1 + 1
+    # 70B MLP batch (up and down projections, r 16): both layers take both kernels
+    assert bench.launches_per_step(_w("mixed_70b", 8192, 16, 16, [1, 1])) == 1 + 2 + 2
+    # two slices of 64 ranks stack to 128: still the tensor-core kernel
+    assert bench.launches_per_step(_w("prefill", 4096, 8, 64, [2])) == 1 + 2
+    # more than 128 stacked ranks, r_max not a multiple of 16, or fp32: no tensor-core kernel
+    assert bench.launches_per_step(_w("prefill", 2048, 8, 64, [3])) == 1 + 1
+    assert bench.launches_per_step(_w("prefill", 2048, 8, 24, [1])) == 1 + 1
+    assert bench.launches_per_step(_w("prefill", 2048, 8, 16, [1], torch.float32)) == 1 + 1
+
+
+def test_launches_per_step_grouping_boundaries():
+    assert bench.launches_per_step(_w("decode_qproj", 2048, 5000, 16, [1])) == 2
+    assert bench.launches_per_step(_w("decode_qproj", 2049, 5000, 16, [1])) == 8
+    assert bench.launches_per_step(_w("decode_qproj", 8192, 1023, 16, [1])) == 2
+    assert bench.launches_per_step(_w("decode_qproj", 8192, 1024, 16, [1])) == 8
+    assert bench.launches_per_step(_w("decode_qproj", 8193, 8, 16, [1])) == 8
