@@ -37,6 +37,19 @@
  *         y      [T][ld_y]            slice s owns columns col_off_s .. +d_out_s
  *         ranks  [N] int32 device,    r_n in [1, r_max]
  *         scales [N] fp32 device,     alpha / r_n (page "Multi-LoRA Serving", 3.1)
+ *
+ * Tuning overrides (environment, read at each call; unset = the library's own
+ * choice).  They change only the launch shape: results stay within the same
+ * tolerance of the exact value, and a fixed setting gives bit-identical results
+ * from run to run.  A value outside the range is ignored.
+ *   LORA_BG_CLUSTER     1, 2, 4 or 8: blocks per cluster of the gathered-tile kernel
+ *   LORA_TC_CLUSTER     1, 2, 4 or 8: blocks per cluster of the tensor-core kernel;
+ *                       when the shape cannot use it, the contiguous tiles run on
+ *                       the gathered-tile kernel instead
+ *   LORA_TC_STAGES      2 to 6: depth of the tensor-core kernel's load ring (ignored
+ *                       when shared memory cannot hold that many stages)
+ *   LORA_TC_LOAD_ROWS   8 to 128, a power of two: rows per x / y load box
+ *   LORA_TC_STORE_ROWS  8 to 128, a power of two: rows per y store box
  */
 #ifndef LORA_DELTA_H
 #define LORA_DELTA_H
