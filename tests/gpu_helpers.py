@@ -65,3 +65,27 @@ def sample_rows(w, k, seed=0):
         where = np.nonzero(ids == n)[0]
         rows.update([int(where[0]), int(where[-1])])
     return np.array(sorted(rows), dtype=np.int32)
+
+
+def kernels_of(fn, tries=5):
+    """Runs fn under the torch profiler (CUPTI) and returns (fn's result, names of
+    the device kernels it launched, in order, and the number of kernel-launch API
+    calls).  CUPTI hands kernel records over asynchronously, and after earlier
+    sessions in the same process it has been seen to deliver fewer records than
+    there were launches; such a session is run again, so fn must be safe to
+    repeat."""
+    from torch.autograd import DeviceType
+    from torch.profiler import ProfilerActivity, profile
+    for _ in range(tries):
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            out = fn()
+            torch.cuda.synchronize()
+        ev = prof.events()
+        kernels = [e.name for e in ev if e.device_type == DeviceType.CUDA
+                   and not e.name.startswith(("Memcpy", "Memset"))]
+        launches = sum(1 for e in ev if e.device_type == DeviceType.CPU and "LaunchKernel" in e.name)
+        if len(kernels) == launches:
+            return out, kernels, launches
+    raise AssertionError(f"kernel records never matched the {launches} launches in {tries} "
+                         f"profiler sessions (last: {kernels})")

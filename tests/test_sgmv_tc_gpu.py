@@ -15,7 +15,7 @@ import torch
 import lora_adapter_application_b200 as lora
 import oracle
 import workloads
-from gpu_helpers import DeviceLayer, assert_within, build_meta, oracle_rows, run_fused
+from gpu_helpers import DeviceLayer, assert_within, build_meta, kernels_of, oracle_rows, run_fused
 
 pytestmark = pytest.mark.gpu
 
@@ -48,13 +48,9 @@ def _ids(c):
 
 
 def _kernels_of(fn):
-    """Names of the CUDA kernels fn launches (torch profiler, CUPTI)."""
-    from torch.profiler import ProfilerActivity, profile
-    torch.cuda.synchronize()
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        out = fn()
-        torch.cuda.synchronize()
-    return out, {e.name for e in prof.events()}
+    """Names of the CUDA kernels fn launches (fn may run more than once)."""
+    out, kernels, _ = kernels_of(fn)
+    return out, set(kernels)
 
 
 def _on_tensor_cores(names):
@@ -104,8 +100,12 @@ def test_shrink_expand_contiguous_tiles(cuda_lib, C, monkeypatch):
         assert np.isnan(vg[i, :, r:]).all()                            # k >= r_n not written
     vin = torch.as_tensor(vref, dtype=torch.float32).permute(1, 0, 2).contiguous().cuda()
     y = dl.y0.clone()
-    _, names = _kernels_of(lambda: lora.lora_sgmv_expand(y, vin, dl.B, dl.col_off, ranks, scales,
-                                                         meta, status))
+
+    def expand():                                     # y += ...: start from y0 on every run
+        y.copy_(dl.y0)
+        lora.lora_sgmv_expand(y, vin, dl.B, dl.col_off, ranks, scales, meta, status)
+
+    _, names = _kernels_of(expand)
     assert _on_tensor_cores(names), sorted(names)
     assert int(status.item()) == 0
     assert_within(y.cpu().double().numpy(), oracle_rows(w, lay, None), torch.bfloat16, "expand")
