@@ -100,9 +100,12 @@ struct Geo {          // chunk geometry of one block for one unit
     int n_shrink, n_chunks;
 };
 
-// Shared-memory bytes of a chunk: 16 padded rows, then 1 KB TMA boxes (1 KB aligned).
-__device__ __forceinline__ int chunk_bytes(int row_stride, int boxes) {
-    return ((BG_ROWS * row_stride + 1023) & ~1023) + boxes * 1024;
+// Shared-memory bytes of a chunk `cols` columns wide: 16 bf16 rows of x or y
+// (padded by 16 bytes, 1 KB aligned), then the adapter boxes, which hold per
+// 64 columns one 1 KB box per 8 ranks, or one 2 KB box per 16 ranks (ab16).
+__device__ __forceinline__ int chunk_bytes(int cols, int nb8, bool ab16) {
+    const int box_kb = ab16 ? 2 * ((nb8 + 1) >> 1) : nb8;   // per 64 columns
+    return ((BG_ROWS * (cols * 2 + 16) + 1023) & ~1023) + box_kb * (cols >> 6) * 1024;
 }
 
 // Position in a block's chunk stream, advanced without divisions: shrink
@@ -153,7 +156,7 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         G.j_hi = min((int)((int64_t)(crank + 1) * n64 / C) * 64, a.d_in);
         // widest power-of-two chunk (>= 64 columns) whose x rows and A boxes fit a stage
         int jc = 64;
-        while (chunk_bytes(jc * 4 + 16, G.nb8 * (jc / 32)) <= BG_STAGE_BYTES) jc *= 2;
+        while (chunk_bytes(jc * 2, G.nb8, a.ab16) <= BG_STAGE_BYTES) jc *= 2;
         const int span = max(0, G.j_hi - G.j_lo);
         while (jc > 64 && jc / 2 >= span) jc /= 2;
         G.JC = jc;
@@ -175,7 +178,7 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         G.c_hi = (int)((int64_t)(crank + 1) * n8 / C) * 8;
         // widest power-of-two chunk (>= 64 columns) whose y rows and B boxes fit a stage
         int cc = 64;
-        while (chunk_bytes(cc * 4 + 16, G.nb8 * (cc / 32)) <= BG_STAGE_BYTES) cc *= 2;
+        while (chunk_bytes(cc * 2, G.nb8, a.ab16) <= BG_STAGE_BYTES) cc *= 2;
         G.CC = cc;
         G.YS = G.CC * 2 + 16;   // 16 (mod 128) bytes: the 8 rows of an mma tile hit 8 bank groups
         G.B0 = (BG_ROWS * G.YS + 1023) & ~1023;
