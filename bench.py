@@ -265,33 +265,40 @@ def _event(external):
         return torch.cuda.Event(enable_timing=True)
 
 
-def time_device(sets, K, W, dist, graph=True):
-    """Time exactly K steps on the device.  The K steps (with a CUDA-event pair
-    around each step's layer calls) are captured into one CUDA graph and replayed
-    once, so host launch overhead does not enter the timed region; without a
-    graph the steps are launched one by one."""
+KERNEL_SAMPLE = 8   # a CUDA-event pair around the layer calls of every 8th timed step
+
+
+def time_device(sets, K, W, dist, graph=True, every=KERNEL_SAMPLE):
+    """Time exactly K steps on the device.  The K steps are captured into one
+    CUDA graph and replayed once, so host launch overhead does not enter the
+    timed region; without a graph the steps are launched one by one.  Every
+    `every`-th step also records a CUDA-event pair around its layer calls (the
+    kernel time of the roofline), measured inside the same timed region; an
+    event node between two kernels lengthens that step, so the pair is not put
+    on every step."""
     for i in range(W):
         step(sets[i % len(sets)])
     torch.cuda.synchronize()
+    sampled = list(range(0, K, every))
     ka = kb = g = None
     if graph:
         try:
-            ka = [_event(True) for _ in range(K)]
-            kb = [_event(True) for _ in range(K)]
+            ka = {i: _event(True) for i in sampled}
+            kb = {i: _event(True) for i in sampled}
             s = torch.cuda.Stream()
             s.wait_stream(torch.cuda.current_stream())
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 for i in range(K):
-                    step(sets[i % len(sets)], ka[i], kb[i])
+                    step(sets[i % len(sets)], ka.get(i), kb.get(i))
             torch.cuda.synchronize()
         except Exception as e:  # capture not available: launch eagerly
             print(f"graph capture failed ({e}); timing eager launches", file=sys.stderr)
             g = None
             torch.cuda.synchronize()
     if g is None:
-        ka = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ka = {i: torch.cuda.Event(enable_timing=True) for i in sampled}
+        kb = {i: torch.cuda.Event(enable_timing=True) for i in sampled}
     dist.barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -301,13 +308,13 @@ def time_device(sets, K, W, dist, graph=True):
         g.replay()
     else:
         for i in range(K):
-            step(sets[i % len(sets)], ka[i], kb[i])
+            step(sets[i % len(sets)], ka.get(i), kb.get(i))
     end.record()
     torch.cuda.synchronize()
     t1 = time.perf_counter()
     dist.barrier()
     step_ms = start.elapsed_time(end) / K
-    kern_ms = sum(a.elapsed_time(b) for a, b in zip(ka, kb)) / K
+    kern_ms = sum(ka[i].elapsed_time(kb[i]) for i in sampled) / len(sampled)
     for st in sets:
         code = int(st.status.item())
         if code:
@@ -443,7 +450,8 @@ def bench_ours(args, dist):
                    "l2": f"{n_sets} rotating input sets of {per_set / 1e6:.1f} MB "
                          f"(inputs {n_sets * per_set / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
                    "parallelism": f"dp{dist.world} (independent batch per GPU)",
-                   "launch": "CUDA graph of the K timed steps" if graphed else "eager",
+                   "launch": ("CUDA graph of the K timed steps" if graphed else "eager") +
+                             f"; kernel events on every {KERNEL_SAMPLE}th step",
                    "seed": args.seed},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(pk["hbm_gbs"]),
                      "unit": "GB/s", "frac": achieved / float(pk["hbm_gbs"]),

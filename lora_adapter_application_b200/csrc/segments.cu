@@ -538,7 +538,9 @@ __global__ void __launch_bounds__(SEG_THREADS) seg_small_kernel(SegArgs a) {
     scatter_block(ids_s, 0, a.T, a.N, hist, hw, nwr, perm_s, brk_s);
     __syncthreads();
     for (int i = tid; i < a.T; i += SEG_THREADS) a.perm[i] = perm_s[i];
-    dev_tiles(ids_s, perm_s, brk_s, a.seg_start, a.N, a.out, tsm);
+    // hist holds seg_start[0..N] (scan above, read-only since): the tile pass reads
+    // it from shared memory instead of the global copy this block just wrote
+    dev_tiles(ids_s, perm_s, brk_s, hist, a.N, a.out, tsm);
 }
 
 __global__ void __launch_bounds__(SEG_HIST_THREADS) seg_hist_kernel(SegArgs a) {
