@@ -43,6 +43,7 @@
  * tolerance of the exact value, and a fixed setting gives bit-identical results
  * from run to run.  A value outside the range is ignored.
  *   LORA_BG_CLUSTER     1, 2, 4 or 8: blocks per cluster of the gathered-tile kernel
+ *   LORA_BG_STAGES      2 or 3: stages of the gathered-tile kernel's 72 KB load ring
  *   LORA_TC_CLUSTER     1, 2, 4 or 8: blocks per cluster of the tensor-core kernel;
  *                       when the shape cannot use it, the contiguous tiles run on
  *                       the gathered-tile kernel instead

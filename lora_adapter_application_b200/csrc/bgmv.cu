@@ -9,8 +9,8 @@
 // k + #clusters, ... of those counted on the device.  Each block is
 // warp-specialised:
 //
-//   producer warp   walks the block's chunk stream and fills a 3-stage
-//                   shared-memory ring through the TMA engine: 2-D tensor
+//   producer warp   walks the block's chunk stream and fills a 72 KB
+//                   shared-memory ring (3 or 2 stages) through the TMA engine: 2-D tensor
 //                   copies of 1-2 KB boxes for the adapters (A: 8 or 16 ranks
 //                   x 64 columns, 128-byte swizzle; B: 64 output columns x 8
 //                   or 16 ranks) and one 1-D bulk copy per gathered x or y
@@ -32,7 +32,7 @@
 //     expand chunks  B rows [CC][r_n] and y rows [cnt][CC] -> y += (s v) B^T in
 //                    fp32, rounded once, written back with 16-byte stores
 //
-// The producer runs up to 3 chunks ahead, across the exchange, so HBM stays
+// The producer runs a ring's worth of chunks ahead, across the exchange, so HBM stays
 // busy; every byte of x, A, B and y crosses HBM once and v never leaves the
 // chip.  s v enters the expand products as a bf16 hi + lo pair (about 16
 // mantissa bits): a single bf16 copy (2^-9 relative) is not enough when the
@@ -53,6 +53,8 @@
 
 #include <cooperative_groups.h>
 
+#include <cstdlib>
+
 #include <mutex>
 
 namespace cg = cooperative_groups;
@@ -63,8 +65,8 @@ constexpr int BG_CONSUMERS = 8;                      // consumer warps
 constexpr int BG_THREADS = (BG_CONSUMERS + 1) * 32;  // + 1 producer warp
 constexpr int BG_ROWS = 16;
 constexpr int BG_RMAX = 64;
-constexpr int BG_STAGES = 3;
-constexpr int BG_STAGE_BYTES = 24576;
+constexpr int BG_MAX_STAGES = 3;                    // mbarrier pairs reserved
+constexpr int BG_RING_BYTES = 73728;                // 3 x 24 KB or 2 x 36 KB (1 KB multiples)
 constexpr int BG_VF_STRIDE = 80;   // floats per row of the reduced v (bank spread)
 
 
@@ -89,7 +91,7 @@ __device__ __forceinline__ uint4 zero_if(bool z, uint4 v) { return z ? make_uint
 //   for the elements e with e % C == this block's rank.
 size_t bgmv_smem_bytes(int n_slices) {
     return 1024 /* alignment of the ring to the 128-byte swizzle atom */ +
-           (size_t)BG_STAGES * BG_STAGE_BYTES + (size_t)n_slices * BG_ROWS * BG_RMAX * 4 +
+           (size_t)BG_RING_BYTES + (size_t)n_slices * BG_ROWS * BG_RMAX * 4 +
            (size_t)n_slices * BG_ROWS * BG_VF_STRIDE * 4 + (size_t)BG_ROWS * BG_RMAX * 4 + 128;
 }
 
@@ -146,6 +148,8 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
     const int cnt = u.cnt;
 
     // ------------------------------------------------------------ geometry
+    const int NS = a.stages == 2 ? 2 : 3;                   // ring stages
+    const int SB = BG_RING_BYTES / NS;                      // bytes per stage
     Geo G;
     G.r8 = (r_n + 7) & ~7;
     G.nb8 = G.r8 >> 3;
@@ -156,7 +160,7 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         G.j_hi = min((int)((int64_t)(crank + 1) * n64 / C) * 64, a.d_in);
         // widest power-of-two chunk (>= 64 columns) whose x rows and A boxes fit a stage
         int jc = 64;
-        while (chunk_bytes(jc * 2, G.nb8, a.ab16) <= BG_STAGE_BYTES) jc *= 2;
+        while (chunk_bytes(jc * 2, G.nb8, a.ab16) <= SB) jc *= 2;
         const int span = max(0, G.j_hi - G.j_lo);
         while (jc > 64 && jc / 2 >= span) jc /= 2;
         G.JC = jc;
@@ -178,7 +182,7 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         G.c_hi = (int)((int64_t)(crank + 1) * n8 / C) * 8;
         // widest power-of-two chunk (>= 64 columns) whose y rows and B boxes fit a stage
         int cc = 64;
-        while (chunk_bytes(cc * 2, G.nb8, a.ab16) <= BG_STAGE_BYTES) cc *= 2;
+        while (chunk_bytes(cc * 2, G.nb8, a.ab16) <= SB) cc *= 2;
         G.CC = cc;
         G.YS = G.CC * 2 + 16;   // 16 (mod 128) bytes: the 8 rows of an mma tile hit 8 bank groups
         G.B0 = (BG_ROWS * G.YS + 1023) & ~1023;
@@ -240,10 +244,10 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
         first(it);
         for (; it.i < G.n_chunks; advance(it)) {
             const uint32_t gi = base + (uint32_t)it.i;   // position in the block's ring stream
-            const int st = (int)(gi % BG_STAGES);
-            const uint32_t full = full0 + 8 * st, dst = ring_s + st * BG_STAGE_BYTES;
-            if (gi >= BG_STAGES)
-                mbar_wait(empty0 + 8 * st, ((gi / BG_STAGES) - 1) & 1, a.status, failed);
+            const int st = (int)(gi % (uint32_t)NS);
+            const uint32_t full = full0 + 8 * st, dst = ring_s + st * SB;
+            if (gi >= (uint32_t)NS)
+                mbar_wait(empty0 + 8 * st, ((gi / NS) - 1) & 1, a.status, failed);
             if (failed) break;
             if (it.i < G.n_shrink) {
                 const int jc0 = G.j_lo + it.q * G.JC;
@@ -499,13 +503,13 @@ __device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm,
     bool exchanged = false;
     for (; it.i < G.n_chunks; advance(it)) {
         const uint32_t gi = base + (uint32_t)it.i;
-        const int st = (int)(gi % BG_STAGES);
-        const uint32_t sta = ring_s + st * BG_STAGE_BYTES;
+        const int st = (int)(gi % (uint32_t)NS);
+        const uint32_t sta = ring_s + st * SB;
         if (!exchanged && it.i >= G.n_shrink) {
             exchange();
             exchanged = true;
         }
-        const bool ready = mbar_wait(full0 + 8 * st, (gi / BG_STAGES) & 1, a.status, failed);
+        const bool ready = mbar_wait(full0 + 8 * st, (gi / NS) & 1, a.status, failed);
         if (ready) {
             if (it.i < G.n_shrink)
                 shrink_chunk(it, sta);
@@ -530,15 +534,15 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
     BgSmem sm;
     // ring on a 1 KB boundary: swizzled TMA boxes need their 1 KB atom aligned
     sm.ring = bg_sm + ((1024u - (smem_u32(bg_sm) & 1023u)) & 1023u);
-    sm.recv = reinterpret_cast<float *>(sm.ring + BG_STAGES * BG_STAGE_BYTES);
+    sm.recv = reinterpret_cast<float *>(sm.ring + BG_RING_BYTES);
     sm.vfull = sm.recv + S * BG_ROWS * BG_RMAX;
     sm.part = sm.vfull + S * BG_ROWS * BG_VF_STRIDE;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm.part + BG_ROWS * BG_RMAX);
     sm.rows = rows_sm;
     sm.ring_s = smem_u32(sm.ring);
     sm.full0 = smem_u32(bars);
-    sm.empty0 = sm.full0 + 8 * BG_STAGES;
-    sm.xready = sm.full0 + 16 * BG_STAGES;
+    sm.empty0 = sm.full0 + 8 * BG_MAX_STAGES;
+    sm.xready = sm.full0 + 16 * BG_MAX_STAGES;
     sm.vready = sm.xready + 8;
 
     const int tid = threadIdx.x;
@@ -548,7 +552,7 @@ __global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_consta
         if (MODE != MODE_SHRINK) prefetch_tmap(&a.tmB[s]);
     }
     if (tid == 0) {
-        for (int st = 0; st < BG_STAGES; ++st) {
+        for (int st = 0; st < BG_MAX_STAGES; ++st) {
             mbar_init(sm.full0 + 8 * st, 1);
             mbar_init(sm.empty0 + 8 * st, BG_CONSUMERS);
         }
@@ -637,8 +641,17 @@ int bg_active_clusters(int mode, int cluster, size_t smem) {
 
 // Persistent launch: as many clusters as fit the device at once (at most one
 // per unit of the tile-list capacity); each walks the live units.
-int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_t st) {
+int launch_bgmv(int mode, const BgArgs &args, int n_units, int cluster, cudaStream_t st) {
     if (n_units <= 0) return LORA_OK;
+    // Two 36 KB stages: chunks twice as wide as with three 24 KB stages up to rank
+    // 48 (half the gathered-row copies), and the whole shrink stream of a decode
+    // unit in flight at once.  Measured on B200 (graph-timed): decode q_proj
+    // kernel 21.8 us against 24.8 with three stages; Llama-3-8B layer set at
+    // decode 583 against 587 us.
+    BgArgs a = args;
+    a.stages = 2;
+    if (const char *e = std::getenv("LORA_BG_STAGES"))   // tuning override: 2 or 3
+        if (std::atoi(e) == 3) a.stages = 3;
     const size_t smem = bgmv_smem_bytes(a.sl.n);
     int clusters = bg_active_clusters(mode, cluster, smem);
     if (clusters < 1) {

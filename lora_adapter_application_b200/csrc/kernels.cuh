@@ -37,6 +37,7 @@ struct BgArgs {
     Tiles tiles;
     int32_t *status;
     int ab16;          // adapters in 16-rank boxes (r_max % 16 == 0): A 64 x 16, B 16 x 64
+    int stages;        // ring stages, 2 or 3, over the same ring bytes (set by launch_bgmv)
 };
 
 struct SimtArgs {

@@ -52,11 +52,13 @@ def test_small_bf16_cases(cuda_lib, case, fn):
 
 @pytest.mark.parametrize("r_max", [32, 64])
 @pytest.mark.parametrize("C", ["4", "8"])
-def test_ranks_17_to_24_in_16_rank_boxes(cuda_lib, r_max, C, monkeypatch):
+@pytest.mark.parametrize("stages", ["2", "3"])
+def test_ranks_17_to_24_in_16_rank_boxes(cuda_lib, r_max, C, stages, monkeypatch):
     """Ranks 17-24 with r_max a multiple of 16: the adapters arrive as two 16-rank
     boxes per 64 columns (32 ranks, 8 of them padding), and every 64-column box of
-    a wide chunk is loaded (4096 columns over 4 or 8 blocks)."""
+    a wide chunk is loaded (4096 columns over 4 or 8 blocks, 2 or 3 ring stages)."""
     monkeypatch.setenv("LORA_BG_CLUSTER", C)
+    monkeypatch.setenv("LORA_BG_STAGES", stages)
     ranks = [17 + (i % 8) for i in range(12)]
     w = workloads.random_case(41, 256, 12, 4096, [4096], r_max, ranks=ranks, none_frac=0.05,
                               dtype=torch.bfloat16)
