@@ -9,6 +9,8 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import torch
 
 import oracle
@@ -292,7 +294,21 @@ def _check_segments_against_library_sort(ids, N, R, min_run, LT):
         prev = (n, q0)
     assert list(grow) == sorted(grow, key=lambda i: (ids[i], i))
     np.testing.assert_array_equal(covered, valid.astype(np.int32))
-    # gathered rows are exactly the rows outside long runs
+    # gathered rows are exactly the rows outside long runs (run lengths by brute force)
+    run_lo, run_len = np.zeros(T, np.int64), np.zeros(T, np.int64)
+    i = 0
+    while i < T:
+        j = i
+        while j < T and ids[j] == ids[i]:
+            j += 1
+        run_lo[i:j], run_len[i:j] = i, j - i
+        i = j
+    long_row = valid & (run_len >= min_run) if min_run > 0 else np.zeros(T, bool)
+    assert sorted(grow) == sorted(np.nonzero(valid & ~long_row)[0])
+    # contiguous tiles: each long run cut every LT rows from its first row
+    for n, row0, cnt, _ in got["contig_tiles"]:
+        assert (row0 - run_lo[row0]) % LT == 0
+        assert cnt == min(LT, run_lo[row0] + run_len[row0] - row0)
     if min_run == 0:
         assert len(got["contig_tiles"]) == 0
         np.testing.assert_array_equal(grow, got["perm"][:valid.sum()])
@@ -313,6 +329,19 @@ def test_segments_against_library_sort_random(seed):
         ids = np.repeat(rng.integers(-1, N, size=12), lens)
     _check_segments_against_library_sort(ids, N, int(rng.integers(1, 17)),
                                          int(rng.choice([0, 8, 32])), int(rng.choice([16, 128])))
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.integers(1, 9).flatmap(lambda N: st.tuples(
+           st.just(N),
+           st.lists(st.tuples(st.integers(-1, N - 1), st.integers(1, 40)), min_size=0, max_size=12),
+           st.integers(1, 16), st.sampled_from([0, 1, 5, 24]), st.sampled_from([4, 16, 128]))))
+def test_segments_properties_hypothesis(case):
+    """Random batches as runs of (id, length): the grouping's definition checked
+    by brute force (stable order, offsets, every row once, long runs tiled)."""
+    N, runs, R, min_run, LT = case
+    ids = np.array([i for (i, L) in runs for _ in range(L)], np.int32)
+    _check_segments_against_library_sort(ids, N, R, min_run, LT)
 
 
 @pytest.mark.parametrize("ids,N", [
