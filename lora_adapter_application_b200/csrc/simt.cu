@@ -9,6 +9,8 @@
 //   expand  one thread per output column: y += s * sum_k B[c][k] v[k]
 #include "kernels.cuh"
 
+#include <mutex>
+
 namespace lora {
 
 constexpr int SIMT_THREADS = 256;
@@ -94,12 +96,19 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_kernel(SimtArgs a) {
 template <typename E>
 static cudaError_t launch_simt_t(int mode, const SimtArgs &a, int n_units, cudaStream_t st) {
     const size_t smem = simt_smem_bytes(a.sl.n, a.r_max);
-    static bool attr_done[3] = {false, false, false};
+    // the shared-memory limit is a per-device attribute of the kernel: set it once
+    // per device and mode (devices 0-63)
+    static std::mutex mu;
+    static uint64_t attr_done[3] = {0, 0, 0};
+    int dev = 0;
+    cudaGetDevice(&dev);
     auto set = [&](const void *fn) {
-        if (!attr_done[mode]) {
+        std::lock_guard<std::mutex> lock(mu);
+        const uint64_t bit = 1ull << (dev & 63);
+        if (!(attr_done[mode] & bit)) {
             cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)simt_smem_bytes(LORA_MAX_SLICES, LORA_MAX_RANK));
-            attr_done[mode] = true;
+            attr_done[mode] |= bit;
         }
     };
     if (mode == 0) {
