@@ -34,7 +34,8 @@
  *         x      [T][ld_x]            d_in columns used
  *         A_s    [N][r_max][d_in]     rank rows k >= r_n are padding, never read
  *         B_s    [N][d_out_s][r_max]  rank columns k >= r_n are padding, never read
- *         y      [T][ld_y]            slice s owns columns col_off_s .. +d_out_s
+ *         y      [T][ld_y]            slice s owns columns col_off_s .. +d_out_s; slices
+ *                                     that overlap, or run past ld_y, are LORA_ERR_SHAPE
  *         ranks  [N] int32 device,    r_n in [1, r_max]
  *         scales [N] fp32 device,     alpha / r_n (page "Multi-LoRA Serving", 3.1)
  *

@@ -148,7 +148,30 @@ int check_call(const Call &c, bool need_x, bool need_y, bool need_scales, bool n
         if (need_y && (sl.d_out < 1 || sl.col_off < 0 || (int64_t)sl.col_off + sl.d_out > c.ld_y))
             return LORA_ERR_SHAPE;
     }
+    if (need_y) {   // each slice owns its columns of y: no two slices overlap
+        int64_t total = 0;
+        for (int s = 0; s < c.n_slices; ++s) {
+            const lora_slice &a = c.slices[s];
+            total += a.d_out;
+            for (int t = 0; t < s; ++t) {
+                const lora_slice &b = c.slices[t];
+                if (a.col_off < (int64_t)b.col_off + b.d_out && b.col_off < (int64_t)a.col_off + a.d_out)
+                    return LORA_ERR_SHAPE;
+            }
+        }
+        if (total > (int64_t)1 << 30) return LORA_ERR_SHAPE;
+    }
     return LORA_OK;
+}
+
+// Adapter rows of every slice addressable by 32-bit tensor coordinates
+// (row n * d_out + column of the stacked B, n * r_max + rank of A).
+bool rows_fit_int32(const Call &c) {
+    const int64_t lim = ((int64_t)1 << 31) - 256;
+    if ((int64_t)c.meta->N * c.r_max > lim) return false;
+    for (int s = 0; s < c.n_slices; ++s)
+        if ((int64_t)c.meta->N * c.slices[s].d_out > lim) return false;
+    return true;
 }
 
 Slices make_slices(const Call &c) {
@@ -184,7 +207,7 @@ int n_units(const Tiles &t) { return t.max_gather + (t.subs ? t.max_contig * t.s
 // The vectorised bf16 tensor-pipe kernel takes the call?  It moves 16-byte
 // pieces, so every row start and width must be a multiple of 8 elements.
 bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
-    if (c.dtype != LORA_BF16 || c.r_max > 64 || (c.r_max & 7)) return false;
+    if (c.dtype != LORA_BF16 || c.r_max > 64 || (c.r_max & 7) || !rows_fit_int32(c)) return false;
     if (need_x) {
         if ((c.d_in & 7) || (c.ld_x & 7) || !aligned(c.x, 16)) return false;
         for (int s = 0; s < c.n_slices; ++s)
@@ -204,7 +227,7 @@ bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
 // 16-byte aligned rows and slices (TMA).
 bool tc_ok(const Call &c, bool need_x, bool need_y) {
     if (c.dtype != LORA_BF16 || c.meta->min_run <= 0 || c.meta->max_contig_tiles <= 0) return false;
-    if ((c.r_max & 15) || c.n_slices * c.r_max > 128) return false;
+    if ((c.r_max & 15) || c.n_slices * c.r_max > 128 || !rows_fit_int32(c)) return false;
     if (need_x) {
         if ((c.d_in & 7) || (c.ld_x & 7) || !aligned(c.x, 16)) return false;
         for (int s = 0; s < c.n_slices; ++s)

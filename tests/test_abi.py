@@ -106,6 +106,12 @@ def test_host_checks(lib):
     assert lib.lora_add_linear(*args(n=9)) == c["SHAPE"]
     assert lib.lora_add_linear(*args(ld_y=8)) == c["SHAPE"]   # slice runs past the row
     assert lib.lora_bgmv_fused(*args(ld_y=8)) == c["SHAPE"]
+    two = (lora.lora_slice * 2)()                                  # q [0, 16) and k [8, 24): overlap
+    two[0].A, two[0].B, two[0].d_out, two[0].col_off = 0x1000, 0x1000, 16, 0
+    two[1].A, two[1].B, two[1].d_out, two[1].col_off = 0x1000, 0x1000, 16, 8
+    assert lib.lora_add_linear(*args(n=2, ld_y=32, sl=two)) == c["SHAPE"]
+    assert lib.lora_sgmv_expand(fake, 32, fake, two, 2, 16, fake, fake, ctypes.byref(m), 0, fake,
+                                None) == c["SHAPE"]
     nul = (lora.lora_slice * 1)()
     nul[0].A, nul[0].B, nul[0].d_out = None, 0x1000, 16
     assert lib.lora_add_linear(*args(sl=nul)) == c["NULL"]
