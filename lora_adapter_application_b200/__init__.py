@@ -232,15 +232,64 @@ def _slices(A, B, d_out, col_off):
     return arr, n
 
 
-def _adapters(A, B):
-    ref = A[0] if A is not None else B[0]
+def _shapes(meta, x=None, y=None, A=None, B=None, col_off=None, ranks=None, scales=None,
+            v=None):
+    """Shape, dtype and layout agreement of a call's operands (the library sees
+    only pointers, so a mismatch here would be an out-of-bounds read there).
+    Runs before any device check.  Returns (N slots, r_max, n_slices)."""
+    T = meta.T
+    stacks = [t for t in (A or []) + (B or [])]
+    if not stacks:
+        raise LoraError("at least one adapter slice")
+    if A is not None and B is not None and len(A) != len(B):
+        raise LoraError("one A and one B per slice")
+    n = len(A) if A is not None else len(B)
+    if not 1 <= n <= MAX_SLICES:
+        raise LoraError("1 to 8 slices")
+    ref = stacks[0]
+    for t in stacks:
+        if not isinstance(t, torch.Tensor) or t.dim() != 3 or not t.is_contiguous() or \
+                t.dtype != ref.dtype:
+            raise LoraError("stacked adapters must be contiguous 3-D tensors of one dtype")
     N = ref.shape[0]
-    r_max = ref.shape[1] if A is not None else ref.shape[2]
+    r_max = A[0].shape[1] if A is not None else B[0].shape[2]
+    if N < meta.N:
+        raise LoraError(f"adapter stacks hold {N} slots, the batch metadata {meta.N}")
+    if A is not None:
+        d_in = A[0].shape[2]
+        if any(a.shape != (N, r_max, d_in) for a in A):
+            raise LoraError("every A slice is [N, r_max, d_in] with the same N, r_max, d_in")
+        if x is not None:
+            if not isinstance(x, torch.Tensor) or x.dim() != 2 or x.shape[0] < T or x.shape[1] < d_in:
+                raise LoraError("x must be 2-D with at least T rows and d_in columns")
+            if x.dtype != ref.dtype:
+                raise LoraError("x, y, A and B share one dtype")
+    if B is not None:
+        if any(b.shape[0] != N or b.shape[2] != r_max for b in B):
+            raise LoraError("every B slice is [N, d_out, r_max] with the same N and r_max")
+        if col_off is None or len(col_off) != n:
+            raise LoraError("one column offset per slice")
+        if y is not None:
+            if not isinstance(y, torch.Tensor) or y.dim() != 2 or y.shape[0] < T:
+                raise LoraError("y must be 2-D with at least T rows")
+            if y.dtype != ref.dtype:
+                raise LoraError("x, y, A and B share one dtype")
+            for b, c in zip(B, col_off):
+                if int(c) < 0 or int(c) + b.shape[1] > y.shape[1]:
+                    raise LoraError("a slice's columns run past y")
+    for t, what, dt in ((ranks, "ranks", torch.int32), (scales, "scales", torch.float32)):
+        if t is not None and (not isinstance(t, torch.Tensor) or t.dtype != dt or
+                              not t.is_contiguous() or t.numel() < meta.N):
+            raise LoraError(f"{what} must be a contiguous {dt} tensor of at least N entries")
+    if v is not None and (not isinstance(v, torch.Tensor) or v.dtype != torch.float32 or
+                          not v.is_contiguous() or v.numel() < n * T * r_max):
+        raise LoraError("v must be contiguous fp32 [n_slices, T, r_max]")
+    return N, r_max, n
+
+
+def _adapters(A, B):
     for t in (A or []) + (B or []):
         _dev(t, "adapter tensor")
-        if not t.is_contiguous() or t.dtype != ref.dtype or t.shape[0] != N:
-            raise LoraError("stacked adapters must be contiguous, one dtype, N slots each")
-    return N, r_max
 
 
 def scales_for(alpha, ranks):
@@ -250,12 +299,11 @@ def scales_for(alpha, ranks):
 
 def lora_sgmv_shrink(v, x, A, ranks, meta: Meta, status, stream=None):
     """v[s, i, k] = sum_j A[s][n, k, j] x[i, j] for rows with an adapter, k < r_n."""
+    N, r_max, n = _shapes(meta, x=x, A=A, ranks=ranks, v=v)
     ld_x = _rows(x, "x")
-    N, r_max = _adapters(A, None)
+    _adapters(A, None)
     sl, n = _slices(A, None, None, None)
     _dev(v, "v")
-    if v.dtype != torch.float32 or not v.is_contiguous() or v.numel() < n * meta.T * r_max:
-        raise LoraError("v must be contiguous fp32 [n_slices, T, r_max]")
     _check(load().lora_sgmv_shrink(_ptr(v), _ptr(x), ld_x, A[0].shape[2], sl, n, r_max,
                                    _ptr(_dev(ranks, "ranks")), ctypes.byref(meta.c), _dtype_code(x),
                                    _ptr(status), _stream(stream)))
@@ -263,8 +311,9 @@ def lora_sgmv_shrink(v, x, A, ranks, meta: Meta, status, stream=None):
 
 def lora_sgmv_expand(y, v, B, col_off, ranks, scales, meta: Meta, status, stream=None):
     """y[i, col_off_s + c] += scales[n] sum_k B[s][n, c, k] v[s, i, k]."""
+    N, r_max, n = _shapes(meta, y=y, B=B, col_off=col_off, ranks=ranks, scales=scales, v=v)
     ld_y = _rows(y, "y")
-    N, r_max = _adapters(None, B)
+    _adapters(None, B)
     sl, n = _slices(None, B, [b.shape[1] for b in B], col_off)
     _dev(v, "v")
     _check(load().lora_sgmv_expand(_ptr(y), ld_y, _ptr(v), sl, n, r_max, _ptr(_dev(ranks, "ranks")),
@@ -273,14 +322,11 @@ def lora_sgmv_expand(y, v, B, col_off, ranks, scales, meta: Meta, status, stream
 
 
 def _fused(fn, y, x, A, B, col_off, ranks, scales, meta, status, stream):
+    N, r_max, n = _shapes(meta, x=x, y=y, A=A, B=B, col_off=col_off, ranks=ranks, scales=scales)
     ld_y = _rows(y, "y")
     ld_x = _rows(x, "x")
-    N, r_max = _adapters(A, B)
-    if len(A) != len(B):
-        raise LoraError("one A and one B per slice")
+    _adapters(A, B)
     sl, n = _slices(A, B, [b.shape[1] for b in B], col_off)
-    if x.dtype != y.dtype or A[0].dtype != x.dtype:
-        raise LoraError("x, y, A and B share one dtype")
     _check(fn(_ptr(y), ld_y, _ptr(x), ld_x, A[0].shape[2], sl, n, r_max, _ptr(_dev(ranks, "ranks")),
               _ptr(_dev(scales, "scales")), ctypes.byref(meta.c), _dtype_code(x), _ptr(status),
               _stream(stream)))
