@@ -93,3 +93,26 @@ def test_launches_per_step_grouping_boundaries():
     assert bench.launches_per_step(_w("decode_qproj", 8192, 1023, 16, [1])) == 2
     assert bench.launches_per_step(_w("decode_qproj", 8192, 1024, 16, [1])) == 8
     assert bench.launches_per_step(_w("decode_qproj", 8193, 8, 16, [1])) == 8
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """`bench.py --impl reference` launched the way a 2-GPU run is: rank 0 alone
+    times the oracle and prints one JSON line; the other rank exits 0 without work."""
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--ref-seconds", "1", "--cpu-budget", "1"]
+    r = subprocess.run(cmd, cwd=bench.ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["steps"] == 1
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["value"] > 0
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
