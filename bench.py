@@ -36,12 +36,14 @@ import workloads  # noqa: E402
 
 METRIC = "multi-LoRA delta tokens/s + achieved HBM GB/s (% of B200 peak), SGMV & BGMV"
 UNIT = "tokens/s"
-HEADLINE = "decode_qproj"
-SWEEP = ["prefill", "multislice_8b", "mixed_70b"]
+HEADLINE = "multislice_8b"
+SWEEP = ["decode_qproj", "prefill", "mixed_70b"]
 # Runs of at least this many rows become contiguous tiles (the tensor-core SGMV
 # kernel); 0 = gathered tiles only.  A serving engine knows whether a batch
 # holds prompts: decode-only batches are grouped without contiguous tiles.
 MIN_RUN = {"tiny": 0, "decode_qproj": 0, "multislice_8b": 0, "prefill": 64, "mixed_70b": 64}
+# Rows per gathered tile: the fused kernel reads a tile's adapter once for all of its rows.
+ROWS_PER_TILE = 64
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -63,19 +65,24 @@ def code_digest(path):
     return hashlib.sha256(text.encode()).hexdigest()
 
 
-def measured_traffic(workload):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    or None when the kernel's code has changed since that capture."""
+def measured_traffic(workload, n_layers):
+    """DRAM bytes of one step's fused-kernel launches (summed over the workload's
+    layers) from the committed ncu summaries, with the per-layer figures; None when
+    the kernel's code has changed since those captures or a layer is missing."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     src = os.path.join(ROOT, "lora_adapter_application_b200", "csrc", "bgmv.cu")
     try:
         with open(p) as f:
             rec = json.load(f)["bgmv_kernel"]
         if code_digest(src) != rec["code_sha256"]:
-            return None
-        return rec[workload]["dram_bytes_per_launch"]
+            return None, None
+        per = rec[workload]["dram_bytes_per_launch"]
+        per = per if isinstance(per, list) else [per]
+        if len(per) != n_layers:
+            return None, None
+        return float(sum(per)), per
     except (OSError, KeyError, ValueError):
-        return None
+        return None, None
 
 
 def peaks():
@@ -202,7 +209,7 @@ class DeviceSet:
         import lora_adapter_application_b200 as lora
         self.ids = w.ids.to(device)
         self.ranks = w.ranks.to(device)
-        self.scales = lora.scales_for(w.alpha, w.ranks).to(device)
+        self.alphas = lora.alphas_full(w.alpha, w.N, device)
         self.layers = []
         for l in w.layers:
             self.layers.append({"x": l.x.to(device), "y": l.y0.to(device),
@@ -219,16 +226,12 @@ class DeviceSet:
         return n
 
 
-def step(ds, ka=None, kb=None):
+def step(ds):
     import lora_adapter_application_b200 as lora
     lora.lora_build_segments(ds.ids, ds.meta, ds.status)
-    if ka is not None:
-        ka.record()
     for l in ds.layers:
-        lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks, ds.scales,
+        lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks, ds.alphas,
                              ds.meta, ds.status)
-    if kb is not None:
-        kb.record()
 
 
 def min_run_of(w):
@@ -265,40 +268,27 @@ def _event(external):
         return torch.cuda.Event(enable_timing=True)
 
 
-KERNEL_SAMPLE = 8   # a CUDA-event pair around the layer calls of every 8th timed step
-
-
-def time_device(sets, K, W, dist, graph=True, every=KERNEL_SAMPLE):
-    """Time exactly K steps on the device.  The K steps are captured into one
+def time_device(sets, K, W, dist, graph=True):
+    """Time exactly K whole steps on the device.  The K steps are captured into one
     CUDA graph and replayed once, so host launch overhead does not enter the
-    timed region; without a graph the steps are launched one by one.  Every
-    `every`-th step also records a CUDA-event pair around its layer calls (the
-    kernel time of the roofline), measured inside the same timed region; an
-    event node between two kernels lengthens that step, so the pair is not put
-    on every step."""
+    timed region; without a graph the steps are launched one by one."""
     for i in range(W):
         step(sets[i % len(sets)])
     torch.cuda.synchronize()
-    sampled = list(range(0, K, every))
-    ka = kb = g = None
+    g = None
     if graph:
         try:
-            ka = {i: _event(True) for i in sampled}
-            kb = {i: _event(True) for i in sampled}
             s = torch.cuda.Stream()
             s.wait_stream(torch.cuda.current_stream())
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 for i in range(K):
-                    step(sets[i % len(sets)], ka.get(i), kb.get(i))
+                    step(sets[i % len(sets)])
             torch.cuda.synchronize()
         except Exception as e:  # capture not available: launch eagerly
             print(f"graph capture failed ({e}); timing eager launches", file=sys.stderr)
             g = None
             torch.cuda.synchronize()
-    if g is None:
-        ka = {i: torch.cuda.Event(enable_timing=True) for i in sampled}
-        kb = {i: torch.cuda.Event(enable_timing=True) for i in sampled}
     dist.barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -308,20 +298,68 @@ def time_device(sets, K, W, dist, graph=True, every=KERNEL_SAMPLE):
         g.replay()
     else:
         for i in range(K):
-            step(sets[i % len(sets)], ka.get(i), kb.get(i))
+            step(sets[i % len(sets)])
     end.record()
     torch.cuda.synchronize()
     t1 = time.perf_counter()
     dist.barrier()
     step_ms = start.elapsed_time(end) / K
-    kern_ms = sum(ka[i].elapsed_time(kb[i]) for i in sampled) / len(sampled)
     for st in sets:
         code = int(st.status.item())
         if code:
             raise RuntimeError(f"device status {code}")
     graphed = g is not None
     del g
-    return step_ms, kern_ms, t0, t1, graphed
+    return step_ms, t0, t1, graphed
+
+
+KERNEL_STEPS = 40   # steps of the kernel-time pass (at least 20, whatever --steps is)
+
+
+def time_layers(sets, K=KERNEL_STEPS):
+    """Kernel time of the layer calls alone: every input set is grouped once, then
+    K steps of only the lora_add_linear calls are captured into one graph and timed
+    with one event pair around the whole replay (no event node between kernels, so
+    nothing lengthens a step).  The same kernels, shapes and rotating input sets as
+    the step; gaps between dependent kernels are included, so the figure is an upper
+    bound on the kernels' own time and never exceeds the step time."""
+    import lora_adapter_application_b200 as lora
+    for ds in sets:
+        lora.lora_build_segments(ds.ids, ds.meta, ds.status)
+    torch.cuda.synchronize()
+
+    def layers(ds):
+        for l in ds.layers:
+            lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks, ds.alphas,
+                                 ds.meta, ds.status)
+
+    for i in range(len(sets)):
+        layers(sets[i])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(K):
+            layers(sets[i % len(sets)])
+    g.replay()   # warm
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    del g
+    return start.elapsed_time(end) / K
+
+
+def kernel_time(sets, step_ms, K=KERNEL_STEPS):
+    """time_layers, taken again once if it came out above the step time (it cannot
+    exceed it: the step is the same work plus the grouping); None if it still does."""
+    for _ in range(2):
+        k = time_layers(sets, K)
+        if k <= step_ms:
+            return k
+    return None
 
 
 def time_e2e(w, device, K, dist, n_streams=2):
@@ -333,7 +371,7 @@ def time_e2e(w, device, K, dist, n_streams=2):
     serving loop; every step still copies its own inputs in and its result out."""
     import lora_adapter_application_b200 as lora
     n_streams = max(1, int(n_streams))
-    sets = [DeviceSet(w, device, 16, min_run_of(w)) for _ in range(n_streams)]
+    sets = [DeviceSet(w, device, ROWS_PER_TILE, min_run_of(w)) for _ in range(n_streams)]
     streams = [torch.cuda.Stream(device) for _ in range(n_streams)]
     host = {"ids": w.ids.pin_memory(),
             "layers": [{"x": l.x.pin_memory(), "y": l.y0.pin_memory()} for l in w.layers]}
@@ -352,7 +390,7 @@ def time_e2e(w, device, K, dist, n_streams=2):
             lora.lora_build_segments(ds.ids, ds.meta, ds.status, stream=st)
             for l in ds.layers:
                 lora.lora_add_linear(l["y"], l["x"], l["A"], l["B"], l["col_off"], ds.ranks,
-                                     ds.scales, ds.meta, ds.status, stream=st)
+                                     ds.alphas, ds.meta, ds.status, stream=st)
             for l, o in zip(ds.layers, out):
                 o.copy_(l["y"], non_blocking=True)
 
@@ -421,21 +459,18 @@ def bench_ours(args, dist):
     sampler.start()
 
     w = workloads.make(args.workload, seed=args.seed + 1000 * dist.rank)
-    sets, per_set = make_sets(w, device, l2, 16, min_run_of(w))
-    step_ms_local, kern_ms_local, t0, t1, graphed = time_device(sets, args.steps, args.warmup, dist,
-                                                                   not args.no_graph)
+    sets, per_set = make_sets(w, device, l2, ROWS_PER_TILE, min_run_of(w))
+    step_ms_local, t0, t1, graphed = time_device(sets, args.steps, args.warmup, dist,
+                                                 not args.no_graph)
     step_ms = dist.max(step_ms_local)
-    kern_ms = dist.max(kern_ms_local)
     tokens_total = dist.sum(w.T)
     value = tokens_total / (step_ms * 1e-3)
     clocks = sampler.summary(t0, t1)
-
-    alg_bytes = roofline.workload_bytes(w)
-    alg_flops = roofline.workload_flops(w)
-    achieved = alg_bytes / (kern_ms_local * 1e-3) / 1e9
+    kern_ms_local = kernel_time(sets, step_ms_local)
     n_sets = len(sets)
     del sets
     torch.cuda.empty_cache()
+    rl = roofline_entry(w, kern_ms_local, pk)
 
     e2e_ms, h2d, d2h = time_e2e(w, device, min(args.steps, args.e2e_steps), dist, args.e2e_streams)
 
@@ -451,14 +486,11 @@ def bench_ours(args, dist):
                          f"(inputs {n_sets * per_set / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
                    "parallelism": f"dp{dist.world} (independent batch per GPU)",
                    "launch": ("CUDA graph of the K timed steps" if graphed else "eager") +
-                             f"; kernel events on every {KERNEL_SAMPLE}th step",
+                             f"; kernel time from a separate graph of {KERNEL_STEPS} steps of "
+                             "the layer calls alone",
+                   "rows_per_tile": ROWS_PER_TILE, "min_run": min_run_of(w),
                    "seed": args.seed},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(pk["hbm_gbs"]),
-                     "unit": "GB/s", "frac": achieved / float(pk["hbm_gbs"]),
-                     "traffic": measured_traffic(w.name) if len(w.layers) == 1 else None,
-                     "kernel": "bgmv_kernel<MODE_FUSED> (lora_add_linear, gathered tiles)", "kernel_ms": kern_ms_local,
-                     "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
-                     "peak_source": f"{pk.get('source')} hbm_gbs"},
+        "roofline": rl,
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": min(args.steps, args.e2e_steps), "streams": args.e2e_streams},
@@ -481,21 +513,42 @@ def bench_ours(args, dist):
     return result
 
 
-def sweep_one(name, args, device, l2, pk, dist):
+def roofline_entry(w, kern_ms, pk):
+    """Roofline of the fused kernel's launches in one step: algorithmic bytes (x, y
+    read and written, the live ranks of every adapter touched) over the kernel time,
+    against the measured copy bandwidth; the DRAM bytes ncu counted for the same
+    launches when a capture of the current kernel code exists."""
     from lora_adapter_application_b200 import roofline
+    alg = roofline.workload_bytes(w)
+    traffic, per_layer = measured_traffic(w.name, len(w.layers))
+    peak = float(pk["hbm_gbs"])
+    out = {"bound": "hbm", "achieved": None, "peak": peak, "unit": "GB/s", "frac": None,
+           "traffic": traffic, "traffic_per_layer": per_layer,
+           "kernel": "bgmv_kernel<MODE_FUSED>" + (" + sgmv_tc_kernel<MODE_FUSED>"
+                                                  if min_run_of(w) > 0 else ""),
+           "kernel_ms": kern_ms, "algorithmic_bytes": alg,
+           "algorithmic_flops": roofline.workload_flops(w),
+           "peak_source": f"{pk.get('source')} hbm_gbs"}
+    if kern_ms:
+        out["achieved"] = alg / (kern_ms * 1e-3) / 1e9
+        out["frac"] = out["achieved"] / peak
+    return out
+
+
+def sweep_one(name, args, device, l2, pk, dist):
     w = workloads.make(name, seed=args.seed)
-    sets, per_set = make_sets(w, device, l2, 16, min_run_of(w), max_sets=4)
-    probe_ms, _, _, _, _ = time_device(sets, 3, 3, dist, graph=False)
-    K = int(min(500, max(10, args.sweep_seconds * 1e3 / probe_ms)))
-    step_ms, kern_ms, _, _, _ = time_device(sets, K, 3, dist, graph=not args.no_graph)
-    b, f = roofline.workload_bytes(w), roofline.workload_flops(w)
-    gbs = b / (kern_ms * 1e-3) / 1e9
+    sets, per_set = make_sets(w, device, l2, ROWS_PER_TILE, min_run_of(w), max_sets=4)
+    probe_ms, _, _, _ = time_device(sets, 3, 3, dist, graph=False)
+    K = int(min(500, max(20, args.sweep_seconds * 1e3 / probe_ms)))
+    step_ms, _, _, _ = time_device(sets, K, 3, dist, graph=not args.no_graph)
+    kern_ms = kernel_time(sets, step_ms)
     del sets
     torch.cuda.empty_cache()
+    rl = roofline_entry(w, kern_ms, pk)
     return {"desc": w.info.get("desc", ""), "T": w.T, "steps": K, "ms_per_step": step_ms,
-            "kernel_ms": kern_ms, "tokens_per_s": w.T / (step_ms * 1e-3),
-            "algorithmic_bytes": b, "gbs": gbs, "frac_hbm": gbs / float(pk["hbm_gbs"]),
-            "tflops": f / (kern_ms * 1e-3) / 1e12, "launches_per_step": launches_per_step(w)}
+            "tokens_per_s": w.T / (step_ms * 1e-3), "roofline": rl,
+            "frac_hbm_by_step": rl["algorithmic_bytes"] / (step_ms * 1e-3) / 1e9 / rl["peak"],
+            "launches_per_step": launches_per_step(w)}
 
 
 def bench_reference(args, dist):

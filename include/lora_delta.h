@@ -32,19 +32,26 @@
  *     LORA_FP32 (all fp32).  Rounding into y happens once, round-to-nearest-even.
  *   - Layouts are row-major with element strides:
  *         x      [T][ld_x]            d_in columns used
- *         A_s    [N][r_max][d_in]     rank rows k >= r_n are padding, never read
- *         B_s    [N][d_out_s][r_max]  rank columns k >= r_n are padding, never read
+ *         A_s    [N][r_max][d_in]     rank rows k >= r_n are padding: they may be read
+ *                                     (up to r_n rounded up to 8) but never affect the
+ *                                     result, whatever they hold (NaN included)
+ *         B_s    [N][d_out_s][r_max]  rank columns k >= r_n are padding, as for A
  *         y      [T][ld_y]            slice s owns columns col_off_s .. +d_out_s; slices
- *                                     that overlap, or run past ld_y, are LORA_ERR_SHAPE
+ *                                     that overlap, or run past ld_y, are LORA_ERR_SHAPE;
+ *                                     y must not overlap x
  *         ranks  [N] int32 device,    r_n in [1, r_max]
- *         scales [N] fp32 device,     alpha / r_n (page "Multi-LoRA Serving", 3.1)
+ *         alphas [N] fp32 device,     alpha_n of adapter n; the library scales adapter n's
+ *                                     delta by alpha_n / r_n (page "Multi-LoRA Serving",
+ *                                     3.1: y = W x + B(A x) * alpha / r), computed on the
+ *                                     device in fp32 from alphas[n] and ranks[n]
  *
  * Tuning overrides (environment, read at each call; unset = the library's own
  * choice).  They change only the launch shape: results stay within the same
  * tolerance of the exact value, and a fixed setting gives bit-identical results
  * from run to run.  A value outside the range is ignored.
- *   LORA_BG_CLUSTER     1, 2, 4 or 8: blocks per cluster of the gathered-tile kernel
- *   LORA_BG_STAGES      2 or 3: stages of the gathered-tile kernel's 72 KB load ring
+ *   LORA_BG_CLUSTER     1, 2, 4 or 8: blocks per cluster of the fused kernel's shrink
+ *   LORA_BG_STAGES      2 to 6: 32 KB stages of the fused kernel's load ring
+ *   LORA_BG_ITEM_COLS   64 to 8192, a multiple of 64: output columns of one expand item
  *   LORA_TC_CLUSTER     1, 2, 4 or 8: blocks per cluster of the tensor-core kernel;
  *                       when the shape cannot use it, the contiguous tiles run on
  *                       the gathered-tile kernel instead
@@ -52,6 +59,13 @@
  *                       when shared memory cannot hold that many stages)
  *   LORA_TC_LOAD_ROWS   8 to 128, a power of two: rows per x / y load box
  *   LORA_TC_STORE_ROWS  8 to 128, a power of two: rows per y store box
+ *
+ * Test hook (environment, read at each call; never set it in production):
+ *   LORA_DEBUG_STALL=1  the fused kernel runs one-block clusters with bounded waits
+ *                       of about 1 ms, and the first load stage of every block
+ *                       expects 16 bytes that never arrive: its waits run out,
+ *                       LORA_DEV_TIMEOUT is set, the call's results are unreliable,
+ *                       and the kernel still completes (the context stays usable).
  */
 #ifndef LORA_DELTA_H
 #define LORA_DELTA_H
@@ -86,7 +100,7 @@ typedef enum {
 #define LORA_DEV_BAD_ID        1  /* id outside [-1, N): that row is treated as -1 */
 #define LORA_DEV_TILE_OVERFLOW 2  /* tile list full: the rows of dropped tiles are untouched */
 #define LORA_DEV_BAD_RANK      4  /* ranks[n] outside [1, r_max]: rows of adapter n untouched */
-#define LORA_DEV_TIMEOUT       8  /* a bounded on-chip wait ran out: the block's rows are unreliable */
+#define LORA_DEV_TIMEOUT       8  /* a bounded wait ran out: the call's results are unreliable */
 
 typedef enum { LORA_BF16 = 0, LORA_FP32 = 1 } lora_dtype;
 
@@ -95,6 +109,7 @@ typedef enum { LORA_BF16 = 0, LORA_FP32 = 1 } lora_dtype;
 #define LORA_MAX_RANK       128  /* r_max */
 #define LORA_MAX_SLICES       8  /* output slices of one linear layer */
 #define LORA_LONG_TILE      128  /* rows per contiguous tile */
+#define LORA_MAX_TILE_ROWS   64  /* rows per gathered tile (lora_meta.rows_per_tile) */
 
 /*
  * Batch metadata: the grouping of rows by adapter id (page "Multi-LoRA
@@ -116,11 +131,13 @@ typedef enum { LORA_BF16 = 0, LORA_FP32 = 1 } lora_dtype;
  * prefill).  Runs of at least min_run rows (min_run > 0) are cut into
  * contiguous tiles of at most long_tile rows; every other row is gathered,
  * and each id's gathered rows are cut into tiles of at most rows_per_tile.
+ * The fused kernel reads a tile's adapter once for all of the tile's rows, so
+ * decode batches are best grouped with rows_per_tile = LORA_MAX_TILE_ROWS.
  */
 typedef struct {
     int32_t T;
     int32_t N;
-    int32_t rows_per_tile;      /* 1 .. 16 */
+    int32_t rows_per_tile;      /* 1 .. LORA_MAX_TILE_ROWS */
     int32_t min_run;            /* 0 = no contiguous tiles, else >= 1 */
     int32_t long_tile;          /* LORA_LONG_TILE */
     int32_t max_gather_tiles;   /* capacity, >= lora_meta_capacity() */
@@ -168,7 +185,9 @@ LORA_API int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int
  * each part rounded up to 256 bytes: per-chunk id counts (4 * (N+1) per 2048
  * rows), one byte per row, 12 bytes per 32 rows (run bitmaps and offsets) and
  * 16 bytes per 2048 rows (per-block totals).  0 when T <= 2048, or T <= 8192
- * and N <= 1023: the grouping then runs in one thread block, in shared memory. */
+ * and N <= 1023: the grouping then runs in one thread block, in shared memory.
+ * Also 0 for T outside [0, LORA_MAX_ROWS] or N outside [1, LORA_MAX_ADAPTERS]
+ * (lora_build_segments then returns LORA_ERR_SHAPE). */
 LORA_API size_t lora_segments_scratch_bytes(int32_t T, int32_t N);
 
 /*
@@ -196,10 +215,14 @@ LORA_API int lora_build_segments(const int32_t *ids, const lora_meta *meta, void
  * output buffers).  Same ids, meta and status as lora_build_segments, same
  * results; the scratch is one library-owned array of
  * LORA_STATIC_SCRATCH_BYTES bytes per device, so nothing is allocated.
- *   - Returns LORA_ERR_WORKSPACE when lora_segments_scratch_bytes(T, N)
+ *   - Returns what lora_build_segments returns for the same meta (checked
+ *     first), then LORA_ERR_WORKSPACE when lora_segments_scratch_bytes(T, N)
  *     exceeds LORA_STATIC_SCRATCH_BYTES (use lora_build_segments then).
- *   - The first call on a device (that device current) looks up the array's
- *     device address; make it before any stream capture.
+ *   - Every call (that device current) asks the CUDA runtime for the array's
+ *     device address; the first call on a device may load the library's
+ *     module there, so make one call on each device before any stream
+ *     capture.  Nothing is cached across calls, so a cudaDeviceReset between
+ *     calls leaves no stale address behind.
  *   - Every call uses the same array; calls that overlap on the GPU race and
  *     corrupt each other: keep them ordered (one stream).
  */
@@ -225,26 +248,46 @@ LORA_API int lora_sgmv_shrink(float *v, const void *x, int64_t ld_x, int32_t d_i
 /*
  * Expand and merge (page "Multi-LoRA Serving", section 3.4: add_expand,
  * delta = B v * alpha/r, grouped per adapter, added into the base output).
- * For every row i with a valid id n: y_i[col_off_s + c] += scales[n] *
+ * For every row i with a valid id n: y_i[col_off_s + c] += (alphas[n] / r_n) *
  * sum_{k < r_n} B_s[n][c][k] v[(s*T + i)*r_max + k].  v as written by
  * lora_sgmv_shrink.
  */
 LORA_API int lora_sgmv_expand(void *y, int64_t ld_y, const float *v, const lora_slice *slices,
                      int32_t n_slices, int32_t r_max, const int32_t *ranks,
-                     const float *scales, const lora_meta *meta, lora_dtype dtype,
+                     const float *alphas, const lora_meta *meta, lora_dtype dtype,
                      int32_t *status, void *stream);
 
 /*
+ * Bytes of the workspace lora_bgmv_fused and lora_add_linear take for a batch
+ * grouped into *meta and a layer of n_slices slices with rank slots r_max: a
+ * 256-byte head of control words, one int per unit of work (tile capacity of
+ * the meta), then v [n_slices][T][r_max] fp32.  0 for invalid arguments.
+ *
+ * The workspace belongs to the caller.  Its head must hold zeros before the
+ * first call that uses it (allocate it zero-filled, or cudaMemset it once);
+ * every call leaves the head at zero again when its kernel completes, so one
+ * workspace serves call after call, CUDA graph replays included.  Calls that
+ * share a workspace must not overlap on the GPU (keep them on one stream).
+ */
+LORA_API size_t lora_linear_workspace_bytes(const lora_meta *meta, int32_t n_slices, int32_t r_max);
+
+/*
  * Fused shrink + expand for every tile (BGMV: page "Multi-LoRA Serving",
- * section 3.2, SGMV/BGMV-style grouped products).  The rank-r intermediate of
- * each tile never leaves the chip: a cluster of thread blocks reduces A x
- * through distributed shared memory and expands from there.  Same result as
- * lora_sgmv_shrink followed by lora_sgmv_expand.
+ * section 3.2, SGMV/BGMV-style grouped products), in one kernel launch: a
+ * cluster of thread blocks reduces A x for all rows of a tile (up to 64 rows
+ * of one adapter) through distributed shared memory, and blocks then expand
+ * the tile's output columns in small items, each starting as soon as its tile
+ * is reduced.  v passes between the two through the workspace (it stays in
+ * L2; only x, y and the adapters' live ranks cross HBM).  Same result as
+ * lora_sgmv_shrink followed by lora_sgmv_expand.  workspace: device memory of
+ * lora_linear_workspace_bytes() bytes, 256-byte aligned (LORA_ERR_WORKSPACE
+ * otherwise; see there for its contract).
  */
 LORA_API int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
                     const lora_slice *slices, int32_t n_slices, int32_t r_max,
-                    const int32_t *ranks, const float *scales, const lora_meta *meta,
-                    lora_dtype dtype, int32_t *status, void *stream);
+                    const int32_t *ranks, const float *alphas, const lora_meta *meta,
+                    void *workspace, size_t workspace_bytes, lora_dtype dtype,
+                    int32_t *status, void *stream);
 
 /*
  * add_lora_linear (page "Multi-LoRA Serving", section 3.4: one call serves a
@@ -253,15 +296,82 @@ LORA_API int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x,
  * y in place.  Gathered tiles (decode rows) take the fused BGMV kernel;
  * contiguous tiles (prompt runs) take the tensor-core SGMV kernel when the
  * data is bf16; everything else takes the general kernel.  Same result as
- * lora_bgmv_fused.  When both kinds of tiles are present the gathered ones run
- * on a library-owned second stream, forked from and joined back into `stream`
- * with events (also under stream capture); the first such call on a device
- * creates that stream and its events, so make it before any capture.
+ * lora_bgmv_fused; the same workspace contract.  When both kinds of tiles are
+ * present the gathered ones run on a library-owned second stream, forked from
+ * and joined back into `stream` with events (also under stream capture); each
+ * caller stream gets a second stream of its own, created by the first such
+ * call on that stream, so make that call before capturing the stream.
  */
 LORA_API int lora_add_linear(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
                     const lora_slice *slices, int32_t n_slices, int32_t r_max,
-                    const int32_t *ranks, const float *scales, const lora_meta *meta,
-                    lora_dtype dtype, int32_t *status, void *stream);
+                    const int32_t *ranks, const float *alphas, const lora_meta *meta,
+                    void *workspace, size_t workspace_bytes, lora_dtype dtype,
+                    int32_t *status, void *stream);
+
+
+/*
+ * Adapter slots (page "LoRA hot load and adapter routing", adapter lifecycle:
+ * load, check the rank, copy to the GPU, evict the least recently used adapter
+ * when the slots are full; page "Multi-LoRA Serving", section 3.2: max_loras
+ * adapters resident, max_lora_rank the slot size).
+ *
+ * lora_load_adapter: put one adapter of rank r into slot n of every slice's
+ * stacked tensors, on `stream`:
+ *     A_s[n][0:r][:]     = src_A[s]  ([r][d_in] row-major)
+ *     A_s[n][r:r_max][:] = 0
+ *     B_s[n][:][0:r]     = src_B[s]  ([d_out_s][r] row-major)
+ *     B_s[n][:][r:r_max] = 0
+ *     ranks[n] = r, alphas[n] = alpha   (device words, written by a kernel)
+ * slices[s].A / .B are the stacks ([N][r_max][d_in], [N][d_out_s][r_max]);
+ * col_off is not used.  src_A[s] / src_B[s] may be device memory or pinned
+ * host memory (the copy engines read them); they must stay valid until the
+ * stream reaches the call.  Everything is enqueued on the stream: batches
+ * enqueued after it on that stream see the new adapter, batches enqueued before
+ * it see the old one.  Returns LORA_ERR_RANK for r outside [1, r_max],
+ * LORA_ERR_SHAPE for n outside [0, N).
+ */
+LORA_API int lora_load_adapter(const lora_slice *slices, int32_t n_slices, int32_t d_in,
+                               int32_t r_max, int32_t N, int32_t n, int32_t r,
+                               const void *const *src_A, const void *const *src_B, float alpha,
+                               int32_t *ranks, float *alphas, lora_dtype dtype, void *stream);
+
+/*
+ * Host policy for the slots: which slot holds which adapter (a caller-chosen
+ * key >= 0), least recently used first out.  Thread-safe; host memory only.
+ *   acquire  the adapter's slot and one pin on it.  *resident = 1: the slot
+ *            already holds the adapter; 0: the slot was given to it (a free slot
+ *            first, else the least recently acquired slot with no pins) and the
+ *            caller must load it (lora_load_adapter).  LORA_ERR_CAPACITY when
+ *            every slot is pinned.
+ *   release  one pin (a batch that read the slot has completed).
+ *   key      the key a slot holds, -1 if free.
+ *   evict    free the adapter's slot (LORA_ERR_CAPACITY while pinned).
+ */
+typedef struct lora_slot_cache lora_slot_cache;
+LORA_API lora_slot_cache *lora_slot_cache_create(int32_t n_slots);
+LORA_API void lora_slot_cache_destroy(lora_slot_cache *cache);
+LORA_API int lora_slot_cache_acquire(lora_slot_cache *cache, int64_t key, int32_t *slot,
+                                     int32_t *resident);
+LORA_API int lora_slot_cache_release(lora_slot_cache *cache, int32_t slot);
+LORA_API int64_t lora_slot_cache_key(lora_slot_cache *cache, int32_t slot);
+LORA_API int lora_slot_cache_evict(lora_slot_cache *cache, int64_t key);
+
+/*
+ * Merge / unmerge one adapter into a dense base weight (page "LoRA service:
+ * multi-adapter dynamic loading", section 1: W' = W + B A for a single-tenant
+ * deployment, with the scale alpha / r of page "Multi-LoRA Serving", 3.1):
+ *     W[o][i] += sign * (alphas[n] / r_n) * sum_{k < r_n} B[n][o][k] A[n][k][i]
+ * for o < d_out, i < d_in.  W: device [d_out][ld_w] (row o = output feature o,
+ * as in y = W x); A [N][r_max][d_in] and B [N][d_out][r_max]: one slice's
+ * stacks; n: the slot; sign: +1 merges, -1 unmerges.  fp32 products and
+ * accumulation, W rounded once (round-to-nearest-even); unmerging a merged
+ * adapter restores W up to that rounding.  ranks[n] outside [1, r_max] sets
+ * LORA_DEV_BAD_RANK and leaves W unchanged.  Padding ranks never affect W.
+ */
+LORA_API int lora_merge_adapter(void *W, int64_t ld_w, int32_t d_out, int32_t d_in, const void *A,
+                                const void *B, int32_t N, int32_t r_max, int32_t n,
+                                const int32_t *ranks, const float *alphas, int32_t sign,
+                                lora_dtype dtype, int32_t *status, void *stream);
 
 #ifdef __cplusplus
 }

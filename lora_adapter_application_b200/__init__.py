@@ -11,9 +11,10 @@ What is computed (page "Multi-LoRA Serving: one base, many adapters", section
 3.1 and 3.4; page "LoRA service: multi-adapter dynamic loading", section 2):
 for every row i with adapter n = ids[i] != -1,
 
-    y_i[col_off_s : col_off_s + d_out_s] += scales[n] * B_s[n] (A_s[n] x_i)
+    y_i[col_off_s : col_off_s + d_out_s] += (alphas[n] / r_n) * B_s[n] (A_s[n] x_i)
 
-with scales[n] = alpha / r_n and only the first r_n rank rows/columns used.
+with only the first r_n rank rows/columns used; the library computes the
+scale alphas[n] / r_n on the device from the two per-slot tensors.
 """
 from __future__ import annotations
 
@@ -25,8 +26,11 @@ import torch
 __all__ = [
     "load", "LoraError", "Meta", "LORA_BF16", "LORA_FP32", "DEV_BAD_ID", "DEV_TILE_OVERFLOW",
     "DEV_BAD_RANK", "lora_version", "lora_last_error", "lora_meta_capacity", "lora_segments_scratch_bytes",
-    "lora_build_segments", "lora_build_segments_static", "lora_shrink_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand",
-    "lora_bgmv_fused", "lora_add_linear", "scales_for",
+    "lora_build_segments", "lora_build_segments_static", "lora_shrink_workspace_bytes",
+    "lora_linear_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_bgmv_fused",
+    "lora_add_linear", "alphas_full", "lora_load_adapter", "SlotCache", "lora_slot_cache_create",
+    "lora_slot_cache_destroy", "lora_slot_cache_acquire", "lora_slot_cache_release",
+    "lora_slot_cache_key", "lora_slot_cache_evict", "lora_merge_adapter",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +40,7 @@ LORA_BF16, LORA_FP32 = 0, 1
 DEV_BAD_ID, DEV_TILE_OVERFLOW, DEV_BAD_RANK, DEV_TIMEOUT = 1, 2, 4, 8
 ERR_CUDA = -8   # LORA_ERR_CUDA
 MAX_ROWS, MAX_ADAPTERS, MAX_RANK, MAX_SLICES, LONG_TILE = 131072, 4096, 128, 8, 128
+MAX_TILE_ROWS = 64
 
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 
@@ -67,14 +72,28 @@ _SIGS = {
     "lora_build_segments": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _SZ, _P, _P]),
     "lora_build_segments_static": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _P]),
     "lora_shrink_workspace_bytes": (_SZ, [_I32, _I32, _I32]),
+    "lora_linear_workspace_bytes": (_SZ, [ctypes.POINTER(lora_meta), _I32, _I32]),
     "lora_sgmv_shrink": (ctypes.c_int, [_P, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32, _I32,
                                         _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
     "lora_sgmv_expand": (ctypes.c_int, [_P, _I64, _P, ctypes.POINTER(lora_slice), _I32, _I32, _P, _P,
                                         ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
     "lora_bgmv_fused": (ctypes.c_int, [_P, _I64, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32,
-                                       _I32, _P, _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
+                                       _I32, _P, _P, ctypes.POINTER(lora_meta), _P, _SZ, ctypes.c_int,
+                                       _P, _P]),
     "lora_add_linear": (ctypes.c_int, [_P, _I64, _P, _I64, _I32, ctypes.POINTER(lora_slice), _I32,
-                                       _I32, _P, _P, ctypes.POINTER(lora_meta), ctypes.c_int, _P, _P]),
+                                       _I32, _P, _P, ctypes.POINTER(lora_meta), _P, _SZ, ctypes.c_int,
+                                       _P, _P]),
+    "lora_load_adapter": (ctypes.c_int, [ctypes.POINTER(lora_slice), _I32, _I32, _I32, _I32, _I32,
+                                         _I32, ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                         ctypes.c_float, _P, _P, ctypes.c_int, _P]),
+    "lora_merge_adapter": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _I32, _I32, _I32, _P, _P,
+                                          _I32, ctypes.c_int, _P, _P]),
+    "lora_slot_cache_create": (_P, [_I32]),
+    "lora_slot_cache_destroy": (None, [_P]),
+    "lora_slot_cache_acquire": (ctypes.c_int, [_P, _I64, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
+    "lora_slot_cache_release": (ctypes.c_int, [_P, _I32]),
+    "lora_slot_cache_key": (_I64, [_P, _I32]),
+    "lora_slot_cache_evict": (ctypes.c_int, [_P, _I64]),
 }
 
 
@@ -142,7 +161,7 @@ def lora_version():
     return int(load().lora_version())
 
 
-def lora_meta_capacity(T, N, rows_per_tile=16, min_run=64, long_tile=LONG_TILE):
+def lora_meta_capacity(T, N, rows_per_tile=MAX_TILE_ROWS, min_run=64, long_tile=LONG_TILE):
     mg, mc = _I32(), _I32()
     _check(load().lora_meta_capacity(T, N, rows_per_tile, min_run, long_tile, ctypes.byref(mg),
                                      ctypes.byref(mc)))
@@ -170,12 +189,18 @@ def lora_shrink_workspace_bytes(T, r_max, n_slices):
     return int(load().lora_shrink_workspace_bytes(T, r_max, n_slices))
 
 
+def lora_linear_workspace_bytes(meta, n_slices, r_max):
+    return int(load().lora_linear_workspace_bytes(ctypes.byref(meta.c), n_slices, r_max))
+
+
 class Meta:
     """Device buffers of a batch's lora_meta, allocated with torch, plus the
-    builder's scratch.  ``rows_per_tile`` caps a gathered tile; ``min_run``
-    (0 = off) is the shortest run of one id that becomes contiguous tiles."""
+    builder's scratch and the fused calls' workspace.  ``rows_per_tile`` caps a
+    gathered tile; ``min_run`` (0 = off) is the shortest run of one id that
+    becomes contiguous tiles."""
 
-    def __init__(self, T, N, rows_per_tile=16, min_run=64, long_tile=LONG_TILE, device="cuda"):
+    def __init__(self, T, N, rows_per_tile=MAX_TILE_ROWS, min_run=64, long_tile=LONG_TILE,
+                 device="cuda"):
         mg, mc = lora_meta_capacity(T, N, rows_per_tile, min_run, long_tile)
         i32 = dict(dtype=torch.int32, device=device)
         self.T, self.N = T, N
@@ -194,6 +219,18 @@ class Meta:
                            self.seg_adapter.data_ptr(), self.counts.data_ptr(),
                            self.grow.data_ptr(), self.gather_tiles.data_ptr(),
                            self.contig_tiles.data_ptr())
+        self.device = device
+        self._ws = None
+
+    def workspace(self, n_slices, r_max):
+        """The fused calls' workspace for a layer of n_slices slices and rank slots
+        r_max: one zero-filled buffer per Meta, grown when a layer needs more (the
+        library keeps its head at zero from call to call).  Calls that use one
+        Meta's workspace must not overlap on the GPU."""
+        need = lora_linear_workspace_bytes(self, n_slices, r_max)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
 
     def host(self):
         """Copy the metadata to the host (synchronises)."""
@@ -232,7 +269,7 @@ def _slices(A, B, d_out, col_off):
     return arr, n
 
 
-def _shapes(meta, x=None, y=None, A=None, B=None, col_off=None, ranks=None, scales=None,
+def _shapes(meta, x=None, y=None, A=None, B=None, col_off=None, ranks=None, alphas=None,
             v=None):
     """Shape, dtype and layout agreement of a call's operands (the library sees
     only pointers, so a mismatch here would be an out-of-bounds read there).
@@ -277,7 +314,7 @@ def _shapes(meta, x=None, y=None, A=None, B=None, col_off=None, ranks=None, scal
             for b, c in zip(B, col_off):
                 if int(c) < 0 or int(c) + b.shape[1] > y.shape[1]:
                     raise LoraError("a slice's columns run past y")
-    for t, what, dt in ((ranks, "ranks", torch.int32), (scales, "scales", torch.float32)):
+    for t, what, dt in ((ranks, "ranks", torch.int32), (alphas, "alphas", torch.float32)):
         if t is not None and (not isinstance(t, torch.Tensor) or t.dtype != dt or
                               not t.is_contiguous() or t.numel() < meta.N):
             raise LoraError(f"{what} must be a contiguous {dt} tensor of at least N entries")
@@ -292,9 +329,9 @@ def _adapters(A, B):
         _dev(t, "adapter tensor")
 
 
-def scales_for(alpha, ranks):
-    """alpha / r_n per adapter slot (page "Multi-LoRA Serving", section 3.1), fp32."""
-    return (float(alpha) / ranks.to(torch.float64)).to(torch.float32)
+def alphas_full(alpha, N, device="cuda"):
+    """One alpha for all N adapter slots, as the fp32 [N] tensor the calls take."""
+    return torch.full((N,), float(alpha), dtype=torch.float32, device=device)
 
 
 def lora_sgmv_shrink(v, x, A, ranks, meta: Meta, status, stream=None):
@@ -309,34 +346,144 @@ def lora_sgmv_shrink(v, x, A, ranks, meta: Meta, status, stream=None):
                                    _ptr(status), _stream(stream)))
 
 
-def lora_sgmv_expand(y, v, B, col_off, ranks, scales, meta: Meta, status, stream=None):
-    """y[i, col_off_s + c] += scales[n] sum_k B[s][n, c, k] v[s, i, k]."""
-    N, r_max, n = _shapes(meta, y=y, B=B, col_off=col_off, ranks=ranks, scales=scales, v=v)
+def lora_sgmv_expand(y, v, B, col_off, ranks, alphas, meta: Meta, status, stream=None):
+    """y[i, col_off_s + c] += (alphas[n] / r_n) sum_k B[s][n, c, k] v[s, i, k]."""
+    N, r_max, n = _shapes(meta, y=y, B=B, col_off=col_off, ranks=ranks, alphas=alphas, v=v)
     ld_y = _rows(y, "y")
     _adapters(None, B)
     sl, n = _slices(None, B, [b.shape[1] for b in B], col_off)
     _dev(v, "v")
     _check(load().lora_sgmv_expand(_ptr(y), ld_y, _ptr(v), sl, n, r_max, _ptr(_dev(ranks, "ranks")),
-                                   _ptr(_dev(scales, "scales")), ctypes.byref(meta.c),
+                                   _ptr(_dev(alphas, "alphas")), ctypes.byref(meta.c),
                                    _dtype_code(y), _ptr(status), _stream(stream)))
 
 
-def _fused(fn, y, x, A, B, col_off, ranks, scales, meta, status, stream):
-    N, r_max, n = _shapes(meta, x=x, y=y, A=A, B=B, col_off=col_off, ranks=ranks, scales=scales)
+def _fused(fn, y, x, A, B, col_off, ranks, alphas, meta, status, stream, workspace):
+    N, r_max, n = _shapes(meta, x=x, y=y, A=A, B=B, col_off=col_off, ranks=ranks, alphas=alphas)
     ld_y = _rows(y, "y")
     ld_x = _rows(x, "x")
     _adapters(A, B)
     sl, n = _slices(A, B, [b.shape[1] for b in B], col_off)
+    ws = meta.workspace(n, r_max) if workspace is None else _dev(workspace, "workspace")
     _check(fn(_ptr(y), ld_y, _ptr(x), ld_x, A[0].shape[2], sl, n, r_max, _ptr(_dev(ranks, "ranks")),
-              _ptr(_dev(scales, "scales")), ctypes.byref(meta.c), _dtype_code(x), _ptr(status),
-              _stream(stream)))
+              _ptr(_dev(alphas, "alphas")), ctypes.byref(meta.c), _ptr(ws),
+              ws.numel() * ws.element_size(), _dtype_code(x), _ptr(status), _stream(stream)))
 
 
-def lora_bgmv_fused(y, x, A, B, col_off, ranks, scales, meta: Meta, status, stream=None):
-    """Fused shrink + expand of every tile (rank-r intermediate kept on chip)."""
-    _fused(load().lora_bgmv_fused, y, x, A, B, col_off, ranks, scales, meta, status, stream)
+def lora_bgmv_fused(y, x, A, B, col_off, ranks, alphas, meta: Meta, status, stream=None,
+                    workspace=None):
+    """Fused shrink + expand of every tile in one launch."""
+    _fused(load().lora_bgmv_fused, y, x, A, B, col_off, ranks, alphas, meta, status, stream,
+           workspace)
 
 
-def lora_add_linear(y, x, A, B, col_off, ranks, scales, meta: Meta, status, stream=None):
-    """All slices of one linear layer applied to y in place (add_lora_linear)."""
-    _fused(load().lora_add_linear, y, x, A, B, col_off, ranks, scales, meta, status, stream)
+def lora_add_linear(y, x, A, B, col_off, ranks, alphas, meta: Meta, status, stream=None,
+                    workspace=None):
+    """All slices of one linear layer applied to y in place (add_lora_linear).
+    ``workspace`` (optional): a zero-filled uint8 CUDA tensor of at least
+    lora_linear_workspace_bytes bytes; by default the Meta's own."""
+    _fused(load().lora_add_linear, y, x, A, B, col_off, ranks, alphas, meta, status, stream,
+           workspace)
+
+
+# ---------------------------------------------------------------- adapter slots
+def lora_load_adapter(A, B, n, src_A, src_B, alpha, ranks, alphas, stream=None):
+    """Copy one adapter (src_A[s] [r, d_in], src_B[s] [d_out_s, r], device or pinned
+    host tensors) into slot n of the stacks A[s] [N, r_max, d_in], B[s] [N, d_out_s,
+    r_max], zeroing the rank padding, and set ranks[n] = r, alphas[n] = alpha."""
+    if len(A) != len(B) or len(src_A) != len(A) or len(src_B) != len(B):
+        raise LoraError("one source A and B per slice")
+    N, r_max, d_in = A[0].shape
+    r = src_A[0].shape[0]
+    for a, b, sa, sb in zip(A, B, src_A, src_B):
+        _dev(a, "A")
+        _dev(b, "B")
+        if a.shape != (N, r_max, d_in) or b.shape[0] != N or b.shape[2] != r_max:
+            raise LoraError("stacks of one N, r_max, d_in")
+        if sa.shape != (r, d_in) or sb.shape != (b.shape[1], r):
+            raise LoraError("sources are [r, d_in] and [d_out_s, r]")
+        if not (sa.is_contiguous() and sb.is_contiguous()) or sa.dtype != a.dtype or sb.dtype != a.dtype:
+            raise LoraError("contiguous sources of the stacks' dtype")
+        if sa.device.type == "cpu" and not (sa.is_pinned() and sb.is_pinned()):
+            raise LoraError("host sources must be pinned")
+    sl, S = _slices(A, B, [b.shape[1] for b in B], [0] * len(B))
+    pa = (_P * S)(*[t.data_ptr() for t in src_A])
+    pb = (_P * S)(*[t.data_ptr() for t in src_B])
+    _check(load().lora_load_adapter(sl, S, d_in, r_max, N, int(n), int(r), pa, pb, float(alpha),
+                                    _ptr(_dev(ranks, "ranks")), _ptr(_dev(alphas, "alphas")),
+                                    _dtype_code(A[0]), _stream(stream)))
+
+
+def lora_slot_cache_create(n_slots):
+    return load().lora_slot_cache_create(int(n_slots))
+
+
+def lora_slot_cache_destroy(cache):
+    load().lora_slot_cache_destroy(cache)
+
+
+def lora_slot_cache_acquire(cache, key):
+    slot, resident = _I32(), _I32()
+    _check(load().lora_slot_cache_acquire(cache, int(key), ctypes.byref(slot), ctypes.byref(resident)))
+    return slot.value, bool(resident.value)
+
+
+def lora_slot_cache_release(cache, slot):
+    _check(load().lora_slot_cache_release(cache, int(slot)))
+
+
+def lora_slot_cache_key(cache, slot):
+    return int(load().lora_slot_cache_key(cache, int(slot)))
+
+
+def lora_slot_cache_evict(cache, key):
+    _check(load().lora_slot_cache_evict(cache, int(key)))
+
+
+class SlotCache:
+    """The library's LRU slot policy (lora_slot_cache_*), owned by this object."""
+
+    def __init__(self, n_slots):
+        self.h = lora_slot_cache_create(n_slots)
+        if not self.h:
+            raise LoraError("n_slots must be in [1, 4096]")
+        self.n_slots = n_slots
+
+    def acquire(self, key):
+        return lora_slot_cache_acquire(self.h, key)
+
+    def release(self, slot):
+        lora_slot_cache_release(self.h, slot)
+
+    def key(self, slot):
+        return lora_slot_cache_key(self.h, slot)
+
+    def evict(self, key):
+        lora_slot_cache_evict(self.h, key)
+
+    def __del__(self):
+        if getattr(self, "h", None) and _lib is not None:
+            lora_slot_cache_destroy(self.h)
+            self.h = None
+
+
+# ---------------------------------------------------------------- merge / unmerge
+def lora_merge_adapter(W, A, B, n, ranks, alphas, status, sign=1, stream=None):
+    """W += sign * (alphas[n] / r_n) * B[n] @ A[n] in place (one slice's stacks
+    A [N, r_max, d_in], B [N, d_out, r_max]; W [d_out, >= d_in])."""
+    ld_w = _rows(W, "W")
+    _dev(A, "A")
+    _dev(B, "B")
+    N, r_max, d_in = A.shape
+    if B.dim() != 3 or B.shape[0] != N or B.shape[2] != r_max or not (A.is_contiguous() and B.is_contiguous()):
+        raise LoraError("A [N, r_max, d_in] and B [N, d_out, r_max], contiguous")
+    d_out = B.shape[1]
+    if W.shape[0] < d_out or W.shape[1] < d_in or W.dtype != A.dtype or B.dtype != A.dtype:
+        raise LoraError("W is [d_out, >= d_in] of the adapters' dtype")
+    for t, what, dt in ((ranks, "ranks", torch.int32), (alphas, "alphas", torch.float32)):
+        if t.dtype != dt or t.numel() < N:
+            raise LoraError(f"{what} must be {dt} with N entries")
+    _check(load().lora_merge_adapter(_ptr(W), ld_w, d_out, d_in, _ptr(A), _ptr(B), N, r_max, int(n),
+                                     _ptr(_dev(ranks, "ranks")), _ptr(_dev(alphas, "alphas")),
+                                     int(sign), _dtype_code(W), _ptr(_dev(status, "status")),
+                                     _stream(stream)))

@@ -1,74 +1,100 @@
-// Fused decode BGMV (page "Multi-LoRA Serving", section 3.2: BGMV-style
-// grouped products; section 3.4: add_shrink then add_expand, grouped per
-// adapter) for bf16, ranks up to 64.
+// Fused multi-LoRA BGMV over gathered rows, bf16, ranks up to 64 (page
+// "Multi-LoRA Serving", section 3.2: rows grouped per adapter, BGMV-style
+// grouped products; section 3.4: add_shrink then add_expand in one call).
 //
-// One unit of work = up to 16 rows that share an adapter (a gathered tile, or
-// 16 rows of a contiguous tile).  A cluster of C thread blocks takes a unit;
-// block c owns 1/C of the input columns (shrink) and 1/C of the output
-// columns (expand).  Clusters are persistent: cluster k walks the units k,
-// k + #clusters, ... of those counted on the device.  Each block is
-// warp-specialised:
+// Unit of work = up to 64 rows that share an adapter (a gathered tile, or a
+// piece of a contiguous tile).  All rows of a unit share one stream of the
+// adapter's A and B, so an adapter with up to 64 rows in the batch is read
+// from HBM once.  One persistent launch runs two phases:
 //
-//   producer warp   walks the block's chunk stream and fills a 72 KB
-//                   shared-memory ring (3 or 2 stages) through the TMA engine: 2-D tensor
-//                   copies of 1-2 KB boxes for the adapters (A: 8 or 16 ranks
-//                   x 64 columns, 128-byte swizzle; B: 64 output columns x 8
-//                   or 16 ranks) and one 1-D bulk copy per gathered x or y
-//                   row piece.  (Measured on B200: TMA copies leave the
-//                   load/store pipe to the consumers, where a cp.async
-//                   producer competes with their shared-memory traffic; TMA
-//                   pays per copy, so copies should be 1 KB or more.)  A
-//                   full/empty mbarrier pair guards each stage.
-//   8 consumer warps
-//     shrink chunks  x rows [cnt][JC] and A rows [r_n][JC] -> partial v
-//                    (tensor-core mma m16n8k16, bf16 in, fp32 accumulate)
-//     exchange       through distributed shared memory, stores only: every
-//                    block sends each partial element to the block that owns
-//                    it; the owner adds the C partials in a fixed order
-//                    (run-to-run identical), scales by alpha/r_n and stores the
-//                    result into every block's copy of v; the stores are
-//                    st.async, counted in bytes on the receiver's mbarrier, so
-//                    neither side needs a cluster-scope fence
-//     expand chunks  B rows [CC][r_n] and y rows [cnt][CC] -> y += (s v) B^T in
-//                    fp32, rounded once, written back with 16-byte stores
+//   shrink   a cluster of C thread blocks takes a unit; block c reduces 1/C
+//            of the input columns: v_part[rows][S*r8] = x[rows][cols] .
+//            A_s[n][0:r8][cols]^T (tensor-pipe mma m16n8k16, bf16 in, fp32
+//            accumulate).  The C partials meet in distributed shared memory
+//            (st.async stores counted in bytes on the owner's mbarrier; the
+//            owner adds them in rank order, so results are run-to-run
+//            identical) and the owners write v = A x (fp32) for k < r_n.
+//   expand   every block on its own takes an expand item = (unit, slice,
+//            block of output columns): y[rows][cols] += (alpha_n / r_n) v .
+//            B_s[n][cols][0:r8]^T, fp32 accumulation, y rounded once.
 //
-// The producer runs a ring's worth of chunks ahead, across the exchange, so HBM stays
-// busy; every byte of x, A, B and y crosses HBM once and v never leaves the
-// chip.  s v enters the expand products as a bf16 hi + lo pair (about 16
-// mantissa bits): a single bf16 copy (2^-9 relative) is not enough when the
-// delta is large and cancels against y.  The multiply-adds (about 4 per byte)
-// run on the tensor pipe.  Large batches are bounded by HBM bandwidth; a
-// small decode batch is latency-bound: each unit is a chain of dependent
-// loads, the exchange and the expand, a few microseconds each.
+// In the fused mode v moves between the phases through a caller-provided
+// workspace: the shrink owners write it, and an expand item of unit u starts
+// its v copy once u's C blocks have signalled (a per-unit counter, release /
+// acquire at GPU scope).  Its bytes stay in L2 (about 2 KB per row); the
+// adapters and the rows cross HBM once.  Shrink units are taken by clusters
+// and expand items by blocks from atomic tickets, so a block only ever waits
+// for units that a running cluster already holds: the launch makes progress
+// whatever number of its blocks is resident (and beside other kernels).  The
+// tickets, the per-unit counters and an exit counter live at the head of the
+// workspace; the last block to leave puts them back to zero.  The shrink-only
+// and expand-only modes (v from / to the caller) assign work statically and
+// need no workspace.
 //
-// Inside one 16-wide K step each thread assigns 4 consecutive elements of each
-// operand row to its four k-slots of the mma fragment; both operands use the
-// same assignment, so the sum is unchanged and shared-memory reads are vectors.
+// Block layout (288 threads, one block per SM):
+//   warp 8        producer: walks the block's work and fills a ring of
+//                 GB_STAGES x 32 KB stages through the TMA engine - A boxes
+//                 of 8-64 ranks x 64 columns (128-byte swizzle), B boxes of 64
+//                 output columns x 8-64 ranks (swizzle matched to the box
+//                 width), one 1-D bulk copy per gathered x / y / v row piece.
+//                 Each stage carries a header (what the chunk is, its rows)
+//                 written before the stage's arrival; a full/empty mbarrier
+//                 pair guards each stage.
+//   warps 0-7     consumers: follow the headers; shrink chunks -> mma into
+//                 registers, the last chunk of a pass -> exchange; expand
+//                 chunks -> mma with s v as a bf16 hi + lo pair (about 16
+//                 mantissa bits), y updated in shared memory and written back
+//                 with 16-byte stores.
+// Box sizes follow the adapter's own rank (r8 = r_n rounded up to 8), not the
+// slot size r_max: rank rows / columns r8..r_max are never loaded; ranks
+// r_n..r8 are loaded and masked out of every product.
 //
 // Every wait is bounded (a suspend-time hint per try, and a try limit): a wait
-// that runs out sets LORA_DEV_TIMEOUT in the status word and the block skips
-// its remaining work instead of hanging.
+// that runs out sets LORA_DEV_TIMEOUT in the status word and the block stops
+// taking work; consumer threads agree on every outcome through a barrier
+// reduction, so no named barrier is left unpaired.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
-#include <cooperative_groups.h>
-
 #include <cstdlib>
-
 #include <mutex>
-
-namespace cg = cooperative_groups;
 
 namespace lora {
 
-constexpr int BG_CONSUMERS = 8;                      // consumer warps
-constexpr int BG_THREADS = (BG_CONSUMERS + 1) * 32;  // + 1 producer warp
-constexpr int BG_ROWS = 16;
-constexpr int BG_RMAX = 64;
-constexpr int BG_MAX_STAGES = 3;                    // mbarrier pairs reserved
-constexpr int BG_RING_BYTES = 73728;                // 3 x 24 KB or 2 x 36 KB (1 KB multiples)
-constexpr int BG_VF_STRIDE = 80;   // floats per row of the reduced v (bank spread)
+constexpr int GB_CONSUMERS = 8;                      // consumer warps
+constexpr int GB_THREADS = (GB_CONSUMERS + 1) * 32;  // + 1 producer warp
+constexpr int GB_ROWS = LORA_MAX_TILE_ROWS;          // rows of one unit
+constexpr int GB_MAX_STAGES = 6;
+constexpr int GB_STAGES_DEFAULT = 4;
+constexpr int GB_SB = 32768;                         // bytes of one ring stage
+constexpr int GB_HDR = 384;                          // bytes of one stage header
+constexpr int GB_XCAP = 8192;                        // partial elements of one exchange
+constexpr int GB_XBUF = GB_XCAP + 64;                // floats of one exchange buffer
+constexpr int GB_PART = 1024;                        // floats of the k-group staging
+constexpr int GB_TK = 8;                             // shrink tickets in flight per cluster
 
+enum { GB_SHRINK = 0, GB_EXPAND = 1, GB_END = 2 };
+enum { GB_FIRST = 1, GB_LAST = 2, GB_NODATA = 4, GB_UNIT_DONE = 8 };
+
+// What one ring stage holds, written by the producer before the stage's arrival.
+struct GbHdr {
+    int kind, flags;
+    int unit, n, r_n, r8, cnt;   // unit, adapter, rank, rank rounded to 8, rows
+    int s0, sn;                  // shrink: slices [s0, s0+sn) of this chunk; expand: slice s0
+    int c0, w;                   // shrink: first input column, width; expand: slice-local column, width
+    int cw;                      // chunk width: rows sit at 2*cw+16 bytes
+    int bofs;                    // byte offset of the adapter boxes (shrink: A, expand: B)
+    int yofs;                    // expand: byte offset of the y rows (v rows sit at 0)
+    float scale;                 // expand: alpha_n / r_n
+    int pad;
+    int rows[GB_ROWS];
+};
+static_assert(sizeof(GbHdr) <= GB_HDR, "stage header");
+
+// Workspace head of the fused mode (ints): tickets and exit counter, then one
+// counter per unit.
+constexpr int GB_CTL_INTS = 64;
+enum { GB_T_SHRINK = 0, GB_T_EXPAND = 1, GB_T_EXIT = 2 };
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -79,524 +105,876 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-
 __device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;\n" ::"n"(BG_CONSUMERS * 32) : "memory");
+    asm volatile("bar.sync 1, %0;\n" ::"n"(GB_CONSUMERS * 32) : "memory");
 }
-
+// every consumer thread passes p; returns the AND over all of them
+__device__ __forceinline__ bool consumers_all(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, o;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred o, 1, %2, q;\n\tselp.u32 %0, 1, 0, o;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)p), "n"(GB_CONSUMERS * 32)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n"
+                 "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
 __device__ __forceinline__ uint4 zero_if(bool z, uint4 v) { return z ? make_uint4(0, 0, 0, 0) : v; }
-
-// Shared memory: ring | recv [S*16*64] | vfull [S][16][80] | part [16][64] | barriers
-//   recv[c*(S*1024/C) + e/C] holds block c's partial of element e = (s*16+row)*64+k,
-//   for the elements e with e % C == this block's rank.
-size_t bgmv_smem_bytes(int n_slices) {
-    return 1024 /* alignment of the ring to the 128-byte swizzle atom */ +
-           (size_t)BG_RING_BYTES + (size_t)n_slices * BG_ROWS * BG_RMAX * 4 +
-           (size_t)n_slices * BG_ROWS * BG_VF_STRIDE * 4 + (size_t)BG_ROWS * BG_RMAX * 4 + 128;
+// 8 bytes into the shared memory of a block of the cluster, completing 8
+// transaction bytes on that block's mbarrier (no fence on either side)
+__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1,%2}, [%3];\n" ::"r"(addr),
+        "f"(a), "f"(b), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];\n" ::"r"(addr),
+                 "r"(v), "r"(bar)
+                 : "memory");
+}
+// one arrival on an mbarrier of another block of the cluster
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(remote_bar)
+                 : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+    float4 r;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "r"(a));
+    return r;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t a) {
+    float2 r;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];\n" : "=f"(r.x), "=f"(r.y) : "r"(a));
+    return r;
 }
 
-struct Geo {          // chunk geometry of one block for one unit
-    int r8, nb8, nkb16;
-    int j_lo, j_hi, JC, RS, A0, n_sc;    // shrink: columns, chunk width, x row stride, A boxes offset, chunks/slice
-    int c_lo, c_hi, CC, YS, B0;          // expand: concatenated column range, chunk width, y row stride, B boxes offset
-    int n_shrink, n_chunks;
-};
+__device__ __forceinline__ int align_up(int v, int a) { return (v + a - 1) & ~(a - 1); }
 
-// Shared-memory bytes of a chunk `cols` columns wide: 16 bf16 rows of x or y
-// (padded by 16 bytes, 1 KB aligned), then the adapter boxes, which hold per
-// 64 columns one 1 KB box per 8 ranks, or one 2 KB box per 16 ranks (ab16).
-__device__ __forceinline__ int chunk_bytes(int cols, int nb8, bool ab16) {
-    const int box_kb = ab16 ? 2 * ((nb8 + 1) >> 1) : nb8;   // per 64 columns
-    return ((BG_ROWS * (cols * 2 + 16) + 1023) & ~1023) + box_kb * (cols >> 6) * 1024;
+// Byte offset of (output column col, rank k) in the B boxes of an expand
+// chunk.  Per 64 columns: 128*r8 bytes.  r8 a power of two: one box of 64 rows
+// x r8 ranks, rows of 2*r8 bytes, swizzled in 16-byte units by the row bits
+// above 128 bytes (the TMA 32/64/128-byte swizzle for 32/64/128-byte rows);
+// otherwise r8/8 boxes of 64 rows x 8 ranks (16-byte rows, no swizzle).
+__device__ __forceinline__ uint32_t b_off(int col, int k, int r8) {
+    const uint32_t blk = (uint32_t)(col >> 6) * (uint32_t)(128 * r8);
+    const int cr = col & 63;
+    if (r8 & (r8 - 1))
+        return blk + (uint32_t)((k >> 3) * 1024 + cr * 16 + (k & 7) * 2);
+    uint32_t off = (uint32_t)(cr * 2 * r8 + 2 * k);
+    off ^= ((off >> 7) & (uint32_t)((r8 >> 3) - 1)) << 4;
+    return blk + off;
 }
 
-// Position in a block's chunk stream, advanced without divisions: shrink
-// chunks slice by slice, then expand chunks slice by slice.
-struct ChunkIt {
-    int i;                 // chunk index
-    int s, q;              // shrink: slice, chunk in slice
-    int es, c0, w;         // expand: slice, first slice-local column, width
+// ------------------------------------------------------------------ geometry (shared by host tests)
+// Rows of one shrink pass: the exchange holds at most GB_XCAP partial elements.
+__host__ __device__ inline int gb_pass_rows(int cnt, int S, int r8) {
+    int pr = (GB_XCAP / (S * r8)) & ~15;
+    pr = pr < 16 ? 16 : (pr > GB_ROWS ? GB_ROWS : pr);
+    return cnt < pr ? cnt : pr;
+}
+// Slices per shrink chunk: as many as fit a stage beside 64 columns of x rows.
+__host__ __device__ inline int gb_shrink_slices(int pcnt, int S, int r8) {
+    const int xb = (pcnt * (128 + 16) + 1023) & ~1023;
+    int sg = (GB_SB - xb) / (r8 * 128);
+    return sg < 1 ? 1 : (sg > S ? S : sg);
+}
+// Columns per shrink chunk (multiple of 64, at most 1024) for pcnt rows and sn slices.
+__host__ __device__ inline int gb_shrink_cols(int pcnt, int sn, int r8) {
+    int jc = (GB_SB - 16 * pcnt - 1023) / (2 * pcnt + 2 * sn * r8);
+    jc &= ~63;
+    return jc < 64 ? 64 : (jc > 1024 ? 1024 : jc);
+}
+// Columns per expand chunk (multiple of 64, at most 2048) for cnt rows with
+// vbytes of v rows in front; 0 when not even 64 columns fit beside the v rows.
+__host__ __device__ inline int gb_expand_cols(int cnt, int r8, int vbytes) {
+    int cc = (GB_SB - ((vbytes + 15) & ~15) - 16 * cnt - 1023) / (2 * cnt + 2 * r8);
+    cc &= ~63;
+    return cc > 2048 ? 2048 : (cc < 0 ? 0 : cc);
+}
+
+// Shared memory: ring | headers | exchange buffers [2] | k-group staging | pass rows | tickets | barriers
+struct GbSmem {
+    uint32_t ring, hdr, recv, part, xrows, tkslot;
+    uint32_t full0, empty0, xready0, tkbar0, tkfree0;
+    int *flag;   // generic pointer: "this block leaves last"
 };
 
-// Shared-memory carve-up of a block (the same for every unit it takes).
-struct BgSmem {
-    unsigned char *ring;
-    float *recv, *vfull, *part;
-    int *rows;
-    uint32_t ring_s, full0, empty0, xready, vready;
+size_t bgmv_smem_bytes(int mode, int stages) {
+    size_t b = 1024 + (size_t)stages * (GB_SB + GB_HDR);
+    if (mode != MODE_EXPAND) b += (size_t)2 * GB_XBUF * 4 + GB_PART * 4;
+    b += GB_ROWS * 4 + GB_TK * 4 + 16 + (size_t)(2 * GB_MAX_STAGES + 2 + 2 * GB_TK) * 8;
+    return b;
+}
+
+struct UnitInfo {
+    int n, cnt, r_n, r8;
+    bool ok;
 };
 
-// One unit on one block of its cluster.  `base`: chunks this block streamed
-// through the ring for earlier units (slot and phase of every chunk follow
-// from base + its index); `uiter`: units this block took before (phase of the
-// exchange barriers).  Returns the unit's chunk count.
+// Unit u's adapter, rank and rows (all lanes of the producer warp; lane l holds
+// rows l and l + 32 in row0 / row1).
+__device__ __forceinline__ UnitInfo fetch_unit(const GbArgs &a, int u, int &row0, int &row1) {
+    const int lane = threadIdx.x & 31;
+    const Unit un = resolve_live_unit(a.tiles, u);
+    UnitInfo f;
+    f.n = un.id;
+    f.cnt = un.cnt;
+    f.r_n = un.cnt > 0 ? a.ranks[un.id] : 0;
+    f.ok = un.cnt > 0 && f.r_n >= 1 && f.r_n <= a.r_max;
+    f.r8 = (f.r_n + 7) & ~7;
+    row0 = lane < f.cnt ? un.row(a.tiles, lane) : -1;
+    row1 = lane + 32 < f.cnt ? un.row(a.tiles, lane + 32) : -1;
+    return f;
+}
+
+// ================================================================ producer warp
 template <int MODE>
-__device__ __forceinline__ uint32_t bgmv_unit(const BgArgs &a, const BgSmem &sm, const Unit &u,
-                                              int r_n, uint32_t base, uint32_t uiter,
-                                              bool &failed) {
-    const int S = a.sl.n;
-    unsigned char *ring = sm.ring;
-    float *recv = sm.recv, *vfull = sm.vfull, *part = sm.part;
-    const int *rows_sm = sm.rows;
-    const uint32_t ring_s = sm.ring_s, full0 = sm.full0, empty0 = sm.empty0;
-    const uint32_t xready = sm.xready, vready = sm.vready;
+__device__ void gb_producer(const GbArgs &a, const GbSmem &sm, bool &failed) {
+    const int lane = threadIdx.x & 31;
+    const int S = a.sl.n, NS = a.stages;
+    const uint32_t crank = cta_rank_in_cluster(), C = cluster_size();
+    const int cid = blockIdx.x / (int)C, ncl = gridDim.x / (int)C;
+    const int live = n_live_units(a.tiles);
+    uint32_t gi = 0;   // stages filled so far
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int C = gridDim.x, crank = blockIdx.x;
-    const int n = u.id;
-    const int cnt = u.cnt;
+    // next free stage (bounded wait; the whole warp sees the outcome)
+    auto acquire = [&](int &st, uint32_t &dst, GbHdr *&h) -> bool {
+        st = (int)(gi % (uint32_t)NS);
+        bool ok = !failed;
+        if (ok && gi >= (uint32_t)NS && lane == 0)
+            ok = mbar_wait(sm.empty0 + 8 * st, ((gi / NS) - 1) & 1, a.status, failed, a.wait_limit);
+        ok = __shfl_sync(FULL, ok ? 1 : 0, 0) != 0;
+        if (!ok) failed = true;
+        dst = sm.ring + (uint32_t)st * GB_SB;
+        h = reinterpret_cast<GbHdr *>(__cvta_shared_to_generic(sm.hdr + (uint32_t)st * GB_HDR));
+        return ok;
+    };
+    // test hook (a.dbg_stall): the block's first stage expects 16 bytes more than arrive,
+    // so its consumers' bounded wait runs out
+    const unsigned stall = a.dbg_stall ? 16u : 0u;
+    auto commit = [&](int st, unsigned bytes) {   // header written: arrive with the stage's bytes
+        __syncwarp();
+        if (lane == 0) mbar_expect_tx(sm.full0 + 8 * st, bytes + (gi == 0 ? stall : 0u));
+        __syncwarp();
+        ++gi;
+    };
 
-    // ------------------------------------------------------------ geometry
-    const int NS = a.stages == 2 ? 2 : 3;                   // ring stages
-    const int SB = BG_RING_BYTES / NS;                      // bytes per stage
-    Geo G;
-    G.r8 = (r_n + 7) & ~7;
-    G.nb8 = G.r8 >> 3;
-    G.nkb16 = (r_n + 15) >> 4;
+    // ------------------------------------------------------------ phase 1: shrink
     if (MODE != MODE_EXPAND) {
-        const int n64 = (a.d_in + 63) >> 6;
-        G.j_lo = (int)((int64_t)crank * n64 / C) * 64;
-        G.j_hi = min((int)((int64_t)(crank + 1) * n64 / C) * 64, a.d_in);
-        // widest power-of-two chunk (>= 64 columns) whose x rows and A boxes fit a stage
-        int jc = 64;
-        while (chunk_bytes(jc * 2, G.nb8, a.ab16) <= SB) jc *= 2;
-        const int span = max(0, G.j_hi - G.j_lo);
-        while (jc > 64 && jc / 2 >= span) jc /= 2;
-        G.JC = jc;
-        G.RS = G.JC * 2 + 16;
-        G.A0 = (BG_ROWS * G.RS + 1023) & ~1023;
-        G.n_sc = (span + G.JC - 1) / G.JC;
-    } else {
-        G.j_lo = G.j_hi = 0;
-        G.JC = 64;
-        G.RS = 144;
-        G.A0 = 0;
-        G.n_sc = 0;
-    }
-    G.n_shrink = S * G.n_sc;
-    G.n_chunks = G.n_shrink;
-    if (MODE != MODE_SHRINK) {
-        const int n8 = a.sl.cat_off[S] >> 3;
-        G.c_lo = (int)((int64_t)crank * n8 / C) * 8;
-        G.c_hi = (int)((int64_t)(crank + 1) * n8 / C) * 8;
-        // widest power-of-two chunk (>= 64 columns) whose y rows and B boxes fit a stage
-        int cc = 64;
-        while (chunk_bytes(cc * 2, G.nb8, a.ab16) <= SB) cc *= 2;
-        G.CC = cc;
-        G.YS = G.CC * 2 + 16;   // 16 (mod 128) bytes: the 8 rows of an mma tile hit 8 bank groups
-        G.B0 = (BG_ROWS * G.YS + 1023) & ~1023;
-        for (int s = 0; s < S; ++s) {
-            const int lo = max(G.c_lo, a.sl.cat_off[s]), hi = min(G.c_hi, a.sl.cat_off[s + 1]);
-            if (hi > lo) G.n_chunks += (hi - lo + G.CC - 1) / G.CC;
-        }
-    } else {
-        G.c_lo = G.c_hi = 0;
-        G.CC = 64;
-        G.YS = 144;
-        G.B0 = 0;
-    }
-
-    // next position of the chunk stream
-    auto advance = [&](ChunkIt &it) {
-        ++it.i;
-        if (it.i < G.n_shrink) {
-            if (++it.q == G.n_sc) {
-                it.q = 0;
-                ++it.s;
-            }
-            return;
-        }
-        if (it.i >= G.n_chunks) return;
-        if (it.es >= 0) {   // next block of columns in this slice?
-            const int hi = min(G.c_hi, a.sl.cat_off[it.es + 1]) - a.sl.cat_off[it.es];
-            if (it.c0 + G.CC < hi) {
-                it.c0 += G.CC;
-                it.w = min(G.CC, hi - it.c0);
+        // fused mode: cluster rank 0 draws unit tickets and hands them to every block
+        // of the cluster through a ring of GB_TK slots with credits
+        auto send_ticket = [&](uint32_t j) {   // lane 0 of rank 0 only
+            const uint32_t slot = j % GB_TK;
+            if (j >= GB_TK &&
+                !mbar_wait<true>(sm.tkfree0 + 8 * slot, ((j / GB_TK) - 1) & 1, a.status, failed,
+                                 a.wait_limit))
                 return;
-            }
-        }
-        for (int s = it.es + 1; s < S; ++s) {   // first later slice with columns in this block
-            const int lo = max(G.c_lo, a.sl.cat_off[s]), hi = min(G.c_hi, a.sl.cat_off[s + 1]);
-            if (hi > lo) {
-                it.es = s;
-                it.c0 = lo - a.sl.cat_off[s];
-                it.w = min(G.CC, hi - lo);
-                return;
-            }
-        }
-    };
-    auto first = [&](ChunkIt &it) {
-        it.i = 0;
-        it.s = it.q = 0;
-        it.es = -1;
-        it.c0 = it.w = 0;
-        if (G.n_shrink == 0 && G.n_chunks > 0) {   // the stream starts with expand chunks
-            it.i = -1;
-            advance(it);
-        }
-    };
-
-
-    if (warp == BG_CONSUMERS) {
-        // ============================================================ producer
-        ChunkIt it;
-        first(it);
-        for (; it.i < G.n_chunks; advance(it)) {
-            const uint32_t gi = base + (uint32_t)it.i;   // position in the block's ring stream
-            const int st = (int)(gi % (uint32_t)NS);
-            const uint32_t full = full0 + 8 * st, dst = ring_s + st * SB;
-            if (gi >= (uint32_t)NS)
-                mbar_wait(empty0 + 8 * st, ((gi / NS) - 1) & 1, a.status, failed);
-            if (failed) break;
-            if (it.i < G.n_shrink) {
-                const int jc0 = G.j_lo + it.q * G.JC;
-                const int width = min(G.JC, G.j_hi - jc0), nbox = (width + 63) >> 6;
-                const int ncb = G.JC >> 6;
-                const unsigned xbytes = (unsigned)width * 2;
-                const int nkg = a.ab16 ? (G.nb8 + 1) >> 1 : G.nb8;   // rank boxes
-                const unsigned abox = a.ab16 ? 2048u : 1024u;
-                if (lane == 0) mbar_expect_tx(full, xbytes * cnt + (unsigned)(nkg * nbox) * abox);
-                __syncwarp();
-                for (int r = lane; r < cnt; r += 32)   // gathered x rows
-                    bulk_g2s(dst + r * G.RS, a.x + (int64_t)rows_sm[r] * a.ld_x + jc0, xbytes, full);
-                for (int e = lane; e < nkg * nbox; e += 32) {   // A: 8 or 16 ranks x 64 columns per box
-                    const int kg = e / nbox, cb = e - kg * nbox;
-                    tma_2d(dst + G.A0 + (kg * ncb + cb) * abox, &a.tmA[it.s], jc0 + 64 * cb,
-                           n * a.r_max + (a.ab16 ? 16 : 8) * kg, full);
+            const int tk = atomicAdd(a.ctl + GB_T_SHRINK, 1);
+            for (uint32_t c = 0; c < C; ++c)
+                st_async_u32(map_rank(sm.tkslot + 4 * slot, c), (uint32_t)tk,
+                             map_rank(sm.tkbar0 + 8 * slot, c));
+        };
+        if (MODE == MODE_FUSED && crank == 0 && lane == 0) send_ticket(0);
+        for (uint32_t k = 0;; ++k) {
+            int u = 0;
+            if (MODE == MODE_FUSED) {
+                const uint32_t slot = k % GB_TK;
+                int got = -1;
+                if (lane == 0 && !failed) {
+                    mbar_expect_tx(sm.tkbar0 + 8 * slot, 4);
+                    if (mbar_wait<true>(sm.tkbar0 + 8 * slot, (k / GB_TK) & 1, a.status, failed,
+                                       a.wait_limit)) {
+                        got = *reinterpret_cast<volatile int *>(
+                            __cvta_shared_to_generic(sm.tkslot + 4 * slot));
+                        mbar_arrive_cluster(map_rank(sm.tkfree0 + 8 * slot, 0));
+                        if (crank == 0 && got < live) send_ticket(k + 1);
+                    }
                 }
+                got = __shfl_sync(FULL, got, 0);
+                // a wait of lane 0 that ran out (here or in send_ticket) stops the whole warp
+                failed = __any_sync(FULL, failed) != 0;
+                if (got < 0 || failed) {
+                    failed = true;
+                    break;
+                }
+                u = got;
             } else {
-                const int s = it.es, d_out = a.sl.d_out[s];
-                const int nbox = (it.w + 63) >> 6, nbx = G.CC >> 6;
-                const unsigned ybytes = (unsigned)it.w * 2;
-                const int nkg = a.ab16 ? (G.nb8 + 1) >> 1 : G.nb8;
-                const unsigned bbox = a.ab16 ? 2048u : 1024u;
-                if (lane == 0) mbar_expect_tx(full, ybytes * cnt + (unsigned)(nkg * nbox) * bbox);
-                __syncwarp();
-                for (int r = lane; r < cnt; r += 32)   // gathered y rows
-                    bulk_g2s(dst + r * G.YS,
-                             a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0, ybytes, full);
-                for (int e = lane; e < nkg * nbox; e += 32) {   // B: 64 columns x 8 or 16 ranks per box
-                    const int kg = e / nbox, cb = e - kg * nbox;
-                    tma_2d(dst + G.B0 + (kg * nbx + cb) * bbox, &a.tmB[s], (a.ab16 ? 16 : 8) * kg,
-                           n * d_out + it.c0 + 64 * cb, full);
-                }
+                u = cid + (int)k * ncl;
             }
-        }
-        return (uint32_t)G.n_chunks;
-    }
-
-    // ================================================================ consumers
-    const int jg = max(1, BG_CONSUMERS / G.nb8);   // warps per 8-rank block
-    const bool shrink_warp = warp < G.nb8 * jg;
-    const int nbw = warp / jg, jgi = warp - (warp / jg) * jg;
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-    const int ctid = tid;   // 0 .. 255
-    const int per_src = (S * BG_ROWS * BG_RMAX) / C;
-    const uint32_t recv_s = smem_u32(recv), vfull_s = smem_u32(vfull);
-    // Exchange rounds: st.async stores that count their bytes on the receiver's
-    // barrier (no fence on either side).  With C dividing 64, every block
-    // receives S * cnt * r8 partials (4 bytes each) in either round: the
-    // elements it owns from every block, then every owner's scaled sums.
-    if (MODE != MODE_EXPAND && ctid == 0) {
-        const unsigned bytes = (unsigned)(S * cnt * G.r8) * 4u;
-        mbar_expect_tx(xready, bytes);
-        if (MODE == MODE_FUSED) mbar_expect_tx(vready, bytes);
-    }
-
-    // block partial of slice s (from part, or zeros) -> recv of the owning block
-    auto send_partials = [&](int s, bool from_part) {
-        for (int idx = ctid; idx < cnt * G.r8; idx += BG_CONSUMERS * 32) {
-            const int row = idx / G.r8, k = idx - row * G.r8;
-            float sum = 0.f;
-            if (from_part)
-                for (int j = 0; j < jg; ++j) sum += part[(j * BG_ROWS + row) * G.r8 + k];
-            const int e = (s * BG_ROWS + row) * BG_RMAX + k;
-            const uint32_t owner = (uint32_t)(e % C);
-            st_async_f32(map_rank(recv_s + (uint32_t)(crank * per_src + e / C) * 4u, owner), sum,
-                         map_rank(xready, owner));
-        }
-    };
-
-    auto shrink_chunk = [&](const ChunkIt &it, uint32_t st) {
-        if (shrink_warp) {
-            const int jc0 = G.j_lo + it.q * G.JC;
-            const int width = min(G.JC, G.j_hi - jc0);
-            const int nsteps = (width + 63) >> 6;
-            const uint32_t xg = st + g * G.RS, xh = st + (g + 8) * G.RS;
-            // A box (8 or 16 ranks x 64 columns, 128-byte swizzle): rank 8 nbw + g, 16-byte
-            // chunks 2t and 2t+1 (the swizzle follows address bits 7-9, the same in either box)
-            const uint32_t ak = a.ab16 ? st + G.A0 + (nbw >> 1) * (G.JC >> 6) * 2048 + (nbw & 1) * 1024 + g * 128
-                                       : st + G.A0 + nbw * (G.JC >> 6) * 1024 + g * 128;
-            const uint32_t astep = a.ab16 ? 2048u : 1024u;
-            const uint32_t c0 = (uint32_t)(((2 * t) ^ g) << 4), c1 = (uint32_t)(((2 * t + 1) ^ g) << 4);
-            for (int sp = jgi; sp < nsteps; sp += jg) {
-                const int col = sp * 64 + t * 16;
-                const bool z0 = col >= width, z1 = col + 8 >= width;   // beyond the chunk: zero
-                const uint32_t off = (uint32_t)(col * 2);
-                const uint4 xa0 = zero_if(z0, lds128(xg + off)), xa1 = zero_if(z1, lds128(xg + off + 16));
-                const uint4 xb0 = zero_if(z0, lds128(xh + off)), xb1 = zero_if(z1, lds128(xh + off + 16));
-                const uint32_t box = ak + sp * astep;
-                const uint4 a0 = zero_if(z0, lds128(box + c0)), a1 = zero_if(z1, lds128(box + c1));
-                {
-                    const uint32_t f[4] = {xa0.x, xb0.x, xa0.y, xb0.y};
-                    mma16816(acc0, f, a0.x, a0.y);
-                }
-                {
-                    const uint32_t f[4] = {xa0.z, xb0.z, xa0.w, xb0.w};
-                    mma16816(acc1, f, a0.z, a0.w);
-                }
-                {
-                    const uint32_t f[4] = {xa1.x, xb1.x, xa1.y, xb1.y};
-                    mma16816(acc0, f, a1.x, a1.y);
-                }
-                {
-                    const uint32_t f[4] = {xa1.z, xb1.z, xa1.w, xb1.w};
-                    mma16816(acc1, f, a1.z, a1.w);
-                }
+            if (u >= live || failed) break;
+            int row0, row1;
+            const UnitInfo f = fetch_unit(a, u, row0, row1);
+            if (!f.ok) {
+                if (f.cnt > 0 && crank == 0 && lane == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
+                continue;
             }
-        }
-        if (it.q == G.n_sc - 1) {   // slice done: block partial -> owners
-            consumer_sync();        // every warp is past its reads of part from the last slice
-            if (shrink_warp) {
-                const int k = nbw * 8 + 2 * t;
-                part[(jgi * BG_ROWS + g) * G.r8 + k] = acc0[0] + acc1[0];
-                part[(jgi * BG_ROWS + g) * G.r8 + k + 1] = acc0[1] + acc1[1];
-                part[(jgi * BG_ROWS + g + 8) * G.r8 + k] = acc0[2] + acc1[2];
-                part[(jgi * BG_ROWS + g + 8) * G.r8 + k + 1] = acc0[3] + acc1[3];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc0[e] = acc1[e] = 0.f;
-            }
-            consumer_sync();
-            send_partials(it.s, true);
-        }
-    };
-
-    auto exchange = [&]() {
-        if (MODE == MODE_EXPAND) {
-            const float scale = a.scales[n];
-            for (int e = ctid; e < S * BG_ROWS * BG_RMAX; e += BG_CONSUMERS * 32) {
-                const int s = e >> 10, rem = e & 1023;
-                const int row = rem >> 6, k = rem & 63;
-                if (row < cnt && k < G.r8)
-                    vfull[(s * BG_ROWS + row) * BG_VF_STRIDE + k] =
-                        k < r_n ? scale * a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] : 0.f;
-            }
-            consumer_sync();
-            return;
-        }
-        if (G.n_sc == 0)   // no input columns here: the partials are zero
-            for (int s = 0; s < S; ++s) send_partials(s, false);
-        mbar_wait(xready, uiter & 1u, a.status, failed);   // every partial has reached its owner
-        const float scale = MODE == MODE_FUSED ? a.scales[n] : 1.f;
-        const int mine = (S * BG_ROWS * BG_RMAX - crank + C - 1) / C;   // elements e = crank + C*j
-        for (int j = ctid; j < mine; j += BG_CONSUMERS * 32) {
-            const int e = crank + C * j;
-            const int s = e >> 10, rem = e & 1023;
-            const int row = rem >> 6, k = rem & 63;
-            if (row >= cnt || k >= G.r8) continue;
-            float sum = 0.f;
-            for (int c = 0; c < C; ++c) sum += recv[c * per_src + j];
-            const float val = k < r_n ? scale * sum : 0.f;
-            if (MODE == MODE_SHRINK) {
-                if (k < r_n) a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] = val;
-            } else {
-                const uint32_t f = vfull_s + (uint32_t)((s * BG_ROWS + row) * BG_VF_STRIDE + k) * 4u;
-                for (int c = 0; c < C; ++c) st_async_f32(map_rank(f, (uint32_t)c), val, map_rank(vready, (uint32_t)c));
-            }
-        }
-        if (MODE == MODE_FUSED)
-            mbar_wait(vready, uiter & 1u, a.status, failed);   // every block holds the full s*v
-    };
-
-    int cur_s = -1;
-    uint32_t ahi[4][4], alo[4][4];
-    auto expand_chunk = [&](const ChunkIt &it, uint32_t st) {
-        const int s = it.es;
-        if (s != cur_s) {   // mma fragments of s*v (bf16 hi + lo) for this slice
-            cur_s = s;
-            const float *vf = vfull + s * BG_ROWS * BG_VF_STRIDE;
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-                const float4 p = *reinterpret_cast<const float4 *>(&vf[g * BG_VF_STRIDE + kb * 16 + 4 * t]);
-                const float4 q =
-                    *reinterpret_cast<const float4 *>(&vf[(g + 8) * BG_VF_STRIDE + kb * 16 + 4 * t]);
-                ahi[kb][0] = pack_bf16x2(p.x, p.y);
-                ahi[kb][1] = pack_bf16x2(q.x, q.y);
-                ahi[kb][2] = pack_bf16x2(p.z, p.w);
-                ahi[kb][3] = pack_bf16x2(q.z, q.w);
-                alo[kb][0] = pack_bf16x2(p.x - bf16_lo(ahi[kb][0]), p.y - bf16_hi(ahi[kb][0]));
-                alo[kb][1] = pack_bf16x2(q.x - bf16_lo(ahi[kb][1]), q.y - bf16_hi(ahi[kb][1]));
-                alo[kb][2] = pack_bf16x2(p.z - bf16_lo(ahi[kb][2]), p.w - bf16_hi(ahi[kb][2]));
-                alo[kb][3] = pack_bf16x2(q.z - bf16_lo(ahi[kb][3]), q.w - bf16_hi(ahi[kb][3]));
-            }
-        }
-        const int nblk = it.w >> 3;
-        const uint32_t bbase = st + G.B0, nbx = G.CC >> 6;
-        for (int nb0 = warp * 2; nb0 < nblk; nb0 += BG_CONSUMERS * 2) {
-            float d[2][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) d[j][e] = 0.f;
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-                if (kb < G.nkb16) {
-                    const int k = kb * 16 + 4 * t;
-                    uint2 bv[2];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        bv[j] = make_uint2(0, 0);
-                        if (k < r_n && nb0 + j < nblk) {
-                            const int col = (nb0 + j) * 8 + g;   // B box: 64 columns x 8 (16) ranks
-                            bv[j] = a.ab16 ? lds64(bbase + ((k >> 4) * nbx + (col >> 6)) * 2048 +
-                                                   (col & 63) * 32 + (k & 15) * 2)
-                                           : lds64(bbase + ((k >> 3) * nbx + (col >> 6)) * 1024 +
-                                                   (col & 63) * 16 + (k & 7) * 2);
-                            if (k + 4 > r_n) {   // the rank ends inside this group of 4
-                                const int keep = r_n - k;
-                                if (keep < 2) bv[j].x &= 0xffffu;
-                                if (keep < 3) bv[j].y = 0;
-                                else bv[j].y &= 0xffffu;
-                            }
+            const int r8 = f.r8;
+            const int n64 = (a.d_in + 63) >> 6;
+            const int j_lo = (int)((int64_t)crank * n64 / C) * 64;
+            const int j_hi = min((int)((int64_t)(crank + 1) * n64 / C) * 64, a.d_in);
+            const int span = j_hi - j_lo;
+            const int pr = gb_pass_rows(f.cnt, S, r8);
+            for (int p0 = 0; p0 < f.cnt && !failed; p0 += pr) {
+                const int pcnt = min(pr, f.cnt - p0);
+                const bool last_pass = p0 + pcnt >= f.cnt;
+                const int sg = gb_shrink_slices(pcnt, S, r8);
+                const int JC = gb_shrink_cols(pcnt, sg, r8);
+                const int RS = 2 * JC + 16;
+                const int ncol = span > 0 ? (span + JC - 1) / JC : 1;
+                const int nsg = (S + sg - 1) / sg;
+                const int nch = ncol * nsg;
+                for (int q = 0; q < nch; ++q) {
+                    int st;
+                    uint32_t dst;
+                    GbHdr *h;
+                    if (!acquire(st, dst, h)) break;
+                    const int qc = q / nsg, qs = q - qc * nsg;
+                    const int jc0 = j_lo + qc * JC;
+                    const int width = span > 0 ? min(JC, j_hi - jc0) : 0;
+                    const int s0 = qs * sg, sn = min(sg, S - s0);
+                    const int bofs = align_up(pcnt * RS, 1024);
+                    if (lane == 0) {
+                        h->kind = GB_SHRINK;
+                        h->flags = (q == 0 ? GB_FIRST : 0) | (q == nch - 1 ? GB_LAST : 0) |
+                                   (width == 0 ? GB_NODATA : 0) |
+                                   (last_pass && q == nch - 1 ? GB_UNIT_DONE : 0);
+                        h->unit = u;
+                        h->n = f.n;
+                        h->r_n = f.r_n;
+                        h->r8 = r8;
+                        h->cnt = pcnt;
+                        h->s0 = s0;
+                        h->sn = sn;
+                        h->c0 = jc0;
+                        h->w = width;
+                        h->cw = JC;
+                        h->bofs = bofs;
+                        h->yofs = 0;
+                        h->scale = 0.f;
+                    }
+                    // rows p0 .. p0+pcnt-1 of the unit
+                    if (lane >= p0 && lane < p0 + pcnt) h->rows[lane - p0] = row0;
+                    if (lane + 32 >= p0 && lane + 32 < p0 + pcnt) h->rows[lane + 32 - p0] = row1;
+                    __syncwarp();
+                    const int nbox = (width + 63) >> 6, ncb = JC >> 6;
+                    // rank boxes: r8 as a sum of 64/32/16/8-rank boxes
+                    int parts[4], nparts = 0;
+                    for (int R = 64, k0 = 0; R >= 8; R >>= 1)
+                        if (r8 & R) {
+                            parts[nparts++] = (k0 << 8) | R;
+                            k0 += R;
+                        }
+                    const unsigned bytes =
+                        width > 0 ? (unsigned)(pcnt * width * 2 + sn * nbox * r8 * 128) : 0u;
+                    if (width > 0) {
+                        for (int r = lane; r < pcnt; r += 32)
+                            bulk_g2s(dst + r * RS, a.x + (int64_t)h->rows[r] * a.ld_x + jc0,
+                                     (unsigned)width * 2, sm.full0 + 8 * st);
+                        const int nb = sn * nbox * nparts;
+                        for (int e = lane; e < nb; e += 32) {
+                            const int ss = e / (nbox * nparts), rem = e - ss * (nbox * nparts);
+                            const int cb = rem / nparts, pi = rem - cb * nparts;
+                            const int k0 = parts[pi] >> 8, R = parts[pi] & 255;
+                            const int mi = R == 64 ? 3 : (R == 32 ? 2 : (R == 16 ? 1 : 0));
+                            tma_2d(dst + bofs + (uint32_t)(((ss * ncb + cb) * r8 + k0) * 128),
+                                   &a.tmA[s0 + ss][mi], jc0 + 64 * cb, f.n * a.r_max + k0,
+                                   sm.full0 + 8 * st);
                         }
                     }
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) mma16816(d[j], ahi[kb], bv[j].x, bv[j].y);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) mma16816(d[j], alo[kb], bv[j].x, bv[j].y);
-                }
-            }
-            // y += delta in shared memory (rows g and g+8, columns 2t, 2t+1 of each 8-column block)
-            const uint32_t yg = st + g * G.YS + (nb0 * 8 + 2 * t) * 2;
-            const uint32_t yh = yg + 8 * G.YS;
-            uint32_t y0[2], y1[2];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const bool ok = nb0 + j < nblk;
-                y0[j] = (ok && g < cnt) ? lds32(yg + j * 16) : 0u;
-                y1[j] = (ok && g + 8 < cnt) ? lds32(yh + j * 16) : 0u;
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                if (nb0 + j < nblk) {
-                    if (g < cnt)
-                        sts32(yg + j * 16, pack_bf16x2(bf16_lo(y0[j]) + d[j][0], bf16_hi(y0[j]) + d[j][1]));
-                    if (g + 8 < cnt)
-                        sts32(yh + j * 16, pack_bf16x2(bf16_lo(y1[j]) + d[j][2], bf16_hi(y1[j]) + d[j][3]));
+                    commit(st, bytes);
                 }
             }
         }
-        consumer_sync();
-        const int ypc = it.w >> 3;
-        const unsigned char *stp = ring + (st - ring_s);
-        for (int r = warp; r < cnt; r += BG_CONSUMERS) {
-            __nv_bfloat16 *dst = a.y + (int64_t)rows_sm[r] * a.ld_y + a.sl.col_off[s] + it.c0;
-            for (int pc = lane; pc < ypc; pc += 32)
-                *reinterpret_cast<uint4 *>(dst + pc * 8) =
-                    *reinterpret_cast<const uint4 *>(stp + r * G.YS + pc * 16);
-        }
-    };
-
-    ChunkIt it;
-    first(it);
-    bool exchanged = false;
-    for (; it.i < G.n_chunks; advance(it)) {
-        const uint32_t gi = base + (uint32_t)it.i;
-        const int st = (int)(gi % (uint32_t)NS);
-        const uint32_t sta = ring_s + st * SB;
-        if (!exchanged && it.i >= G.n_shrink) {
-            exchange();
-            exchanged = true;
-        }
-        const bool ready = mbar_wait(full0 + 8 * st, (gi / NS) & 1, a.status, failed);
-        if (ready) {
-            if (it.i < G.n_shrink)
-                shrink_chunk(it, sta);
-            else
-                expand_chunk(it, sta);
-        }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * st);
     }
-    if (!exchanged) exchange();
-    return (uint32_t)G.n_chunks;
+
+    // ------------------------------------------------------------ phase 2: expand
+    if (MODE != MODE_SHRINK && !failed) {
+        const int nb = a.blk_off[S];
+        const int64_t total = (int64_t)live * nb;
+        int64_t e = MODE == MODE_FUSED ? -1 : (int64_t)blockIdx.x;
+        if (MODE == MODE_FUSED && lane == 0) e = atomicAdd(a.ctl + GB_T_EXPAND, 1);
+        for (int k = 0;; ++k) {
+            if (MODE == MODE_FUSED) e = __shfl_sync(FULL, (int)e, 0);
+            if (e >= total || failed) break;
+            const int u = (int)(e / nb), b = (int)(e - (int64_t)u * nb);
+            int enext = 0;   // the next ticket, drawn early so its latency overlaps this item
+            if (MODE == MODE_FUSED && lane == 0) enext = atomicAdd(a.ctl + GB_T_EXPAND, 1);
+            int s = 0;
+            while (s + 1 < S && a.blk_off[s + 1] <= b) ++s;
+            const int c_item = (b - a.blk_off[s]) * a.bc;
+            const int w_item = min(a.bc, a.sl.d_out[s] - c_item);
+            int row0, row1;
+            const UnitInfo f = fetch_unit(a, u, row0, row1);
+            if (!f.ok) {
+                if (f.cnt > 0 && b == 0 && lane == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
+            } else {
+                const int r8 = f.r8, cnt = f.cnt;
+                const float scale = a.alphas[f.n] / (float)f.r_n;
+                const int vbytes = cnt * r8 * 4;
+                const int d_out = a.sl.d_out[s];
+                const int mi = r8 == 64 ? 3 : (r8 == 32 ? 2 : (r8 == 16 ? 1 : 0));
+                const bool wide = (r8 & (r8 - 1)) == 0;
+                int c = c_item;
+                bool first = true;
+                while ((c < c_item + w_item || first) && !failed) {
+                    const int vb = first ? vbytes : 0;
+                    int CC = gb_expand_cols(cnt, r8, vb);
+                    int w = min(CC, c_item + w_item - c);
+                    if (CC == 0) w = 0;   // v rows alone in this stage
+                    int st;
+                    uint32_t dst;
+                    GbHdr *h;
+                    if (!acquire(st, dst, h)) break;
+                    const int CCs = CC > 0 ? CC : 64;
+                    const int YS = 2 * CCs + 16;
+                    const int yofs = align_up(vb, 16);
+                    const int bofs = align_up(yofs + cnt * YS, 1024);
+                    const bool last = c + w >= c_item + w_item;
+                    if (lane == 0) {
+                        h->kind = GB_EXPAND;
+                        h->flags = (first ? GB_FIRST : 0) | (last ? GB_LAST : 0);
+                        h->unit = u;
+                        h->n = f.n;
+                        h->r_n = f.r_n;
+                        h->r8 = r8;
+                        h->cnt = cnt;
+                        h->s0 = s;
+                        h->sn = 1;
+                        h->c0 = c;
+                        h->w = w;
+                        h->cw = CCs;
+                        h->bofs = bofs;
+                        h->yofs = yofs;
+                        h->scale = scale;
+                    }
+                    if (lane < cnt) h->rows[lane] = row0;
+                    if (lane + 32 < cnt) h->rows[lane + 32] = row1;
+                    __syncwarp();
+                    const int nbox = (w + 63) >> 6;
+                    const unsigned bytes = (unsigned)(vb + cnt * w * 2 + nbox * 128 * r8);
+                    if (lane == 0) mbar_expect_tx(sm.full0 + 8 * st, bytes + (gi == 0 ? stall : 0u));
+                    __syncwarp();
+                    if (w > 0) {
+                        const __nv_bfloat16 *ybase = a.y + a.sl.col_off[s] + c;
+                        for (int r = lane; r < cnt; r += 32)
+                            bulk_g2s(dst + yofs + r * YS, ybase + (int64_t)h->rows[r] * a.ld_y,
+                                     (unsigned)w * 2, sm.full0 + 8 * st);
+                        const int nbb = wide ? nbox : nbox * (r8 >> 3);
+                        for (int e2 = lane; e2 < nbb; e2 += 32) {
+                            const int cb = wide ? e2 : e2 / (r8 >> 3);
+                            const int kb = wide ? 0 : e2 - cb * (r8 >> 3);
+                            tma_2d(dst + bofs + (uint32_t)(cb * 128 * r8 + kb * 1024),
+                                   &a.tmB[s][wide ? mi : 0], kb * 8, f.n * d_out + c + 64 * cb,
+                                   sm.full0 + 8 * st);
+                        }
+                    }
+                    if (first) {
+                        if (MODE == MODE_FUSED) {
+                            // v of this unit is complete once its C shrink blocks have signalled
+                            bool ok = true;
+                            if (lane == 0) {
+                                unsigned it = 0;
+                                while (ld_acquire_gpu(a.done + u) < (int)C) {
+                                    if (++it >= a.wait_limit * 64u) {
+                                        atomicOr(a.status, LORA_DEV_TIMEOUT);
+                                        ok = false;
+                                        break;
+                                    }
+                                    __nanosleep(128);
+                                }
+                            }
+                            ok = __shfl_sync(FULL, ok ? 1 : 0, 0) != 0;
+                            if (!ok) failed = true;
+                            // the v rows were written by other blocks' generic stores; order
+                            // the copies below (async proxy) after the acquire above
+                            asm volatile("fence.proxy.async.global;\n" ::: "memory");
+                        }
+                        if (!failed) {
+                            for (int r = lane; r < cnt; r += 32)
+                                bulk_g2s(dst + r * r8 * 4,
+                                         a.v + ((int64_t)s * a.T + h->rows[r]) * a.r_max,
+                                         (unsigned)r8 * 4, sm.full0 + 8 * st);
+                        }
+                    }
+                    __syncwarp();
+                    ++gi;
+                    c += w;
+                    first = false;
+                    if (w == 0 && CC > 0) break;
+                }
+            }
+            if (MODE == MODE_FUSED) {
+                e = enext;
+            } else {
+                e += gridDim.x;
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ end of the stream
+    {
+        int st;
+        uint32_t dst;
+        GbHdr *h;
+        const bool was_failed = failed;
+        bool ok = !was_failed;
+        if (ok) ok = acquire(st, dst, h);
+        if (ok) {
+            if (lane == 0) h->kind = GB_END;
+            commit(st, 0);
+        }
+    }
 }
 
-// Persistent clusters: cluster k takes the live units k, k + #clusters, ...
+// ================================================================ consumer warps
+// Wait for stage gi to be full; every consumer thread sees the same outcome.
+__device__ __forceinline__ bool gb_stage_wait(const GbArgs &a, const GbSmem &sm, uint32_t gi,
+                                              bool &failed) {
+    const int st = (int)(gi % (uint32_t)a.stages);
+    bool ok = !failed && mbar_wait(sm.full0 + 8 * st, (gi / a.stages) & 1, a.status, failed,
+                                  a.wait_limit);
+    ok = consumers_all(ok);
+    if (!ok) failed = true;
+    return ok;
+}
+__device__ __forceinline__ const GbHdr *gb_hdr(const GbSmem &sm, int st) {
+    return reinterpret_cast<const GbHdr *>(__cvta_shared_to_generic(sm.hdr + (uint32_t)st * GB_HDR));
+}
+// This warp is done with stage st (its shared memory may be refilled by TMA).
+__device__ __forceinline__ void gb_release(const GbSmem &sm, int st) {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(sm.empty0 + 8 * st);
+}
+
+// Phase 1: shrink chunks until the stream moves on; returns the position of
+// the first stage that is not a shrink chunk.
 template <int MODE>
-__global__ void __launch_bounds__(BG_THREADS, 2) bgmv_kernel(const __grid_constant__ BgArgs a) {
-    extern __shared__ __align__(128) unsigned char bg_sm[];
-    __shared__ int rows_sm[BG_ROWS];
+__device__ uint32_t gb_consume_shrink(const GbArgs &a, const GbSmem &sm, bool &failed) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t crank = cta_rank_in_cluster(), C = cluster_size();
+    const int S = a.sl.n;
+    int *xrows = reinterpret_cast<int *>(__cvta_shared_to_generic(sm.xrows));
+    float *part = reinterpret_cast<float *>(__cvta_shared_to_generic(sm.part));
+
+    float acc[8][4];
+    // per pair i: m16 tile | slice << 4 | A rank row << 8 | first column << 16
+    int pinfo[8];
+    int nt = 0, np = 0, jg = 1, p_lo = 0, p_hi = 0, kgi = 0, W = 0;
+    uint32_t xc = 0;   // exchanges so far (buffer parity)
+    uint32_t gi = 0;
+    for (;; ++gi) {
+        if (!gb_stage_wait(a, sm, gi, failed)) break;
+        const int st = (int)(gi % (uint32_t)a.stages);
+        const GbHdr *h = gb_hdr(sm, st);
+        if (h->kind != GB_SHRINK) break;
+        const uint32_t stg = sm.ring + (uint32_t)st * GB_SB;
+        const int flags = h->flags;
+        const int cnt = h->cnt, r_n = h->r_n, r8 = h->r8;
+        if (flags & GB_FIRST) {   // a new pass: pairs (m16 tile, n8 rank tile) per warp
+            W = S * r8;
+            const int mt = (cnt + 15) >> 4;
+            nt = W >> 3;
+            np = mt * nt;
+            if (np >= GB_CONSUMERS) {
+                jg = 1;
+                const int ppw = (np + GB_CONSUMERS - 1) / GB_CONSUMERS;
+                p_lo = warp * ppw;
+                p_hi = min(np, p_lo + ppw);
+                kgi = 0;
+            } else {
+                jg = GB_CONSUMERS / np;
+                p_lo = warp % np;
+                kgi = warp / np;
+                p_hi = kgi < jg ? p_lo + 1 : p_lo;
+            }
+            const int nkb8 = r8 >> 3;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int p = p_lo + i < p_hi ? p_lo + i : p_lo;
+                const int m = p / nt, nn = p - m * nt;
+                const int s = nn / nkb8;
+                pinfo[i] = m | (s << 4) | (((nn - s * nkb8) * 8 + g) << 8) | ((nn * 8 + 2 * t) << 16);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+            }
+            if (tid < cnt) xrows[tid] = h->rows[tid];
+        }
+        if (!(flags & GB_NODATA)) {
+            const int width = h->w, JC = h->cw, RS = 2 * JC + 16, ncb = JC >> 6;
+            const int s0 = h->s0, sn = h->sn;
+            const uint32_t abase = stg + (uint32_t)h->bofs;
+            const int nbox = (width + 63) >> 6;
+            const uint32_t c0s = (uint32_t)(((2 * t) ^ g) << 4), c1s = (uint32_t)(((2 * t + 1) ^ g) << 4);
+            for (int sp = kgi; sp < nbox; sp += jg) {
+                const int col = sp * 64 + t * 16;
+                const bool z0 = col >= width, z1 = col + 8 >= width;
+                int cm = -1;
+                uint4 xa0 = make_uint4(0, 0, 0, 0), xa1 = xa0, xb0 = xa0, xb1 = xa0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (p_lo + i >= p_hi) break;
+                    const int m = pinfo[i] & 15, s = (pinfo[i] >> 4) & 15, kr = (pinfo[i] >> 8) & 255;
+                    if (s < s0 || s >= s0 + sn) continue;
+                    if (m != cm) {
+                        cm = m;
+                        const uint32_t xg = stg + (uint32_t)((16 * m + g) * RS + col * 2);
+                        const uint32_t xh = xg + 8 * RS;
+                        xa0 = zero_if(z0, lds128(xg));
+                        xa1 = zero_if(z1, lds128(xg + 16));
+                        xb0 = zero_if(z0, lds128(xh));
+                        xb1 = zero_if(z1, lds128(xh + 16));
+                    }
+                    const uint32_t arow = abase + (uint32_t)((((s - s0) * ncb + sp) * r8 + kr) * 128);
+                    const uint4 a0 = zero_if(z0, lds128(arow + c0s));
+                    const uint4 a1 = zero_if(z1, lds128(arow + c1s));
+                    {
+                        const uint32_t fr[4] = {xa0.x, xb0.x, xa0.y, xb0.y};
+                        mma16816(acc[i], fr, a0.x, a0.y);
+                    }
+                    {
+                        const uint32_t fr[4] = {xa0.z, xb0.z, xa0.w, xb0.w};
+                        mma16816(acc[i], fr, a0.z, a0.w);
+                    }
+                    {
+                        const uint32_t fr[4] = {xa1.x, xb1.x, xa1.y, xb1.y};
+                        mma16816(acc[i], fr, a1.x, a1.y);
+                    }
+                    {
+                        const uint32_t fr[4] = {xa1.z, xb1.z, xa1.w, xb1.w};
+                        mma16816(acc[i], fr, a1.z, a1.w);
+                    }
+                }
+            }
+        }
+        const int unit = h->unit;
+        gb_release(sm, st);   // the exchange below reads only registers and its own buffers
+        if (!(flags & GB_LAST)) continue;
+
+        // -------------------------------------------------------- exchange of the pass
+        const uint32_t par = xc & 1u;
+        const uint32_t xr = sm.xready0 + 8 * par;
+        const uint32_t rbuf = sm.recv + par * (uint32_t)GB_XBUF * 4u;
+        const int total_pairs = cnt * W / 2;
+        const int spc = (total_pairs + (int)C - 1) / (int)C;
+        const int mine = total_pairs > (int)crank ? (total_pairs - (int)crank + (int)C - 1) / (int)C : 0;
+        if (tid == 0) mbar_expect_tx(xr, (unsigned)(mine * (int)C * 8));
+        auto send = [&](int row, int col, float v0, float v1) {
+            if (row >= cnt) return;
+            const int P = (row * W + col) >> 1;
+            const uint32_t o = (uint32_t)P % C, slot = (uint32_t)P / C;
+            st_async_v2(map_rank(rbuf + ((crank * (uint32_t)spc + slot) * 2u) * 4u, o), v0, v1,
+                        map_rank(xr, o));
+        };
+        if (jg > 1) {   // k-groups of one pair: add them in shared memory first
+            if (p_lo < p_hi) {
+                float *pp = part + (kgi * np + p_lo) * 128;
+                pp[g * 8 + 2 * t] = acc[0][0];
+                pp[g * 8 + 2 * t + 1] = acc[0][1];
+                pp[(g + 8) * 8 + 2 * t] = acc[0][2];
+                pp[(g + 8) * 8 + 2 * t + 1] = acc[0][3];
+            }
+            consumer_sync();
+            for (int idx = tid; idx < np * 64; idx += GB_CONSUMERS * 32) {
+                const int p = idx >> 6, r = (idx & 63) >> 2, c2 = (idx & 3) * 2;
+                float v0 = 0.f, v1 = 0.f;
+                for (int kg = 0; kg < jg; ++kg) {
+                    v0 += part[(kg * np + p) * 128 + r * 8 + c2];
+                    v1 += part[(kg * np + p) * 128 + r * 8 + c2 + 1];
+                }
+                const int m = p / nt, nn = p - m * nt;
+                send(16 * m + r, nn * 8 + c2, v0, v1);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (p_lo + i >= p_hi) break;
+                const int m = pinfo[i] & 15, col = pinfo[i] >> 16;
+                send(16 * m + g, col, acc[i][0], acc[i][1]);
+                send(16 * m + g + 8, col, acc[i][2], acc[i][3]);
+            }
+        }
+        bool xok = mbar_wait<true>(xr, (xc >> 1) & 1u, a.status, failed, a.wait_limit);
+        xok = consumers_all(xok);
+        ++xc;
+        if (!xok) {
+            failed = true;
+            break;
+        }
+        // owned pairs: the C partials in rank order, v for k < r_n
+        for (int j = tid; j < mine; j += GB_CONSUMERS * 32) {
+            const int P = (int)crank + j * (int)C;
+            float v0 = 0.f, v1 = 0.f;
+            for (uint32_t c = 0; c < C; ++c) {
+                const float2 pv = lds64f(rbuf + ((c * (uint32_t)spc + (uint32_t)j) * 2u) * 4u);
+                v0 += pv.x;
+                v1 += pv.y;
+            }
+            const int e = 2 * P, row = e / W, col = e - row * W;
+            const int s = col / r8, k = col - s * r8;
+            float *vr = a.v + ((int64_t)s * a.T + xrows[row]) * a.r_max;
+            if (k < r_n) vr[k] = v0;
+            if (k + 1 < r_n) vr[k + 1] = v1;
+        }
+        if (MODE == MODE_FUSED && (flags & GB_UNIT_DONE)) {
+            __threadfence();
+            consumer_sync();
+            if (tid == 0) atomicAdd(a.done + unit, 1);
+        } else {
+            consumer_sync();   // xrows and the exchange buffer are reused by the next pass
+        }
+    }
+    return gi;
+}
+
+// Phase 2: expand chunks from stage gi until the end of the stream.
+template <int MODE>
+__device__ void gb_consume_expand(const GbArgs &a, const GbSmem &sm, uint32_t gi, bool &failed) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t vhi[4][4], vlo[4][4];
+    int em = 0, ecg = 0, ewpm = 1, nkb = 0;
+    bool eactive = false;
+    for (;; ++gi) {
+        if (!gb_stage_wait(a, sm, gi, failed)) break;
+        const int st = (int)(gi % (uint32_t)a.stages);
+        const GbHdr *h = gb_hdr(sm, st);
+        if (h->kind != GB_EXPAND) break;   // the end of the stream
+        const uint32_t stg = sm.ring + (uint32_t)st * GB_SB;
+        const int flags = h->flags;
+        const int cnt = h->cnt, r_n = h->r_n, r8 = h->r8;
+        if (flags & GB_FIRST) {   // a new item: s v fragments of this warp's m16 tile
+            const int mtt = (cnt + 15) >> 4;
+            const int mtp = mtt <= 1 ? 1 : (mtt <= 2 ? 2 : 4);
+            ewpm = GB_CONSUMERS / mtp;
+            em = warp % mtp;
+            ecg = warp / mtp;
+            eactive = em < mtt;
+            nkb = (r_n + 15) >> 4;
+            const float scale = h->scale;
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                float p[4] = {0.f, 0.f, 0.f, 0.f}, q[4] = {0.f, 0.f, 0.f, 0.f};
+                const int k = kb * 16 + 4 * t;
+                const int rg = 16 * em + g, rh = rg + 8;
+                if (kb < nkb && k < r8) {
+                    if (rg < cnt) {
+                        const float4 v = lds128f(stg + (uint32_t)((rg * r8 + k) * 4));
+                        p[0] = v.x; p[1] = v.y; p[2] = v.z; p[3] = v.w;
+                    }
+                    if (rh < cnt) {
+                        const float4 v = lds128f(stg + (uint32_t)((rh * r8 + k) * 4));
+                        q[0] = v.x; q[1] = v.y; q[2] = v.z; q[3] = v.w;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    p[i] = k + i < r_n ? scale * p[i] : 0.f;
+                    q[i] = k + i < r_n ? scale * q[i] : 0.f;
+                }
+                vhi[kb][0] = pack_bf16x2(p[0], p[1]);
+                vhi[kb][1] = pack_bf16x2(q[0], q[1]);
+                vhi[kb][2] = pack_bf16x2(p[2], p[3]);
+                vhi[kb][3] = pack_bf16x2(q[2], q[3]);
+                vlo[kb][0] = pack_bf16x2(p[0] - bf16_lo(vhi[kb][0]), p[1] - bf16_hi(vhi[kb][0]));
+                vlo[kb][1] = pack_bf16x2(q[0] - bf16_lo(vhi[kb][1]), q[1] - bf16_hi(vhi[kb][1]));
+                vlo[kb][2] = pack_bf16x2(p[2] - bf16_lo(vhi[kb][2]), p[3] - bf16_hi(vhi[kb][2]));
+                vlo[kb][3] = pack_bf16x2(q[2] - bf16_lo(vhi[kb][3]), q[3] - bf16_hi(vhi[kb][3]));
+            }
+        }
+        const int w = h->w;
+        if (w > 0) {
+            const int YS = 2 * h->cw + 16;
+            const uint32_t ybase = stg + (uint32_t)h->yofs, bbase = stg + (uint32_t)h->bofs;
+            const int nblk = w >> 3;
+            if (eactive) {
+                for (int b0 = ecg * 2; b0 < nblk; b0 += 2 * ewpm) {
+                    float d[2][4];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) d[j][e] = 0.f;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        if (kb < nkb) {
+                            const int k = kb * 16 + 4 * t;
+                            uint2 bv[2];
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                bv[j] = make_uint2(0, 0);
+                                if (k < r_n && b0 + j < nblk) {
+                                    bv[j] = lds64(bbase + b_off((b0 + j) * 8 + g, k, r8));
+                                    if (k + 4 > r_n) {   // the rank ends inside this group of 4
+                                        const int keep = r_n - k;
+                                        if (keep < 2) bv[j].x &= 0xffffu;
+                                        if (keep < 3) bv[j].y = 0;
+                                        else bv[j].y &= 0xffffu;
+                                    }
+                                }
+                            }
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) mma16816(d[j], vhi[kb], bv[j].x, bv[j].y);
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) mma16816(d[j], vlo[kb], bv[j].x, bv[j].y);
+                        }
+                    }
+                    // y += delta in shared memory (rows g, g+8 of the tile; columns 2t, 2t+1)
+                    const int rg = 16 * em + g, rh = rg + 8;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        if (b0 + j >= nblk) continue;
+                        const uint32_t col2 = (uint32_t)(((b0 + j) * 8 + 2 * t) * 2);
+                        if (rg < cnt) {
+                            const uint32_t ad = ybase + (uint32_t)(rg * YS) + col2;
+                            const uint32_t yv = lds32(ad);
+                            sts32(ad, pack_bf16x2(bf16_lo(yv) + d[j][0], bf16_hi(yv) + d[j][1]));
+                        }
+                        if (rh < cnt) {
+                            const uint32_t ad = ybase + (uint32_t)(rh * YS) + col2;
+                            const uint32_t yv = lds32(ad);
+                            sts32(ad, pack_bf16x2(bf16_lo(yv) + d[j][2], bf16_hi(yv) + d[j][3]));
+                        }
+                    }
+                }
+            }
+            consumer_sync();
+            const int ypc = w >> 3;
+            const int s = h->s0;
+            __nv_bfloat16 *ydst = a.y + a.sl.col_off[s] + h->c0;
+            const unsigned char *yg =
+                reinterpret_cast<const unsigned char *>(__cvta_shared_to_generic(ybase));
+            for (int idx = tid; idx < cnt * ypc; idx += GB_CONSUMERS * 32) {
+                const int r = idx / ypc, pc = idx - r * ypc;
+                *reinterpret_cast<uint4 *>(ydst + (int64_t)h->rows[r] * a.ld_y + pc * 8) =
+                    *reinterpret_cast<const uint4 *>(yg + r * YS + pc * 16);
+            }
+        }
+        gb_release(sm, st);
+    }
+}
+
+template <int MODE>
+__device__ void gb_consumers(const GbArgs &a, const GbSmem &sm, bool &failed) {
+    uint32_t gi = 0;
+    if (MODE != MODE_EXPAND) gi = gb_consume_shrink<MODE>(a, sm, failed);
+    if (MODE != MODE_SHRINK && !failed) gb_consume_expand<MODE>(a, sm, gi, failed);
+}
+
+// Persistent launch: clusters of C blocks; every block runs both phases.
+template <int MODE>
+__global__ void __launch_bounds__(GB_THREADS, 1) bgmv_kernel(const __grid_constant__ GbArgs a) {
+    extern __shared__ __align__(128) unsigned char gb_sm[];
+    const int tid = threadIdx.x;
+    const uint32_t base = (smem_u32(gb_sm) + 1023u) & ~1023u;
+    GbSmem sm;
+    const int NS = a.stages;
+    sm.ring = base;
+    sm.hdr = sm.ring + (uint32_t)NS * GB_SB;
+    uint32_t p = sm.hdr + (uint32_t)NS * GB_HDR;
+    sm.recv = p;
+    if (MODE != MODE_EXPAND) p += 2u * GB_XBUF * 4u;
+    sm.part = p;
+    if (MODE != MODE_EXPAND) p += GB_PART * 4u;
+    sm.xrows = p;
+    p += GB_ROWS * 4u;
+    sm.tkslot = p;
+    p += GB_TK * 4u;
+    const uint32_t flag_s = p;
+    p += 16u;
+    p = (p + 7u) & ~7u;
+    sm.full0 = p;
+    sm.empty0 = p + 8u * GB_MAX_STAGES;
+    sm.xready0 = p + 16u * GB_MAX_STAGES;
+    sm.tkbar0 = sm.xready0 + 16u;
+    sm.tkfree0 = sm.tkbar0 + 8u * GB_TK;
+    sm.flag = reinterpret_cast<int *>(__cvta_shared_to_generic(flag_s));
 
     const int S = a.sl.n;
-    BgSmem sm;
-    // ring on a 1 KB boundary: swizzled TMA boxes need their 1 KB atom aligned
-    sm.ring = bg_sm + ((1024u - (smem_u32(bg_sm) & 1023u)) & 1023u);
-    sm.recv = reinterpret_cast<float *>(sm.ring + BG_RING_BYTES);
-    sm.vfull = sm.recv + S * BG_ROWS * BG_RMAX;
-    sm.part = sm.vfull + S * BG_ROWS * BG_VF_STRIDE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm.part + BG_ROWS * BG_RMAX);
-    sm.rows = rows_sm;
-    sm.ring_s = smem_u32(sm.ring);
-    sm.full0 = smem_u32(bars);
-    sm.empty0 = sm.full0 + 8 * BG_MAX_STAGES;
-    sm.xready = sm.full0 + 16 * BG_MAX_STAGES;
-    sm.vready = sm.xready + 8;
-
-    const int tid = threadIdx.x;
-    if (tid >= BG_CONSUMERS * 32 && tid - BG_CONSUMERS * 32 < S) {   // producer lanes: descriptors
-        const int s = tid - BG_CONSUMERS * 32;
-        if (MODE != MODE_EXPAND) prefetch_tmap(&a.tmA[s]);   // only the maps this mode built
-        if (MODE != MODE_SHRINK) prefetch_tmap(&a.tmB[s]);
-    }
+    const uint32_t C = cluster_size();
     if (tid == 0) {
-        for (int st = 0; st < BG_MAX_STAGES; ++st) {
+        for (int st = 0; st < NS; ++st) {
             mbar_init(sm.full0 + 8 * st, 1);
-            mbar_init(sm.empty0 + 8 * st, BG_CONSUMERS);
+            mbar_init(sm.empty0 + 8 * st, GB_CONSUMERS);
         }
-        mbar_init(sm.xready, 1);   // per unit: the expect_tx arrival, then C x the owned partials' bytes
-        mbar_init(sm.vready, 1);
+        mbar_init(sm.xready0, 1);   // per exchange: the expect_tx arrival, then the partials' bytes
+        mbar_init(sm.xready0 + 8, 1);
+        for (int j = 0; j < GB_TK; ++j) {
+            mbar_init(sm.tkbar0 + 8 * j, 1);
+            mbar_init(sm.tkfree0 + 8 * j, C);   // used on cluster rank 0: one arrival per block
+        }
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    cg::cluster_group cluster = cg::this_cluster();
-
-    // Every block of a cluster walks the same units and takes the same branches,
-    // so the cluster barriers below always pair up; a block whose wait ran out
-    // keeps walking (its waits then return at once) instead of leaving early.
-    bool failed = false;
-    uint32_t base = 0, uiter = 0;
-    const int live = n_live_units(a.tiles);
-    for (int v = blockIdx.y; v < live; v += gridDim.y) {
-        const Unit u = resolve_live_unit(a.tiles, v);
-        if (u.cnt == 0) continue;
-        const int r_n = a.ranks[u.id];
-        if (r_n < 1 || r_n > a.r_max) {
-            if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
-            continue;
+    if (tid >= GB_CONSUMERS * 32 && tid - GB_CONSUMERS * 32 < S) {   // descriptors this mode uses
+        const int s = tid - GB_CONSUMERS * 32;
+        for (int i = 0; i < 4; ++i) {
+            if (MODE != MODE_EXPAND && (8 << i) <= a.r_max) prefetch_tmap(&a.tmA[s][i]);
+            if (MODE != MODE_SHRINK && (8 << i) <= a.r_max) prefetch_tmap(&a.tmB[s][i]);
         }
-        if (uiter > 0) cluster.sync();   // the previous unit is done in every block
-        if (tid < BG_ROWS) rows_sm[tid] = tid < u.cnt ? u.row(a.tiles, tid) : -1;
-        for (int e = tid; e < S * BG_ROWS * BG_VF_STRIDE; e += BG_THREADS) sm.vfull[e] = 0.f;
-        cluster.sync();                  // barriers, rows and zeroed s*v ready in every block
-        base += bgmv_unit<MODE>(a, sm, u, r_n, base, uiter, failed);
-        ++uiter;
     }
-    cluster.sync();   // no block leaves while a peer may still write to it
+    cluster_barrier();   // barriers of every block initialised before any remote arrival
+
+    bool failed = false;
+    if (tid >= GB_CONSUMERS * 32)
+        gb_producer<MODE>(a, sm, failed);
+    else
+        gb_consumers<MODE>(a, sm, failed);
+
+    cluster_barrier();   // no block leaves while a peer may still write to it
+    if (MODE == MODE_FUSED) {
+        // the last block out puts the tickets and the per-unit counters back to zero
+        if (tid == 0) {
+            __threadfence();
+            const int old = atomicAdd(a.ctl + GB_T_EXIT, 1);
+            *sm.flag = old == (int)gridDim.x - 1;
+        }
+        __syncthreads();
+        if (*sm.flag) {
+            __threadfence();
+            const int live = n_live_units(a.tiles);
+            for (int u = tid; u < live; u += GB_THREADS) a.done[u] = 0;
+            if (tid == 0) {
+                a.ctl[GB_T_SHRINK] = 0;
+                a.ctl[GB_T_EXPAND] = 0;
+                a.ctl[GB_T_EXIT] = 0;
+            }
+        }
+    }
 }
 
 namespace {
 
-const void *bg_fn(int mode) {
+const void *gb_fn(int mode) {
     return mode == MODE_FUSED    ? (const void *)bgmv_kernel<MODE_FUSED>
            : mode == MODE_SHRINK ? (const void *)bgmv_kernel<MODE_SHRINK>
                                  : (const void *)bgmv_kernel<MODE_EXPAND>;
 }
 
 // Clusters of `cluster` blocks with `smem` bytes each that fit the device at once
-// (0 if the query fails).
-int bg_active_clusters(int mode, int cluster, size_t smem) {
+// (0 if the query fails); the shared-memory limit is set once per device and mode.
+int gb_active_clusters(int mode, int cluster, size_t smem) {
     struct Key {
         int dev, mode, cluster;
         size_t smem;
@@ -614,13 +992,13 @@ int bg_active_clusters(int mode, int cluster, size_t smem) {
                 cache[i].smem == smem)
                 return cache[i].n;
     }
-    const void *fn = bg_fn(mode);
+    const void *fn = gb_fn(mode);
     int n = 0;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)bgmv_smem_bytes(LORA_MAX_SLICES)) == cudaSuccess) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+        cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(cluster, 1, 1);
-        cfg.blockDim = dim3(BG_THREADS, 1, 1);
+        cfg.blockDim = dim3(GB_THREADS, 1, 1);
         cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -639,31 +1017,30 @@ int bg_active_clusters(int mode, int cluster, size_t smem) {
 
 }  // namespace
 
-// Persistent launch: as many clusters as fit the device at once (at most one
-// per unit of the tile-list capacity); each walks the live units.
-int launch_bgmv(int mode, const BgArgs &args, int n_units, int cluster, cudaStream_t st) {
-    if (n_units <= 0) return LORA_OK;
-    // Two 36 KB stages: chunks twice as wide as with three 24 KB stages up to rank
-    // 48 (half the gathered-row copies), and the whole shrink stream of a decode
-    // unit in flight at once.  Measured on B200 (graph-timed): decode q_proj
-    // kernel 21.8 us against 24.8 with three stages; Llama-3-8B layer set at
-    // decode 583 against 587 us.
-    BgArgs a = args;
-    a.stages = 2;
-    if (const char *e = std::getenv("LORA_BG_STAGES"))   // tuning override: 2 or 3
-        if (std::atoi(e) == 3) a.stages = 3;
-    const size_t smem = bgmv_smem_bytes(a.sl.n);
-    int clusters = bg_active_clusters(mode, cluster, smem);
+// Workspace of the fused mode: the control words (GB_CTL_INTS ints), one
+// counter per unit, then v [S][T][r_max] fp32; each part 256-byte aligned.
+size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max) {
+    const size_t head = (size_t)GB_CTL_INTS * 4 + (((size_t)units * 4 + 255) & ~(size_t)255);
+    return head + (size_t)n_slices * (size_t)T * (size_t)r_max * 4;
+}
+
+// Persistent launch: as many clusters as fit the device at once.
+int launch_bgmv(int mode, const GbArgs &args, int cluster, cudaStream_t st) {
+    GbArgs a = args;
+    // the exchange buffers of the shrink modes leave room for 4 stages; expand-only takes 6
+    const int max_stages = mode == MODE_EXPAND ? GB_MAX_STAGES : 4;
+    if (a.stages < 2 || a.stages > max_stages) a.stages = GB_STAGES_DEFAULT;
+    const size_t smem = bgmv_smem_bytes(mode, a.stages);
+    int clusters = gb_active_clusters(mode, cluster, smem);
     if (clusters < 1) {
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         clusters = sms / cluster > 0 ? sms / cluster : 1;
     }
-    clusters = clusters < n_units ? clusters : n_units;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cluster, clusters, 1);
-    cfg.blockDim = dim3(BG_THREADS, 1, 1);
+    cfg.gridDim = dim3(cluster * clusters, 1, 1);
+    cfg.blockDim = dim3(GB_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

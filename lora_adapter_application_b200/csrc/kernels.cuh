@@ -9,35 +9,42 @@ namespace lora {
 
 enum { MODE_FUSED = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 
-// Tensor maps of the fused kernel (bf16 2-D views of the stacked adapters),
-// K = 16 ranks per box when r_max % 16 == 0, else 8:
-//   A_s as [N*r_max rows][d_in], boxes of K rows x 64 columns, 128-byte swizzle
-//   B_s as [N*d_out rows][r_max], boxes of 64 rows x K ranks
+// Tensor maps of the fused kernel, per slice and per box rank R = 8, 16, 32, 64
+// (index 0..3; only R <= r_max are built):
+//   A_s as [N*r_max rows][d_in], boxes of R rows x 64 columns, 128-byte swizzle
+//   B_s as [N*d_out rows][r_max], boxes of 64 rows x R ranks, swizzle of 2R bytes
+//       (none for R = 8)
 constexpr int BG_ABOX_COLS = 64;
 constexpr int BG_BBOX_ROWS = 64;
-// row_stride: elements between consecutive rows (0 = inner, densely packed)
+// row_stride: elements between consecutive rows (0 = inner, densely packed);
+// swizzle: 0 (none), 32, 64 or 128 bytes
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
-                  uint32_t box_inner, uint32_t box_outer, bool swizzle128,
+                  uint32_t box_inner, uint32_t box_outer, int swizzle,
                   uint64_t row_stride = 0);
 
-struct BgArgs {
-    CUtensorMap tmA[LORA_MAX_SLICES];
-    CUtensorMap tmB[LORA_MAX_SLICES];
+struct GbArgs {
+    CUtensorMap tmA[LORA_MAX_SLICES][4];
+    CUtensorMap tmB[LORA_MAX_SLICES][4];
     const __nv_bfloat16 *x;
     int64_t ld_x;
     int d_in;
     __nv_bfloat16 *y;
     int64_t ld_y;
-    float *v;          // [S][T][r_max] fp32 (shrink / expand modes)
+    float *v;          // [S][T][r_max] fp32: the caller's (shrink / expand modes) or the workspace's
     int T;
     Slices sl;
     int r_max;
     const int32_t *ranks;
-    const float *scales;
+    const float *alphas;
     Tiles tiles;
     int32_t *status;
-    int ab16;          // adapters in 16-rank boxes (r_max % 16 == 0): A 64 x 16, B 16 x 64
-    int stages;        // ring stages, 2 or 3, over the same ring bytes (set by launch_bgmv)
+    int *ctl;          // fused mode: tickets and exit counter (workspace head)
+    int *done;         // fused mode: per unit, shrink blocks finished
+    int bc;            // columns of one expand item (multiple of 64)
+    int blk_off[LORA_MAX_SLICES + 1];   // expand items per unit: slice s owns [blk_off[s], blk_off[s+1])
+    int stages;        // ring stages (2 .. 6)
+    unsigned wait_limit;   // tries of a bounded wait (WAIT_LIMIT; shorter for the stall test hook)
+    int dbg_stall;     // test hook: every block's first stage expects 16 bytes that never come
 };
 
 struct SimtArgs {
@@ -51,7 +58,7 @@ struct SimtArgs {
     Slices sl;
     int r_max;
     const int32_t *ranks;
-    const float *scales;
+    const float *alphas;
     Tiles tiles;
     int32_t *status;
 };
@@ -79,7 +86,7 @@ struct TcArgs {
     Slices sl;
     int r_max;
     const int32_t *ranks;
-    const float *scales;
+    const float *alphas;
     const int4 *contig;
     const int32_t *counts;
     int max_contig;
@@ -93,14 +100,21 @@ int cuda_rc(cudaError_t e);
 // records a failure without a runtime error code (e.g. a driver call) and returns LORA_ERR_CUDA
 int cuda_fail(const char *what);
 
+// lora_api.cu: the lora_meta checks every entry point makes (LORA_OK or an error)
+int check_meta_args(const lora_meta *m);
+
 // segments.cu
 size_t segments_scratch_bytes(int T, int N);
 int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
                           size_t scratch_bytes, int32_t *status, cudaStream_t st);
 
-// bgmv.cu: bf16, r_max <= 64, vector-aligned data; grid = cluster x n_units
-size_t bgmv_smem_bytes(int n_slices);
-int launch_bgmv(int mode, const BgArgs &a, int n_units, int cluster, cudaStream_t st);
+// bgmv.cu: bf16, r_max <= 64 and a multiple of 8, n_slices * r_max <= 512,
+// 16-byte aligned rows; units of up to LORA_MAX_TILE_ROWS rows; persistent
+// clusters of `cluster` blocks (1 for the expand-only mode)
+size_t bgmv_smem_bytes(int mode, int stages);
+int launch_bgmv(int mode, const GbArgs &a, int cluster, cudaStream_t st);
+// workspace of the fused mode: control words, then one int per unit, then v
+size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max);
 
 // sgmv_tc.cu: bf16, r_max % 16 == 0, n_slices * r_max <= 128, 16-byte aligned rows;
 // chooses the cluster size and ring depth, launches persistent clusters

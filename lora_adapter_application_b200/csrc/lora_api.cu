@@ -1,6 +1,7 @@
 // C ABI of the multi-LoRA delta library: argument checks and the choice of
 // kernel for each unit of work.  Declarations and contracts: lora_delta.h.
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 #include <cstdint>
 #include <cstdio>
@@ -32,62 +33,59 @@ int cuda_fail(const char *what) {
 
 namespace {
 
-// Blocks per unit of the fused kernel.  Measured on B200 (persistent grid,
-// about two blocks per SM): 4 suits decode batches from the q_proj shape to
-// the Llama-3-8B layer set; 8 when the units are few - the gathered rows of a
-// batch whose prompt runs went to the tensor-core kernel (est_units = 1), or
-// a tile list of a handful of units; 2 when those gathered rows run beside a
-// tensor-core launch that leaves SMs free (idle_sms): 2-block clusters fit
-// there, 8-block ones wait for it to finish.
-int bgmv_cluster(int est_units, int idle_sms = 0) {
-    if (const char *e = std::getenv("LORA_BG_CLUSTER")) {   // tuning override: 1, 2, 4 or 8
-        const int c = std::atoi(e);
-        if (c == 1 || c == 2 || c == 4 || c == 8) return c;
-    }
-    if (idle_sms >= 16) return 2;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return (int64_t)est_units * 4 * 2 < sms ? 8 : 4;
-}
-
-// A second stream per device for the gathered-tile launch of a call whose
-// contiguous tiles take the tensor-core kernel: forked from and joined back to
-// the caller's stream with events (also under stream capture), so that its
-// blocks fill the SMs the persistent tensor-core grid leaves free.  The two
-// launches touch disjoint rows.
+// A second stream for the gathered-tile launch of a call whose contiguous
+// tiles take the tensor-core kernel: forked from and joined back to the
+// caller's stream with events, so that its blocks fill the SMs the persistent
+// tensor-core grid leaves free.  The two launches touch disjoint rows.  Each
+// (device, caller stream) pair has a side stream and events of its own, so
+// calls on different caller streams never meet on a shared stream - neither in
+// eager use nor while one of them is being captured into a CUDA graph.
 struct SideStream {
+    int dev = -1;
+    cudaStream_t caller = nullptr;
     cudaStream_t stream = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
 };
-constexpr int kSideDevices = 64;
+constexpr int kSideStreams = 256;
 std::mutex g_side_mu;
-SideStream g_side[kSideDevices];
+SideStream g_side[kSideStreams];
+int g_side_used = 0;
 
 // fn(side stream) between a fork from and a join into `caller`: work fn puts on
 // `caller` after the fork and work it puts on the side stream may overlap.
+// Past kSideStreams distinct caller streams, both launches go to `caller`.
 template <class F>
 int with_side_stream(cudaStream_t caller, F &&fn) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_rc(e);
-    if (dev < 0 || dev >= kSideDevices) return fn(caller);
-    std::lock_guard<std::mutex> lock(g_side_mu);   // one fork/join sequence at a time
-    SideStream &ss = g_side[dev];
-    if (!ss.stream) {
-        if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess ||
-            (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
-            (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) {
-            ss = SideStream{};
-            return cuda_rc(e);
+    SideStream *ss = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_side_mu);
+        for (int i = 0; i < g_side_used; ++i)
+            if (g_side[i].dev == dev && g_side[i].caller == caller) {
+                ss = &g_side[i];
+                break;
+            }
+        if (!ss && g_side_used < kSideStreams) {
+            SideStream n;
+            n.dev = dev;
+            n.caller = caller;
+            if ((e = cudaStreamCreateWithFlags(&n.stream, cudaStreamNonBlocking)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_rc(e);
+            g_side[g_side_used] = n;
+            ss = &g_side[g_side_used++];
         }
     }
-    if ((e = cudaEventRecord(ss.fork, caller)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(ss.stream, ss.fork, 0)) != cudaSuccess)
+    if (!ss) return fn(caller);
+    if ((e = cudaEventRecord(ss->fork, caller)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess)
         return cuda_rc(e);
-    const int rc = fn(ss.stream);
-    if ((e = cudaEventRecord(ss.join, ss.stream)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(caller, ss.join, 0)) != cudaSuccess)
+    const int rc = fn(ss->stream);
+    if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(caller, ss->join, 0)) != cudaSuccess)
         return cuda_rc(e);
     return rc;
 }
@@ -98,7 +96,7 @@ int check_meta(const lora_meta *m) {
     if (!m) return LORA_ERR_NULL;
     if (m->T < 0 || m->T > LORA_MAX_ROWS || m->N < 1 || m->N > LORA_MAX_ADAPTERS)
         return LORA_ERR_SHAPE;
-    if (m->rows_per_tile < 1 || m->rows_per_tile > 16 || m->min_run < 0 || m->long_tile < 1 ||
+    if (m->rows_per_tile < 1 || m->rows_per_tile > LORA_MAX_TILE_ROWS || m->min_run < 0 || m->long_tile < 1 ||
         m->long_tile > LORA_LONG_TILE)
         return LORA_ERR_SHAPE;
     int32_t mg = 0, mc = 0;
@@ -120,21 +118,23 @@ struct Call {
     int32_t n_slices;
     int32_t r_max;
     const int32_t *ranks;
-    const float *scales;
+    const float *alphas;
     const float *v_in;
     float *v_out;
     const lora_meta *meta;
+    void *ws;
+    size_t ws_bytes;
     lora_dtype dtype;
     int32_t *status;
     cudaStream_t stream;
 };
 
-// need_x / need_y / need_scales: which operands the mode reads
-int check_call(const Call &c, bool need_x, bool need_y, bool need_scales, bool need_v) {
+// need_x / need_y / need_alphas: which operands the mode reads
+int check_call(const Call &c, bool need_x, bool need_y, bool need_alphas, bool need_v) {
     if (!c.slices || !c.ranks || !c.status) return LORA_ERR_NULL;
     if (need_x && !c.x) return LORA_ERR_NULL;
     if (need_y && !c.y) return LORA_ERR_NULL;
-    if (need_scales && !c.scales) return LORA_ERR_NULL;
+    if (need_alphas && !c.alphas) return LORA_ERR_NULL;
     if (need_v && !(c.v_in || c.v_out)) return LORA_ERR_NULL;
     if (c.dtype != LORA_BF16 && c.dtype != LORA_FP32) return LORA_ERR_DTYPE;
     int rc = check_meta(c.meta);
@@ -204,10 +204,12 @@ Tiles make_tiles(const lora_meta *m, bool gather, bool contig) {
 
 int n_units(const Tiles &t) { return t.max_gather + (t.subs ? t.max_contig * t.subs : 0); }
 
-// The vectorised bf16 tensor-pipe kernel takes the call?  It moves 16-byte
-// pieces, so every row start and width must be a multiple of 8 elements.
-bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
+// The fused BGMV kernel takes the call?  bf16, rank slots of at most 64 in
+// multiples of 8, and 16-byte aligned rows, slices and v (it moves data with
+// TMA copies).
+bool bgmv_ok(int mode, const Call &c, bool need_x, bool need_y) {
     if (c.dtype != LORA_BF16 || c.r_max > 64 || (c.r_max & 7) || !rows_fit_int32(c)) return false;
+    if ((int64_t)c.meta->T * c.n_slices * c.r_max > ((int64_t)1 << 31) - 1) return false;
     if (need_x) {
         if ((c.d_in & 7) || (c.ld_x & 7) || !aligned(c.x, 16)) return false;
         for (int s = 0; s < c.n_slices; ++s)
@@ -219,6 +221,8 @@ bool bgmv_ok(const Call &c, bool need_x, bool need_y) {
             if ((c.slices[s].d_out & 7) || (c.slices[s].col_off & 7) || !aligned(c.slices[s].B, 16))
                 return false;
     }
+    if (mode != MODE_FUSED && !aligned(mode == MODE_SHRINK ? (const void *)c.v_out : (const void *)c.v_in, 16))
+        return false;
     return true;
 }
 
@@ -284,7 +288,7 @@ bool run_tc(int mode, const Call &c, int *rc, int *idle_sms) {
     a.sl = make_slices(c);
     a.r_max = c.r_max;
     a.ranks = c.ranks;
-    a.scales = c.scales;
+    a.alphas = c.alphas;
     a.contig = reinterpret_cast<const int4 *>(c.meta->contig_tiles);
     a.counts = c.meta->counts;
     a.max_contig = c.meta->max_contig_tiles;
@@ -293,47 +297,108 @@ bool run_tc(int mode, const Call &c, int *rc, int *idle_sms) {
     return *rc != LORA_ERR_SHAPE;
 }
 
+int env_int(const char *name, int dflt) {
+    const char *e = std::getenv(name);
+    return e ? std::atoi(e) : dflt;
+}
+
+int device_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// Blocks per cluster of the fused kernel's shrink: one per 1024 input columns
+// (up to 8), so that a unit's A reaches the cluster in about 1024 columns per
+// block; the expand-only mode needs no cluster.  Tuning override:
+// LORA_BG_CLUSTER = 1, 2, 4 or 8.
+int bgmv_cluster(int mode, int d_in) {
+    if (mode == MODE_EXPAND) return 1;
+    const int e = env_int("LORA_BG_CLUSTER", 0);
+    if (e == 1 || e == 2 || e == 4 || e == 8) return e;
+    return d_in <= 1536 ? 1 : (d_in <= 3072 ? 2 : (d_in <= 6144 ? 4 : 8));
+}
+
+// Output columns of one expand item: the widest of 2048 .. 256 that still gives
+// about six items per block for the batch's expected units (the expand phase
+// is balanced by handing out many items of similar size).  Tuning override:
+// LORA_BG_ITEM_COLS, a multiple of 64 from 64 to 8192.
+int bgmv_item_cols(const Call &c, int est_units) {
+    const int e = env_int("LORA_BG_ITEM_COLS", 0);
+    if (e >= 64 && e <= 8192 && (e & 63) == 0) return e;
+    const int target = 6 * device_sms();
+    for (int bc = 2048; bc > 256; bc >>= 1) {
+        int64_t items = 0;
+        for (int s = 0; s < c.n_slices; ++s) items += (c.slices[s].d_out + bc - 1) / bc;
+        if (items * est_units >= target) return bc;
+    }
+    return 256;
+}
+
 // The gathered tiles (and the contiguous ones unless tc_took) on the fused
 // kernel, or the general kernel when the data does not suit it, on `stream`.
-int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took, int idle_sms,
-                cudaStream_t stream) {
+int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took, cudaStream_t stream) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
     Tiles tiles = make_tiles(c.meta, gather, contig);
     const int units = n_units(tiles);
     if (c.meta->T == 0 || units == 0) return LORA_OK;
-    bool maps_ok = units <= 65535 && bgmv_ok(c, need_x, need_y);
-    if (maps_ok) {
-        BgArgs bg{};
-        for (int s = 0; s < c.n_slices && maps_ok; ++s) {
-            const int N = c.meta->N;
-            // 16-rank boxes when the slot rank allows: half the TMA operations, and B
-            // comes in 32-byte pieces (full sectors) instead of 16-byte ones
-            const uint32_t kbox = (c.r_max & 15) == 0 ? 16 : 8;
-            if (need_x)
-                maps_ok = tensor_map_2d(&bg.tmA[s], c.slices[s].A, (uint64_t)c.d_in,
-                                        (uint64_t)N * c.r_max, BG_ABOX_COLS, kbox, true) == LORA_OK;
-            if (need_y && maps_ok)
-                maps_ok = tensor_map_2d(&bg.tmB[s], c.slices[s].B, (uint64_t)c.r_max,
-                                        (uint64_t)N * c.slices[s].d_out, kbox, BG_BBOX_ROWS,
-                                        false) == LORA_OK;
-        }
+    (void)tc_took;
+    if (bgmv_ok(mode, c, need_x, need_y)) {
+        GbArgs g{};
+        bool maps_ok = true;
+        const int N = c.meta->N;
+        for (int s = 0; s < c.n_slices && maps_ok; ++s)
+            for (int i = 0; i < 4 && maps_ok; ++i) {
+                const int R = 8 << i;
+                if (R > c.r_max) break;
+                if (need_x)
+                    maps_ok = tensor_map_2d(&g.tmA[s][i], c.slices[s].A, (uint64_t)c.d_in,
+                                            (uint64_t)N * c.r_max, BG_ABOX_COLS, (uint32_t)R, 128) == LORA_OK;
+                if (need_y && maps_ok)
+                    maps_ok = tensor_map_2d(&g.tmB[s][i], c.slices[s].B, (uint64_t)c.r_max,
+                                            (uint64_t)N * c.slices[s].d_out, (uint32_t)R, BG_BBOX_ROWS,
+                                            R == 8 ? 0 : 2 * R) == LORA_OK;
+            }
         if (maps_ok) {
-            bg.x = static_cast<const __nv_bfloat16 *>(c.x);
-            bg.ld_x = c.ld_x;
-            bg.d_in = c.d_in;
-            bg.y = static_cast<__nv_bfloat16 *>(c.y);
-            bg.ld_y = c.ld_y;
-            bg.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
-            bg.T = c.meta->T;
-            bg.sl = make_slices(c);
-            bg.r_max = c.r_max;
-            bg.ranks = c.ranks;
-            bg.scales = c.scales;
-            bg.tiles = tiles;
-            bg.status = c.status;
-            bg.ab16 = (c.r_max & 15) == 0 ? 1 : 0;
-            const int cl = tc_took ? bgmv_cluster(1, idle_sms) : bgmv_cluster(units);
-            return launch_bgmv(mode, bg, units, cl, stream);
+            g.x = static_cast<const __nv_bfloat16 *>(c.x);
+            g.ld_x = c.ld_x;
+            g.d_in = c.d_in;
+            g.y = static_cast<__nv_bfloat16 *>(c.y);
+            g.ld_y = c.ld_y;
+            g.T = c.meta->T;
+            g.sl = make_slices(c);
+            g.r_max = c.r_max;
+            g.ranks = c.ranks;
+            g.alphas = c.alphas;
+            g.tiles = tiles;
+            g.status = c.status;
+            if (mode == MODE_FUSED) {   // control words, per-unit counters, v: the workspace
+                unsigned char *ws = static_cast<unsigned char *>(c.ws);
+                g.ctl = reinterpret_cast<int *>(ws);
+                g.done = g.ctl + 64;
+                g.v = reinterpret_cast<float *>(ws + bgmv_workspace_bytes(units, 0, 1, 8));
+            } else {
+                g.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
+            }
+            const int est = std::min(units, std::min(c.meta->N, c.meta->T) +
+                                                (c.meta->T + c.meta->rows_per_tile - 1) / c.meta->rows_per_tile);
+            g.bc = bgmv_item_cols(c, std::max(1, est));
+            g.blk_off[0] = 0;
+            for (int s = 0; s < c.n_slices; ++s)
+                g.blk_off[s + 1] = g.blk_off[s] + (c.slices[s].d_out + g.bc - 1) / g.bc;
+            // tuning override: LORA_BG_STAGES = 2 .. 6 ring stages of 32 KB
+            g.stages = env_int("LORA_BG_STAGES", 4);
+            if (g.stages < 2 || g.stages > 6) g.stages = 4;
+            g.wait_limit = WAIT_LIMIT;
+            int cl = bgmv_cluster(mode, c.d_in);
+            if (env_int("LORA_DEBUG_STALL", 0) == 1) {
+                // test hook for the bounded waits: one-block clusters (every wait bounded,
+                // no peer to leave behind), short waits, and a first stage that never fills
+                g.dbg_stall = 1;
+                g.wait_limit = 64;
+                cl = 1;
+            }
+            return launch_bgmv(mode, g, cl, stream);
         }
     }
     SimtArgs a{};
@@ -347,7 +412,7 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
     a.sl = make_slices(c);
     a.r_max = c.r_max;
     a.ranks = c.ranks;
-    a.scales = c.scales;
+    a.alphas = c.alphas;
     a.tiles = tiles;
     a.status = c.status;
     return launch_simt(mode, c.dtype == LORA_BF16, a, units, stream);
@@ -361,19 +426,37 @@ int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = tr
         return with_side_stream(c.stream, [&](cudaStream_t side) -> int {
             int rc = LORA_OK, idle_sms = 0;
             if (!run_tc(mode, c, &rc, &idle_sms))   // a tensor map could not be encoded
-                return launch_rest(mode, c, gather, true, false, 0, c.stream);
+                return launch_rest(mode, c, gather, true, false, c.stream);
             if (rc != LORA_OK) return rc;
-            return launch_rest(mode, c, gather, false, true, idle_sms, side);
+            return launch_rest(mode, c, gather, false, true, side);
         });
     }
-    return launch_rest(mode, c, gather, contig, false, 0, c.stream);
+    return launch_rest(mode, c, gather, contig, false, c.stream);
+}
+
+// Workspace a fused call needs for this batch metadata and layer shape.
+size_t linear_ws_bytes(const lora_meta *m, int n_slices, int r_max) {
+    const Tiles t = make_tiles(m, true, m->min_run > 0);
+    return bgmv_workspace_bytes(n_units(t), m->T, n_slices, r_max);
+}
+
+// The fused entry points' workspace: present, large enough, 256-byte aligned.
+int check_ws(const Call &c) {
+    if (!c.ws) return LORA_ERR_NULL;
+    if (!aligned(c.ws, 256) || c.ws_bytes < linear_ws_bytes(c.meta, c.n_slices, c.r_max))
+        return LORA_ERR_WORKSPACE;
+    return LORA_OK;
 }
 
 }  // namespace
 
+namespace lora {
+int check_meta_args(const lora_meta *m) { return check_meta(m); }
+}  // namespace lora
+
 extern "C" {
 
-int lora_version(void) { return 100; }
+int lora_version(void) { return 20000; }
 
 const char *lora_last_error(void) { return g_last_error; }
 
@@ -396,7 +479,7 @@ int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int32_t min_
                        int32_t long_tile, int32_t *max_gather, int32_t *max_contig) {
     if (!max_gather || !max_contig) return LORA_ERR_NULL;
     if (T < 0 || T > LORA_MAX_ROWS || N < 1 || N > LORA_MAX_ADAPTERS || rows_per_tile < 1 ||
-        rows_per_tile > 16 || min_run < 0 || long_tile < 1 || long_tile > LORA_LONG_TILE)
+        rows_per_tile > LORA_MAX_TILE_ROWS || min_run < 0 || long_tile < 1 || long_tile > LORA_LONG_TILE)
         return LORA_ERR_SHAPE;
     *max_gather = (T + rows_per_tile - 1) / rows_per_tile + (N < T ? N : T);
     *max_contig = min_run > 0 ? (T + long_tile - 1) / long_tile + T / min_run : 0;
@@ -404,7 +487,7 @@ int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int32_t min_
 }
 
 size_t lora_segments_scratch_bytes(int32_t T, int32_t N) {
-    if (T < 0 || N < 1) return 0;
+    if (T < 0 || T > LORA_MAX_ROWS || N < 1 || N > LORA_MAX_ADAPTERS) return 0;
     return segments_scratch_bytes(T, N);
 }
 
@@ -422,12 +505,19 @@ size_t lora_shrink_workspace_bytes(int32_t T, int32_t r_max, int32_t n_slices) {
     return (size_t)n_slices * (size_t)T * (size_t)r_max * sizeof(float);
 }
 
+size_t lora_linear_workspace_bytes(const lora_meta *meta, int32_t n_slices, int32_t r_max) {
+    if (check_meta(meta) != LORA_OK || n_slices < 1 || n_slices > LORA_MAX_SLICES || r_max < 1 ||
+        r_max > LORA_MAX_RANK)
+        return 0;
+    return linear_ws_bytes(meta, n_slices, r_max);
+}
+
 int lora_sgmv_shrink(float *v, const void *x, int64_t ld_x, int32_t d_in,
                      const lora_slice *slices, int32_t n_slices, int32_t r_max,
                      const int32_t *ranks, const lora_meta *meta, lora_dtype dtype,
                      int32_t *status, void *stream) {
     Call c{nullptr, 0, x, ld_x, d_in, slices, n_slices, r_max, ranks, nullptr, nullptr, v,
-           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+           meta, nullptr, 0, dtype, status, static_cast<cudaStream_t>(stream)};
     int rc = check_call(c, true, false, false, true);
     if (rc != LORA_OK) return rc;
     return run(MODE_SHRINK, c, true, true);
@@ -435,10 +525,10 @@ int lora_sgmv_shrink(float *v, const void *x, int64_t ld_x, int32_t d_in,
 
 int lora_sgmv_expand(void *y, int64_t ld_y, const float *v, const lora_slice *slices,
                      int32_t n_slices, int32_t r_max, const int32_t *ranks,
-                     const float *scales, const lora_meta *meta, lora_dtype dtype,
+                     const float *alphas, const lora_meta *meta, lora_dtype dtype,
                      int32_t *status, void *stream) {
-    Call c{y, ld_y, nullptr, 0, 0, slices, n_slices, r_max, ranks, scales, v, nullptr,
-           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+    Call c{y, ld_y, nullptr, 0, 0, slices, n_slices, r_max, ranks, alphas, v, nullptr,
+           meta, nullptr, 0, dtype, status, static_cast<cudaStream_t>(stream)};
     int rc = check_call(c, false, true, true, true);
     if (rc != LORA_OK) return rc;
     return run(MODE_EXPAND, c, true, true);
@@ -446,22 +536,26 @@ int lora_sgmv_expand(void *y, int64_t ld_y, const float *v, const lora_slice *sl
 
 int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
                     const lora_slice *slices, int32_t n_slices, int32_t r_max,
-                    const int32_t *ranks, const float *scales, const lora_meta *meta,
-                    lora_dtype dtype, int32_t *status, void *stream) {
-    Call c{y, ld_y, x, ld_x, d_in, slices, n_slices, r_max, ranks, scales, nullptr, nullptr,
-           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+                    const int32_t *ranks, const float *alphas, const lora_meta *meta,
+                    void *workspace, size_t workspace_bytes, lora_dtype dtype, int32_t *status,
+                    void *stream) {
+    Call c{y, ld_y, x, ld_x, d_in, slices, n_slices, r_max, ranks, alphas, nullptr, nullptr,
+           meta, workspace, workspace_bytes, dtype, status, static_cast<cudaStream_t>(stream)};
     int rc = check_call(c, true, true, true, false);
+    if (rc == LORA_OK) rc = check_ws(c);
     if (rc != LORA_OK) return rc;
     return run(MODE_FUSED, c, true, true, false);
 }
 
 int lora_add_linear(void *y, int64_t ld_y, const void *x, int64_t ld_x, int32_t d_in,
                     const lora_slice *slices, int32_t n_slices, int32_t r_max,
-                    const int32_t *ranks, const float *scales, const lora_meta *meta,
-                    lora_dtype dtype, int32_t *status, void *stream) {
-    Call c{y, ld_y, x, ld_x, d_in, slices, n_slices, r_max, ranks, scales, nullptr, nullptr,
-           meta, dtype, status, static_cast<cudaStream_t>(stream)};
+                    const int32_t *ranks, const float *alphas, const lora_meta *meta,
+                    void *workspace, size_t workspace_bytes, lora_dtype dtype, int32_t *status,
+                    void *stream) {
+    Call c{y, ld_y, x, ld_x, d_in, slices, n_slices, r_max, ranks, alphas, nullptr, nullptr,
+           meta, workspace, workspace_bytes, dtype, status, static_cast<cudaStream_t>(stream)};
     int rc = check_call(c, true, true, true, false);
+    if (rc == LORA_OK) rc = check_ws(c);
     if (rc != LORA_OK) return rc;
     return run(MODE_FUSED, c, true, true);
 }

@@ -46,12 +46,12 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, unsigned parity) {
             : "memory");
     return ok != 0;
 }
-// Bounded wait; false (and the status bit) once the limit is reached.
+// Bounded wait; false (and the status bit) once `limit` tries have failed.
 template <bool CLUSTER_ACQUIRE = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, int32_t *status,
-                                          bool &failed) {
+                                          bool &failed, unsigned limit = WAIT_LIMIT) {
     if (failed) return false;
-    for (unsigned it = 0; it < WAIT_LIMIT; ++it)
+    for (unsigned it = 0; it < limit; ++it)
         if (mbar_try<CLUSTER_ACQUIRE>(bar, parity)) return true;
     atomicOr(status, LORA_DEV_TIMEOUT);
     failed = true;

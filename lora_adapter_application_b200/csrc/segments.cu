@@ -844,13 +844,13 @@ __global__ void __launch_bounds__(SEG_THREADS) seg_gtiles_kernel(SegArgs a) {
     if (overflow) atomicOr(a.out.status, LORA_DEV_TILE_OVERFLOW);
 }
 
-static size_t ws_bytes(int T, int N) {
-    const size_t n_chunks = (T + SEG_CHUNK - 1) / SEG_CHUNK;
-    return (n_chunks * (size_t)(N + 1) * sizeof(int) + 255) & ~(size_t)255;
+static size_t ws_bytes(int T, int N) {   // size_t throughout: no int overflow for any T, N
+    const size_t n_chunks = ((size_t)T + SEG_CHUNK - 1) / SEG_CHUNK;
+    return (n_chunks * ((size_t)N + 1) * sizeof(int) + 255) & ~(size_t)255;
 }
 
 static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
-static int tw_words(int T) { return (T + 31) / 32; }
+static int tw_words(int T) { return (int)(((int64_t)T + 31) / 32); }
 static int tw_blocks(int T) { return (tw_words(T) + TW_WORDS - 1) / TW_WORDS; }
 
 // per-chunk id counts | run-start byte per row | 3 words per 32 rows | 4 ints per block

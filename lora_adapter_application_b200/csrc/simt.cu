@@ -37,58 +37,62 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_kernel(SimtArgs a) {
         if (tid == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
         return;
     }
-    if (tid < SIMT_ROWS) rows_sm[tid] = tid < u.cnt ? u.row(a.tiles, tid) : -1;
-    __syncthreads();
-    const int cnt = u.cnt;
+    const float scale = MODE == 1 ? 1.f : a.alphas[n] / (float)r_n;
     const E *x = static_cast<const E *>(a.x);
     E *y = static_cast<E *>(a.y);
 
-    if (MODE == 2) {   // expand only: v from global, scaled
-        const float scale = a.scales[n];
-        for (int e = tid; e < S * cnt * r_n; e += SIMT_THREADS) {
-            const int s = e / (cnt * r_n), rem = e - s * cnt * r_n;
-            const int row = rem / r_n, k = rem - row * r_n;
-            vfull[(s * SIMT_ROWS + row) * a.r_max + k] =
-                scale * a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k];
-        }
-    } else {
-        const float scale = MODE == 0 ? a.scales[n] : 1.f;
-        for (int e = warp; e < S * cnt * r_n; e += SIMT_THREADS / 32) {
-            const int s = e / (cnt * r_n), rem = e - s * cnt * r_n;
-            const int row = rem / r_n, k = rem - row * r_n;
-            const E *Ak = static_cast<const E *>(a.sl.A[s]) + ((int64_t)n * a.r_max + k) * a.d_in;
-            const E *xr = x + (int64_t)rows_sm[row] * a.ld_x;
-            float acc = 0.f;
-            for (int j = lane; j < a.d_in; j += 32) acc = fmaf(load_elem(Ak + j), load_elem(xr + j), acc);
+    // the unit's rows, 16 at a time
+    for (int q0 = 0; q0 < u.cnt; q0 += SIMT_ROWS) {
+        const int cnt = min(SIMT_ROWS, u.cnt - q0);
+        __syncthreads();   // the previous group is done with rows_sm and vfull
+        if (tid < SIMT_ROWS) rows_sm[tid] = tid < cnt ? u.row(a.tiles, q0 + tid) : -1;
+        __syncthreads();
+
+        if (MODE == 2) {   // expand only: v from global, scaled
+            for (int e = tid; e < S * cnt * r_n; e += SIMT_THREADS) {
+                const int s = e / (cnt * r_n), rem = e - s * cnt * r_n;
+                const int row = rem / r_n, k = rem - row * r_n;
+                vfull[(s * SIMT_ROWS + row) * a.r_max + k] =
+                    scale * a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k];
+            }
+        } else {
+            for (int e = warp; e < S * cnt * r_n; e += SIMT_THREADS / 32) {
+                const int s = e / (cnt * r_n), rem = e - s * cnt * r_n;
+                const int row = rem / r_n, k = rem - row * r_n;
+                const E *Ak = static_cast<const E *>(a.sl.A[s]) + ((int64_t)n * a.r_max + k) * a.d_in;
+                const E *xr = x + (int64_t)rows_sm[row] * a.ld_x;
+                float acc = 0.f;
+                for (int j = lane; j < a.d_in; j += 32) acc = fmaf(load_elem(Ak + j), load_elem(xr + j), acc);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-            if (lane == 0) vfull[(s * SIMT_ROWS + row) * a.r_max + k] = scale * acc;
+                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+                if (lane == 0) vfull[(s * SIMT_ROWS + row) * a.r_max + k] = scale * acc;
+            }
         }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    if (MODE == 1) {   // shrink only: write v
-        for (int e = tid; e < S * cnt * r_n; e += SIMT_THREADS) {
-            const int s = e / (cnt * r_n), rem = e - s * cnt * r_n;
-            const int row = rem / r_n, k = rem - row * r_n;
-            a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] =
-                vfull[(s * SIMT_ROWS + row) * a.r_max + k];
+        if (MODE == 1) {   // shrink only: write v
+            for (int e = tid; e < S * cnt * r_n; e += SIMT_THREADS) {
+                const int s = e / (cnt * r_n), rem = e - s * cnt * r_n;
+                const int row = rem / r_n, k = rem - row * r_n;
+                a.v[((int64_t)s * a.T + rows_sm[row]) * a.r_max + k] =
+                    vfull[(s * SIMT_ROWS + row) * a.r_max + k];
+            }
+            continue;
         }
-        return;
-    }
 
-    const int total = a.sl.cat_off[S];
-    for (int e = tid; e < total; e += SIMT_THREADS) {
-        int s = 0;
-        while (e >= a.sl.cat_off[s + 1]) ++s;
-        const int c = e - a.sl.cat_off[s];
-        const E *Bc = static_cast<const E *>(a.sl.B[s]) + ((int64_t)n * a.sl.d_out[s] + c) * a.r_max;
-        const float *vs = vfull + s * SIMT_ROWS * a.r_max;
-        for (int row = 0; row < cnt; ++row) {
-            float acc = 0.f;
-            for (int k = 0; k < r_n; ++k) acc = fmaf(load_elem(Bc + k), vs[row * a.r_max + k], acc);
-            E *yp = y + (int64_t)rows_sm[row] * a.ld_y + a.sl.col_off[s] + c;
-            store_elem(yp, load_elem(yp) + acc);
+        const int total = a.sl.cat_off[S];
+        for (int e = tid; e < total; e += SIMT_THREADS) {
+            int s = 0;
+            while (e >= a.sl.cat_off[s + 1]) ++s;
+            const int c = e - a.sl.cat_off[s];
+            const E *Bc = static_cast<const E *>(a.sl.B[s]) + ((int64_t)n * a.sl.d_out[s] + c) * a.r_max;
+            const float *vs = vfull + s * SIMT_ROWS * a.r_max;
+            for (int row = 0; row < cnt; ++row) {
+                float acc = 0.f;
+                for (int k = 0; k < r_n; ++k) acc = fmaf(load_elem(Bc + k), vs[row * a.r_max + k], acc);
+                E *yp = y + (int64_t)rows_sm[row] * a.ld_y + a.sl.col_off[s] + c;
+                store_elem(yp, load_elem(yp) + acc);
+            }
         }
     }
 }

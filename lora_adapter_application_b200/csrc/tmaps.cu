@@ -42,7 +42,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 }  // namespace
 
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
-                  uint32_t box_inner, uint32_t box_outer, bool swizzle128, uint64_t row_stride) {
+                  uint32_t box_inner, uint32_t box_outer, int swizzle, uint64_t row_stride) {
     if (row_stride == 0) row_stride = inner;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -51,7 +51,7 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
         const Entry &e = g_cache[i];
         if (e.base == base && e.inner == inner && e.outer == outer && e.stride == row_stride &&
             e.box_inner == box_inner &&
-            e.box_outer == box_outer && e.swizzle == (int)swizzle128 && e.dev == dev) {
+            e.box_outer == box_outer && e.swizzle == swizzle && e.dev == dev) {
             *out = e.map;
             return LORA_OK;
         }
@@ -65,7 +65,10 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
     CUtensorMap m;
     const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          swizzle == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : swizzle == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                          : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail("cuTensorMapEncodeTiled failed");
     Entry &e = g_cache[g_used < kCache ? g_used++ : (g_next++ % kCache)];
@@ -75,7 +78,7 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
     e.stride = row_stride;
     e.box_inner = box_inner;
     e.box_outer = box_outer;
-    e.swizzle = (int)swizzle128;
+    e.swizzle = swizzle;
     e.dev = dev;
     e.map = m;
     *out = m;

@@ -29,6 +29,8 @@ def main(argv=None):
     ap.add_argument("--layer", type=int, default=0)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--min-run", type=int, default=64, help="shortest run that becomes contiguous tiles (0 = none)")
+    ap.add_argument("--rows-per-tile", type=int, default=lora.MAX_TILE_ROWS,
+                    help="rows per gathered tile (1 .. 64)")
     ap.add_argument("--requests", type=int, default=0, help="prefill / mixed_70b: number of prompts (0 = default)")
     ap.add_argument("--seed", type=int, default=0)
     args = ap.parse_args(argv)
@@ -40,12 +42,12 @@ def main(argv=None):
     x, y = lay.x.to(dev), lay.y0.to(dev)
     A, B = [a.to(dev) for a in lay.A], [b.to(dev) for b in lay.B]
     ids, ranks = w.ids.to(dev), w.ranks.to(dev)
-    scales = lora.scales_for(w.alpha, w.ranks).to(dev)
-    meta = lora.Meta(w.T, w.N, 16, args.min_run, device=dev)
+    alphas = lora.alphas_full(w.alpha, w.N, dev)
+    meta = lora.Meta(w.T, w.N, args.rows_per_tile, args.min_run, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     lora.lora_build_segments(ids, meta, status)
     for _ in range(args.reps):
-        lora.lora_add_linear(y, x, A, B, lay.col_off, ranks, scales, meta, status)
+        lora.lora_add_linear(y, x, A, B, lay.col_off, ranks, alphas, meta, status)
     torch.cuda.synchronize()
     code = int(status.item())
     print(f"{w.name}/{lay.name}: T={w.T} counts={meta.counts.cpu().tolist()} status={code}")

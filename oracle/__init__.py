@@ -50,6 +50,8 @@ def _load():
         lib.oracle_build_segments.restype = ctypes.c_int
         lib.oracle_build_segments.argtypes = [P, I32, I32, I32, I32, I32, I32, I32,
                                               P, P, P, P, P, P, P]
+        lib.oracle_lora_merge.restype = ctypes.c_int
+        lib.oracle_lora_merge.argtypes = [ctypes.c_int, P, I64, I32, I32, P, P, I32, I32, D, I32, P]
         lib.oracle_lora_param_count.restype = I64
         lib.oracle_lora_param_count.argtypes = [I64, I64, I64]
         lib.oracle_adapter_bytes.restype = I64
@@ -184,6 +186,24 @@ def build_segments(ids, N, rows_per_tile, min_run, long_tile=128,
         "gather_tiles": gt[:n_gather].copy(),
         "contig_tiles": ct[:n_contig].copy(),
     }
+
+
+def lora_merge(W, A, B, r, alpha, sign=1):
+    """W + sign * (alpha / r) * B[:, :r] A[:r, :] in fp64 for one adapter: W [d_out,
+    ld_w] (d_in = A's width used), A [r_max, d_in], B [d_out, r_max]."""
+    lib = _load()
+    W, A, B = _cpu(W), _cpu(A), _cpu(B)
+    code = _dtype_code(W)
+    assert _dtype_code(A) == code and _dtype_code(B) == code, "one dtype"
+    d_out, ld_w = W.shape
+    r_max, d_in = A.shape
+    assert B.shape == (d_out, r_max)
+    out = np.empty((d_out, d_in), dtype=np.float64)
+    rc = lib.oracle_lora_merge(code, W.data_ptr(), ld_w, d_out, d_in, A.data_ptr(), B.data_ptr(),
+                               r_max, int(r), float(alpha), int(sign), out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_lora_merge rejected its arguments")
+    return out
 
 
 def lora_param_count(d: int, k: int, r: int) -> int:

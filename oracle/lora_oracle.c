@@ -268,6 +268,36 @@ int oracle_build_segments(const int32_t *ids, int32_t T, int32_t N,
     return status;
 }
 
+/*
+ * Merged weight (page "LoRA service: multi-adapter dynamic loading", section 1:
+ * a single-tenant deployment folds the adapter into the base weight,
+ * W' = W + B A; the scale alpha / r of page "Multi-LoRA Serving", section 3.1),
+ * in fp64:
+ *   out[o][i] = W[o][i] + sign * (alpha / r) * sum_{k < r} B[o][k] * A[k][i]
+ * for o < d_out, i < d_in.  W is [d_out][ld_w]; A is one adapter [r_max][d_in]
+ * and B one adapter [d_out][r_max] (rank rows / columns k >= r are padding,
+ * never read); out is [d_out][d_in].  Returns 0, or -1 on a bad argument.
+ */
+int oracle_lora_merge(int dtype, const void *W, int64_t ld_w, int32_t d_out, int32_t d_in,
+                      const void *A, const void *B, int32_t r_max, int32_t r, double alpha,
+                      int32_t sign, double *out)
+{
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP32)
+        return -1;
+    if (d_out <= 0 || d_in <= 0 || ld_w < d_in || r <= 0 || r > r_max || (sign != 1 && sign != -1))
+        return -1;
+    double s = (double)sign * alpha / (double)r;
+#pragma omp parallel for schedule(static)
+    for (int32_t o = 0; o < d_out; ++o)
+        for (int32_t i = 0; i < d_in; ++i) {
+            double acc = 0.0;
+            for (int32_t k = 0; k < r; ++k)
+                acc += widen(dtype, B, (int64_t)o * r_max + k) * widen(dtype, A, (int64_t)k * d_in + i);
+            out[(int64_t)o * d_in + i] = widen(dtype, W, (int64_t)o * ld_w + i) + s * acc;
+        }
+    return 0;
+}
+
 /* Adapter parameter count r(d + k) against the full d*k (page "Multi-LoRA
  * Serving", section 3.1, last paragraph). */
 int64_t oracle_lora_param_count(int64_t d, int64_t k, int64_t r) { return r * (d + k); }

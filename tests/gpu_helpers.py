@@ -42,9 +42,9 @@ def build_meta(ids_cpu, N, rows_per_tile=16, min_run=64, device="cuda"):
 def run_fused(w, dl, meta, status, fn=None):
     fn = fn or lora.lora_add_linear
     ranks = w.ranks.cuda()
-    scales = lora.scales_for(w.alpha, w.ranks).cuda()
+    alphas = lora.alphas_full(w.alpha, w.N)
     y = dl.y0.clone()
-    fn(y, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status)
+    fn(y, dl.x, dl.A, dl.B, dl.col_off, ranks, alphas, meta, status)
     torch.cuda.synchronize()
     return y
 

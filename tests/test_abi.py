@@ -51,7 +51,8 @@ def test_capacity_bounds(lib):
     with pytest.raises(lora.LoraError):
         lora.lora_meta_capacity(-1, 4, 16, 0, 128)
     with pytest.raises(lora.LoraError):
-        lora.lora_meta_capacity(10, 4, 17, 0, 128)
+        lora.lora_meta_capacity(10, 4, 65, 0, 128)
+    assert lora.lora_meta_capacity(1024, 100, 64, 0, 128) == (16 + 100, 0)
 
 
 def test_scratch_and_workspace_sizes(lib):
@@ -70,6 +71,29 @@ def test_scratch_and_workspace_sizes(lib):
         want = r256(4 * (N + 1) * chunks) + r256(T) + r256(12 * words) + r256(16 * blocks)
         assert lora.lora_segments_scratch_bytes(T, N) == want, (T, N)
     assert lora.lora_shrink_workspace_bytes(1024, 64, 3) == 3 * 1024 * 64 * 4
+    # out-of-range sizes: 0, and no integer overflow on the way
+    INT_MAX = 2 ** 31 - 1
+    assert lora.lora_segments_scratch_bytes(INT_MAX, 8) == 0
+    assert lora.lora_segments_scratch_bytes(1024, INT_MAX) == 0
+    assert lora.lora_segments_scratch_bytes(lora.MAX_ROWS + 1, 8) == 0
+
+
+def test_linear_workspace_size(lib):
+    """256-byte head, one int per unit of the meta's tile capacity (rounded up to
+    256 bytes), then v [n_slices][T][r_max] fp32."""
+    def r256(b):
+        return (b + 255) // 256 * 256
+    for T, N, R, min_run, S, r_max in [(1024, 100, 64, 0, 3, 64), (256, 32, 64, 0, 1, 16),
+                                       (8192, 16, 64, 64, 1, 16), (77431, 8, 16, 64, 2, 32)]:
+        m = _meta(T, N, R, min_run)
+        mg, mc = lora.lora_meta_capacity(T, N, R, min_run, 128)
+        units = mg + (mc * -(-128 // R) if min_run > 0 else 0)
+        want = 256 + r256(4 * units) + S * T * r_max * 4
+        assert lib.lora_linear_workspace_bytes(ctypes.byref(m), S, r_max) == want, (T, N, R)
+    m = _meta()
+    assert lib.lora_linear_workspace_bytes(ctypes.byref(m), 0, 16) == 0
+    assert lib.lora_linear_workspace_bytes(ctypes.byref(m), 1, 129) == 0
+    assert lib.lora_linear_workspace_bytes(None, 1, 16) == 0
 
 
 def _meta(T=8, N=4, R=4, min_run=0):
@@ -97,8 +121,10 @@ def test_host_checks(lib):
     assert lib.lora_build_segments(fake, ctypes.byref(bad), None, 0, fake, None) == c["SHAPE"]
     sl = (lora.lora_slice * 1)()
     sl[0].A, sl[0].B, sl[0].d_out, sl[0].col_off = 0x1000, 0x1000, 16, 0
-    args = lambda dtype=0, r_max=16, n=1, ld_y=16, sl=sl: (
-        fake, ld_y, fake, 16, 16, sl, n, r_max, fake, fake, ctypes.byref(m), dtype, fake, None)
+    ws_need = lib.lora_linear_workspace_bytes(ctypes.byref(m), 1, 16)
+    args = lambda dtype=0, r_max=16, n=1, ld_y=16, sl=sl, ws=ctypes.c_void_p(0x10000), wsb=ws_need: (
+        fake, ld_y, fake, 16, 16, sl, n, r_max, fake, fake, ctypes.byref(m), ws, wsb, dtype, fake,
+        None)
     assert lib.lora_add_linear(*args(dtype=7)) == c["DTYPE"]
     assert lib.lora_add_linear(*args(r_max=0)) == c["RANK"]
     assert lib.lora_add_linear(*args(r_max=129)) == c["RANK"]
@@ -121,4 +147,24 @@ def test_host_checks(lib):
                                 None) == c["SHAPE"]
     assert lib.lora_sgmv_expand(fake, 16, None, sl, 1, 16, fake, fake, ctypes.byref(m), 0, fake,
                                 None) == c["NULL"]
+    # the fused calls' workspace: present, large enough, 256-byte aligned
+    for fn in (lib.lora_add_linear, lib.lora_bgmv_fused):
+        assert fn(*args(ws=None)) == c["NULL"]
+        assert fn(*args(wsb=ws_need - 1)) == c["WORKSPACE"]
+        assert fn(*args(ws=ctypes.c_void_p(0x10010))) == c["WORKSPACE"]
     assert lib.lora_status_string(-7) == b"LORA_ERR_CAPACITY"
+
+
+def test_static_grouping_checks_the_meta_first(lib):
+    """lora_build_segments_static refuses an out-of-range meta with the same code as
+    lora_build_segments (LORA_ERR_SHAPE), before sizing any scratch: no integer
+    overflow, no LORA_ERR_WORKSPACE for sizes that are simply invalid."""
+    c = _codes(lib)
+    fake = ctypes.c_void_p(0x1000)
+    for T, N in [(2 ** 31 - 1, 8), (lora.MAX_ROWS + 1, 8), (1024, 2 ** 31 - 1), (-1, 8)]:
+        m = _meta()
+        m.T, m.N = T, N
+        assert lib.lora_build_segments_static(fake, ctypes.byref(m), fake, None) == c["SHAPE"], (T, N)
+        assert lib.lora_build_segments(fake, ctypes.byref(m), None, 0, fake, None) == c["SHAPE"]
+    m = _meta()
+    assert lib.lora_build_segments_static(fake, ctypes.byref(m), None, None) == c["NULL"]

@@ -44,26 +44,30 @@ def _fake_root(tmp_path, src_text, recorded_text):
     rec_src = tmp_path / "recorded.cu"
     _write(rec_src, recorded_text)
     rec = {"bgmv_kernel": {"code_sha256": bench.code_digest(rec_src),
-                           "decode_qproj": {"dram_bytes_per_launch": 123456.0}}}
+                           "decode_qproj": {"dram_bytes_per_launch": [123456.0]},
+                           "multislice_8b": {"dram_bytes_per_launch": [1.0, 2.0, 3.0, 4.0]}}}
     _write(tmp_path / "profiles" / "traffic.json", json.dumps(rec))
 
 
 def test_traffic_kept_while_code_unchanged(tmp_path, monkeypatch):
     _fake_root(tmp_path, CODE + "// a note added after the capture\n", CODE)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.measured_traffic("decode_qproj") == 123456.0
-    assert bench.measured_traffic("prefill") is None          # no capture for it
+    assert bench.measured_traffic("decode_qproj", 1) == (123456.0, [123456.0])
+    # a layer set: one figure per layer, summed over the step
+    assert bench.measured_traffic("multislice_8b", 4) == (10.0, [1.0, 2.0, 3.0, 4.0])
+    assert bench.measured_traffic("multislice_8b", 3) == (None, None)   # layers missing
+    assert bench.measured_traffic("prefill", 1) == (None, None)         # no capture for it
 
 
 def test_traffic_dropped_once_code_changes(tmp_path, monkeypatch):
     _fake_root(tmp_path, CODE.replace("+=", "-="), CODE)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.measured_traffic("decode_qproj") is None
+    assert bench.measured_traffic("decode_qproj", 1) == (None, None)
 
 
 def test_traffic_missing_record(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.measured_traffic("decode_qproj") is None
+    assert bench.measured_traffic("decode_qproj", 1) == (None, None)
 
 
 def _w(name, T, N, r_max, slices_per_layer, dtype=torch.bfloat16):

@@ -17,9 +17,9 @@ def _ops(dtype=torch.bfloat16):
     x = torch.zeros(T, D_IN, dtype=dtype)
     y = torch.zeros(T, sum(D_OUT), dtype=dtype)
     ranks = torch.full((N,), R, dtype=torch.int32)
-    scales = torch.ones(N, dtype=torch.float32)
+    alphas = torch.ones(N, dtype=torch.float32)
     meta = lora.Meta(T, N, 16, 0, device="cpu")
-    return dict(y=y, x=x, A=A, B=B, col_off=[0, 32], ranks=ranks, scales=scales, meta=meta,
+    return dict(y=y, x=x, A=A, B=B, col_off=[0, 32], ranks=ranks, alphas=alphas, meta=meta,
                 status=torch.zeros(1, dtype=torch.int32))
 
 
@@ -27,7 +27,7 @@ def _call(**over):
     o = _ops()
     o.update(over)
     return lora.lora_add_linear(o["y"], o["x"], o["A"], o["B"], o["col_off"], o["ranks"],
-                                o["scales"], o["meta"], o["status"])
+                                o["alphas"], o["meta"], o["status"])
 
 
 def test_well_formed_operands_reach_the_device_check():
@@ -46,7 +46,7 @@ def test_well_formed_operands_reach_the_device_check():
     (lambda o: {"col_off": [0, 40]}, "run past y"),
     (lambda o: {"col_off": [0]}, "one column offset"),
     (lambda o: {"ranks": o["ranks"].long()}, "ranks"),
-    (lambda o: {"scales": o["scales"][:N - 1]}, "scales"),
+    (lambda o: {"alphas": o["alphas"][:N - 1]}, "alphas"),
     (lambda o: {"x": o["x"].float()}, "one dtype"),
     (lambda o: {"B": o["B"][:1]}, "one A and one B"),
     (lambda o: {"A": [a.transpose(1, 2) for a in o["A"]]}, "contiguous 3-D"),
@@ -61,7 +61,7 @@ def test_expand_and_shrink_check_v():
     o = _ops()
     v_small = torch.zeros(2, T, R - 1)
     with pytest.raises(LoraError, match="v must be"):
-        lora.lora_sgmv_expand(o["y"], v_small, o["B"], o["col_off"], o["ranks"], o["scales"],
+        lora.lora_sgmv_expand(o["y"], v_small, o["B"], o["col_off"], o["ranks"], o["alphas"],
                               o["meta"], o["status"])
     with pytest.raises(LoraError, match="v must be"):
         lora.lora_sgmv_shrink(torch.zeros(2, T, R, dtype=torch.float64), o["x"], o["A"],

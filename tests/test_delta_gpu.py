@@ -11,8 +11,7 @@ import torch
 import lora_adapter_application_b200 as lora
 import oracle
 import workloads
-from gpu_helpers import (DeviceLayer, assert_within, build_meta, oracle_rows, run_fused,
-                         sample_rows)
+from gpu_helpers import DeviceLayer, assert_within, build_meta, oracle_rows, run_fused
 
 pytestmark = pytest.mark.gpu
 
@@ -44,28 +43,29 @@ SMALL = [
 
 @pytest.mark.parametrize("case", SMALL)
 @pytest.mark.parametrize("fn", ["add_linear", "bgmv_fused"])
-def test_small_bf16_cases(cuda_lib, case, fn):
+@pytest.mark.parametrize("R", [16, 64])
+def test_small_bf16_cases(cuda_lib, case, fn, R):
     seed, T, N, d_in, d_out, r_max, ranks = case
     w = workloads.random_case(seed, T, N, d_in, d_out, r_max, ranks=ranks, dtype=torch.bfloat16)
-    _check_full(w, fn=fn, R=16, min_run=0)
+    _check_full(w, fn=fn, R=R, min_run=0)
 
 
 @pytest.mark.parametrize("r_max", [32, 64])
-@pytest.mark.parametrize("C", ["4", "8"])
-@pytest.mark.parametrize("stages", ["2", "3"])
-def test_ranks_17_to_24_in_16_rank_boxes(cuda_lib, r_max, C, stages, monkeypatch):
-    """Ranks 17-24 with r_max a multiple of 16: the adapters arrive as two 16-rank
-    boxes per 64 columns (32 ranks, 8 of them padding), and every 64-column box of
-    a wide chunk is loaded (4096 columns over 4 or 8 blocks, 2 or 3 ring stages)."""
+@pytest.mark.parametrize("C", ["1", "2", "4", "8"])
+@pytest.mark.parametrize("stages", ["2", "4"])
+def test_ranks_17_to_24(cuda_lib, r_max, C, stages, monkeypatch):
+    """Ranks 17-24 (24 or 32 loaded ranks: a 16- and an 8-rank A box, three 8-rank
+    B boxes, or one 32-rank B box) over 4096 columns, every cluster size and two
+    ring depths."""
     monkeypatch.setenv("LORA_BG_CLUSTER", C)
     monkeypatch.setenv("LORA_BG_STAGES", stages)
     ranks = [17 + (i % 8) for i in range(12)]
     w = workloads.random_case(41, 256, 12, 4096, [4096], r_max, ranks=ranks, none_frac=0.05,
                               dtype=torch.bfloat16)
-    _check_full(w, fn="bgmv_fused", R=16, min_run=0)
+    _check_full(w, fn="bgmv_fused", R=64, min_run=0)
 
 
-@pytest.mark.parametrize("R,min_run", [(16, 8), (5, 0), (1, 0), (16, 200)])
+@pytest.mark.parametrize("R,min_run", [(16, 8), (5, 0), (1, 0), (16, 200), (64, 0), (64, 8), (37, 16)])
 def test_tiles_and_runs(cuda_lib, R, min_run):
     """Long same-adapter segments over several tiles, prompt-like runs that become
     contiguous tiles, and ragged tails."""
@@ -102,10 +102,10 @@ def test_strided_rows_and_offsets(cuda_lib):
     yw = torch.randn(w.T, 72, generator=g).to(torch.bfloat16)
     col_off = [8, 48]
     meta, status = build_meta(w.ids, w.N, 16, 0)
-    ranks, scales = w.ranks.cuda(), lora.scales_for(w.alpha, w.ranks).cuda()
+    ranks, alphas = w.ranks.cuda(), lora.alphas_full(w.alpha, w.N)
     y = yw.cuda()
     lora.lora_add_linear(y, xw.cuda()[:, :96], [a.cuda() for a in lay.A],
-                         [b.cuda() for b in lay.B], col_off, ranks, scales, meta, status)
+                         [b.cuda() for b in lay.B], col_off, ranks, alphas, meta, status)
     torch.cuda.synchronize()
     ref = oracle.lora_apply(xw, lay.A, lay.B, col_off, w.ranks, w.alpha, w.ids, yw)
     assert_within(y.cpu().double().numpy(), ref, torch.bfloat16, "strided")
@@ -121,9 +121,9 @@ def test_bad_rank_is_flagged_and_rows_untouched(cuda_lib):
     dl = DeviceLayer(lay)
     meta, status = build_meta(w.ids, w.N, 16, 0)
     ranks = torch.tensor([8, 9, 8], dtype=torch.int32).cuda()   # 9 > r_max
-    scales = lora.scales_for(w.alpha, w.ranks).cuda()
+    alphas = lora.alphas_full(w.alpha, w.N)
     y = dl.y0.clone()
-    lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status)
+    lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, alphas, meta, status)
     torch.cuda.synchronize()
     assert int(status.item()) & lora.DEV_BAD_RANK
     rows1 = (w.ids == 1)
@@ -141,7 +141,7 @@ def test_shrink_then_expand_matches_oracle(cuda_lib):
     for min_run in (0, 16):
         meta, status = build_meta(w.ids, w.N, 16, min_run)
         v = torch.full((3, w.T, w.r_max), float("nan"), device="cuda")
-        ranks, scales = w.ranks.cuda(), lora.scales_for(w.alpha, w.ranks).cuda()
+        ranks, alphas = w.ranks.cuda(), lora.alphas_full(w.alpha, w.N)
         lora.lora_sgmv_shrink(v, dl.x, dl.A, ranks, meta, status)
         torch.cuda.synchronize()
         vref = oracle.lora_shrink(lay.x, lay.A, w.ranks, w.ids)          # [T, S, r_max]
@@ -156,13 +156,13 @@ def test_shrink_then_expand_matches_oracle(cuda_lib):
         # expand from the oracle's v gives the oracle's y
         vin = torch.as_tensor(vref, dtype=torch.float32).permute(1, 0, 2).contiguous().cuda()
         y = dl.y0.clone()
-        lora.lora_sgmv_expand(y, vin, dl.B, dl.col_off, ranks, scales, meta, status)
+        lora.lora_sgmv_expand(y, vin, dl.B, dl.col_off, ranks, alphas, meta, status)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert_within(y.cpu().double().numpy(), oracle_rows(w, lay, None), torch.bfloat16, "expand")
         # and shrink -> expand on the GPU equals the fused kernel within tolerance
         y2 = dl.y0.clone()
-        lora.lora_sgmv_expand(y2, v, dl.B, dl.col_off, ranks, scales, meta, status)
+        lora.lora_sgmv_expand(y2, v, dl.B, dl.col_off, ranks, alphas, meta, status)
         torch.cuda.synchronize()
         assert_within(y2.cpu().double().numpy(), oracle_rows(w, lay, None), torch.bfloat16, "pair")
 
@@ -178,15 +178,16 @@ def test_fused_is_deterministic(cuda_lib):
 
 # ------------------------------------------------------------------ full-size workloads
 
-def _full_size(w, layer_idx, k=96):
+def _full_size(w, layer_idx, R=64, min_run=64):
+    """Every row of a full-size workload layer against the oracle (fp64, OpenMP over
+    the host cores); rows without an adapter bit-identical."""
     lay = w.layers[layer_idx]
     dl = DeviceLayer(lay)
-    meta, status = build_meta(w.ids, w.N, 16, 64)
+    meta, status = build_meta(w.ids, w.N, R, min_run)
     y = run_fused(w, dl, meta, status).cpu()
     assert int(status.item()) == 0
-    rows = sample_rows(w, k)
-    ref = oracle_rows(w, lay, rows)
-    assert_within(y[rows].double().numpy(), ref, w.dtype, f"{w.name}/{lay.name}")
+    ref = oracle_rows(w, lay, None)
+    assert_within(y.double().numpy(), ref, w.dtype, f"{w.name}/{lay.name}")
     none = (w.ids < 0)
     assert torch.equal(y[none], lay.y0[none])
     return y, dl, meta, status
@@ -194,21 +195,22 @@ def _full_size(w, layer_idx, k=96):
 
 def test_decode_qproj_full(cuda_lib):
     w = workloads.decode_qproj()
-    _check_full(w)
+    _check_full(w, R=64, min_run=0)
+    _check_full(w, R=16, min_run=0)
 
 
-def test_prefill_full_sampled(cuda_lib):
+def test_prefill_full(cuda_lib):
     w = workloads.prefill()
     _full_size(w, 0)
 
 
 @pytest.mark.parametrize("layer_idx", [0, 1, 2, 3])
-def test_multislice_8b_full_sampled(cuda_lib, layer_idx):
+def test_multislice_8b_full(cuda_lib, layer_idx):
     w = workloads.multislice_8b()
-    _full_size(w, layer_idx, k=48)
+    _full_size(w, layer_idx, min_run=0)
 
 
 @pytest.mark.parametrize("layer_idx", [0, 1])
-def test_mixed_70b_full_sampled(cuda_lib, layer_idx):
+def test_mixed_70b_full(cuda_lib, layer_idx):
     w = workloads.mixed_70b()
-    _full_size(w, layer_idx, k=64)
+    _full_size(w, layer_idx)

@@ -83,7 +83,7 @@ def test_shrink_expand_contiguous_tiles(cuda_lib, C, monkeypatch):
     lay = w.layers[0]
     dl = DeviceLayer(lay)
     meta, status = build_meta(w.ids, w.N, 16, 16)
-    ranks, scales = w.ranks.cuda(), lora.scales_for(w.alpha, w.ranks).cuda()
+    ranks, alphas = w.ranks.cuda(), lora.alphas_full(w.alpha, w.N)
     v = torch.full((2, w.T, w.r_max), float("nan"), device="cuda")
     _, names = _kernels_of(lambda: lora.lora_sgmv_shrink(v, dl.x, dl.A, ranks, meta, status))
     assert _on_tensor_cores(names), sorted(names)
@@ -103,7 +103,7 @@ def test_shrink_expand_contiguous_tiles(cuda_lib, C, monkeypatch):
 
     def expand():                                     # y += ...: start from y0 on every run
         y.copy_(dl.y0)
-        lora.lora_sgmv_expand(y, vin, dl.B, dl.col_off, ranks, scales, meta, status)
+        lora.lora_sgmv_expand(y, vin, dl.B, dl.col_off, ranks, alphas, meta, status)
 
     _, names = _kernels_of(expand)
     assert _on_tensor_cores(names), sorted(names)
@@ -118,9 +118,9 @@ def test_contiguous_bad_rank_flagged(cuda_lib):
     dl = DeviceLayer(lay)
     meta, status = build_meta(w.ids, w.N, 16, 16)
     ranks = torch.tensor([16, 17, 16], dtype=torch.int32).cuda()      # 17 > r_max
-    scales = lora.scales_for(w.alpha, w.ranks).cuda()
+    alphas = lora.alphas_full(w.alpha, w.N)
     y = dl.y0.clone()
-    lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status)
+    lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, alphas, meta, status)
     torch.cuda.synchronize()
     assert int(status.item()) & lora.DEV_BAD_RANK
     rows1 = (w.ids == 1)
@@ -159,16 +159,16 @@ def test_captured_graph_matches_eager(cuda_lib):
     w = _case(CASES[0])          # prompt runs and decode rows: both kernels, both streams
     dl = DeviceLayer(w.layers[0])
     meta, status = build_meta(w.ids, w.N, 16, 16)
-    ranks, scales = w.ranks.cuda(), lora.scales_for(w.alpha, w.ranks).cuda()
+    ranks, alphas = w.ranks.cuda(), lora.alphas_full(w.alpha, w.N)
     eager = dl.y0.clone()
-    lora.lora_add_linear(eager, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status)
+    lora.lora_add_linear(eager, dl.x, dl.A, dl.B, dl.col_off, ranks, alphas, meta, status)
     torch.cuda.synchronize()
     y = dl.y0.clone()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, scales, meta, status,
+        lora.lora_add_linear(y, dl.x, dl.A, dl.B, dl.col_off, ranks, alphas, meta, status,
                              stream=s)
     for _ in range(2):
         y.copy_(dl.y0)
