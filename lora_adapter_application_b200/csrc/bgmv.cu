@@ -152,6 +152,9 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(remote_bar)
                  : "memory");
 }
+__device__ __forceinline__ void red_release_gpu(int *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
@@ -188,10 +191,14 @@ __device__ __forceinline__ uint32_t b_off(int col, int k, int r8) {
 }
 
 // ------------------------------------------------------------------ geometry (shared by host tests)
-// Rows of one shrink pass: the exchange holds at most GB_XCAP partial elements.
+// Rows of one shrink pass.  Each consumer warp owns one m16 tile of the pass
+// and a run of its S*r8/8 rank tiles: mtp warps-groups (1, 2 or 4) cover the
+// m16 tiles, and a warp holds at most 8 (m16, n8) accumulators, so
+// pow2(m16 tiles) * S*r8 <= 512; that also bounds the exchange (16 * 512
+// partial elements = GB_XCAP).
 __host__ __device__ inline int gb_pass_rows(int cnt, int S, int r8) {
-    int pr = (GB_XCAP / (S * r8)) & ~15;
-    pr = pr < 16 ? 16 : (pr > GB_ROWS ? GB_ROWS : pr);
+    const int mt_max = 512 / (S * r8);
+    const int pr = mt_max >= 4 ? 64 : (mt_max >= 2 ? 32 : 16);
     return cnt < pr ? cnt : pr;
 }
 // Slices per shrink chunk: as many as fit a stage beside 64 columns of x rows.
@@ -247,6 +254,48 @@ __device__ __forceinline__ UnitInfo fetch_unit(const GbArgs &a, int u, int &row0
     row0 = lane < f.cnt ? un.row(a.tiles, lane) : -1;
     row1 = lane + 32 < f.cnt ? un.row(a.tiles, lane + 32) : -1;
     return f;
+}
+
+// Tile record of unit v (one dependent load): adapter, first row (contiguous) or
+// first index into grow (gathered), rows.  ng = live gathered tiles.
+struct URec {
+    int id, base, cnt, gathered;
+};
+__device__ __forceinline__ URec unit_rec(const Tiles &t, int ng, int v) {
+    URec r{0, 0, 0, 1};
+    if (v < ng) {
+        const int4 g = t.gather[v];
+        r.id = g.x;
+        r.base = g.y;
+        r.cnt = g.z;
+        return r;
+    }
+    v -= ng;
+    const int tile = v / t.subs, sub = v - tile * t.subs;
+    const int4 c = t.contig[tile];
+    const int first = sub * t.rows_per_unit;
+    if (first < c.z) {
+        r.id = c.x;
+        r.base = c.y + first;
+        r.cnt = min(t.rows_per_unit, c.z - first);
+        r.gathered = 0;
+    }
+    return r;
+}
+// What the producer needs beyond the record: rank, alpha, rows (lane l: rows l, l+32).
+struct UMeta {
+    int r_n;
+    float alpha;
+    int row0, row1;
+};
+__device__ __forceinline__ UMeta unit_meta(const GbArgs &a, const URec &r) {
+    const int lane = threadIdx.x & 31;
+    UMeta m;
+    m.r_n = r.cnt > 0 ? a.ranks[r.id] : 0;
+    m.alpha = r.cnt > 0 ? a.alphas[r.id] : 0.f;
+    m.row0 = lane < r.cnt ? (r.gathered ? a.tiles.grow[r.base + lane] : r.base + lane) : -1;
+    m.row1 = lane + 32 < r.cnt ? (r.gathered ? a.tiles.grow[r.base + lane + 32] : r.base + lane + 32) : -1;
+    return m;
 }
 
 // ================================================================ producer warp
@@ -410,28 +459,40 @@ __device__ void gb_producer(const GbArgs &a, const GbSmem &sm, bool &failed) {
     }
 
     // ------------------------------------------------------------ phase 2: expand
+    // Items are drawn two ahead and their metadata one ahead: at the start of item i
+    // the ticket of item i+2 and the tile record of item i+1 are requested, and the
+    // rank, alpha and rows of item i+1 right after item i's chunks are issued, so
+    // the dependent global reads overlap the ring's drain instead of stalling it.
     if (MODE != MODE_SHRINK && !failed) {
         const int nb = a.blk_off[S];
-        const int64_t total = (int64_t)live * nb;
-        int64_t e = MODE == MODE_FUSED ? -1 : (int64_t)blockIdx.x;
-        if (MODE == MODE_FUSED && lane == 0) e = atomicAdd(a.ctl + GB_T_EXPAND, 1);
-        for (int k = 0;; ++k) {
-            if (MODE == MODE_FUSED) e = __shfl_sync(FULL, (int)e, 0);
-            if (e >= total || failed) break;
-            const int u = (int)(e / nb), b = (int)(e - (int64_t)u * nb);
-            int enext = 0;   // the next ticket, drawn early so its latency overlaps this item
-            if (MODE == MODE_FUSED && lane == 0) enext = atomicAdd(a.ctl + GB_T_EXPAND, 1);
+        const int total = live * nb;
+        const int ng = a.tiles.use_gather ? min(a.tiles.counts[1], a.tiles.max_gather) : 0;
+        auto claim = [&](int prev) -> int {   // the next item (fused: lane 0's ticket)
+            if (MODE == MODE_FUSED) return lane == 0 ? atomicAdd(a.ctl + GB_T_EXPAND, 1) : 0;
+            return prev + (int)gridDim.x;
+        };
+        auto bcast = [&](int v) -> int { return MODE == MODE_FUSED ? __shfl_sync(FULL, v, 0) : v; };
+        int e_cur = bcast(claim((int)blockIdx.x - (int)gridDim.x));
+        int e_raw = claim(e_cur);   // item i+1, not yet broadcast
+        URec rec = e_cur < total ? unit_rec(a.tiles, ng, e_cur / nb) : URec{0, 0, 0, 1};
+        UMeta meta = unit_meta(a, rec);
+        for (;;) {
+            if (e_cur >= total || failed) break;
+            const int e_nxt = bcast(e_raw);
+            const URec rec_nxt = e_nxt < total ? unit_rec(a.tiles, ng, e_nxt / nb) : URec{0, 0, 0, 1};
+            e_raw = claim(e_nxt);
+            const int u = e_cur / nb, b = e_cur - u * nb;
             int s = 0;
             while (s + 1 < S && a.blk_off[s + 1] <= b) ++s;
             const int c_item = (b - a.blk_off[s]) * a.bc;
             const int w_item = min(a.bc, a.sl.d_out[s] - c_item);
-            int row0, row1;
-            const UnitInfo f = fetch_unit(a, u, row0, row1);
-            if (!f.ok) {
-                if (f.cnt > 0 && b == 0 && lane == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
+            const int cnt = rec.cnt, r_n = meta.r_n;
+            const bool ok_rank = cnt > 0 && r_n >= 1 && r_n <= a.r_max;
+            if (!ok_rank) {
+                if (cnt > 0 && b == 0 && lane == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
             } else {
-                const int r8 = f.r8, cnt = f.cnt;
-                const float scale = a.alphas[f.n] / (float)f.r_n;
+                const int r8 = (r_n + 7) & ~7;
+                const float scale = meta.alpha / (float)r_n;
                 const int vbytes = cnt * r8 * 4;
                 const int d_out = a.sl.d_out[s];
                 const int mi = r8 == 64 ? 3 : (r8 == 32 ? 2 : (r8 == 16 ? 1 : 0));
@@ -456,8 +517,8 @@ __device__ void gb_producer(const GbArgs &a, const GbSmem &sm, bool &failed) {
                         h->kind = GB_EXPAND;
                         h->flags = (first ? GB_FIRST : 0) | (last ? GB_LAST : 0);
                         h->unit = u;
-                        h->n = f.n;
-                        h->r_n = f.r_n;
+                        h->n = rec.id;
+                        h->r_n = r_n;
                         h->r8 = r8;
                         h->cnt = cnt;
                         h->s0 = s;
@@ -469,8 +530,8 @@ __device__ void gb_producer(const GbArgs &a, const GbSmem &sm, bool &failed) {
                         h->yofs = yofs;
                         h->scale = scale;
                     }
-                    if (lane < cnt) h->rows[lane] = row0;
-                    if (lane + 32 < cnt) h->rows[lane + 32] = row1;
+                    if (lane < cnt) h->rows[lane] = meta.row0;
+                    if (lane + 32 < cnt) h->rows[lane + 32] = meta.row1;
                     __syncwarp();
                     const int nbox = (w + 63) >> 6;
                     const unsigned bytes = (unsigned)(vb + cnt * w * 2 + nbox * 128 * r8);
@@ -486,7 +547,7 @@ __device__ void gb_producer(const GbArgs &a, const GbSmem &sm, bool &failed) {
                             const int cb = wide ? e2 : e2 / (r8 >> 3);
                             const int kb = wide ? 0 : e2 - cb * (r8 >> 3);
                             tma_2d(dst + bofs + (uint32_t)(cb * 128 * r8 + kb * 1024),
-                                   &a.tmB[s][wide ? mi : 0], kb * 8, f.n * d_out + c + 64 * cb,
+                                   &a.tmB[s][wide ? mi : 0], kb * 8, rec.id * d_out + c + 64 * cb,
                                    sm.full0 + 8 * st);
                         }
                     }
@@ -525,11 +586,9 @@ __device__ void gb_producer(const GbArgs &a, const GbSmem &sm, bool &failed) {
                     if (w == 0 && CC > 0) break;
                 }
             }
-            if (MODE == MODE_FUSED) {
-                e = enext;
-            } else {
-                e += gridDim.x;
-            }
+            meta = unit_meta(a, rec_nxt);   // the next item's rank, alpha and rows
+            rec = rec_nxt;
+            e_cur = e_nxt;
         }
     }
 
@@ -569,6 +628,52 @@ __device__ __forceinline__ void gb_release(const GbSmem &sm, int st) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(sm.empty0 + 8 * st);
 }
 
+// One warp's MMAs for one 64-column box of a shrink chunk: NPW pairs (this warp's
+// m16 tile x NPW rank tiles), compile-time so that no branch surrounds the
+// warp-synchronous MMAs; a pair whose slice is not in this chunk gets zero A
+// fragments (loaded from a safe address).  One pair: two accumulators take
+// alternate k-steps.
+template <int NPW>
+__device__ __forceinline__ void shrink_box(float (&acc)[8][4], const int (&pinfo)[8], uint32_t xrow,
+                                           int RS, uint32_t abase, int ncb, int sp, int r8, int s0,
+                                           int sn, int width, int g, int t) {
+    const int col = sp * 64 + t * 16;
+    const bool z0 = col >= width, z1 = col + 8 >= width;
+    const uint32_t c0s = (uint32_t)(((2 * t) ^ g) << 4), c1s = (uint32_t)(((2 * t + 1) ^ g) << 4);
+    const uint32_t xg = xrow + (uint32_t)(col * 2), xh = xg + 8 * RS;
+    const uint4 xa0 = zero_if(z0, lds128(xg)), xa1 = zero_if(z1, lds128(xg + 16));
+    const uint4 xb0 = zero_if(z0, lds128(xh)), xb1 = zero_if(z1, lds128(xh + 16));
+    uint32_t arow[NPW];
+    bool on[NPW];
+#pragma unroll
+    for (int i = 0; i < NPW; ++i) {
+        const int s = pinfo[i] >> 8;
+        on[i] = s >= s0 && s < s0 + sn;
+        arow[i] = on[i] ? abase + (uint32_t)((((s - s0) * ncb + sp) * r8 + (pinfo[i] & 255)) * 128) : abase;
+    }
+    const uint32_t f0[4] = {xa0.x, xb0.x, xa0.y, xb0.y}, f1[4] = {xa0.z, xb0.z, xa0.w, xb0.w};
+    const uint32_t f2[4] = {xa1.x, xb1.x, xa1.y, xb1.y}, f3[4] = {xa1.z, xb1.z, xa1.w, xb1.w};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {   // k-steps 0-1, then 2-3: each half's loads first
+        const bool zh = half ? z1 : z0;
+        const uint32_t cs = half ? c1s : c0s;
+        uint4 af[NPW];
+#pragma unroll
+        for (int i = 0; i < NPW; ++i) af[i] = zero_if(zh || !on[i], lds128(arow[i] + cs));
+        const uint32_t(&fa)[4] = half ? f2 : f0;
+        const uint32_t(&fb)[4] = half ? f3 : f1;
+        if (NPW == 1) {
+            mma16816(acc[0], fa, af[0].x, af[0].y);
+            mma16816(acc[1], fb, af[0].z, af[0].w);
+        } else {
+#pragma unroll
+            for (int i = 0; i < NPW; ++i) mma16816(acc[i], fa, af[i].x, af[i].y);
+#pragma unroll
+            for (int i = 0; i < NPW; ++i) mma16816(acc[i], fb, af[i].z, af[i].w);
+        }
+    }
+}
+
 // Phase 1: shrink chunks until the stream moves on; returns the position of
 // the first stage that is not a shrink chunk.
 template <int MODE>
@@ -581,9 +686,10 @@ __device__ uint32_t gb_consume_shrink(const GbArgs &a, const GbSmem &sm, bool &f
     float *part = reinterpret_cast<float *>(__cvta_shared_to_generic(sm.part));
 
     float acc[8][4];
-    // per pair i: m16 tile | slice << 4 | A rank row << 8 | first column << 16
+    // this warp's pairs: m16 tile wm, rank tiles n_lo .. n_lo + npw - 1 (k-group kgi of jg
+    // when the rank tiles are fewer than the tile's warps); per pair i: slice << 8 | A rank row
     int pinfo[8];
-    int nt = 0, np = 0, jg = 1, p_lo = 0, p_hi = 0, kgi = 0, W = 0;
+    int nt = 0, np = 0, jg = 1, npw = 0, n_lo = 0, kgi = 0, W = 0, wm = 0;
     uint32_t xc = 0;   // exchanges so far (buffer parity)
     uint32_t gi = 0;
     for (;; ++gi) {
@@ -594,80 +700,62 @@ __device__ uint32_t gb_consume_shrink(const GbArgs &a, const GbSmem &sm, bool &f
         const uint32_t stg = sm.ring + (uint32_t)st * GB_SB;
         const int flags = h->flags;
         const int cnt = h->cnt, r_n = h->r_n, r8 = h->r8;
-        if (flags & GB_FIRST) {   // a new pass: pairs (m16 tile, n8 rank tile) per warp
+        if (flags & GB_FIRST) {   // a new pass
             W = S * r8;
             const int mt = (cnt + 15) >> 4;
+            const int mtp = mt <= 1 ? 1 : (mt <= 2 ? 2 : 4);
+            const int wpm = GB_CONSUMERS / mtp;   // warps per m16 tile
             nt = W >> 3;
             np = mt * nt;
-            if (np >= GB_CONSUMERS) {
-                jg = 1;
-                const int ppw = (np + GB_CONSUMERS - 1) / GB_CONSUMERS;
-                p_lo = warp * ppw;
-                p_hi = min(np, p_lo + ppw);
-                kgi = 0;
-            } else {
-                jg = GB_CONSUMERS / np;
-                p_lo = warp % np;
-                kgi = warp / np;
-                p_hi = kgi < jg ? p_lo + 1 : p_lo;
+            wm = warp % mtp;
+            const int wj = warp / mtp;
+            // jg is the same in every consumer warp (idle ones included): it decides
+            // whether the exchange takes the shared-memory staging and its barrier
+            jg = nt >= wpm ? 1 : wpm / nt;
+            npw = 0;
+            kgi = 0;
+            n_lo = 0;
+            if (wm < mt) {
+                if (jg == 1) {
+                    const int per = (nt + wpm - 1) / wpm;
+                    n_lo = wj * per;
+                    npw = max(0, min(nt, n_lo + per) - n_lo);
+                } else {
+                    n_lo = wj % nt;
+                    kgi = wj / nt;
+                    npw = kgi < jg ? 1 : 0;
+                }
             }
             const int nkb8 = r8 >> 3;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int p = p_lo + i < p_hi ? p_lo + i : p_lo;
-                const int m = p / nt, nn = p - m * nt;
+                const int nn = n_lo + (i < npw ? i : 0);
                 const int s = nn / nkb8;
-                pinfo[i] = m | (s << 4) | (((nn - s * nkb8) * 8 + g) << 8) | ((nn * 8 + 2 * t) << 16);
+                pinfo[i] = (s << 8) | ((nn - s * nkb8) * 8 + g);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
             }
             if (tid < cnt) xrows[tid] = h->rows[tid];
         }
-        if (!(flags & GB_NODATA)) {
+        if (!(flags & GB_NODATA) && npw > 0) {
             const int width = h->w, JC = h->cw, RS = 2 * JC + 16, ncb = JC >> 6;
             const int s0 = h->s0, sn = h->sn;
             const uint32_t abase = stg + (uint32_t)h->bofs;
             const int nbox = (width + 63) >> 6;
-            const uint32_t c0s = (uint32_t)(((2 * t) ^ g) << 4), c1s = (uint32_t)(((2 * t + 1) ^ g) << 4);
+            const uint32_t xrow = stg + (uint32_t)((16 * wm + g) * RS);
             for (int sp = kgi; sp < nbox; sp += jg) {
-                const int col = sp * 64 + t * 16;
-                const bool z0 = col >= width, z1 = col + 8 >= width;
-                int cm = -1;
-                uint4 xa0 = make_uint4(0, 0, 0, 0), xa1 = xa0, xb0 = xa0, xb1 = xa0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (p_lo + i >= p_hi) break;
-                    const int m = pinfo[i] & 15, s = (pinfo[i] >> 4) & 15, kr = (pinfo[i] >> 8) & 255;
-                    if (s < s0 || s >= s0 + sn) continue;
-                    if (m != cm) {
-                        cm = m;
-                        const uint32_t xg = stg + (uint32_t)((16 * m + g) * RS + col * 2);
-                        const uint32_t xh = xg + 8 * RS;
-                        xa0 = zero_if(z0, lds128(xg));
-                        xa1 = zero_if(z1, lds128(xg + 16));
-                        xb0 = zero_if(z0, lds128(xh));
-                        xb1 = zero_if(z1, lds128(xh + 16));
-                    }
-                    const uint32_t arow = abase + (uint32_t)((((s - s0) * ncb + sp) * r8 + kr) * 128);
-                    const uint4 a0 = zero_if(z0, lds128(arow + c0s));
-                    const uint4 a1 = zero_if(z1, lds128(arow + c1s));
-                    {
-                        const uint32_t fr[4] = {xa0.x, xb0.x, xa0.y, xb0.y};
-                        mma16816(acc[i], fr, a0.x, a0.y);
-                    }
-                    {
-                        const uint32_t fr[4] = {xa0.z, xb0.z, xa0.w, xb0.w};
-                        mma16816(acc[i], fr, a0.z, a0.w);
-                    }
-                    {
-                        const uint32_t fr[4] = {xa1.x, xb1.x, xa1.y, xb1.y};
-                        mma16816(acc[i], fr, a1.x, a1.y);
-                    }
-                    {
-                        const uint32_t fr[4] = {xa1.z, xb1.z, xa1.w, xb1.w};
-                        mma16816(acc[i], fr, a1.z, a1.w);
-                    }
+#define LORA_SHRINK(N) shrink_box<N>(acc, pinfo, xrow, RS, abase, ncb, sp, r8, s0, sn, width, g, t)
+                switch (npw) {
+                    case 1: LORA_SHRINK(1); break;
+                    case 2: LORA_SHRINK(2); break;
+                    case 3: LORA_SHRINK(3); break;
+                    case 4: LORA_SHRINK(4); break;
+                    case 5: LORA_SHRINK(5); break;
+                    case 6: LORA_SHRINK(6); break;
+                    case 7: LORA_SHRINK(7); break;
+                    default: LORA_SHRINK(8); break;
                 }
+#undef LORA_SHRINK
             }
         }
         const int unit = h->unit;
@@ -689,9 +777,16 @@ __device__ uint32_t gb_consume_shrink(const GbArgs &a, const GbSmem &sm, bool &f
             st_async_v2(map_rank(rbuf + ((crank * (uint32_t)spc + slot) * 2u) * 4u, o), v0, v1,
                         map_rank(xr, o));
         };
+        if (npw == 1) {   // the two alternating accumulators of a single pair
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[0][e] += acc[1][e];
+                acc[1][e] = 0.f;
+            }
+        }
         if (jg > 1) {   // k-groups of one pair: add them in shared memory first
-            if (p_lo < p_hi) {
-                float *pp = part + (kgi * np + p_lo) * 128;
+            if (npw > 0) {
+                float *pp = part + (kgi * np + wm * nt + n_lo) * 128;
                 pp[g * 8 + 2 * t] = acc[0][0];
                 pp[g * 8 + 2 * t + 1] = acc[0][1];
                 pp[(g + 8) * 8 + 2 * t] = acc[0][2];
@@ -711,10 +806,10 @@ __device__ uint32_t gb_consume_shrink(const GbArgs &a, const GbSmem &sm, bool &f
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                if (p_lo + i >= p_hi) break;
-                const int m = pinfo[i] & 15, col = pinfo[i] >> 16;
-                send(16 * m + g, col, acc[i][0], acc[i][1]);
-                send(16 * m + g + 8, col, acc[i][2], acc[i][3]);
+                if (i >= npw) break;
+                const int col = (n_lo + i) * 8 + 2 * t;
+                send(16 * wm + g, col, acc[i][0], acc[i][1]);
+                send(16 * wm + g + 8, col, acc[i][2], acc[i][3]);
             }
         }
         bool xok = mbar_wait<true>(xr, (xc >> 1) & 1u, a.status, failed, a.wait_limit);
@@ -740,14 +835,86 @@ __device__ uint32_t gb_consume_shrink(const GbArgs &a, const GbSmem &sm, bool &f
             if (k + 1 < r_n) vr[k + 1] = v1;
         }
         if (MODE == MODE_FUSED && (flags & GB_UNIT_DONE)) {
-            __threadfence();
+            // every consumer's v stores are ordered before thread 0's release by the barrier
             consumer_sync();
-            if (tid == 0) atomicAdd(a.done + unit, 1);
+            if (tid == 0) red_release_gpu(a.done + unit, 1);
         } else {
             consumer_sync();   // xrows and the exchange buffer are reused by the next pass
         }
     }
     return gi;
+}
+
+// One warp's share of an expand chunk: y[rows of its m16 tile][its 8-column blocks]
+// += (s v) B^T.  RB: ranks of one B box (8, 16, 32 or 64: one box per 64 columns,
+// rows of 2*RB bytes swizzled in 16-byte units by the row bits above 128 bytes),
+// or 0 for stacked 8-rank boxes (r8 / 8 boxes of 1 KB per 64 columns); NKB: 16-rank
+// steps.  Both are compile-time so that the loop has no branch around the
+// warp-synchronous MMAs and computes every shared-memory address without one.
+// Loads are unconditional (out-of-chunk addresses stay inside the block's shared
+// memory and their values are masked or never stored).
+template <int RB, int NKB>
+__device__ __forceinline__ void expand_warp(uint32_t bbase, uint32_t yg_ad, uint32_t yh_ad, bool okg,
+                                            bool okh, int nblk, int b_first, int b_step, int r8,
+                                            const uint32_t (&vhi)[4][4], const uint32_t (&vlo)[4][4],
+                                            const uint32_t (&bmx)[4], const uint32_t (&bmy)[4], int g,
+                                            int t) {
+    constexpr int NB = 4;
+    constexpr int SWM = RB >= 16 ? RB / 8 - 1 : 0;              // swizzle mask of the box rows
+    constexpr int SWS = RB == 64 ? 0 : (RB == 32 ? 1 : 2);      // row bits above 128 bytes
+    const int blk_bytes = 128 * (RB ? RB : r8);                // B bytes per 64 columns
+    uint32_t kterm[NKB];                                       // rank part of the address
+#pragma unroll
+    for (int kb = 0; kb < NKB; ++kb)
+        kterm[kb] = RB ? (uint32_t)(2 * (kb * 16 + 4 * t))
+                       : (uint32_t)((2 * kb + (t >> 1)) * 1024 + 8 * (t & 1));
+    for (int b0 = b_first; b0 < nblk; b0 += b_step) {
+        uint2 bv[NB][NKB];
+        uint32_t y0[NB], y1[NB];
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            const int col = (b0 + j) * 8 + g, cr = col & 63;
+            const uint32_t cbase = bbase + (uint32_t)((col >> 6) * blk_bytes);
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) {
+                uint32_t off;
+                if (RB) {
+                    const uint32_t sw = SWM ? (uint32_t)(((RB == 64 ? cr : (cr >> SWS)) & SWM) << 4) : 0u;
+                    off = (uint32_t)(cr * 2 * RB) + (kterm[kb] ^ sw);
+                } else {
+                    off = (uint32_t)(cr * 16) + kterm[kb];
+                }
+                bv[j][kb] = lds64(cbase + off);
+            }
+            y0[j] = lds32(yg_ad + (uint32_t)((b0 + j) * 16));
+            y1[j] = lds32(yh_ad + (uint32_t)((b0 + j) * 16));
+        }
+        float d[NB][4];
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[j][e] = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < NKB; ++kb) {
+#pragma unroll
+            for (int j = 0; j < NB; ++j)
+                mma16816(d[j], vhi[kb], bv[j][kb].x & bmx[kb], bv[j][kb].y & bmy[kb]);
+#pragma unroll
+            for (int j = 0; j < NB; ++j)
+                mma16816(d[j], vlo[kb], bv[j][kb].x & bmx[kb], bv[j][kb].y & bmy[kb]);
+        }
+        // y += delta in shared memory (rows g, g+8 of the tile; columns 2t, 2t+1)
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            const bool okb = b0 + j < nblk;
+            if (okb && okg)
+                sts32(yg_ad + (uint32_t)((b0 + j) * 16),
+                      pack_bf16x2(bf16_lo(y0[j]) + d[j][0], bf16_hi(y0[j]) + d[j][1]));
+            if (okb && okh)
+                sts32(yh_ad + (uint32_t)((b0 + j) * 16),
+                      pack_bf16x2(bf16_lo(y1[j]) + d[j][2], bf16_hi(y1[j]) + d[j][3]));
+        }
+    }
 }
 
 // Phase 2: expand chunks from stage gi until the end of the stream.
@@ -756,6 +923,7 @@ __device__ void gb_consume_expand(const GbArgs &a, const GbSmem &sm, uint32_t gi
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     uint32_t vhi[4][4], vlo[4][4];
+    uint32_t bmx[4], bmy[4];   // per 16-rank step: B's ranks 4t..4t+3 that are below r_n
     int em = 0, ecg = 0, ewpm = 1, nkb = 0;
     bool eactive = false;
     for (;; ++gi) {
@@ -774,6 +942,12 @@ __device__ void gb_consume_expand(const GbArgs &a, const GbSmem &sm, uint32_t gi
             ecg = warp / mtp;
             eactive = em < mtt;
             nkb = (r_n + 15) >> 4;
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                const int keep = r_n - (kb * 16 + 4 * t);   // ranks of this thread's 4 below r_n
+                bmx[kb] = keep >= 2 ? 0xffffffffu : (keep == 1 ? 0xffffu : 0u);
+                bmy[kb] = keep >= 4 ? 0xffffffffu : (keep == 3 ? 0xffffu : 0u);
+            }
             const float scale = h->scale;
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
@@ -811,54 +985,24 @@ __device__ void gb_consume_expand(const GbArgs &a, const GbSmem &sm, uint32_t gi
             const uint32_t ybase = stg + (uint32_t)h->yofs, bbase = stg + (uint32_t)h->bofs;
             const int nblk = w >> 3;
             if (eactive) {
-                for (int b0 = ecg * 2; b0 < nblk; b0 += 2 * ewpm) {
-                    float d[2][4];
-#pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) d[j][e] = 0.f;
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        if (kb < nkb) {
-                            const int k = kb * 16 + 4 * t;
-                            uint2 bv[2];
-#pragma unroll
-                            for (int j = 0; j < 2; ++j) {
-                                bv[j] = make_uint2(0, 0);
-                                if (k < r_n && b0 + j < nblk) {
-                                    bv[j] = lds64(bbase + b_off((b0 + j) * 8 + g, k, r8));
-                                    if (k + 4 > r_n) {   // the rank ends inside this group of 4
-                                        const int keep = r_n - k;
-                                        if (keep < 2) bv[j].x &= 0xffffu;
-                                        if (keep < 3) bv[j].y = 0;
-                                        else bv[j].y &= 0xffffu;
-                                    }
-                                }
-                            }
-#pragma unroll
-                            for (int j = 0; j < 2; ++j) mma16816(d[j], vhi[kb], bv[j].x, bv[j].y);
-#pragma unroll
-                            for (int j = 0; j < 2; ++j) mma16816(d[j], vlo[kb], bv[j].x, bv[j].y);
-                        }
-                    }
-                    // y += delta in shared memory (rows g, g+8 of the tile; columns 2t, 2t+1)
-                    const int rg = 16 * em + g, rh = rg + 8;
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        if (b0 + j >= nblk) continue;
-                        const uint32_t col2 = (uint32_t)(((b0 + j) * 8 + 2 * t) * 2);
-                        if (rg < cnt) {
-                            const uint32_t ad = ybase + (uint32_t)(rg * YS) + col2;
-                            const uint32_t yv = lds32(ad);
-                            sts32(ad, pack_bf16x2(bf16_lo(yv) + d[j][0], bf16_hi(yv) + d[j][1]));
-                        }
-                        if (rh < cnt) {
-                            const uint32_t ad = ybase + (uint32_t)(rh * YS) + col2;
-                            const uint32_t yv = lds32(ad);
-                            sts32(ad, pack_bf16x2(bf16_lo(yv) + d[j][2], bf16_hi(yv) + d[j][3]));
-                        }
-                    }
+                const int rg = 16 * em + g;
+                const uint32_t yg_ad = ybase + (uint32_t)(rg * YS) + (uint32_t)(4 * t);
+                const uint32_t yh_ad = yg_ad + (uint32_t)(8 * YS);
+                const bool okg = rg < cnt, okh = rg + 8 < cnt;
+                const int bf = ecg * 4, bs = 4 * ewpm;
+#define LORA_EXPAND(RB, NKB)                                                                      \
+    expand_warp<RB, NKB>(bbase, yg_ad, yh_ad, okg, okh, nblk, bf, bs, r8, vhi, vlo, bmx, bmy, g, t)
+                if ((r8 & (r8 - 1)) == 0) {   // one box per 64 columns
+                    if (r8 == 8) LORA_EXPAND(8, 1);
+                    else if (r8 == 16) LORA_EXPAND(16, 1);
+                    else if (r8 == 32) LORA_EXPAND(32, 2);
+                    else LORA_EXPAND(64, 4);
+                } else {                      // stacked 8-rank boxes: r8 = 24, 40, 48, 56
+                    if (nkb == 2) LORA_EXPAND(0, 2);
+                    else if (nkb == 3) LORA_EXPAND(0, 3);
+                    else LORA_EXPAND(0, 4);
                 }
+#undef LORA_EXPAND
             }
             consumer_sync();
             const int ypc = w >> 3;
@@ -994,7 +1138,10 @@ int gb_active_clusters(int mode, int cluster, size_t smem) {
     }
     const void *fn = gb_fn(mode);
     int n = 0;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+    // the limit is a per-device attribute of the kernel: always the mode's largest
+    // launch, so no query for a smaller size can lower it under another launch
+    const size_t smem_max = bgmv_smem_bytes(mode, mode == MODE_EXPAND ? GB_MAX_STAGES : 4);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) ==
         cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(cluster, 1, 1);

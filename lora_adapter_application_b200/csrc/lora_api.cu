@@ -262,22 +262,22 @@ bool run_tc(int mode, const Call &c, int *rc, int *idle_sms) {
     a.lbr = box_rows("LORA_TC_LOAD_ROWS", 128);
     a.sbr = box_rows("LORA_TC_STORE_ROWS", 128);
     if (need_x &&
-        tensor_map_2d(&a.tmX, c.x, (uint64_t)c.d_in, (uint64_t)c.meta->T, 64, (uint32_t)a.lbr, true,
+        tensor_map_2d(&a.tmX, c.x, (uint64_t)c.d_in, (uint64_t)c.meta->T, 64, (uint32_t)a.lbr, 128,
                       (uint64_t)c.ld_x) != LORA_OK)
         return false;
     for (int s = 0; s < c.n_slices; ++s) {
         const lora_slice &sl = c.slices[s];
         if (need_x && tensor_map_2d(&a.tmA[s], sl.A, (uint64_t)c.d_in, (uint64_t)N * c.r_max, 64,
-                                    (uint32_t)c.r_max, true) != LORA_OK)
+                                    (uint32_t)c.r_max, 128) != LORA_OK)
             return false;
         const __nv_bfloat16 *ys = static_cast<const __nv_bfloat16 *>(c.y) + sl.col_off;
         if (need_y &&
             (tensor_map_2d(&a.tmB[s], sl.B, (uint64_t)c.r_max, (uint64_t)N * sl.d_out, 8, 128,
-                           false) != LORA_OK ||
+                           0) != LORA_OK ||
              tensor_map_2d(&a.tmY[s], ys, (uint64_t)sl.d_out, (uint64_t)c.meta->T, 64,
-                           (uint32_t)a.lbr, true, (uint64_t)c.ld_y) != LORA_OK ||
+                           (uint32_t)a.lbr, 128, (uint64_t)c.ld_y) != LORA_OK ||
              tensor_map_2d(&a.tmYs[s], ys, (uint64_t)sl.d_out, (uint64_t)c.meta->T, 64,
-                           (uint32_t)a.sbr, true, (uint64_t)c.ld_y) != LORA_OK))
+                           (uint32_t)a.sbr, 128, (uint64_t)c.ld_y) != LORA_OK))
             return false;
     }
     a.y = static_cast<__nv_bfloat16 *>(c.y);

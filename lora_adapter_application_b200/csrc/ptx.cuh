@@ -67,6 +67,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, unsigned
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// 16 bytes global -> shared on the load/store path (L2 only), completion tracked by
+// cp_async_arrive.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+// One arrival on bar once every cp.async this thread issued so far has landed (the
+// barrier's expected arrival count includes it).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
 // Pull a tensor map (kernel parameter) into the TMA unit's descriptor cache
 // ahead of its first copy.
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {

@@ -363,3 +363,22 @@ def test_stalled_stage_times_out_and_the_context_survives(cuda_lib, monkeypatch)
     status.zero_()
     _check(w, lay, _apply(lora.lora_add_linear, w, lay, dl.A, dl.B, meta, status), status,
            "after a timed-out call")
+
+
+# ------------------------------------------------------------------ tile row counts
+@pytest.mark.parametrize("rows", [1, 15, 16, 17, 31, 33, 40, 47, 48, 49, 63, 64])
+@pytest.mark.parametrize("S,ranks", [(1, [8, 64]), (3, [16, 40]), (2, [8, 33])])
+def test_every_tile_row_count(cuda_lib, rows, S, ranks):
+    """Two adapters with `rows` rows each, in 64-row tiles: every count of m16 tiles
+    per pass (1 to 4, idle warps when it is 3) and every split of a pass's rank
+    tiles over the warps (one pair per warp with k-groups, or several pairs)."""
+    T = 2 * rows + 5
+    ids = [0] * rows + [1] * rows + [-1] * 5
+    perm = torch.randperm(T, generator=torch.Generator().manual_seed(rows))
+    w = workloads.random_case(70 + rows, T, 2, 384, [256] * S if S > 1 else [512], 64, ranks=ranks)
+    w.ids = torch.tensor(ids, dtype=torch.int32)[perm]
+    lay = w.layers[0]
+    dl = DeviceLayer(lay)
+    meta, status = build_meta(w.ids, w.N, 64, 0)
+    _check(w, lay, _apply(lora.lora_add_linear, w, lay, dl.A, dl.B, meta, status), status,
+           f"rows {rows} S={S}")
