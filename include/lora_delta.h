@@ -49,9 +49,10 @@
  * choice).  They change only the launch shape: results stay within the same
  * tolerance of the exact value, and a fixed setting gives bit-identical results
  * from run to run.  A value outside the range is ignored.
- *   LORA_BG_CLUSTER     1, 2, 4 or 8: blocks per cluster of the fused kernel's shrink
- *   LORA_BG_STAGES      2 to 6: 32 KB stages of the fused kernel's load ring
- *   LORA_BG_ITEM_COLS   64 to 8192, a multiple of 64: output columns of one expand item
+ *   LORA_BG_BLOCKS      1 to 4096: blocks of the gathered-tile kernel's persistent
+ *                       grid (default: one per SM)
+ *   LORA_BG_STAGES      2 to 4: steps in flight per warp of the gathered-tile kernel
+ *   LORA_BG_ITEM_COLS   32 to 8192, a multiple of 32: output columns of one expand item
  *   LORA_TC_CLUSTER     1, 2, 4 or 8: blocks per cluster of the tensor-core kernel;
  *                       when the shape cannot use it, the contiguous tiles run on
  *                       the gathered-tile kernel instead
@@ -61,11 +62,11 @@
  *   LORA_TC_STORE_ROWS  8 to 128, a power of two: rows per y store box
  *
  * Test hook (environment, read at each call; never set it in production):
- *   LORA_DEBUG_STALL=1  the fused kernel runs one-block clusters with bounded waits
- *                       of about 1 ms, and the first load stage of every block
- *                       expects 16 bytes that never arrive: its waits run out,
- *                       LORA_DEV_TIMEOUT is set, the call's results are unreliable,
- *                       and the kernel still completes (the context stays usable).
+ *   LORA_DEBUG_STALL=1  the gathered-tile kernel's expand items wait, with a bound of
+ *                       a few ms, for one shrink signal more than their unit gives:
+ *                       the waits run out, LORA_DEV_TIMEOUT is set, the call's
+ *                       results are unreliable, and the kernel still completes (the
+ *                       context stays usable).
  */
 #ifndef LORA_DELTA_H
 #define LORA_DELTA_H
@@ -274,11 +275,11 @@ LORA_API size_t lora_linear_workspace_bytes(const lora_meta *meta, int32_t n_sli
 /*
  * Fused shrink + expand for every tile (BGMV: page "Multi-LoRA Serving",
  * section 3.2, SGMV/BGMV-style grouped products), in one kernel launch: a
- * cluster of thread blocks reduces A x for all rows of a tile (up to 64 rows
- * of one adapter) through distributed shared memory, and blocks then expand
- * the tile's output columns in small items, each starting as soon as its tile
- * is reduced.  v passes between the two through the workspace (it stays in
- * L2; only x, y and the adapters' live ranks cross HBM).  Same result as
+ * thread block reduces A x for all rows of a tile (up to 64 rows of one
+ * adapter) and 32 of its ranks, its warps splitting the input columns, and
+ * warps then expand the tile's output columns in small items, each starting as
+ * soon as its tile is reduced.  v passes between the two through the workspace
+ * (it stays in L2; only x, y and the adapters' live ranks cross HBM).  Same result as
  * lora_sgmv_shrink followed by lora_sgmv_expand.  workspace: device memory of
  * lora_linear_workspace_bytes() bytes, 256-byte aligned (LORA_ERR_WORKSPACE
  * otherwise; see there for its contract).

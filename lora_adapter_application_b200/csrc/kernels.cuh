@@ -9,22 +9,14 @@ namespace lora {
 
 enum { MODE_FUSED = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 
-// Tensor maps of the fused kernel, per slice and per box rank R = 8, 16, 32, 64
-// (index 0..3; only R <= r_max are built):
-//   A_s as [N*r_max rows][d_in], boxes of R rows x 64 columns, 128-byte swizzle
-//   B_s as [N*d_out rows][r_max], boxes of 64 rows x R ranks, swizzle of 2R bytes
-//       (none for R = 8)
-constexpr int BG_ABOX_COLS = 64;
-constexpr int BG_BBOX_ROWS = 64;
 // row_stride: elements between consecutive rows (0 = inner, densely packed);
 // swizzle: 0 (none), 32, 64 or 128 bytes
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
                   uint32_t box_inner, uint32_t box_outer, int swizzle,
                   uint64_t row_stride = 0);
 
+// The gathered-tile kernel (bgmv.cu): plain pointers, no tensor maps.
 struct GbArgs {
-    CUtensorMap tmA[LORA_MAX_SLICES][4];
-    CUtensorMap tmB[LORA_MAX_SLICES][4];
     const __nv_bfloat16 *x;
     int64_t ld_x;
     int d_in;
@@ -39,12 +31,12 @@ struct GbArgs {
     Tiles tiles;
     int32_t *status;
     int *ctl;          // fused mode: tickets and exit counter (workspace head)
-    int *done;         // fused mode: per unit, shrink blocks finished
-    int bc;            // columns of one expand item (multiple of 64)
+    int *done;         // fused mode: per unit, shrink items finished
+    int bc;            // output columns of one expand item (multiple of 32)
     int blk_off[LORA_MAX_SLICES + 1];   // expand items per unit: slice s owns [blk_off[s], blk_off[s+1])
-    int stages;        // ring stages (2 .. 6)
-    unsigned wait_limit;   // tries of a bounded wait (WAIT_LIMIT; shorter for the stall test hook)
-    int dbg_stall;     // test hook: every block's first stage expects 16 bytes that never come
+    int stages;        // steps in flight per warp (2 .. 4)
+    unsigned wait_limit;   // tries of the bounded wait (WAIT_LIMIT; shorter for the stall test hook)
+    int dbg_stall;     // test hook: expand items wait for one shrink signal more than exists
 };
 
 struct SimtArgs {
@@ -108,11 +100,11 @@ size_t segments_scratch_bytes(int T, int N);
 int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
                           size_t scratch_bytes, int32_t *status, cudaStream_t st);
 
-// bgmv.cu: bf16, r_max <= 64 and a multiple of 8, n_slices * r_max <= 512,
-// 16-byte aligned rows; units of up to LORA_MAX_TILE_ROWS rows; persistent
-// clusters of `cluster` blocks (1 for the expand-only mode)
+// bgmv.cu: bf16, r_max <= 64 and a multiple of 8, 16-byte aligned rows; units
+// of up to LORA_MAX_TILE_ROWS rows; a persistent grid of one block per SM
+// (`blocks` blocks when positive)
 size_t bgmv_smem_bytes(int mode, int stages);
-int launch_bgmv(int mode, const GbArgs &a, int cluster, cudaStream_t st);
+int launch_bgmv(int mode, const GbArgs &a, int blocks, cudaStream_t st);
 // workspace of the fused mode: control words, then one int per unit, then v
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max);
 

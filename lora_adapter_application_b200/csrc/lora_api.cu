@@ -308,31 +308,28 @@ int device_sms() {
     return sms;
 }
 
-// Blocks per cluster of the fused kernel's shrink: one per 1024 input columns
-// (up to 8), so that a unit's A reaches the cluster in about 1024 columns per
-// block; the expand-only mode needs no cluster.  Tuning override:
-// LORA_BG_CLUSTER = 1, 2, 4 or 8.
-int bgmv_cluster(int mode, int d_in) {
-    if (mode == MODE_EXPAND) return 1;
-    const int e = env_int("LORA_BG_CLUSTER", 0);
-    if (e == 1 || e == 2 || e == 4 || e == 8) return e;
-    return d_in <= 1536 ? 1 : (d_in <= 3072 ? 2 : (d_in <= 6144 ? 4 : 8));
+// Grid of the gathered-tile kernel: one block per SM.  Tuning / test override:
+// LORA_BG_BLOCKS = 1 .. 4096 blocks (the kernel makes progress with any number
+// resident).
+int bgmv_blocks() {
+    const int e = env_int("LORA_BG_BLOCKS", 0);
+    return e >= 1 && e <= 4096 ? e : 0;
 }
 
-// Output columns of one expand item: the widest of 2048 .. 256 that still gives
-// about six items per block for the batch's expected units (the expand phase
-// is balanced by handing out many items of similar size).  Tuning override:
-// LORA_BG_ITEM_COLS, a multiple of 64 from 64 to 8192.
+// Output columns of one expand item (one warp's): the widest of 1024 .. 128
+// that still gives about six items per warp for the batch's expected units
+// (the expand phase is balanced by handing out many items of similar size).
+// Tuning override: LORA_BG_ITEM_COLS, a multiple of 32 from 32 to 8192.
 int bgmv_item_cols(const Call &c, int est_units) {
     const int e = env_int("LORA_BG_ITEM_COLS", 0);
-    if (e >= 64 && e <= 8192 && (e & 63) == 0) return e;
-    const int target = 6 * device_sms();
-    for (int bc = 2048; bc > 256; bc >>= 1) {
+    if (e >= 32 && e <= 8192 && (e & 31) == 0) return e;
+    const int target = 6 * 8 * device_sms();
+    for (int bc = 1024; bc > 128; bc >>= 1) {
         int64_t items = 0;
         for (int s = 0; s < c.n_slices; ++s) items += (c.slices[s].d_out + bc - 1) / bc;
         if (items * est_units >= target) return bc;
     }
-    return 256;
+    return 128;
 }
 
 // The gathered tiles (and the contiguous ones unless tc_took) on the fused
@@ -345,61 +342,43 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
     (void)tc_took;
     if (bgmv_ok(mode, c, need_x, need_y)) {
         GbArgs g{};
-        bool maps_ok = true;
-        const int N = c.meta->N;
-        for (int s = 0; s < c.n_slices && maps_ok; ++s)
-            for (int i = 0; i < 4 && maps_ok; ++i) {
-                const int R = 8 << i;
-                if (R > c.r_max) break;
-                if (need_x)
-                    maps_ok = tensor_map_2d(&g.tmA[s][i], c.slices[s].A, (uint64_t)c.d_in,
-                                            (uint64_t)N * c.r_max, BG_ABOX_COLS, (uint32_t)R, 128) == LORA_OK;
-                if (need_y && maps_ok)
-                    maps_ok = tensor_map_2d(&g.tmB[s][i], c.slices[s].B, (uint64_t)c.r_max,
-                                            (uint64_t)N * c.slices[s].d_out, (uint32_t)R, BG_BBOX_ROWS,
-                                            R == 8 ? 0 : 2 * R) == LORA_OK;
-            }
-        if (maps_ok) {
-            g.x = static_cast<const __nv_bfloat16 *>(c.x);
-            g.ld_x = c.ld_x;
-            g.d_in = c.d_in;
-            g.y = static_cast<__nv_bfloat16 *>(c.y);
-            g.ld_y = c.ld_y;
-            g.T = c.meta->T;
-            g.sl = make_slices(c);
-            g.r_max = c.r_max;
-            g.ranks = c.ranks;
-            g.alphas = c.alphas;
-            g.tiles = tiles;
-            g.status = c.status;
-            if (mode == MODE_FUSED) {   // control words, per-unit counters, v: the workspace
-                unsigned char *ws = static_cast<unsigned char *>(c.ws);
-                g.ctl = reinterpret_cast<int *>(ws);
-                g.done = g.ctl + 64;
-                g.v = reinterpret_cast<float *>(ws + bgmv_workspace_bytes(units, 0, 1, 8));
-            } else {
-                g.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
-            }
-            const int est = std::min(units, std::min(c.meta->N, c.meta->T) +
-                                                (c.meta->T + c.meta->rows_per_tile - 1) / c.meta->rows_per_tile);
-            g.bc = bgmv_item_cols(c, std::max(1, est));
-            g.blk_off[0] = 0;
-            for (int s = 0; s < c.n_slices; ++s)
-                g.blk_off[s + 1] = g.blk_off[s] + (c.slices[s].d_out + g.bc - 1) / g.bc;
-            // tuning override: LORA_BG_STAGES = 2 .. 6 ring stages of 32 KB
-            g.stages = env_int("LORA_BG_STAGES", 4);
-            if (g.stages < 2 || g.stages > 6) g.stages = 4;
-            g.wait_limit = WAIT_LIMIT;
-            int cl = bgmv_cluster(mode, c.d_in);
-            if (env_int("LORA_DEBUG_STALL", 0) == 1) {
-                // test hook for the bounded waits: one-block clusters (every wait bounded,
-                // no peer to leave behind), short waits, and a first stage that never fills
-                g.dbg_stall = 1;
-                g.wait_limit = 64;
-                cl = 1;
-            }
-            return launch_bgmv(mode, g, cl, stream);
+        g.x = static_cast<const __nv_bfloat16 *>(c.x);
+        g.ld_x = c.ld_x;
+        g.d_in = c.d_in;
+        g.y = static_cast<__nv_bfloat16 *>(c.y);
+        g.ld_y = c.ld_y;
+        g.T = c.meta->T;
+        g.sl = make_slices(c);
+        g.r_max = c.r_max;
+        g.ranks = c.ranks;
+        g.alphas = c.alphas;
+        g.tiles = tiles;
+        g.status = c.status;
+        if (mode == MODE_FUSED) {   // control words, per-unit counters, v: the workspace
+            unsigned char *ws = static_cast<unsigned char *>(c.ws);
+            g.ctl = reinterpret_cast<int *>(ws);
+            g.done = g.ctl + 64;
+            g.v = reinterpret_cast<float *>(ws + bgmv_workspace_bytes(units, 0, 1, 8));
+        } else {
+            g.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
         }
+        const int est = std::min(units, std::min(c.meta->N, c.meta->T) +
+                                            (c.meta->T + c.meta->rows_per_tile - 1) / c.meta->rows_per_tile);
+        g.bc = bgmv_item_cols(c, std::max(1, est));
+        g.blk_off[0] = 0;
+        for (int s = 0; s < c.n_slices; ++s)
+            g.blk_off[s + 1] = g.blk_off[s] + (c.slices[s].d_out + g.bc - 1) / g.bc;
+        // tuning override: LORA_BG_STAGES = 2 .. 4 steps in flight per warp
+        g.stages = env_int("LORA_BG_STAGES", 4);
+        if (g.stages < 2 || g.stages > 4) g.stages = 4;
+        g.wait_limit = WAIT_LIMIT;
+        if (env_int("LORA_DEBUG_STALL", 0) == 1) {
+            // test hook for the bounded wait: expand items wait for a shrink signal
+            // that never comes, with a short limit
+            g.dbg_stall = 1;
+            g.wait_limit = 64;
+        }
+        return launch_bgmv(mode, g, bgmv_blocks(), stream);
     }
     SimtArgs a{};
     a.x = c.x;

@@ -51,13 +51,13 @@ def test_small_bf16_cases(cuda_lib, case, fn, R):
 
 
 @pytest.mark.parametrize("r_max", [32, 64])
-@pytest.mark.parametrize("C", ["1", "2", "4", "8"])
-@pytest.mark.parametrize("stages", ["2", "4"])
-def test_ranks_17_to_24(cuda_lib, r_max, C, stages, monkeypatch):
-    """Ranks 17-24 (24 or 32 loaded ranks: a 16- and an 8-rank A box, three 8-rank
-    B boxes, or one 32-rank B box) over 4096 columns, every cluster size and two
-    ring depths."""
-    monkeypatch.setenv("LORA_BG_CLUSTER", C)
+@pytest.mark.parametrize("blocks", ["1", "3", "0"])
+@pytest.mark.parametrize("stages", ["2", "3", "4"])
+def test_ranks_17_to_24(cuda_lib, r_max, blocks, stages, monkeypatch):
+    """Ranks 17-24 (24 loaded ranks, masked to r_n: two m16 rank tiles in the shrink,
+    one 32-rank chunk with a masked tail in the expand) over 4096 columns, on one
+    block, three blocks and the full grid, and every ring depth."""
+    monkeypatch.setenv("LORA_BG_BLOCKS", blocks)
     monkeypatch.setenv("LORA_BG_STAGES", stages)
     ranks = [17 + (i % 8) for i in range(12)]
     w = workloads.random_case(41, 256, 12, 4096, [4096], r_max, ranks=ranks, none_frac=0.05,

@@ -189,25 +189,25 @@ def test_workspace_serves_call_after_call(cuda_lib):
 
 
 # ------------------------------------------------------------------ passes and slice groups
-@pytest.mark.parametrize("C", ["1", "4"])
-def test_eight_slices_rank_64_multi_pass(cuda_lib, C, monkeypatch):
-    """8 slices of rank 64 and 64-row tiles: 64 x 512 partials exceed one exchange
-    (tiles reduce in 4 passes of 16 rows) and 64 columns of 8 slices' A exceed a
-    stage (chunks stream 3 slices at a time)."""
-    monkeypatch.setenv("LORA_BG_CLUSTER", C)
+@pytest.mark.parametrize("blocks", ["1", "0"])
+def test_eight_slices_rank_64_multi_pass(cuda_lib, blocks, monkeypatch):
+    """8 slices of rank 64 and 64-row tiles: 16 shrink items per unit (8 slices x two
+    32-rank groups), expand items in two 32-row passes, on one block and on the
+    full grid."""
+    monkeypatch.setenv("LORA_BG_BLOCKS", blocks)
     w = workloads.random_case(57, 260, 3, 256, [64] * 8, 64, ranks=[64, 64, 40], none_frac=0.0)
     lay = w.layers[0]
     dl = DeviceLayer(lay)
     meta, status = build_meta(w.ids, w.N, 64, 0)
     _check(w, lay, _apply(lora.lora_bgmv_fused, w, lay, dl.A, dl.B, meta, status), status,
-           f"8 slices C={C}")
+           f"8 slices blocks={blocks}")
 
 
 # ------------------------------------------------------------------ launch-shape overrides
 @pytest.mark.parametrize("env", [
-    {"LORA_BG_ITEM_COLS": "64"}, {"LORA_BG_ITEM_COLS": "192"}, {"LORA_BG_ITEM_COLS": "4096"},
-    {"LORA_BG_STAGES": "2"}, {"LORA_BG_STAGES": "3"}, {"LORA_BG_CLUSTER": "1"},
-    {"LORA_BG_CLUSTER": "2"}, {"LORA_BG_CLUSTER": "8"},
+    {"LORA_BG_ITEM_COLS": "32"}, {"LORA_BG_ITEM_COLS": "96"}, {"LORA_BG_ITEM_COLS": "192"},
+    {"LORA_BG_ITEM_COLS": "4096"}, {"LORA_BG_STAGES": "2"}, {"LORA_BG_STAGES": "3"},
+    {"LORA_BG_BLOCKS": "1"}, {"LORA_BG_BLOCKS": "2"}, {"LORA_BG_BLOCKS": "7"},
 ])
 def test_overrides_keep_parity(cuda_lib, env, monkeypatch):
     for k, v in env.items():
@@ -347,9 +347,10 @@ def test_capture_beside_an_eager_caller(cuda_lib):
 
 # ------------------------------------------------------------------ bounded waits
 def test_stalled_stage_times_out_and_the_context_survives(cuda_lib, monkeypatch):
-    """LORA_DEBUG_STALL=1: each block's first stage waits for 16 bytes that never
-    come; the bounded waits run out (~1 ms), LORA_DEV_TIMEOUT is set and the call
-    returns.  The same workspace then serves a normal call, exactly."""
+    """LORA_DEBUG_STALL=1: every expand item waits for one shrink signal more than
+    its unit ever gives; the bounded wait runs out (a few ms), LORA_DEV_TIMEOUT is
+    set and the call returns.  The same workspace then serves a normal call,
+    exactly."""
     w = workloads.random_case(64, 300, 5, 512, [256], 32)
     lay = w.layers[0]
     dl = DeviceLayer(lay)
@@ -366,12 +367,13 @@ def test_stalled_stage_times_out_and_the_context_survives(cuda_lib, monkeypatch)
 
 
 # ------------------------------------------------------------------ tile row counts
-@pytest.mark.parametrize("rows", [1, 15, 16, 17, 31, 33, 40, 47, 48, 49, 63, 64])
+@pytest.mark.parametrize("rows", [1, 7, 8, 9, 15, 16, 17, 24, 31, 32, 33, 40, 47, 48, 49, 63, 64])
 @pytest.mark.parametrize("S,ranks", [(1, [8, 64]), (3, [16, 40]), (2, [8, 33])])
 def test_every_tile_row_count(cuda_lib, rows, S, ranks):
-    """Two adapters with `rows` rows each, in 64-row tiles: every count of m16 tiles
-    per pass (1 to 4, idle warps when it is 3) and every split of a pass's rank
-    tiles over the warps (one pair per warp with k-groups, or several pairs)."""
+    """Two adapters with `rows` rows each, in 64-row tiles: every count of n8 row
+    tiles in the shrink (1, 2, 4 or 8 loaded, the rest zero-filled), one or two
+    32-row expand passes of one or two m16 tiles, and ranks that use one or two
+    m16 rank tiles and the 16-, 32- and 64-rank expand loads."""
     T = 2 * rows + 5
     ids = [0] * rows + [1] * rows + [-1] * 5
     perm = torch.randperm(T, generator=torch.Generator().manual_seed(rows))
