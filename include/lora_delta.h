@@ -51,7 +51,6 @@
  * from run to run.  A value outside the range is ignored.
  *   LORA_BG_BLOCKS      1 to 4096: blocks of the gathered-tile kernel's persistent
  *                       grid (default: one per SM)
- *   LORA_BG_STAGES      2 to 4: steps in flight per warp of the gathered-tile kernel
  *   LORA_BG_ITEM_COLS   32 to 8192, a multiple of 32: output columns of one expand item
  *   LORA_TC_CLUSTER     1, 2, 4 or 8: blocks per cluster of the tensor-core kernel;
  *                       when the shape cannot use it, the contiguous tiles run on

@@ -21,9 +21,9 @@
 // per operand row per step with cp.async, straight into the order the mma
 // fragments want (lane (g, t) of an 8-row operand reads columns 8t..8t+7 of row
 // g; both operands of a product use the same permutation of the 32 columns of
-// a step, so the sum over k is unchanged).  Each warp keeps a private ring of
-// `stages` steps in flight (6 KB per step), so loads issue from all warps of
-// the SM and no thread walks the work for the others; an 8-row x 64-byte load
+// a step, so the sum over k is unchanged).  Each warp keeps a private 24 KB
+// ring of steps in flight (2 to 16 of them, by step size), so loads issue from
+// all warps of the SM and no thread walks the work for the others; an 8-row x 64-byte load
 // keeps whole 32-byte sectors, and a warp's stream runs along its rows for its
 // whole column range.  Output columns of an expand step are permuted the same
 // way (lane t's accumulators are columns 8t..8t+7 of its rows), so y moves in
@@ -56,13 +56,16 @@ namespace {
 constexpr int BG_WARPS = 8;
 constexpr int BG_THREADS = BG_WARPS * 32;
 constexpr int BG_ROWS = LORA_MAX_TILE_ROWS;      // rows of one unit
-constexpr int BG_LD = 12;                        // 16-byte loads per lane per ring step
-constexpr int BG_STEP = BG_LD * 32 * 16;         // bytes of one step of a warp's ring
-constexpr int BG_MAX_STAGES = 4;
+constexpr int BG_RING = 24576;                   // bytes of one warp's ring of steps
 constexpr int BG_RG = 32;                        // ranks of one shrink item
 constexpr int BG_RED_LD = BG_RG + 4;             // floats per row of the shrink reduction
 constexpr int BG_RED_BYTES = BG_WARPS * BG_ROWS * BG_RED_LD * 4;
-static_assert(BG_RED_BYTES <= 2 * BG_WARPS * BG_STEP, "the reduction fits the smallest ring");
+static_assert(BG_RED_BYTES <= BG_WARPS * BG_RING, "the reduction overlays the rings");
+
+// Steps of nld 16-byte loads per lane (nld * 512 bytes per warp) that a ring holds.
+__host__ __device__ constexpr int ring_depth(int nld) {
+    return BG_RING / (nld * 512) > 16 ? 16 : BG_RING / (nld * 512);
+}
 
 // Workspace head of the fused mode (ints): tickets and exit counter, then one
 // counter per unit.
@@ -72,34 +75,29 @@ enum { GB_T_SHRINK = 0, GB_T_EXPAND = 1, GB_T_EXIT = 2 };
 constexpr unsigned FULL = 0xffffffffu;
 
 // ------------------------------------------------------------------ PTX helpers
+// (not volatile: the compiler may interleave independent products)
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// 16 (8) bytes global -> shared through L2; zero-filled (nothing read) when !valid
-__device__ __forceinline__ void cp16(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-                 "r"(valid ? 16 : 0)
+// 16 (8) bytes global -> shared through L2, of which the first `bytes` are read and
+// the rest zero-filled (0: nothing read)
+__device__ __forceinline__ void cp16(uint32_t dst, const void *src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ void cp8(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(src),
-                 "r"(valid ? 8 : 0)
+__device__ __forceinline__ void cp8(uint32_t dst, const void *src, int bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
                  : "memory");
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-// wait until at most n of this thread's copy groups are still in flight
-__device__ __forceinline__ void cp_wait(int n) {
-    switch (n) {
-        case 0: asm volatile("cp.async.wait_group 0;\n" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;\n" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;\n" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 3;\n" ::: "memory"); break;
-    }
+// wait until at most N of this thread's copy groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 r;
@@ -133,10 +131,7 @@ __device__ __forceinline__ void split2(float v0, float v1, uint32_t &hi, uint32_
     hi = pack_bf16x2(v0, v1);
     lo = pack_bf16x2(v0 - bf_lo(hi), v1 - bf_hi(hi));
 }
-// halves of a bf16 pair word that hold ranks k, k+1: all ones where the rank is below r_n
-__device__ __forceinline__ uint32_t rank_mask(int k, int r_n) {
-    return (k < r_n ? 0x0000ffffu : 0u) | (k + 1 < r_n ? 0xffff0000u : 0u);
-}
+__device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
 // ------------------------------------------------------------------ shrink
 // One warp's part of a shrink item: rank rows [0, rv) of the item's 32 (A_rows,
@@ -147,42 +142,45 @@ __device__ __forceinline__ uint32_t rank_mask(int k, int r_n) {
 template <int MG, int NTR>
 __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int rv, const char *x,
                                             int64_t ldx, const int *rows_s, int d_in, int k_lo,
-                                            int k_hi, uint32_t ring, int NS, float *red) {
+                                            int k_hi, uint32_t ring, float *red) {
+    constexpr int NLD = 2 * MG + NTR;
+    constexpr int NSL = ring_depth(NLD);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const char *pa[MG][2];
-    bool va[MG][2];
+    // row starts (a row past the item reads nothing: its start stands in)
+    const char *p[NLD];
+    int sz[NLD];
 #pragma unroll
     for (int mi = 0; mi < MG; ++mi)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int rr = 16 * mi + 8 * h + g;
-            va[mi][h] = rr < rv;
-            pa[mi][h] = A_rows + (va[mi][h] ? rr : 0) * lda + 16 * t;
+            const bool ok = rr < rv;
+            p[2 * mi + h] = A_rows + (ok ? rr : 0) * lda;
+            sz[2 * mi + h] = ok ? 16 : 0;
         }
-    const char *px[NTR];
-    bool vx[NTR];
 #pragma unroll
     for (int i = 0; i < NTR; ++i) {
         const int r = rows_s[8 * i + g];
-        vx[i] = r >= 0;
-        px[i] = x + (int64_t)(vx[i] ? r : 0) * ldx + 16 * t;
+        const bool ok = r >= 0;
+        p[2 * MG + i] = x + (int64_t)(ok ? r : 0) * ldx;
+        sz[2 * MG + i] = ok ? 16 : 0;
     }
+    const int nst = k_hi - k_lo;
+    const int nfull = clampi((d_in >> 5) - k_lo, 0, nst);   // steps inside d_in for every lane
+    const int jv = max(0, (d_in - 8 * t - 32 * k_lo + 31) >> 5);   // steps inside d_in for this lane
     const uint32_t lbase = ring + (uint32_t)lane * 16u;
-    auto issue = [&](int ks, int slot) {
-        const uint32_t b = lbase + (uint32_t)slot * BG_STEP;
-        const bool cv = 32 * ks + 8 * t < d_in;
+    auto issue = [&](int j, int slot) {
+        const uint32_t b = lbase + (uint32_t)(slot * NLD * 512);
+        if (j < nfull) {
+            const int off = 64 * (k_lo + j) + 16 * t;
 #pragma unroll
-        for (int mi = 0; mi < MG; ++mi)
+            for (int l = 0; l < NLD; ++l) cp16(b + l * 512, p[l] + off, sz[l]);
+        } else {
+            const bool cv = j < jv;
+            const int off = cv ? 64 * (k_lo + j) + 16 * t : 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const bool ok = va[mi][h] && cv;
-                cp16(b + (2 * mi + h) * 512, ok ? pa[mi][h] + 64 * ks : A_rows, ok);
-            }
-#pragma unroll
-        for (int i = 0; i < NTR; ++i) {
-            const bool ok = vx[i] && cv;
-            cp16(b + (2 * MG + i) * 512, ok ? px[i] + 64 * ks : x, ok);
+            for (int l = 0; l < NLD; ++l) cp16(b + l * 512, p[l] + off, cv ? sz[l] : 0);
         }
     };
     float acc[MG][NTR][4];
@@ -193,37 +191,35 @@ __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[mi][i][e] = 0.f;
 
-    const int nst = k_hi - k_lo;
-    for (int j = 0; j < NS - 1; ++j) {
-        if (j < nst) issue(k_lo + j, j);
+#pragma unroll
+    for (int j = 0; j < NSL - 1; ++j) {
+        if (j < nst) issue(j, j);
         cp_commit();
     }
+    int si = NSL - 1, sc = 0;   // slots of the next issue and of the next step consumed
     for (int j = 0; j < nst; ++j) {
-        const int jn = j + NS - 1;
-        if (jn < nst) issue(k_lo + jn, jn % NS);
+        if (j + NSL - 1 < nst) issue(j + NSL - 1, si);
+        si = si + 1 == NSL ? 0 : si + 1;
         cp_commit();
-        cp_wait(NS - 1);
-        const uint32_t b = lbase + (uint32_t)(j % NS) * BG_STEP;
-        uint4 qa[MG][2], qx[NTR];
+        cp_wait<NSL - 1>();
+        const uint32_t b = lbase + (uint32_t)(sc * NLD * 512);
+        sc = sc + 1 == NSL ? 0 : sc + 1;
+        uint4 q[NLD];
 #pragma unroll
-        for (int mi = 0; mi < MG; ++mi) {
-            qa[mi][0] = lds128(b + (2 * mi) * 512);
-            qa[mi][1] = lds128(b + (2 * mi + 1) * 512);
-        }
+        for (int l = 0; l < NLD; ++l) q[l] = lds128(b + l * 512);
 #pragma unroll
-        for (int i = 0; i < NTR; ++i) qx[i] = lds128(b + (2 * MG + i) * 512);
+        for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int mi = 0; mi < MG; ++mi) {
-            const uint32_t a0[4] = {qa[mi][0].x, qa[mi][1].x, qa[mi][0].y, qa[mi][1].y};
-            const uint32_t a1[4] = {qa[mi][0].z, qa[mi][1].z, qa[mi][0].w, qa[mi][1].w};
+            for (int mi = 0; mi < MG; ++mi) {
+                const uint32_t a[4] = {kb ? q[2 * mi].z : q[2 * mi].x, kb ? q[2 * mi + 1].z : q[2 * mi + 1].x,
+                                       kb ? q[2 * mi].w : q[2 * mi].y, kb ? q[2 * mi + 1].w : q[2 * mi + 1].y};
 #pragma unroll
-            for (int i = 0; i < NTR; ++i) {
-                mma16816(acc[mi][i], a0, qx[i].x, qx[i].y);
-                mma16816(acc[mi][i], a1, qx[i].z, qx[i].w);
+                for (int i = 0; i < NTR; ++i)
+                    mma16816(acc[mi][i], a, kb ? q[2 * MG + i].z : q[2 * MG + i].x,
+                             kb ? q[2 * MG + i].w : q[2 * MG + i].y);
             }
-        }
     }
-    cp_wait(0);
+    cp_wait<0>();
     __syncthreads();   // every warp is done with its ring: the reduction buffer overlays them
     float *rw = red + warp * BG_ROWS * BG_RED_LD;
 #pragma unroll
@@ -241,15 +237,15 @@ __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int
 template <int MG>
 __device__ __forceinline__ void shrink_dispatch(int ntr, const char *A_rows, int64_t lda, int rv,
                                                 const char *x, int64_t ldx, const int *rows_s, int d_in,
-                                                int k_lo, int k_hi, uint32_t ring, int NS, float *red) {
+                                                int k_lo, int k_hi, uint32_t ring, float *red) {
     if (ntr <= 1)
-        shrink_warp<MG, 1>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, NS, red);
+        shrink_warp<MG, 1>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
     else if (ntr <= 2)
-        shrink_warp<MG, 2>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, NS, red);
+        shrink_warp<MG, 2>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
     else if (ntr <= 4)
-        shrink_warp<MG, 4>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, NS, red);
+        shrink_warp<MG, 4>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
     else
-        shrink_warp<MG, 8>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, NS, red);
+        shrink_warp<MG, 8>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
 }
 
 // ------------------------------------------------------------------ expand
@@ -257,17 +253,22 @@ __device__ __forceinline__ void shrink_dispatch(int ntr, const char *A_rows, int
 // to 32 rows of a unit (row_l: this lane's row, -1 past the unit; rows 16*mi+g
 // and 16*mi+g+8 of the pass are m16 tile mi).  RK: ranks loaded per row,
 // 16 (8-byte loads of ranks 4t..4t+3), 32 or 64 (16-byte loads of ranks
-// 32c+8t..32c+8t+7).  m = rows, n = output columns: n-tile j's column for
-// n-index q is c0 + 8*(q>>1) + 2*j + (q&1), so lane t ends with columns
-// c0+8t .. c0+8t+7.
+// 32c+8t..32c+8t+7); bytes past rank r_n are zero-filled, not read.  m = rows,
+// n = output columns: n-tile j's column for n-index q is
+// c0 + 8*(q>>1) + 2*j + (q&1), so lane t ends with columns c0+8t .. c0+8t+7.
+// The accumulators start from the y values, so y + scale * v . B^T is rounded
+// to bf16 once.
 template <int MR, int RK>
 __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max, int r_n,
                                             float scale, int c_lo, int c_hi,
                                             __nv_bfloat16 *ys, int64_t ld_y, const float *vs,
-                                            uint32_t ring, int NS) {
+                                            uint32_t ring) {
     constexpr int CH = RK == 64 ? 2 : 1;            // rank chunks per step
     constexpr int NB = 4 * CH;                      // B loads per step
+    constexpr int NLD = NB + 2 * MR;
+    constexpr int NSL = ring_depth(NLD);
     constexpr int KB = RK == 16 ? 1 : 2;            // k16 products per chunk
+    constexpr int LB = RK == 16 ? 8 : 16;           // bytes of one B load
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int r8 = (r_n + 7) & ~7;
     // rows of this lane's y pieces and v fragments
@@ -276,43 +277,79 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
     for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
         for (int h = 0; h < 2; ++h) yrow[mi][h] = __shfl_sync(FULL, row_l, 16 * mi + 8 * h + g);
-    // B rank offset of chunk c for this lane, and the masks of ranks r_n..r8
     const int rk0 = RK == 16 ? 4 * t : 8 * t;
-    uint32_t bm[CH][4];
+    int szb[CH];   // bytes of chunk c below rank r_n
 #pragma unroll
-    for (int c = 0; c < CH; ++c)
+    for (int c = 0; c < CH; ++c) szb[c] = clampi(2 * (r_n - 32 * c - rk0), 0, LB);
+    // B column of n-tile j at step ks: cb + 2j + 32ks (B rows are r_max ranks long); a
+    // chunk that this lane reads nothing of points at Bn and does not move
+    const int cb = c_lo + 8 * (g >> 1) + (g & 1);
+    const char *pbc[CH];
+    int bs[CH], bj[CH];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) bm[c][p] = rank_mask(32 * c + rk0 + 2 * p, r_n);
-    const int bcol = 8 * (g >> 1) + (g & 1);
+    for (int c = 0; c < CH; ++c) {
+        const bool any = szb[c] > 0 && cb < c_hi;
+        pbc[c] = any ? Bn + ((int64_t)cb * r_max + rk0 + 32 * c) * 2 : Bn;
+        bs[c] = any ? 64 * r_max : 0;
+        bj[c] = any ? 4 * r_max : 0;
+    }
+    // y piece of row (mi, h) at step ks: columns c_lo + 8t + 32ks .. +7
+    const char *py[MR][2];
+    int sy[MR][2];
+#pragma unroll
+    for (int mi = 0; mi < MR; ++mi)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const bool ok = yrow[mi][h] >= 0;
+            py[mi][h] = reinterpret_cast<const char *>(ys + (int64_t)(ok ? yrow[mi][h] : 0) * ld_y) +
+                        (ok ? 2 * (c_lo + 8 * t) : 0);
+            sy[mi][h] = ok ? 16 : 0;
+        }
+    const int nst = (c_hi - c_lo + 31) >> 5;
+    const int nfull = (c_hi - c_lo) >> 5;   // steps whose 32 columns are all inside
     const uint32_t lbase = ring + (uint32_t)lane * 16u;
     auto issue = [&](int ks, int slot) {
-        const uint32_t b = lbase + (uint32_t)slot * BG_STEP;
-        const int c0 = c_lo + 32 * ks;
+        const uint32_t b = lbase + (uint32_t)(slot * NLD * 512);
+        if (ks < nfull) {
 #pragma unroll
-        for (int c = 0; c < CH; ++c)
+            for (int c = 0; c < CH; ++c)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int col = c0 + bcol + 2 * j;
-                const bool ok = col < c_hi && 32 * c + rk0 < r8;
-                const char *src = Bn + ((int64_t)col * r_max + 32 * c + rk0) * 2;
-                if (RK == 16)
-                    cp8(b + (4 * c + j) * 512, ok ? src : Bn, ok);
-                else
-                    cp16(b + (4 * c + j) * 512, ok ? src : Bn, ok);
-            }
-        const bool cv = c0 + 8 * t < c_hi;
+                for (int j = 0; j < 4; ++j) {
+                    const char *src = pbc[c] + (ks * bs[c] + j * bj[c]);
+                    if (RK == 16)
+                        cp8(b + (4 * c + j) * 512, src, szb[c]);
+                    else
+                        cp16(b + (4 * c + j) * 512, src, szb[c]);
+                }
 #pragma unroll
-        for (int mi = 0; mi < MR; ++mi)
+            for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const bool ok = cv && yrow[mi][h] >= 0;
-                const char *src = reinterpret_cast<const char *>(ys + (int64_t)(ok ? yrow[mi][h] : 0) * ld_y +
-                                                                 (ok ? c0 + 8 * t : 0));
-                cp16(b + (NB + 2 * mi + h) * 512, src, ok);
-            }
+                for (int h = 0; h < 2; ++h)
+                    cp16(b + (NB + 2 * mi + h) * 512, py[mi][h] + (sy[mi][h] ? 64 * ks : 0), sy[mi][h]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < CH; ++c)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const bool ok = cb + 2 * j + 32 * ks < c_hi;
+                    const char *src = ok ? pbc[c] + (ks * bs[c] + j * bj[c]) : Bn;
+                    if (RK == 16)
+                        cp8(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
+                    else
+                        cp16(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
+                }
+            const bool cv = c_lo + 8 * t + 32 * ks < c_hi;
+#pragma unroll
+            for (int mi = 0; mi < MR; ++mi)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const bool ok = cv && sy[mi][h];
+                    cp16(b + (NB + 2 * mi + h) * 512, py[mi][h] + (ok ? 64 * ks : 0), ok ? 16 : 0);
+                }
+        }
     };
-    const int nst = (c_hi - c_lo + 31) >> 5;
-    for (int j = 0; j < NS - 1; ++j) {   // the first steps fly while v is read
+#pragma unroll
+    for (int j = 0; j < NSL - 1; ++j) {   // the first steps fly while v is read
         if (j < nst) issue(j, j);
         cp_commit();
     }
@@ -328,11 +365,11 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
                 const int k = 32 * c + rk0;
                 float f[8];
                 if (row >= 0 && k < r8) {
-                    const float4 *p = reinterpret_cast<const float4 *>(vs + (int64_t)row * r_max + k);
-                    const float4 lo4 = p[0];
+                    const float4 *pv = reinterpret_cast<const float4 *>(vs + (int64_t)row * r_max + k);
+                    const float4 lo4 = pv[0];
                     f[0] = lo4.x; f[1] = lo4.y; f[2] = lo4.z; f[3] = lo4.w;
                     if (RK != 16) {
-                        const float4 hi4 = p[1];
+                        const float4 hi4 = pv[1];
                         f[4] = hi4.x; f[5] = hi4.y; f[6] = hi4.z; f[7] = hi4.w;
                     } else {
                         f[4] = f[5] = f[6] = f[7] = 0.f;
@@ -347,19 +384,28 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
                 for (int p = 0; p < 4; ++p) split2(f[2 * p], f[2 * p + 1], vh[mi][c][h][p], vl[mi][c][h][p]);
             }
 
+    int si = NSL - 1, sc = 0;
     for (int ks = 0; ks < nst; ++ks) {
-        const int jn = ks + NS - 1;
-        if (jn < nst) issue(jn, jn % NS);
+        if (ks + NSL - 1 < nst) issue(ks + NSL - 1, si);
+        si = si + 1 == NSL ? 0 : si + 1;
         cp_commit();
-        cp_wait(NS - 1);
-        const uint32_t b = lbase + (uint32_t)(ks % NS) * BG_STEP;
+        cp_wait<NSL - 1>();
+        const uint32_t b = lbase + (uint32_t)(sc * NLD * 512);
+        sc = sc + 1 == NSL ? 0 : sc + 1;
+        // accumulators from the y values: word j of row (mi, h) = columns 8t+2j, 8t+2j+1
         float acc[MR][4][4];
 #pragma unroll
         for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int h = 0; h < 2; ++h) {
+                const uint4 w = lds128(b + (NB + 2 * mi + h) * 512);
+                const uint32_t win[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[mi][j][e] = 0.f;
+                for (int j = 0; j < 4; ++j) {
+                    acc[mi][j][2 * h] = bf_lo(win[j]);
+                    acc[mi][j][2 * h + 1] = bf_hi(win[j]);
+                }
+            }
 #pragma unroll
         for (int c = 0; c < CH; ++c)
 #pragma unroll
@@ -367,60 +413,75 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
                 uint32_t q[4];
                 if (RK == 16) {
                     const uint2 w = lds64(b + (4 * c + j) * 512);
-                    q[0] = w.x & bm[c][0];
-                    q[1] = w.y & bm[c][1];
+                    q[0] = w.x;
+                    q[1] = w.y;
                     q[2] = q[3] = 0u;
                 } else {
                     const uint4 w = lds128(b + (4 * c + j) * 512);
-                    q[0] = w.x & bm[c][0];
-                    q[1] = w.y & bm[c][1];
-                    q[2] = w.z & bm[c][2];
-                    q[3] = w.w & bm[c][3];
+                    q[0] = w.x;
+                    q[1] = w.y;
+                    q[2] = w.z;
+                    q[3] = w.w;
                 }
 #pragma unroll
-                for (int mi = 0; mi < MR; ++mi) {
+                for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-                    for (int kb = 0; kb < KB; ++kb) {
-                        const uint32_t ah[4] = {vh[mi][c][0][2 * kb], vh[mi][c][1][2 * kb],
-                                                vh[mi][c][0][2 * kb + 1], vh[mi][c][1][2 * kb + 1]};
-                        const uint32_t al[4] = {vl[mi][c][0][2 * kb], vl[mi][c][1][2 * kb],
-                                                vl[mi][c][0][2 * kb + 1], vl[mi][c][1][2 * kb + 1]};
-                        mma16816(acc[mi][j], ah, q[2 * kb], q[2 * kb + 1]);
-                        mma16816(acc[mi][j], al, q[2 * kb], q[2 * kb + 1]);
-                    }
-                }
+                    for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+                        for (int mi = 0; mi < MR; ++mi) {
+                            const uint32_t(&vv)[2][4] = hl ? vl[mi][c] : vh[mi][c];
+                            const uint32_t av[4] = {vv[0][2 * kb], vv[1][2 * kb], vv[0][2 * kb + 1],
+                                                    vv[1][2 * kb + 1]};
+                            mma16816(acc[mi][j], av, q[2 * kb], q[2 * kb + 1]);
+                        }
             }
-        // y rows: lane t's 8 columns, word j = columns 8t+2j, 8t+2j+1 = accumulators (j, 2h), (j, 2h+1)
         const int c0 = c_lo + 32 * ks;
         const bool cv = c0 + 8 * t < c_hi;
 #pragma unroll
         for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 w = lds128(b + (NB + 2 * mi + h) * 512);
-                const uint32_t win[4] = {w.x, w.y, w.z, w.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    o[j] = pack_bf16x2(bf_lo(win[j]) + acc[mi][j][2 * h],
-                                       bf_hi(win[j]) + acc[mi][j][2 * h + 1]);
+            for (int h = 0; h < 2; ++h)
                 if (cv && yrow[mi][h] >= 0)
-                    stg128(ys + (int64_t)yrow[mi][h] * ld_y + c0 + 8 * t, make_uint4(o[0], o[1], o[2], o[3]));
-            }
+                    stg128(ys + (int64_t)yrow[mi][h] * ld_y + c0 + 8 * t,
+                           make_uint4(pack_bf16x2(acc[mi][0][2 * h], acc[mi][0][2 * h + 1]),
+                                      pack_bf16x2(acc[mi][1][2 * h], acc[mi][1][2 * h + 1]),
+                                      pack_bf16x2(acc[mi][2][2 * h], acc[mi][2][2 * h + 1]),
+                                      pack_bf16x2(acc[mi][3][2 * h], acc[mi][3][2 * h + 1])));
     }
-    cp_wait(0);
+    cp_wait<0>();
 }
 
 template <int MR>
 __device__ __forceinline__ void expand_dispatch(int r8, int row_l, const char *Bn, int r_max, int r_n,
                                                 float scale, int c_lo, int c_hi, __nv_bfloat16 *ys,
-                                                int64_t ld_y, const float *vs, uint32_t ring, int NS) {
+                                                int64_t ld_y, const float *vs, uint32_t ring) {
     if (r8 <= 16)
-        expand_warp<MR, 16>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, NS);
+        expand_warp<MR, 16>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
     else if (r8 <= 32)
-        expand_warp<MR, 32>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, NS);
+        expand_warp<MR, 32>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
     else
-        expand_warp<MR, 64>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, NS);
+        expand_warp<MR, 64>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
+}
+
+// What an expand warp needs of one item before it starts: unit, rank, this
+// lane's row among the first 32 (loaded one item ahead).
+struct ERec {
+    Unit un;
+    int r_n;
+    int row_l;
+};
+__device__ __forceinline__ ERec erec_load(const GbArgs &a, int e, int total, int nb) {
+    ERec r{};
+    r.un = Unit{0, 0, 0, true};
+    r.r_n = 0;
+    r.row_l = -1;
+    if (e < total) {
+        r.un = resolve_live_unit(a.tiles, e / nb);
+        if (r.un.cnt > 0) r.r_n = a.ranks[r.un.id];
+        const int lane = threadIdx.x & 31;
+        r.row_l = lane < r.un.cnt ? r.un.row(a.tiles, lane) : -1;
+    }
+    return r;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -430,8 +491,7 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
     __shared__ int rows_s[BG_ROWS];
     __shared__ int info_s[4];   // current shrink ticket, next ticket, "this block leaves last"
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int NS = a.stages;
-    const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NS * BG_STEP);
+    const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * BG_RING);
     float *red = reinterpret_cast<float *>(smem);
     const int S = a.sl.n;
     const int live = n_live_units(a.tiles);
@@ -462,16 +522,15 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                 const char *A_rows = static_cast<const char *>(a.sl.A[s]) +
                                      ((int64_t)un.id * a.r_max + BG_RG * grp) * a.d_in * 2;
                 const char *x = reinterpret_cast<const char *>(a.x);
+                const int64_t lda = (int64_t)a.d_in * 2;
+                float *vb = a.v + (int64_t)s * a.T * a.r_max;
                 const int ntr = (un.cnt + 7) >> 3;
                 if (rv > 16)
-                    shrink_dispatch<2>(ntr, A_rows, (int64_t)a.d_in * 2, rv, x, a.ld_x * 2, rows_s, a.d_in,
-                                       k_lo, k_hi, ring, NS, red);
+                    shrink_dispatch<2>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring, red);
                 else
-                    shrink_dispatch<1>(ntr, A_rows, (int64_t)a.d_in * 2, rv, x, a.ld_x * 2, rows_s, a.d_in,
-                                       k_lo, k_hi, ring, NS, red);
+                    shrink_dispatch<1>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring, red);
                 __syncthreads();
                 // the 8 partials in warp order; v rows of the unit, ranks of the group below r_n
-                float *vb = a.v + (int64_t)s * a.T * a.r_max;
                 for (int p = tid; p < un.cnt * BG_RG; p += BG_THREADS) {
                     const int row = p / BG_RG, rl = p - row * BG_RG, k = BG_RG * grp + rl;
                     if (rl < rv && k < r_n) {
@@ -493,30 +552,33 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
     }
 
     // ------------------------------------------------------------ phase 2: expand
+    // Items are drawn two ahead and their records one ahead: while item i runs,
+    // the ticket of item i+2 and the unit, rank, alpha and first rows of item i+1
+    // are on their way.
     if (MODE != MODE_SHRINK) {
         const int nb = a.blk_off[S];
         const int total = live * nb;
         const int need = S * GM + (a.dbg_stall ? 1 : 0);   // the stall test hook waits for one more
-        int cur;
-        if (MODE == MODE_FUSED) {
-            cur = lane == 0 ? atomicAdd(a.ctl + GB_T_EXPAND, 1) : 0;
-            cur = __shfl_sync(FULL, cur, 0);
-        } else {
-            cur = (int)blockIdx.x * BG_WARPS + warp;
-        }
+        auto claim = [&](int prev) -> int {
+            if (MODE == MODE_FUSED) {
+                const int v = lane == 0 ? atomicAdd(a.ctl + GB_T_EXPAND, 1) : 0;
+                return __shfl_sync(FULL, v, 0);
+            }
+            return prev + (int)gridDim.x * BG_WARPS;
+        };
+        int cur = claim((int)blockIdx.x * BG_WARPS + warp - (int)gridDim.x * BG_WARPS);
+        ERec rc = erec_load(a, cur, total, nb);
+        int nxt = claim(cur);
         while (cur < total) {
-            int nxt;
-            if (MODE == MODE_FUSED)
-                nxt = lane == 0 ? atomicAdd(a.ctl + GB_T_EXPAND, 1) : 0;
-            else
-                nxt = cur + (int)gridDim.x * BG_WARPS;
+            const ERec rn = erec_load(a, nxt, total, nb);
+            const int nxt2 = nxt < total ? claim(nxt) : nxt;
             const int u = cur / nb, b = cur - u * nb;
             int s = 0;
             while (s + 1 < S && a.blk_off[s + 1] <= b) ++s;
             const int c_lo = (b - a.blk_off[s]) * a.bc;
             const int c_hi = min(c_lo + a.bc, (int)a.sl.d_out[s]);
-            const Unit un = resolve_live_unit(a.tiles, u);
-            const int r_n = un.cnt > 0 ? a.ranks[un.id] : 0;
+            const Unit &un = rc.un;
+            const int r_n = rc.r_n;
             const bool ok = un.cnt > 0 && r_n >= 1 && r_n <= a.r_max;
             if (!ok && un.cnt > 0 && b == 0 && lane == 0 && MODE == MODE_EXPAND)
                 atomicOr(a.status, LORA_DEV_BAD_RANK);
@@ -545,16 +607,16 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                 const float *vs = a.v + (int64_t)s * a.T * a.r_max;
                 for (int rg = 0; rg * 32 < un.cnt; ++rg) {
                     const int q = 32 * rg + lane;
-                    const int row_l = q < un.cnt ? un.row(a.tiles, q) : -1;
+                    const int row_l = rg == 0 ? rc.row_l : (q < un.cnt ? un.row(a.tiles, q) : -1);
                     if (un.cnt - 32 * rg > 16)
-                        expand_dispatch<2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs,
-                                           ring, NS);
+                        expand_dispatch<2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
                     else
-                        expand_dispatch<1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs,
-                                           ring, NS);
+                        expand_dispatch<1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
                 }
             }
-            cur = MODE == MODE_FUSED ? __shfl_sync(FULL, nxt, 0) : nxt;
+            cur = nxt;
+            nxt = nxt2;
+            rc = rn;
         }
     }
 
@@ -586,9 +648,9 @@ const void *bg_fn(int mode) {
 
 }  // namespace
 
-size_t bgmv_smem_bytes(int mode, int stages) {
+size_t bgmv_smem_bytes(int mode) {
     (void)mode;
-    return (size_t)stages * BG_WARPS * BG_STEP;
+    return (size_t)BG_WARPS * BG_RING;
 }
 
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max) {
@@ -598,9 +660,8 @@ size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max) {
 
 // Persistent launch: one block per SM (or `blocks` when positive).
 int launch_bgmv(int mode, const GbArgs &args, int blocks, cudaStream_t st) {
-    GbArgs a = args;
-    if (a.stages < 2 || a.stages > BG_MAX_STAGES) a.stages = BG_MAX_STAGES;
-    const size_t smem = bgmv_smem_bytes(mode, a.stages);
+    const GbArgs &a = args;
+    const size_t smem = bgmv_smem_bytes(mode);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -611,8 +672,8 @@ int launch_bgmv(int mode, const GbArgs &args, int blocks, cudaStream_t st) {
         std::lock_guard<std::mutex> lock(mu);
         const int d = dev & 63;
         if (!set[d][mode]) {
-            const cudaError_t e = cudaFuncSetAttribute(bg_fn(mode), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)bgmv_smem_bytes(mode, BG_MAX_STAGES));
+            const cudaError_t e =
+                cudaFuncSetAttribute(bg_fn(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return cuda_rc(e);
             set[d][mode] = true;
         }

@@ -34,7 +34,6 @@ struct GbArgs {
     int *done;         // fused mode: per unit, shrink items finished
     int bc;            // output columns of one expand item (multiple of 32)
     int blk_off[LORA_MAX_SLICES + 1];   // expand items per unit: slice s owns [blk_off[s], blk_off[s+1])
-    int stages;        // steps in flight per warp (2 .. 4)
     unsigned wait_limit;   // tries of the bounded wait (WAIT_LIMIT; shorter for the stall test hook)
     int dbg_stall;     // test hook: expand items wait for one shrink signal more than exists
 };
@@ -103,7 +102,7 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
 // bgmv.cu: bf16, r_max <= 64 and a multiple of 8, 16-byte aligned rows; units
 // of up to LORA_MAX_TILE_ROWS rows; a persistent grid of one block per SM
 // (`blocks` blocks when positive)
-size_t bgmv_smem_bytes(int mode, int stages);
+size_t bgmv_smem_bytes(int mode);
 int launch_bgmv(int mode, const GbArgs &a, int blocks, cudaStream_t st);
 // workspace of the fused mode: control words, then one int per unit, then v
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max);

@@ -368,9 +368,6 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
         g.blk_off[0] = 0;
         for (int s = 0; s < c.n_slices; ++s)
             g.blk_off[s + 1] = g.blk_off[s] + (c.slices[s].d_out + g.bc - 1) / g.bc;
-        // tuning override: LORA_BG_STAGES = 2 .. 4 steps in flight per warp
-        g.stages = env_int("LORA_BG_STAGES", 4);
-        if (g.stages < 2 || g.stages > 4) g.stages = 4;
         g.wait_limit = WAIT_LIMIT;
         if (env_int("LORA_DEBUG_STALL", 0) == 1) {
             // test hook for the bounded wait: expand items wait for a shrink signal
