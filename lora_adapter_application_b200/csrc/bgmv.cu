@@ -93,6 +93,17 @@ __device__ __forceinline__ void cp8(uint32_t dst, const void *src, int bytes) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
                  : "memory");
 }
+// The same for B rows: their ranks past r8 are padding, so L2 fetches 64 bytes for
+// them instead of its default line (a rank-8..32 adapter in a 64-rank slot then moves
+// 64 bytes per output column through HBM, not 128)
+__device__ __forceinline__ void cp16_64(uint32_t dst, const void *src, int bytes) {
+    asm volatile("cp.async.cg.shared.global.L2::64B [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp8_64(uint32_t dst, const void *src, int bytes) {
+    asm volatile("cp.async.ca.shared.global.L2::64B [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 // wait until at most N of this thread's copy groups are still in flight
 template <int N>
@@ -249,34 +260,59 @@ __device__ __forceinline__ void shrink_dispatch(int ntr, const char *A_rows, int
 }
 
 // ------------------------------------------------------------------ expand
+// L2 policy for the y rows: read once and written once, they go first, so the
+// repeats of A, B and x stay longer.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void cp16_hint(uint32_t dst, const void *src, int bytes, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src),
+                 "r"(bytes), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void stg128_hint(void *p, uint4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;\n" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w), "l"(pol)
+                 : "memory");
+}
+
 // One warp's expand pass over output columns [c_lo, c_hi) of one slice for up
 // to 32 rows of a unit (row_l: this lane's row, -1 past the unit; rows 16*mi+g
-// and 16*mi+g+8 of the pass are m16 tile mi).  RK: ranks loaded per row,
-// 16 (8-byte loads of ranks 4t..4t+3), 32 or 64 (16-byte loads of ranks
-// 32c+8t..32c+8t+7); bytes past rank r_n are zero-filled, not read.  m = rows,
-// n = output columns: n-tile j's column for n-index q is
+// and 16*mi+g+8 of the pass are m16 tile mi; H = 1 when the pass has at most 8
+// rows, so the g+8 halves hold none and are neither read nor written).  RK:
+// ranks loaded per row, 16 (8-byte loads of ranks 4t..4t+3), 32 or 64 (16-byte
+// loads of ranks 32c+8t..32c+8t+7); bytes past rank r_n are zero-filled, not
+// read.  m = rows, n = output columns: n-tile j's column for n-index q is
 // c0 + 8*(q>>1) + 2*j + (q&1), so lane t ends with columns c0+8t .. c0+8t+7.
 // The accumulators start from the y values, so y + scale * v . B^T is rounded
-// to bf16 once.
-template <int MR, int RK>
+// to bf16 once.  Single-tile passes take two steps per iteration (independent
+// accumulators for the scheduler to interleave).
+template <int MR, int RK, int H>
 __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max, int r_n,
                                             float scale, int c_lo, int c_hi,
                                             __nv_bfloat16 *ys, int64_t ld_y, const float *vs,
                                             uint32_t ring) {
     constexpr int CH = RK == 64 ? 2 : 1;            // rank chunks per step
     constexpr int NB = 4 * CH;                      // B loads per step
-    constexpr int NLD = NB + 2 * MR;
+    constexpr int NLD = NB + MR * H;
     constexpr int NSL = ring_depth(NLD);
     constexpr int KB = RK == 16 ? 1 : 2;            // k16 products per chunk
     constexpr int LB = RK == 16 ? 8 : 16;           // bytes of one B load
+    constexpr int U = MR == 1 && NSL >= 4 ? 2 : 1;  // steps per iteration
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int r8 = (r_n + 7) & ~7;
+    const uint64_t pol = policy_evict_first();
     // rows of this lane's y pieces and v fragments
     int yrow[MR][2];
 #pragma unroll
     for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) yrow[mi][h] = __shfl_sync(FULL, row_l, 16 * mi + 8 * h + g);
+        for (int h = 0; h < 2; ++h) {
+            const int r = __shfl_sync(FULL, row_l, 16 * mi + 8 * h + g);
+            yrow[mi][h] = h < H ? r : -1;
+        }
     const int rk0 = RK == 16 ? 4 * t : 8 * t;
     int szb[CH];   // bytes of chunk c below rank r_n
 #pragma unroll
@@ -293,16 +329,16 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
         bs[c] = any ? 64 * r_max : 0;
         bj[c] = any ? 4 * r_max : 0;
     }
-    // y piece of row (mi, h) at step ks: columns c_lo + 8t + 32ks .. +7
-    const char *py[MR][2];
-    int sy[MR][2];
+    // y piece of row (mi, h) at step ks: columns c_lo + 32ks + 8t .. +7 (the row's
+    // first column of the item stands in for a piece that is not read)
+    const char *py[MR][H];
+    int sy[MR][H];
 #pragma unroll
     for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < H; ++h) {
             const bool ok = yrow[mi][h] >= 0;
-            py[mi][h] = reinterpret_cast<const char *>(ys + (int64_t)(ok ? yrow[mi][h] : 0) * ld_y) +
-                        (ok ? 2 * (c_lo + 8 * t) : 0);
+            py[mi][h] = reinterpret_cast<const char *>(ys + (int64_t)(ok ? yrow[mi][h] : 0) * ld_y + c_lo);
             sy[mi][h] = ok ? 16 : 0;
         }
     const int nst = (c_hi - c_lo + 31) >> 5;
@@ -317,15 +353,16 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
                 for (int j = 0; j < 4; ++j) {
                     const char *src = pbc[c] + (ks * bs[c] + j * bj[c]);
                     if (RK == 16)
-                        cp8(b + (4 * c + j) * 512, src, szb[c]);
+                        cp8_64(b + (4 * c + j) * 512, src, szb[c]);
                     else
-                        cp16(b + (4 * c + j) * 512, src, szb[c]);
+                        cp16_64(b + (4 * c + j) * 512, src, szb[c]);
                 }
 #pragma unroll
             for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    cp16(b + (NB + 2 * mi + h) * 512, py[mi][h] + (sy[mi][h] ? 64 * ks : 0), sy[mi][h]);
+                for (int h = 0; h < H; ++h)
+                    cp16_hint(b + (NB + H * mi + h) * 512, py[mi][h] + (sy[mi][h] ? 64 * ks + 16 * t : 0),
+                              sy[mi][h], pol);
         } else {
 #pragma unroll
             for (int c = 0; c < CH; ++c)
@@ -334,22 +371,26 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
                     const bool ok = cb + 2 * j + 32 * ks < c_hi;
                     const char *src = ok ? pbc[c] + (ks * bs[c] + j * bj[c]) : Bn;
                     if (RK == 16)
-                        cp8(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
+                        cp8_64(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
                     else
-                        cp16(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
+                        cp16_64(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
                 }
             const bool cv = c_lo + 8 * t + 32 * ks < c_hi;
 #pragma unroll
             for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < H; ++h) {
                     const bool ok = cv && sy[mi][h];
-                    cp16(b + (NB + 2 * mi + h) * 512, py[mi][h] + (ok ? 64 * ks : 0), ok ? 16 : 0);
+                    cp16_hint(b + (NB + H * mi + h) * 512, py[mi][h] + (ok ? 64 * ks + 16 * t : 0), ok ? 16 : 0,
+                              pol);
                 }
         }
     };
+    // the first steps fly while v is read: NSL-1 of them (NSL-2 when two steps are
+    // taken per iteration, each iteration refilling the two slots it freed before)
+    constexpr int PRO = U == 2 ? NSL - 2 : NSL - 1;
 #pragma unroll
-    for (int j = 0; j < NSL - 1; ++j) {   // the first steps fly while v is read
+    for (int j = 0; j < PRO; ++j) {
         if (j < nst) issue(j, j);
         cp_commit();
     }
@@ -384,26 +425,24 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
                 for (int p = 0; p < 4; ++p) split2(f[2 * p], f[2 * p + 1], vh[mi][c][h][p], vl[mi][c][h][p]);
             }
 
-    int si = NSL - 1, sc = 0;
-    for (int ks = 0; ks < nst; ++ks) {
-        if (ks + NSL - 1 < nst) issue(ks + NSL - 1, si);
-        si = si + 1 == NSL ? 0 : si + 1;
-        cp_commit();
-        cp_wait<NSL - 1>();
-        const uint32_t b = lbase + (uint32_t)(sc * NLD * 512);
-        sc = sc + 1 == NSL ? 0 : sc + 1;
-        // accumulators from the y values: word j of row (mi, h) = columns 8t+2j, 8t+2j+1
+    // one step from ring slot b: accumulators from the y pieces, products, y rounded and stored
+    auto step = [&](uint32_t b, int ks) {
         float acc[MR][4][4];
 #pragma unroll
         for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint4 w = lds128(b + (NB + 2 * mi + h) * 512);
-                const uint32_t win[4] = {w.x, w.y, w.z, w.w};
+                if (h < H) {
+                    const uint4 w = lds128(b + (NB + H * mi + h) * 512);
+                    const uint32_t win[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc[mi][j][2 * h] = bf_lo(win[j]);
-                    acc[mi][j][2 * h + 1] = bf_hi(win[j]);
+                    for (int j = 0; j < 4; ++j) {
+                        acc[mi][j][2 * h] = bf_lo(win[j]);
+                        acc[mi][j][2 * h + 1] = bf_hi(win[j]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[mi][j][2 * h] = acc[mi][j][2 * h + 1] = 0.f;
                 }
             }
 #pragma unroll
@@ -440,27 +479,64 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
 #pragma unroll
         for (int mi = 0; mi < MR; ++mi)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < H; ++h)
                 if (cv && yrow[mi][h] >= 0)
-                    stg128(ys + (int64_t)yrow[mi][h] * ld_y + c0 + 8 * t,
-                           make_uint4(pack_bf16x2(acc[mi][0][2 * h], acc[mi][0][2 * h + 1]),
-                                      pack_bf16x2(acc[mi][1][2 * h], acc[mi][1][2 * h + 1]),
-                                      pack_bf16x2(acc[mi][2][2 * h], acc[mi][2][2 * h + 1]),
-                                      pack_bf16x2(acc[mi][3][2 * h], acc[mi][3][2 * h + 1])));
+                    stg128_hint(ys + (int64_t)yrow[mi][h] * ld_y + c0 + 8 * t,
+                                make_uint4(pack_bf16x2(acc[mi][0][2 * h], acc[mi][0][2 * h + 1]),
+                                           pack_bf16x2(acc[mi][1][2 * h], acc[mi][1][2 * h + 1]),
+                                           pack_bf16x2(acc[mi][2][2 * h], acc[mi][2][2 * h + 1]),
+                                           pack_bf16x2(acc[mi][3][2 * h], acc[mi][3][2 * h + 1])),
+                                pol);
+    };
+
+    int si = PRO, sc = 0;
+    int ks = 0;
+    if (U == 2) {
+        // iteration at ks: steps up to ks+NSL-3 are in flight; steps ks+NSL-2 and ks+NSL-1
+        // take the slots of ks-2 and ks-1, then ks and ks+1 are waited for
+        for (; ks + 1 < nst; ks += 2) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                if (ks + e + NSL - 2 < nst) issue(ks + e + NSL - 2, si);
+                si = si + 1 == NSL ? 0 : si + 1;
+                cp_commit();
+            }
+            cp_wait<(U == 2 ? NSL - 2 : 0)>();
+            const uint32_t b0 = lbase + (uint32_t)(sc * NLD * 512);
+            sc = sc + 1 == NSL ? 0 : sc + 1;
+            const uint32_t b1 = lbase + (uint32_t)(sc * NLD * 512);
+            sc = sc + 1 == NSL ? 0 : sc + 1;
+            step(b0, ks);
+            step(b1, ks + 1);
+        }
+        if (ks < nst) {   // an odd last step: already issued
+            cp_wait<0>();
+            step(lbase + (uint32_t)(sc * NLD * 512), ks);
+        }
+    } else {
+        for (; ks < nst; ++ks) {
+            if (ks + NSL - 1 < nst) issue(ks + NSL - 1, si);
+            si = si + 1 == NSL ? 0 : si + 1;
+            cp_commit();
+            cp_wait<NSL - 1>();
+            const uint32_t b = lbase + (uint32_t)(sc * NLD * 512);
+            sc = sc + 1 == NSL ? 0 : sc + 1;
+            step(b, ks);
+        }
     }
     cp_wait<0>();
 }
 
-template <int MR>
+template <int MR, int H>
 __device__ __forceinline__ void expand_dispatch(int r8, int row_l, const char *Bn, int r_max, int r_n,
                                                 float scale, int c_lo, int c_hi, __nv_bfloat16 *ys,
                                                 int64_t ld_y, const float *vs, uint32_t ring) {
     if (r8 <= 16)
-        expand_warp<MR, 16>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
+        expand_warp<MR, 16, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
     else if (r8 <= 32)
-        expand_warp<MR, 32>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
+        expand_warp<MR, 32, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
     else
-        expand_warp<MR, 64>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
+        expand_warp<MR, 64, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
 }
 
 // What an expand warp needs of one item before it starts: unit, rank, this
@@ -608,10 +684,13 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                 for (int rg = 0; rg * 32 < un.cnt; ++rg) {
                     const int q = 32 * rg + lane;
                     const int row_l = rg == 0 ? rc.row_l : (q < un.cnt ? un.row(a.tiles, q) : -1);
-                    if (un.cnt - 32 * rg > 16)
-                        expand_dispatch<2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
+                    const int rows = un.cnt - 32 * rg;
+                    if (rows > 16)
+                        expand_dispatch<2, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
+                    else if (rows > 8)
+                        expand_dispatch<1, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
                     else
-                        expand_dispatch<1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
+                        expand_dispatch<1, 1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
                 }
             }
             cur = nxt;
