@@ -278,6 +278,34 @@ __device__ __forceinline__ void stg128_hint(void *p, uint4 v, uint64_t pol) {
                  : "memory");
 }
 
+// The fused mode's wait of an expand item for its unit's v: until *done reaches
+// need (bounded; nullptr = nothing to wait for).  Every lane then acquires the
+// count itself, ordering its v reads after the shrink's writes.
+struct EWait {
+    const int *done;
+    int need;
+    unsigned limit;
+    int32_t *status;
+};
+__device__ __forceinline__ bool e_wait(const EWait &w) {
+    if (!w.done) return true;
+    bool ready = true;
+    if ((threadIdx.x & 31) == 0) {
+        unsigned it = 0;
+        while (ld_acquire_gpu(w.done) < w.need) {
+            if (++it >= w.limit * 64u) {
+                atomicOr(w.status, LORA_DEV_TIMEOUT);
+                ready = false;
+                break;
+            }
+            __nanosleep(128);
+        }
+    }
+    if (__shfl_sync(FULL, ready ? 1 : 0, 0) == 0) return false;
+    (void)ld_acquire_gpu(w.done);
+    return true;
+}
+
 // One warp's expand pass over output columns [c_lo, c_hi) of one slice for up
 // to 32 rows of a unit (row_l: this lane's row, -1 past the unit; rows 16*mi+g
 // and 16*mi+g+8 of the pass are m16 tile mi; H = 1 when the pass has at most 8
@@ -290,10 +318,10 @@ __device__ __forceinline__ void stg128_hint(void *p, uint4 v, uint64_t pol) {
 // to bf16 once.  Single-tile passes take two steps per iteration (independent
 // accumulators for the scheduler to interleave).
 template <int MR, int RK, int H>
-__device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max, int r_n,
+__device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max, int r_n,
                                             float scale, int c_lo, int c_hi,
                                             __nv_bfloat16 *ys, int64_t ld_y, const float *vs,
-                                            uint32_t ring) {
+                                            uint32_t ring, const EWait &wt) {
     constexpr int CH = RK == 64 ? 2 : 1;            // rank chunks per step
     constexpr int NB = 4 * CH;                      // B loads per step
     constexpr int NLD = NB + MR * H;
@@ -393,6 +421,11 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
     for (int j = 0; j < PRO; ++j) {
         if (j < nst) issue(j, j);
         cp_commit();
+    }
+    // B and y do not depend on v: the first steps fly while the unit's shrink finishes
+    if (!e_wait(wt)) {
+        cp_wait<0>();
+        return false;
     }
     // scale * v as bf16 hi / lo pairs: vh[mi][c][h][p] = ranks 32c + rk0 + 2p, +1 of row (mi, h)
     uint32_t vh[MR][CH][2][4], vl[MR][CH][2][4];
@@ -525,18 +558,18 @@ __device__ __forceinline__ void expand_warp(int row_l, const char *Bn, int r_max
         }
     }
     cp_wait<0>();
+    return true;
 }
 
 template <int MR, int H>
-__device__ __forceinline__ void expand_dispatch(int r8, int row_l, const char *Bn, int r_max, int r_n,
+__device__ __forceinline__ bool expand_dispatch(int r8, int row_l, const char *Bn, int r_max, int r_n,
                                                 float scale, int c_lo, int c_hi, __nv_bfloat16 *ys,
-                                                int64_t ld_y, const float *vs, uint32_t ring) {
+                                                int64_t ld_y, const float *vs, uint32_t ring, const EWait &wt) {
     if (r8 <= 16)
-        expand_warp<MR, 16, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
-    else if (r8 <= 32)
-        expand_warp<MR, 32, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
-    else
-        expand_warp<MR, 64, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring);
+        return expand_warp<MR, 16, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
+    if (r8 <= 32)
+        return expand_warp<MR, 32, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
+    return expand_warp<MR, 64, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
 }
 
 // What an expand warp needs of one item before it starts: unit, rank, this
@@ -659,39 +692,32 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
             if (!ok && un.cnt > 0 && b == 0 && lane == 0 && MODE == MODE_EXPAND)
                 atomicOr(a.status, LORA_DEV_BAD_RANK);
             if (ok) {
-                if (MODE == MODE_FUSED) {   // v of unit u: all its shrink items have signalled
-                    bool ready = true;
-                    if (lane == 0) {
-                        unsigned it = 0;
-                        while (ld_acquire_gpu(a.done + u) < need) {
-                            if (++it >= a.wait_limit * 64u) {
-                                atomicOr(a.status, LORA_DEV_TIMEOUT);
-                                ready = false;
-                                break;
-                            }
-                            __nanosleep(128);
-                        }
-                    }
-                    if (__shfl_sync(FULL, ready ? 1 : 0, 0) == 0) break;   // the warp takes no more work
-                    (void)ld_acquire_gpu(a.done + u);   // every lane orders its v reads after the count
-                }
                 const float scale = a.alphas[un.id] / (float)r_n;
                 const int r8 = (r_n + 7) & ~7;
                 const char *Bn = static_cast<const char *>(a.sl.B[s]) +
                                  (int64_t)un.id * a.sl.d_out[s] * a.r_max * 2;
                 __nv_bfloat16 *ys = a.y + a.sl.col_off[s];
                 const float *vs = a.v + (int64_t)s * a.T * a.r_max;
-                for (int rg = 0; rg * 32 < un.cnt; ++rg) {
+                // the first pass waits (fused mode) for unit u's shrink items, after issuing
+                // its first steps
+                EWait wt{MODE == MODE_FUSED ? a.done + u : nullptr, need, a.wait_limit, a.status};
+                bool ok_pass = true;
+                for (int rg = 0; rg * 32 < un.cnt && ok_pass; ++rg) {
                     const int q = 32 * rg + lane;
                     const int row_l = rg == 0 ? rc.row_l : (q < un.cnt ? un.row(a.tiles, q) : -1);
                     const int rows = un.cnt - 32 * rg;
                     if (rows > 16)
-                        expand_dispatch<2, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
+                        ok_pass = expand_dispatch<2, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
+                                                        vs, ring, wt);
                     else if (rows > 8)
-                        expand_dispatch<1, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
+                        ok_pass = expand_dispatch<1, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
+                                                        vs, ring, wt);
                     else
-                        expand_dispatch<1, 1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y, vs, ring);
+                        ok_pass = expand_dispatch<1, 1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
+                                                        vs, ring, wt);
+                    wt.done = nullptr;
                 }
+                if (!ok_pass) break;   // the wait ran out: the warp takes no more work
             }
             cur = nxt;
             nxt = nxt2;
