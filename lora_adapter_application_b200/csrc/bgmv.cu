@@ -57,9 +57,15 @@ constexpr int BG_WARPS = 8;
 constexpr int BG_THREADS = BG_WARPS * 32;
 constexpr int BG_ROWS = LORA_MAX_TILE_ROWS;      // rows of one unit
 constexpr int BG_RING = 24576;                   // bytes of one warp's ring of steps
-constexpr int BG_RG = 32;                        // ranks of one shrink item
-constexpr int BG_RED_LD = BG_RG + 4;             // floats per row of the shrink reduction
-constexpr int BG_RED_BYTES = BG_WARPS * BG_ROWS * BG_RED_LD * 4;
+// Ranks of one shrink item: 32 (units of up to 64 rows), or all of the slot's 64 when
+// units have at most 16 rows (the accumulators of 4 x 2 tiles fit a warp)
+constexpr int BG_RG = 32;
+constexpr int BG_RG_SMALL = 64;
+constexpr int BG_SMALL_ROWS = 16;
+// floats per row of the shrink reduction: the item's ranks + 4 (bank spread)
+__host__ __device__ constexpr int red_ld(int rg) { return rg + 4; }
+constexpr int BG_RED_BYTES = BG_WARPS * BG_ROWS * (BG_RG + 4) * 4;
+static_assert(BG_WARPS * BG_SMALL_ROWS * (BG_RG_SMALL + 4) * 4 <= BG_RED_BYTES, "small-unit reduction");
 static_assert(BG_RED_BYTES <= BG_WARPS * BG_RING, "the reduction overlays the rings");
 
 // Steps of nld 16-byte loads per lane (nld * 512 bytes per warp) that a ring holds.
@@ -149,11 +155,11 @@ __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? l
 // lda bytes apart), the unit's rows (rows_s, -1 past the unit), k-steps
 // [k_lo, k_hi) of 32 columns.  m = ranks (MG m16 tiles), n = rows (NTR n8
 // tiles).  Ends with a block barrier and the warp's partial in red
-// [warp][row][rank].
+// [warp][row][rank] (8*NTR rows of ld floats per warp).
 template <int MG, int NTR>
 __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int rv, const char *x,
                                             int64_t ldx, const int *rows_s, int d_in, int k_lo,
-                                            int k_hi, uint32_t ring, float *red) {
+                                            int k_hi, uint32_t ring, float *red, int ld) {
     constexpr int NLD = 2 * MG + NTR;
     constexpr int NSL = ring_depth(NLD);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -232,31 +238,39 @@ __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int
     }
     cp_wait<0>();
     __syncthreads();   // every warp is done with its ring: the reduction buffer overlays them
-    float *rw = red + warp * BG_ROWS * BG_RED_LD;
+    float *rw = red + warp * 8 * NTR * ld;
 #pragma unroll
     for (int mi = 0; mi < MG; ++mi)
 #pragma unroll
         for (int i = 0; i < NTR; ++i) {
             const int r0 = 8 * i + 2 * t, k0 = 16 * mi + g;
-            rw[r0 * BG_RED_LD + k0] = acc[mi][i][0];
-            rw[(r0 + 1) * BG_RED_LD + k0] = acc[mi][i][1];
-            rw[r0 * BG_RED_LD + k0 + 8] = acc[mi][i][2];
-            rw[(r0 + 1) * BG_RED_LD + k0 + 8] = acc[mi][i][3];
+            rw[r0 * ld + k0] = acc[mi][i][0];
+            rw[(r0 + 1) * ld + k0] = acc[mi][i][1];
+            rw[r0 * ld + k0 + 8] = acc[mi][i][2];
+            rw[(r0 + 1) * ld + k0 + 8] = acc[mi][i][3];
         }
 }
 
+// n8 row tiles of the item: 1, 2, 4 or 8 (the loaded rows past the unit are zero-filled);
+// returns the tile count used (the reduction buffer's rows per warp / 8)
 template <int MG>
-__device__ __forceinline__ void shrink_dispatch(int ntr, const char *A_rows, int64_t lda, int rv,
-                                                const char *x, int64_t ldx, const int *rows_s, int d_in,
-                                                int k_lo, int k_hi, uint32_t ring, float *red) {
-    if (ntr <= 1)
-        shrink_warp<MG, 1>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
-    else if (ntr <= 2)
-        shrink_warp<MG, 2>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
-    else if (ntr <= 4)
-        shrink_warp<MG, 4>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
-    else
-        shrink_warp<MG, 8>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red);
+__device__ __forceinline__ int shrink_dispatch(int ntr, const char *A_rows, int64_t lda, int rv,
+                                               const char *x, int64_t ldx, const int *rows_s, int d_in,
+                                               int k_lo, int k_hi, uint32_t ring, float *red, int ld) {
+    if (ntr <= 1) {
+        shrink_warp<MG, 1>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red, ld);
+        return 1;
+    }
+    if (ntr <= 2) {
+        shrink_warp<MG, 2>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red, ld);
+        return 2;
+    }
+    if (MG <= 2 && ntr <= 4) {
+        shrink_warp<MG, 4>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red, ld);
+        return 4;
+    }
+    shrink_warp<(MG <= 2 ? MG : 2), 8>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red, ld);
+    return 8;
 }
 
 // ------------------------------------------------------------------ expand
@@ -604,7 +618,11 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
     float *red = reinterpret_cast<float *>(smem);
     const int S = a.sl.n;
     const int live = n_live_units(a.tiles);
-    const int GM = (a.r_max + BG_RG - 1) / BG_RG;   // shrink items per unit and slice
+    // shrink items per unit and slice: one for units of up to 16 rows, else one per 32 ranks
+    const bool small = a.tiles.rows_per_unit <= BG_SMALL_ROWS;
+    const int RGW = small ? BG_RG_SMALL : BG_RG;
+    const int GM = (a.r_max + RGW - 1) / RGW;
+    const int rld = red_ld(RGW);
 
     // ------------------------------------------------------------ phase 1: shrink
     if (MODE != MODE_EXPAND) {
@@ -625,27 +643,37 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
             const int r_n = un.cnt > 0 ? a.ranks[un.id] : 0;
             const bool ok = un.cnt > 0 && r_n >= 1 && r_n <= a.r_max;
             if (!ok && un.cnt > 0 && s == 0 && grp == 0 && tid == 0) atomicOr(a.status, LORA_DEV_BAD_RANK);
-            const int rv = ok ? min(BG_RG, ((r_n + 7) & ~7) - BG_RG * grp) : 0;
+            const int rv = ok ? min(RGW, ((r_n + 7) & ~7) - RGW * grp) : 0;
             __syncthreads();
             if (rv > 0) {
                 const char *A_rows = static_cast<const char *>(a.sl.A[s]) +
-                                     ((int64_t)un.id * a.r_max + BG_RG * grp) * a.d_in * 2;
+                                     ((int64_t)un.id * a.r_max + RGW * grp) * a.d_in * 2;
                 const char *x = reinterpret_cast<const char *>(a.x);
                 const int64_t lda = (int64_t)a.d_in * 2;
                 float *vb = a.v + (int64_t)s * a.T * a.r_max;
                 const int ntr = (un.cnt + 7) >> 3;
-                if (rv > 16)
-                    shrink_dispatch<2>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring, red);
+                int nt;
+                if (rv > 48)
+                    nt = shrink_dispatch<4>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
+                                            red, rld);
+                else if (rv > 32)
+                    nt = shrink_dispatch<3>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
+                                            red, rld);
+                else if (rv > 16)
+                    nt = shrink_dispatch<2>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
+                                            red, rld);
                 else
-                    shrink_dispatch<1>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring, red);
+                    nt = shrink_dispatch<1>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
+                                            red, rld);
                 __syncthreads();
                 // the 8 partials in warp order; v rows of the unit, ranks of the group below r_n
-                for (int p = tid; p < un.cnt * BG_RG; p += BG_THREADS) {
-                    const int row = p / BG_RG, rl = p - row * BG_RG, k = BG_RG * grp + rl;
+                const int wst = 8 * nt * rld;   // floats of one warp's partial
+                for (int p = tid; p < un.cnt * RGW; p += BG_THREADS) {
+                    const int row = p / RGW, rl = p - row * RGW, k = RGW * grp + rl;
                     if (rl < rv && k < r_n) {
                         float sum = 0.f;
 #pragma unroll
-                        for (int w = 0; w < BG_WARPS; ++w) sum += red[(w * BG_ROWS + row) * BG_RED_LD + rl];
+                        for (int w = 0; w < BG_WARPS; ++w) sum += red[w * wst + row * rld + rl];
                         vb[(int64_t)rows_s[row] * a.r_max + k] = sum;
                     }
                 }
