@@ -316,20 +316,26 @@ int bgmv_blocks() {
     return e >= 1 && e <= 4096 ? e : 0;
 }
 
-// Output columns of one expand item (one warp's): the widest of 1024 .. 128
-// that still gives about six items per warp for the batch's expected units
-// (the expand phase is balanced by handing out many items of similar size).
-// Tuning override: LORA_BG_ITEM_COLS, a multiple of 32 from 32 to 8192.
+// Output columns of one expand item (one warp's): the narrowest of 128 .. 2048
+// that keeps the batch's expected items at most five per warp of the grid (more
+// items balance better, each item pays one pipeline fill), and at least 256 when
+// the batch has fewer than 64 units (a small batch is bound by one item's
+// latency).  Measured on the Llama-3-8B decode layer set (16-row tiles: best
+// 256 / 128 / 768-1024 / 128 for qkv / o / gate-up / down) and decode q_proj
+// (256).  Tuning override: LORA_BG_ITEM_COLS, a multiple of 32 from 32 to 8192.
 int bgmv_item_cols(const Call &c, int est_units) {
     const int e = env_int("LORA_BG_ITEM_COLS", 0);
     if (e >= 32 && e <= 8192 && (e & 31) == 0) return e;
-    const int target = 6 * 8 * device_sms();
-    for (int bc = 1024; bc > 128; bc >>= 1) {
+    const int64_t cap = 5LL * 8 * device_sms();
+    const int lo = est_units < 64 ? 256 : 128;
+    static const int cand[] = {128, 256, 384, 512, 768, 1024, 1536, 2048};
+    for (int bc : cand) {
+        if (bc < lo) continue;
         int64_t items = 0;
         for (int s = 0; s < c.n_slices; ++s) items += (c.slices[s].d_out + bc - 1) / bc;
-        if (items * est_units >= target) return bc;
+        if (items * est_units <= cap) return bc;
     }
-    return 128;
+    return 2048;
 }
 
 // The gathered tiles (and the contiguous ones unless tc_took) on the fused
