@@ -89,14 +89,10 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// 16 (8) bytes global -> shared through L2, of which the first `bytes` are read and
-// the rest zero-filled (0: nothing read)
+// 16 bytes global -> shared through L2, of which the first `bytes` are read and the
+// rest zero-filled (0: nothing read)
 __device__ __forceinline__ void cp16(uint32_t dst, const void *src, int bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp8(uint32_t dst, const void *src, int bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
                  : "memory");
 }
 // The same for B rows: their ranks past r8 are padding, so L2 fetches 64 bytes for
@@ -104,10 +100,6 @@ __device__ __forceinline__ void cp8(uint32_t dst, const void *src, int bytes) {
 // 64 bytes per output column through HBM, not 128)
 __device__ __forceinline__ void cp16_64(uint32_t dst, const void *src, int bytes) {
     asm volatile("cp.async.cg.shared.global.L2::64B [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp8_64(uint32_t dst, const void *src, int bytes) {
-    asm volatile("cp.async.ca.shared.global.L2::64B [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
                  : "memory");
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
@@ -122,16 +114,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                  : "r"(a));
     return r;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 r;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(r.x), "=r"(r.y) : "r"(a));
-    return r;
-}
-__device__ __forceinline__ void stg128(void *p, uint4 v) {
-    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
 }
 __device__ __forceinline__ void red_release_gpu(int *p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
@@ -251,16 +233,13 @@ __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int
         }
 }
 
-// n8 row tiles of the item: 1, 2, 4 or 8 (the loaded rows past the unit are zero-filled);
+// n8 row tiles of the item: 2, 4 or 8 (the loaded rows past the unit are zero-filled; a
+// unit of up to 8 rows takes the 2-tile form, one variant fewer in the instruction cache);
 // returns the tile count used (the reduction buffer's rows per warp / 8)
 template <int MG>
 __device__ __forceinline__ int shrink_dispatch(int ntr, const char *A_rows, int64_t lda, int rv,
                                                const char *x, int64_t ldx, const int *rows_s, int d_in,
                                                int k_lo, int k_hi, uint32_t ring, float *red, int ld) {
-    if (ntr <= 1) {
-        shrink_warp<MG, 1>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red, ld);
-        return 1;
-    }
     if (ntr <= 2) {
         shrink_warp<MG, 2>(A_rows, lda, rv, x, ldx, rows_s, d_in, k_lo, k_hi, ring, red, ld);
         return 2;
@@ -322,27 +301,26 @@ __device__ __forceinline__ bool e_wait(const EWait &w) {
 
 // One warp's expand pass over output columns [c_lo, c_hi) of one slice for up
 // to 32 rows of a unit (row_l: this lane's row, -1 past the unit; rows 16*mi+g
-// and 16*mi+g+8 of the pass are m16 tile mi; H = 1 when the pass has at most 8
-// rows, so the g+8 halves hold none and are neither read nor written).  RK:
-// ranks loaded per row, 16 (8-byte loads of ranks 4t..4t+3), 32 or 64 (16-byte
-// loads of ranks 32c+8t..32c+8t+7); bytes past rank r_n are zero-filled, not
-// read.  m = rows, n = output columns: n-tile j's column for n-index q is
+// and 16*mi+g+8 of the pass are m16 tile mi).  RK: ranks loaded per row, 32 or
+// 64 (16-byte loads of ranks 32c+8t..32c+8t+7; a rank-8 or rank-16 adapter takes
+// the 32-rank form with its upper lanes reading nothing: one variant fewer keeps
+// the hot code inside the instruction cache, which measured faster); bytes past
+// rank r_n are zero-filled, not read.  m = rows, n = output columns: n-tile j's column for n-index q is
 // c0 + 8*(q>>1) + 2*j + (q&1), so lane t ends with columns c0+8t .. c0+8t+7.
 // The accumulators start from the y values, so y + scale * v . B^T is rounded
-// to bf16 once.  Single-tile passes take two steps per iteration (independent
-// accumulators for the scheduler to interleave).
-template <int MR, int RK, int H>
+// to bf16 once.
+template <int MR, int RK>
 __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max, int r_n,
                                             float scale, int c_lo, int c_hi,
                                             __nv_bfloat16 *ys, int64_t ld_y, const float *vs,
                                             uint32_t ring, const EWait &wt) {
+    constexpr int H = 2;                            // row halves (g, g+8) of an m16 tile
     constexpr int CH = RK == 64 ? 2 : 1;            // rank chunks per step
     constexpr int NB = 4 * CH;                      // B loads per step
     constexpr int NLD = NB + MR * H;
     constexpr int NSL = ring_depth(NLD);
-    constexpr int KB = RK == 16 ? 1 : 2;            // k16 products per chunk
-    constexpr int LB = RK == 16 ? 8 : 16;           // bytes of one B load
-    constexpr int U = MR == 1 && NSL >= 4 ? 2 : 1;  // steps per iteration
+    constexpr int KB = 2;                           // k16 products per chunk
+    constexpr int LB = 16;                          // bytes of one B load
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int r8 = (r_n + 7) & ~7;
     const uint64_t pol = policy_evict_first();
@@ -355,7 +333,7 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
             const int r = __shfl_sync(FULL, row_l, 16 * mi + 8 * h + g);
             yrow[mi][h] = h < H ? r : -1;
         }
-    const int rk0 = RK == 16 ? 4 * t : 8 * t;
+    const int rk0 = 8 * t;
     int szb[CH];   // bytes of chunk c below rank r_n
 #pragma unroll
     for (int c = 0; c < CH; ++c) szb[c] = clampi(2 * (r_n - 32 * c - rk0), 0, LB);
@@ -394,10 +372,7 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const char *src = pbc[c] + (ks * bs[c] + j * bj[c]);
-                    if (RK == 16)
-                        cp8_64(b + (4 * c + j) * 512, src, szb[c]);
-                    else
-                        cp16_64(b + (4 * c + j) * 512, src, szb[c]);
+                    cp16_64(b + (4 * c + j) * 512, src, szb[c]);
                 }
 #pragma unroll
             for (int mi = 0; mi < MR; ++mi)
@@ -412,10 +387,7 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
                 for (int j = 0; j < 4; ++j) {
                     const bool ok = cb + 2 * j + 32 * ks < c_hi;
                     const char *src = ok ? pbc[c] + (ks * bs[c] + j * bj[c]) : Bn;
-                    if (RK == 16)
-                        cp8_64(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
-                    else
-                        cp16_64(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
+                    cp16_64(b + (4 * c + j) * 512, src, ok ? szb[c] : 0);
                 }
             const bool cv = c_lo + 8 * t + 32 * ks < c_hi;
 #pragma unroll
@@ -428,9 +400,8 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
                 }
         }
     };
-    // the first steps fly while v is read: NSL-1 of them (NSL-2 when two steps are
-    // taken per iteration, each iteration refilling the two slots it freed before)
-    constexpr int PRO = U == 2 ? NSL - 2 : NSL - 1;
+    // the first steps fly while the unit's shrink finishes and v is read
+    constexpr int PRO = NSL - 1;
 #pragma unroll
     for (int j = 0; j < PRO; ++j) {
         if (j < nst) issue(j, j);
@@ -456,12 +427,8 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
                     const float4 *pv = reinterpret_cast<const float4 *>(vs + (int64_t)row * r_max + k);
                     const float4 lo4 = pv[0];
                     f[0] = lo4.x; f[1] = lo4.y; f[2] = lo4.z; f[3] = lo4.w;
-                    if (RK != 16) {
-                        const float4 hi4 = pv[1];
-                        f[4] = hi4.x; f[5] = hi4.y; f[6] = hi4.z; f[7] = hi4.w;
-                    } else {
-                        f[4] = f[5] = f[6] = f[7] = 0.f;
-                    }
+                    const float4 hi4 = pv[1];
+                    f[4] = hi4.x; f[5] = hi4.y; f[6] = hi4.z; f[7] = hi4.w;
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = 0.f;
@@ -496,19 +463,8 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
         for (int c = 0; c < CH; ++c)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                uint32_t q[4];
-                if (RK == 16) {
-                    const uint2 w = lds64(b + (4 * c + j) * 512);
-                    q[0] = w.x;
-                    q[1] = w.y;
-                    q[2] = q[3] = 0u;
-                } else {
-                    const uint4 w = lds128(b + (4 * c + j) * 512);
-                    q[0] = w.x;
-                    q[1] = w.y;
-                    q[2] = w.z;
-                    q[3] = w.w;
-                }
+                const uint4 w = lds128(b + (4 * c + j) * 512);
+                const uint32_t q[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
@@ -537,53 +493,26 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
     };
 
     int si = PRO, sc = 0;
-    int ks = 0;
-    if (U == 2) {
-        // iteration at ks: steps up to ks+NSL-3 are in flight; steps ks+NSL-2 and ks+NSL-1
-        // take the slots of ks-2 and ks-1, then ks and ks+1 are waited for
-        for (; ks + 1 < nst; ks += 2) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                if (ks + e + NSL - 2 < nst) issue(ks + e + NSL - 2, si);
-                si = si + 1 == NSL ? 0 : si + 1;
-                cp_commit();
-            }
-            cp_wait<(U == 2 ? NSL - 2 : 0)>();
-            const uint32_t b0 = lbase + (uint32_t)(sc * NLD * 512);
-            sc = sc + 1 == NSL ? 0 : sc + 1;
-            const uint32_t b1 = lbase + (uint32_t)(sc * NLD * 512);
-            sc = sc + 1 == NSL ? 0 : sc + 1;
-            step(b0, ks);
-            step(b1, ks + 1);
-        }
-        if (ks < nst) {   // an odd last step: already issued
-            cp_wait<0>();
-            step(lbase + (uint32_t)(sc * NLD * 512), ks);
-        }
-    } else {
-        for (; ks < nst; ++ks) {
-            if (ks + NSL - 1 < nst) issue(ks + NSL - 1, si);
-            si = si + 1 == NSL ? 0 : si + 1;
-            cp_commit();
-            cp_wait<NSL - 1>();
-            const uint32_t b = lbase + (uint32_t)(sc * NLD * 512);
-            sc = sc + 1 == NSL ? 0 : sc + 1;
-            step(b, ks);
-        }
+    for (int ks = 0; ks < nst; ++ks) {
+        if (ks + NSL - 1 < nst) issue(ks + NSL - 1, si);
+        si = si + 1 == NSL ? 0 : si + 1;
+        cp_commit();
+        cp_wait<NSL - 1>();
+        const uint32_t b = lbase + (uint32_t)(sc * NLD * 512);
+        sc = sc + 1 == NSL ? 0 : sc + 1;
+        step(b, ks);
     }
     cp_wait<0>();
     return true;
 }
 
-template <int MR, int H>
+template <int MR>
 __device__ __forceinline__ bool expand_dispatch(int r8, int row_l, const char *Bn, int r_max, int r_n,
                                                 float scale, int c_lo, int c_hi, __nv_bfloat16 *ys,
                                                 int64_t ld_y, const float *vs, uint32_t ring, const EWait &wt) {
-    if (r8 <= 16)
-        return expand_warp<MR, 16, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
     if (r8 <= 32)
-        return expand_warp<MR, 32, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
-    return expand_warp<MR, 64, H>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
+        return expand_warp<MR, 32>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
+    return expand_warp<MR, 64>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
 }
 
 // What an expand warp needs of one item before it starts: unit, rank, this
@@ -653,11 +582,8 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                 float *vb = a.v + (int64_t)s * a.T * a.r_max;
                 const int ntr = (un.cnt + 7) >> 3;
                 int nt;
-                if (rv > 48)
+                if (rv > 32)
                     nt = shrink_dispatch<4>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
-                                            red, rld);
-                else if (rv > 32)
-                    nt = shrink_dispatch<3>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
                                             red, rld);
                 else if (rv > 16)
                     nt = shrink_dispatch<2>(ntr, A_rows, lda, rv, x, a.ld_x * 2, rows_s, a.d_in, k_lo, k_hi, ring,
@@ -735,13 +661,10 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                     const int row_l = rg == 0 ? rc.row_l : (q < un.cnt ? un.row(a.tiles, q) : -1);
                     const int rows = un.cnt - 32 * rg;
                     if (rows > 16)
-                        ok_pass = expand_dispatch<2, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
-                                                        vs, ring, wt);
-                    else if (rows > 8)
-                        ok_pass = expand_dispatch<1, 2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
+                        ok_pass = expand_dispatch<2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
                                                         vs, ring, wt);
                     else
-                        ok_pass = expand_dispatch<1, 1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
+                        ok_pass = expand_dispatch<1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
                                                         vs, ring, wt);
                     wt.done = nullptr;
                 }
