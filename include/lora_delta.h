@@ -52,6 +52,12 @@
  *   LORA_BG_BLOCKS      1 to 4096: blocks of the gathered-tile kernel's persistent
  *                       grid (default: one per SM)
  *   LORA_BG_ITEM_COLS   32 to 8192, a multiple of 32: output columns of one expand item
+ *   LORA_BG_TC          1: fused calls whose tiles have at most 16 rows run on the
+ *                       tensor-core gathered-tile kernel (tcgen05 MMAs, TMA copies,
+ *                       accumulators in tensor memory) instead of the mma.sync one;
+ *                       off by default (correct, slower on the decode layer set)
+ *   LORA_BT_COLS        128 to 512, a multiple of 128: output columns of one expand
+ *                       item of the tensor-core gathered-tile kernel
  *   LORA_TC_CLUSTER     1, 2, 4 or 8: blocks per cluster of the tensor-core kernel;
  *                       when the shape cannot use it, the contiguous tiles run on
  *                       the gathered-tile kernel instead
@@ -261,7 +267,10 @@ LORA_API int lora_sgmv_expand(void *y, int64_t ld_y, const float *v, const lora_
  * Bytes of the workspace lora_bgmv_fused and lora_add_linear take for a batch
  * grouped into *meta and a layer of n_slices slices with rank slots r_max: a
  * 256-byte head of control words, one int per unit of work (tile capacity of
- * the meta), then v [n_slices][T][r_max] fp32.  0 for invalid arguments.
+ * the meta, rounded up to 256 bytes), then room for v: the larger of
+ * [n_slices][T][r_max] fp32 and, per unit and slice, a bf16 hi + lo pair of 16
+ * rows by r_max rounded up to 16 ranks (the tensor-core gathered-tile kernel's
+ * form).  0 for invalid arguments.
  *
  * The workspace belongs to the caller.  Its head must hold zeros before the
  * first call that uses it (allocate it zero-filled, or cudaMemset it once);

@@ -75,8 +75,6 @@ __host__ __device__ constexpr int ring_depth(int nld) {
 
 // Workspace head of the fused mode (ints): tickets and exit counter, then one
 // counter per unit.
-constexpr int GB_CTL_INTS = 64;
-enum { GB_T_SHRINK = 0, GB_T_EXPAND = 1, GB_T_EXIT = 2 };
 
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -709,9 +707,14 @@ size_t bgmv_smem_bytes(int mode) {
     return (size_t)BG_WARPS * BG_RING;
 }
 
+size_t bgmv_workspace_head(int units) {
+    return (size_t)GB_CTL_INTS * 4 + (((size_t)units * 4 + 255) & ~(size_t)255);
+}
+
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max) {
-    const size_t head = (size_t)GB_CTL_INTS * 4 + (((size_t)units * 4 + 255) & ~(size_t)255);
-    return head + (size_t)n_slices * (size_t)T * (size_t)r_max * 4;
+    const size_t v32 = (size_t)n_slices * (size_t)T * (size_t)r_max * 4;   // this kernel's fp32 v
+    const size_t vtc = bgmv_tc_v_bytes(units, n_slices, r_max);            // the tensor-core kernel's v pairs
+    return bgmv_workspace_head(units) + (v32 > vtc ? v32 : vtc);
 }
 
 // Persistent launch: one block per SM (or `blocks` when positive).

@@ -15,6 +15,11 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
                   uint32_t box_inner, uint32_t box_outer, int swizzle,
                   uint64_t row_stride = 0);
 
+// Fused-mode workspace head shared by the gathered-tile kernels: GB_CTL_INTS
+// control words (tickets and the exit counter), then one done word per unit.
+constexpr int GB_CTL_INTS = 64;
+enum { GB_T_SHRINK = 0, GB_T_EXPAND = 1, GB_T_EXIT = 2 };
+
 // The gathered-tile kernel (bgmv.cu): plain pointers, no tensor maps.
 struct GbArgs {
     const __nv_bfloat16 *x;
@@ -36,6 +41,20 @@ struct GbArgs {
     int blk_off[LORA_MAX_SLICES + 1];   // expand items per unit: slice s owns [blk_off[s], blk_off[s+1])
     unsigned wait_limit;   // tries of the bounded wait (WAIT_LIMIT; shorter for the stall test hook)
     int dbg_stall;     // test hook: expand items wait for one shrink signal more than exists
+};
+
+// The gathered-tile kernel on the tensor cores (bgmv_tc.cu, fused mode only):
+// GbArgs (bc a multiple of 128) plus maps over
+//   A_s  [N*r_max][d_in], boxes of 64 columns x 8 ranks, 128-byte swizzle
+//   B_s  [N*d_out_s][r_max], boxes of 8 ranks x 128 columns, no swizzle
+//   y_s  y + col_off_s as [T][d_out_s] (row stride ld_y), boxes of 128 columns x 1 row
+// and the workspace's v pairs (s_n v as bf16 hi + lo per unit and slice).
+struct BtArgs {
+    CUtensorMap tmA[LORA_MAX_SLICES];
+    CUtensorMap tmB[LORA_MAX_SLICES];
+    CUtensorMap tmY[LORA_MAX_SLICES];
+    GbArgs g;
+    unsigned char *vws;
 };
 
 struct SimtArgs {
@@ -104,8 +123,20 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
 // (`blocks` blocks when positive)
 size_t bgmv_smem_bytes(int mode);
 int launch_bgmv(int mode, const GbArgs &a, int blocks, cudaStream_t st);
-// workspace of the fused mode: control words, then one int per unit, then v
+// workspace of the fused mode: control words, then one int per unit (the head),
+// then v: fp32 [S][T][r_max] for this kernel or the v pairs of bgmv_tc.cu,
+// whichever is larger
+size_t bgmv_workspace_head(int units);
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max);
+
+// bgmv_tc.cu: bf16, r_max <= 64 and a multiple of 8, units of at most 16 rows,
+// the 16-byte alignments of bgmv.cu; a persistent grid of two blocks per SM
+size_t bgmv_tc_smem_bytes();
+// widest expand item the kernel's operand ring holds (columns, a multiple of 128)
+int bgmv_tc_max_item_cols();
+// v pairs of the fused workspace (after the head)
+size_t bgmv_tc_v_bytes(int units, int n_slices, int r_max);
+int launch_bgmv_tc(const BtArgs &a, int blocks, cudaStream_t st);
 
 // sgmv_tc.cu: bf16, r_max % 16 == 0, n_slices * r_max <= 128, 16-byte aligned rows;
 // chooses the cluster size and ring depth, launches persistent clusters

@@ -338,8 +338,40 @@ int bgmv_item_cols(const Call &c, int est_units) {
     return 2048;
 }
 
-// The gathered tiles (and the contiguous ones unless tc_took) on the fused
-// kernel, or the general kernel when the data does not suit it, on `stream`.
+// The tensor-core gathered-tile kernel takes a fused call whose units have at
+// most 16 rows (the MMA's N) when LORA_BG_TC=1.  It is opt-in: on the Llama-3-8B
+// decode layer set it is correct but slower than the mma.sync kernel (one
+// producer warp per block issues every copy and bounds the block).
+bool bgmv_tc_ok(const Call &c) {
+    return c.meta->rows_per_tile <= 16 && env_int("LORA_BG_TC", 0) == 1;
+}
+
+// Output columns of one tensor-core expand item: the widest the kernel's ring
+// holds (up to four 128-column tiles behind one v pair); tuning override
+// LORA_BT_COLS, a multiple of 128 up to that width.
+int bgmv_tc_item_cols() {
+    const int cap = bgmv_tc_max_item_cols();
+    const int e = env_int("LORA_BT_COLS", 0);
+    return e >= 128 && e <= cap && (e & 127) == 0 ? e : cap;
+}
+
+// Tensor maps of the tensor-core gathered-tile kernel; false when one cannot be encoded.
+bool bgmv_tc_maps(const Call &c, BtArgs &b) {
+    const int64_t N = c.meta->N;
+    for (int s = 0; s < c.n_slices; ++s) {
+        const lora_slice &sl = c.slices[s];
+        const __nv_bfloat16 *ys = static_cast<const __nv_bfloat16 *>(c.y) + sl.col_off;
+        if (tensor_map_2d(&b.tmA[s], sl.A, (uint64_t)c.d_in, (uint64_t)N * c.r_max, 64, 8, 128) != LORA_OK ||
+            tensor_map_2d(&b.tmB[s], sl.B, (uint64_t)c.r_max, (uint64_t)N * sl.d_out, 8, 128, 0) != LORA_OK ||
+            tensor_map_2d(&b.tmY[s], ys, (uint64_t)sl.d_out, (uint64_t)c.meta->T, 128, 1, 0,
+                          (uint64_t)c.ld_y) != LORA_OK)
+            return false;
+    }
+    return true;
+}
+
+// The gathered tiles (and the contiguous ones unless tc_took) on a gathered-tile
+// kernel, or the general kernel when the data does not suit them, on `stream`.
 int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took, cudaStream_t stream) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
     Tiles tiles = make_tiles(c.meta, gather, contig);
@@ -364,16 +396,18 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
             unsigned char *ws = static_cast<unsigned char *>(c.ws);
             g.ctl = reinterpret_cast<int *>(ws);
             g.done = g.ctl + 64;
-            g.v = reinterpret_cast<float *>(ws + bgmv_workspace_bytes(units, 0, 1, 8));
+            g.v = reinterpret_cast<float *>(ws + bgmv_workspace_head(units));
         } else {
             g.v = mode == MODE_SHRINK ? c.v_out : const_cast<float *>(c.v_in);
         }
         const int est = std::min(units, std::min(c.meta->N, c.meta->T) +
                                             (c.meta->T + c.meta->rows_per_tile - 1) / c.meta->rows_per_tile);
-        g.bc = bgmv_item_cols(c, std::max(1, est));
-        g.blk_off[0] = 0;
-        for (int s = 0; s < c.n_slices; ++s)
-            g.blk_off[s + 1] = g.blk_off[s] + (c.slices[s].d_out + g.bc - 1) / g.bc;
+        auto set_cols = [&](int bc) {
+            g.bc = bc;
+            g.blk_off[0] = 0;
+            for (int s = 0; s < c.n_slices; ++s)
+                g.blk_off[s + 1] = g.blk_off[s] + (c.slices[s].d_out + g.bc - 1) / g.bc;
+        };
         g.wait_limit = WAIT_LIMIT;
         if (env_int("LORA_DEBUG_STALL", 0) == 1) {
             // test hook for the bounded wait: expand items wait for a shrink signal
@@ -381,6 +415,20 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
             g.dbg_stall = 1;
             g.wait_limit = 64;
         }
+        if (mode == MODE_FUSED && bgmv_tc_ok(c)) {
+            static BtArgs bt;   // ~3.5 KB: kept off the stack; filled and launched under the lock
+            static std::mutex bt_mu;
+            std::lock_guard<std::mutex> lock(bt_mu);
+            bt = BtArgs{};
+            if (bgmv_tc_maps(c, bt)) {
+                set_cols(bgmv_tc_item_cols());
+                bt.g = g;
+                bt.vws = reinterpret_cast<unsigned char *>(g.v);
+                return launch_bgmv_tc(bt, bgmv_blocks(), stream);
+            }
+            // a map could not be encoded: the mma.sync kernel takes the call
+        }
+        set_cols(bgmv_item_cols(c, std::max(1, est)));
         return launch_bgmv(mode, g, bgmv_blocks(), stream);
     }
     SimtArgs a{};

@@ -18,7 +18,7 @@ SHAPES = {
     "multi_block_grouping": lambda: workloads.random_case(3, 3000, 1100, 256, [128], 16,
                                                           ranks=[16] * 1100),
 }
-OURS = ("seg_", "bgmv_kernel", "sgmv_tc_kernel", "simt_", "lora_")
+OURS = ("seg_", "bgmv_kernel", "bgmv_tc_kernel", "sgmv_tc_kernel", "simt_", "lora_")
 
 
 @pytest.mark.parametrize("shape", list(SHAPES))
