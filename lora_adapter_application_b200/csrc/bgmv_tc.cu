@@ -67,7 +67,7 @@ namespace {
 // shrink chunk or expand tile per 0.3-0.5 us) bounds its block; the rings shrink
 // with the count so that the SM's bytes in flight stay about the same.
 constexpr int BT_PER_SM = BT_BLOCKS_PER_SM;
-static_assert(BT_PER_SM >= 1 && BT_PER_SM <= 3, "blocks per SM");
+static_assert(BT_PER_SM >= 1 && BT_PER_SM <= 2, "blocks per SM");
 constexpr int BT_THREADS = 192;
 constexpr uint32_t BT_RB = BT_PER_SM == 1 ? (128u << 10) : BT_PER_SM == 2 ? (64u << 10) : (32u << 10);   // operand ring
 constexpr uint32_t BT_RY = BT_PER_SM == 1 ? (48u << 10) : (16u << 10);    // y ring
@@ -95,9 +95,13 @@ constexpr uint32_t OFF_BAR = OFF_YEND + BT_NYB * 4;
 constexpr uint32_t BT_NBARS = 2 * BT_NSB + 2 * BT_NYB + 2 * BT_NQ + 2 * BT_NT + 2 * BT_NV;
 constexpr uint32_t BT_SMEM = OFF_BAR + 8 * BT_NBARS + 1024;   // + room to align the base
 static_assert(BT_PER_SM * (BT_SMEM + 1024) <= 228 * 1024, "shared memory");
-// a shrink chunk's A box is read as 128 rows (16 KB) from its start: the bytes
-// past the operand ring that such a read may reach are the y ring's
+// A shrink chunk's A rows are read as 128 rows (16 KB) from the chunk's start,
+// which may reach up to 8 KB past its stage (r8 * 128 B per chunk, x after the
+// last): the bytes past the operand ring that such a read may reach are the y ring's
 static_assert(BT_RY >= 16384, "A over-read stays inside the allocation");
+// the largest allocations (a 256-column shrink stage at r_max 64: 32 KB of A and
+// 8 KB of x; 16 rows of y) fit their rings with room for the next
+static_assert(BT_RB >= 40960 + 16384 && BT_RY >= 2 * 4096, "ring sizes");
 
 // item record fields
 enum { IT_KIND = 0, IT_U, IT_S, IT_ID, IT_CNT, IT_RN, IT_N, IT_CLO, IT_SCALE, IT_FAIL, IT_ROWS = 16 };
@@ -231,47 +235,63 @@ __global__ void __launch_bounds__(BT_THREADS, BT_PER_SM) bgmv_tc_kernel(const __
         uint32_t bhead = 0, btail = 0, yhead = 0, ytail = 0;
         int sbh = 0, sbt = 0, ybh = 0, ybt = 0, qc = 0, vc = 0;
         bool failed = false;
-        // n bytes (a multiple of 1 KB) of the operand ring; its allocation index in *idx
+        // n bytes (a multiple of 1 KB) of the operand ring; its allocation index in *idx.
+        // Allocations never wrap: one that would run past the end starts at the
+        // beginning, the skipped tail counted with it; an empty ring restarts there.
         auto alloc_b = [&](uint32_t n, int *idx) -> uint32_t {
-            const uint32_t off = bhead & (BT_RB - 1);
-            const uint32_t pad = off + n > BT_RB ? BT_RB - off : 0u;
-            while (bhead + pad + n - btail > BT_RB || sbh - sbt >= BT_NSB) {
-                const int i = sbt % BT_NSB;
+            for (;;) {
+                const uint32_t off = bhead & (BT_RB - 1);
+                const uint32_t pad = off + n > BT_RB ? BT_RB - off : 0u;
+                if (pad && sbh == sbt) {   // nothing live: move to the beginning
+                    bhead += pad;
+                    btail = bhead;
+                    continue;
+                }
+                if (bhead + pad + n - btail <= BT_RB && sbh - sbt < BT_NSB) {
+                    bhead += pad;
+                    const uint32_t addr = rb + (bhead & (BT_RB - 1));
+                    bhead += n;
+                    *idx = sbh % BT_NSB;
+                    if (lane == 0) {
+                        send[*idx] = bhead;
+                        saddr[*idx] = addr;
+                    }
+                    ++sbh;
+                    return addr;
+                }
+                const int i = sbt % BT_NSB;   // the oldest live allocation comes back
                 if (!warp_wait(sempty + 8 * i, (unsigned)(sbt / BT_NSB) & 1u, a.status, failed)) return 0u;
                 btail = send[i];
                 ++sbt;
             }
-            bhead += pad;
-            const uint32_t addr = rb + (bhead & (BT_RB - 1));
-            bhead += n;
-            *idx = sbh % BT_NSB;
-            if (lane == 0) {
-                send[*idx] = bhead;
-                saddr[*idx] = addr;
-            }
-            ++sbh;
-            return addr;
         };
-        // n bytes (a multiple of 256) of the y ring
+        // n bytes (a multiple of 256) of the y ring, the same way
         auto alloc_y = [&](uint32_t n, int *idx) -> uint32_t {
-            const uint32_t off = yhead % BT_RY;
-            const uint32_t pad = off + n > BT_RY ? BT_RY - off : 0u;
-            while (yhead + pad + n - ytail > BT_RY || ybh - ybt >= BT_NYB) {
+            for (;;) {
+                const uint32_t off = yhead % BT_RY;
+                const uint32_t pad = off + n > BT_RY ? BT_RY - off : 0u;
+                if (pad && ybh == ybt) {
+                    yhead += pad;
+                    ytail = yhead;
+                    continue;
+                }
+                if (yhead + pad + n - ytail <= BT_RY && ybh - ybt < BT_NYB) {
+                    yhead += pad;
+                    const uint32_t addr = ry + yhead % BT_RY;
+                    yhead += n;
+                    *idx = ybh % BT_NYB;
+                    if (lane == 0) {
+                        yend[*idx] = yhead;
+                        yaddr[*idx] = addr;
+                    }
+                    ++ybh;
+                    return addr;
+                }
                 const int i = ybt % BT_NYB;
                 if (!warp_wait(yempty + 8 * i, (unsigned)(ybt / BT_NYB) & 1u, a.status, failed)) return 0u;
                 ytail = yend[i];
                 ++ybt;
             }
-            yhead += pad;
-            const uint32_t addr = ry + yhead % BT_RY;
-            yhead += n;
-            *idx = ybh % BT_NYB;
-            if (lane == 0) {
-                yend[*idx] = yhead;
-                yaddr[*idx] = addr;
-            }
-            ++ybh;
-            return addr;
         };
         // the next item record (waits until both consumers are done with its slot)
         auto take_record = [&]() -> int * {
@@ -291,7 +311,9 @@ __global__ void __launch_bounds__(BT_THREADS, BT_PER_SM) bgmv_tc_kernel(const __
 
         // ------------------------------------------------ shrink items
         const int total1 = live * S;
+        const int ks = p.ks;                       // 64-column chunks per stage
         const int nch = (a.d_in + 63) >> 6;
+        const int nst = (nch + ks - 1) / ks;
         int cur = ticket(GB_T_SHRINK);
         while (cur < total1 && !failed) {
             const int nxt = ticket(GB_T_SHRINK);   // in flight during this item
@@ -329,27 +351,38 @@ __global__ void __launch_bounds__(BT_THREADS, BT_PER_SM) bgmv_tc_kernel(const __
                 it[IT_ID] = un.id;
                 it[IT_CNT] = un.cnt;
                 it[IT_RN] = r_n;
-                it[IT_N] = nch;
+                it[IT_N] = nst;
                 it[IT_SCALE] = __float_as_int(a.alphas[un.id] / (float)r_n);
                 it[IT_FAIL] = 0;
             }
             publish();
             const int arow = un.id * a.r_max;
             const uint32_t pc = (uint32_t)(lane & 7);
-            for (int kc = 0; kc < nch; ++kc) {
+            for (int st = 0; st < nst; ++st) {
+                const int c0 = st * ks, nsub = min(ks, nch - c0);
                 int si = 0;
-                const uint32_t sa = alloc_b((uint32_t)g8 * 1024u + 2048u, &si);
+                // A: the item's r8 rank rows of ks chunks (one box), then x: ks chunks of 16 rows x 128 B
+                const uint32_t sa = alloc_b((uint32_t)(g8 * ks) * 1024u + (uint32_t)ks * 2048u, &si);
                 if (failed) break;
-                const uint32_t xa = sa + (uint32_t)g8 * 1024u;
-                if (lane == 0) mbar_expect_tx(sfull + 8 * si, (uint32_t)g8 * 1024u);
+                const uint32_t xa = sa + (uint32_t)(g8 * ks) * 1024u;
+                if (lane == 0) mbar_expect_tx(sfull + 8 * si, (uint32_t)(g8 * ks) * 1024u);
                 __syncwarp();
-                if (lane < g8) tma_2d(sa + (uint32_t)lane * 1024u, &p.tmA[s], kc * 64, arow + 8 * lane, sfull + 8 * si);
-                const int col = kc * 64 + (int)pc * 8;
-                const int sz = min(max(2 * (a.d_in - col), 0), 16);
+                if (ks == 4) {
+                    if (lane == 0) tma_3d(sa, &p.tmA4[g8 - 1][s], 0, arow, c0, sfull + 8 * si);
+                } else if (lane < g8) {
+                    tma_2d(sa + (uint32_t)lane * 1024u, &p.tmA[s], c0 * 64, arow + 8 * lane, sfull + 8 * si);
+                }
+                for (int c = 0; c < nsub; ++c) {
+                    const int col = (c0 + c) * 64 + (int)pc * 8;
+                    const int sz = min(max(2 * (a.d_in - col), 0), 16);
+                    const uint32_t xc = xa + (uint32_t)c * 2048u;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const uint32_t j = (uint32_t)((lane >> 3) + 4 * m);
-                    if (xv[m]) cp16z(xa + j * 128u + ((pc ^ (j & 7u)) << 4), sz ? (const void *)(xr[m] + col) : (const void *)xr[m], sz);
+                    for (int m = 0; m < 4; ++m) {
+                        const uint32_t j = (uint32_t)((lane >> 3) + 4 * m);
+                        if (xv[m])
+                            cp16z(xc + j * 128u + ((pc ^ (j & 7u)) << 4),
+                                  sz ? (const void *)(xr[m] + col) : (const void *)xr[m], sz);
+                    }
                 }
                 cp_async_arrive(sfull + 8 * si);   // once this lane's x pieces have landed
             }
@@ -452,17 +485,23 @@ __global__ void __launch_bounds__(BT_THREADS, BT_PER_SM) bgmv_tc_kernel(const __
                 if (!warp_wait(aempty + 8 * slot, ((unsigned)(ts / BT_NT) & 1u) ^ 1u, a.status, failed)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)slot * 16u;
-                for (int c = 0; c < n; ++c) {
+                const int ks = p.ks, nch = (a.d_in + 63) >> 6;
+                for (int st = 0; st < n; ++st) {
                     const int i = sc % BT_NSB;
                     if (!warp_wait(sfull + 8 * i, (unsigned)(sc / BT_NSB) & 1u, a.status, failed)) break;
                     tc_fence_after();
-                    const uint32_t sa = saddr[i], xa = sa + (uint32_t)g8 * 1024u;
+                    const int nsub = min(ks, nch - st * ks);
+                    const uint32_t sa = saddr[i], xa = sa + (uint32_t)(g8 * ks) * 1024u;
                     if (lane == 0) {
                         fence_proxy_async();   // x arrived by cp.async (generic proxy); the MMA reads it as an operand
+                        for (int c = 0; c < nsub; ++c) {
+                            // chunk c: its r8 rank rows are contiguous (8-row atoms 1 KB apart)
+                            const uint32_t ac = sa + (uint32_t)(c * g8) * 1024u, xc = xa + (uint32_t)c * 2048u;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma(d, desc_sw128(sa + 32u * kk), desc_sw128(xa + 32u * kk), BT_IDESC,
-                                   (c | kk) ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_mma(d, desc_sw128(ac + 32u * kk), desc_sw128(xc + 32u * kk), BT_IDESC,
+                                       (st | c | kk) ? 1u : 0u);
+                        }
                         tc_commit(sempty + 8 * i);
                     }
                     __syncwarp();

@@ -14,6 +14,10 @@ enum { MODE_FUSED = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t outer,
                   uint32_t box_inner, uint32_t box_outer, int swizzle,
                   uint64_t row_stride = 0);
+// [rows][inner] viewed as [inner / 64][rows][64] (inner a multiple of 64): boxes of
+// 64 columns x box_rows x box_chunks chunks, 128-byte swizzle
+int tensor_map_chunks(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t row_stride, uint32_t box_rows, uint32_t box_chunks);
 
 // Fused-mode workspace head shared by the gathered-tile kernels: GB_CTL_INTS
 // control words (tickets and the exit counter), then one done word per unit.
@@ -45,12 +49,16 @@ struct GbArgs {
 
 // The gathered-tile kernel on the tensor cores (bgmv_tc.cu, fused mode only):
 // GbArgs (bc a multiple of 128) plus maps over
-//   A_s  [N*r_max][d_in], boxes of 64 columns x 8 ranks, 128-byte swizzle
+//   A_s  [N*r_max][d_in], boxes of 64 columns x 8 ranks, 128-byte swizzle (and the
+//        chunked view above, one box per 256-column shrink stage)
 //   B_s  [N*d_out_s][r_max], boxes of 8 ranks x 128 columns, no swizzle
 //   y_s  y + col_off_s as [T][d_out_s] (row stride ld_y), boxes of 128 columns x 1 row
 // and the workspace's v pairs (s_n v as bf16 hi + lo per unit and slice).
 struct BtArgs {
     CUtensorMap tmA[LORA_MAX_SLICES];
+    // A_s as [d_in/64][N*r_max][64] (d_in % 64 == 0): tmA4[g - 1][s] boxes 8g ranks x 4 chunks
+    CUtensorMap tmA4[8][LORA_MAX_SLICES];
+    int ks;                              // 64-column chunks per shrink stage: 4 with tmA4, else 1
     CUtensorMap tmB[LORA_MAX_SLICES];
     CUtensorMap tmY[LORA_MAX_SLICES];
     GbArgs g;

@@ -361,6 +361,10 @@ bool bgmv_tc_maps(const Call &c, BtArgs &b) {
     for (int s = 0; s < c.n_slices; ++s) {
         const lora_slice &sl = c.slices[s];
         const __nv_bfloat16 *ys = static_cast<const __nv_bfloat16 *>(c.y) + sl.col_off;
+        for (int g = 1; b.ks == 4 && g <= c.r_max / 8; ++g)
+            if (tensor_map_chunks(&b.tmA4[g - 1][s], sl.A, (uint64_t)c.d_in, (uint64_t)N * c.r_max,
+                                  (uint64_t)c.d_in, (uint32_t)(8 * g), 4) != LORA_OK)
+                return false;
         if (tensor_map_2d(&b.tmA[s], sl.A, (uint64_t)c.d_in, (uint64_t)N * c.r_max, 64, 8, 128) != LORA_OK ||
             tensor_map_2d(&b.tmB[s], sl.B, (uint64_t)c.r_max, (uint64_t)N * sl.d_out, 8, 128, 0) != LORA_OK ||
             tensor_map_2d(&b.tmY[s], ys, (uint64_t)sl.d_out, (uint64_t)c.meta->T, 128, 1, 0,
@@ -420,6 +424,7 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
             static std::mutex bt_mu;
             std::lock_guard<std::mutex> lock(bt_mu);
             bt = BtArgs{};
+            bt.ks = c.d_in % 64 == 0 ? 4 : 1;   // 256-column shrink stages when the chunks are whole
             if (bgmv_tc_maps(c, bt)) {
                 set_cols(bgmv_tc_item_cols());
                 bt.g = g;

@@ -91,6 +91,15 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap *map, int
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
+// 3-D tensor copy (one box) global -> shared through the TMA engine.
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                       uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3, %4}], [%5];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 r;

@@ -85,4 +85,55 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
     return LORA_OK;
 }
 
+// A [rows][inner] bf16 matrix (row stride `row_stride` elements) viewed as
+// [inner / 64][rows][64]: boxes of 64 columns x box_rows rows x box_chunks
+// consecutive 64-column chunks, 128-byte swizzle.  inner must be a multiple
+// of 64; chunks past the end read as zero.
+int tensor_map_chunks(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t row_stride, uint32_t box_rows, uint32_t box_chunks) {
+    struct E3 {
+        const void *base;
+        uint64_t inner, rows, stride;
+        uint32_t br, bc;
+        int dev;
+        CUtensorMap map;
+    };
+    static E3 cache[64];
+    static int used = 0, next = 0;
+    if (inner % 64) return LORA_ERR_SHAPE;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < used; ++i) {
+        const E3 &e = cache[i];
+        if (e.base == base && e.inner == inner && e.rows == rows && e.stride == row_stride && e.br == box_rows &&
+            e.bc == box_chunks && e.dev == dev) {
+            *out = e.map;
+            return LORA_OK;
+        }
+    }
+    auto fn = encoder();
+    if (!fn) return cuda_fail("cuTensorMapEncodeTiled: driver entry point not found");
+    const cuuint64_t dims[3] = {64, rows, inner / 64};
+    const cuuint64_t strides[2] = {row_stride * 2, 128};   // bytes: next row, next 64-column chunk
+    const cuuint32_t box[3] = {64, box_rows, box_chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMap m;
+    const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail("cuTensorMapEncodeTiled failed");
+    E3 &e = cache[used < 64 ? used++ : (next++ % 64)];
+    e.base = base;
+    e.inner = inner;
+    e.rows = rows;
+    e.stride = row_stride;
+    e.br = box_rows;
+    e.bc = box_chunks;
+    e.dev = dev;
+    e.map = m;
+    *out = m;
+    return LORA_OK;
+}
+
 }  // namespace lora
