@@ -52,6 +52,9 @@
  *   LORA_BG_BLOCKS      1 to 4096: blocks of the gathered-tile kernel's persistent
  *                       grid (default: one per SM)
  *   LORA_BG_ITEM_COLS   32 to 8192, a multiple of 32: output columns of one expand item
+ *   LORA_BG_KSPLIT      1 or 2: pieces a fused call's shrink items are split into along
+ *                       d_in (default 2 for batches small enough to leave most SMs idle
+ *                       in the shrink, else 1)
  *   LORA_BG_TC          1: fused calls whose tiles have at most 16 rows run on the
  *                       tensor-core gathered-tile kernel (tcgen05 MMAs, TMA copies,
  *                       accumulators in tensor memory) instead of the mma.sync one;
@@ -268,7 +271,8 @@ LORA_API int lora_sgmv_expand(void *y, int64_t ld_y, const float *v, const lora_
  * grouped into *meta and a layer of n_slices slices with rank slots r_max: a
  * 256-byte head of control words, one int per unit of work (tile capacity of
  * the meta, rounded up to 256 bytes), then room for v: the larger of
- * [n_slices][T][r_max] fp32 and, per unit and slice, a bf16 hi + lo pair of 16
+ * [2][n_slices][T][r_max] fp32 (a small batch's shrink items may be split in two
+ * along d_in, each half with its own partial v) and, per unit and slice, a bf16 hi + lo pair of 16
  * rows by r_max rounded up to 16 ranks (the tensor-core gathered-tile kernel's
  * form).  0 for invalid arguments.
  *

@@ -310,7 +310,7 @@ __device__ __forceinline__ bool e_wait(const EWait &w) {
 template <int MR, int RK>
 __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max, int r_n,
                                             float scale, int c_lo, int c_hi,
-                                            __nv_bfloat16 *ys, int64_t ld_y, const float *vs,
+                                            __nv_bfloat16 *ys, int64_t ld_y, const float *vs, int64_t vpiece,
                                             uint32_t ring, const EWait &wt) {
     constexpr int H = 2;                            // row halves (g, g+8) of an m16 tile
     constexpr int CH = RK == 64 ? 2 : 1;            // rank chunks per step
@@ -423,9 +423,14 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
                 float f[8];
                 if (row >= 0 && k < r8) {
                     const float4 *pv = reinterpret_cast<const float4 *>(vs + (int64_t)row * r_max + k);
-                    const float4 lo4 = pv[0];
+                    float4 lo4 = pv[0], hi4 = pv[1];
+                    if (vpiece) {   // a split shrink: the second piece's partial, added in piece order
+                        const float4 *pw = pv + vpiece / 4;
+                        const float4 lo2 = pw[0], hi2 = pw[1];
+                        lo4 = make_float4(lo4.x + lo2.x, lo4.y + lo2.y, lo4.z + lo2.z, lo4.w + lo2.w);
+                        hi4 = make_float4(hi4.x + hi2.x, hi4.y + hi2.y, hi4.z + hi2.z, hi4.w + hi2.w);
+                    }
                     f[0] = lo4.x; f[1] = lo4.y; f[2] = lo4.z; f[3] = lo4.w;
-                    const float4 hi4 = pv[1];
                     f[4] = hi4.x; f[5] = hi4.y; f[6] = hi4.z; f[7] = hi4.w;
                 } else {
 #pragma unroll
@@ -507,10 +512,11 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
 template <int MR>
 __device__ __forceinline__ bool expand_dispatch(int r8, int row_l, const char *Bn, int r_max, int r_n,
                                                 float scale, int c_lo, int c_hi, __nv_bfloat16 *ys,
-                                                int64_t ld_y, const float *vs, uint32_t ring, const EWait &wt) {
+                                                int64_t ld_y, const float *vs, int64_t vpiece, uint32_t ring,
+                                                const EWait &wt) {
     if (r8 <= 32)
-        return expand_warp<MR, 32>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
-    return expand_warp<MR, 64>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, ring, wt);
+        return expand_warp<MR, 32>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, vpiece, ring, wt);
+    return expand_warp<MR, 64>(row_l, Bn, r_max, r_n, scale, c_lo, c_hi, ys, ld_y, vs, vpiece, ring, wt);
 }
 
 // What an expand warp needs of one item before it starts: unit, rank, this
@@ -535,7 +541,10 @@ __device__ __forceinline__ ERec erec_load(const GbArgs &a, int e, int total, int
 }
 
 // ------------------------------------------------------------------ kernel
-template <int MODE>
+// SPLIT (fused mode): every shrink item is two pieces along d_in, each writing
+// its own partial v; the expand adds them.  A separate instantiation, so that the
+// unsplit kernel's hot code is unchanged.
+template <int MODE, bool SPLIT = false>
 __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int rows_s[BG_ROWS];
@@ -553,18 +562,22 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
 
     // ------------------------------------------------------------ phase 1: shrink
     if (MODE != MODE_EXPAND) {
-        const int total = live * S * GM;
+        constexpr int KS = MODE == MODE_FUSED && SPLIT ? 2 : 1;   // pieces of an item along d_in
+        const int total = live * S * GM * KS;
         if (tid == 0) info_s[0] = MODE == MODE_FUSED ? atomicAdd(a.ctl + GB_T_SHRINK, 1) : (int)blockIdx.x;
         __syncthreads();
         const int nsteps = (a.d_in + 31) >> 5;
-        const int k_lo = warp * nsteps / BG_WARPS, k_hi = (warp + 1) * nsteps / BG_WARPS;
         for (;;) {
             const int item = info_s[0];
             if (item >= total) break;
             if (tid == 0)   // the next ticket flies during this item
                 info_s[1] = MODE == MODE_FUSED ? atomicAdd(a.ctl + GB_T_SHRINK, 1) : item + (int)gridDim.x;
-            const int u = item / (S * GM), rem = item - u * S * GM;
+            const int piece = item % KS, ig = item / KS;
+            const int u = ig / (S * GM), rem = ig - u * S * GM;
             const int s = rem / GM, grp = rem - s * GM;
+            // the piece's 32-column steps, split over the block's warps
+            const int p_lo = piece * nsteps / KS, p_n = (piece + 1) * nsteps / KS - p_lo;
+            const int k_lo = p_lo + warp * p_n / BG_WARPS, k_hi = p_lo + (warp + 1) * p_n / BG_WARPS;
             const Unit un = resolve_live_unit(a.tiles, u);
             if (tid < BG_ROWS) rows_s[tid] = tid < un.cnt ? un.row(a.tiles, tid) : -1;
             const int r_n = un.cnt > 0 ? a.ranks[un.id] : 0;
@@ -577,7 +590,7 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                                      ((int64_t)un.id * a.r_max + RGW * grp) * a.d_in * 2;
                 const char *x = reinterpret_cast<const char *>(a.x);
                 const int64_t lda = (int64_t)a.d_in * 2;
-                float *vb = a.v + (int64_t)s * a.T * a.r_max;
+                float *vb = a.v + piece * a.vpiece + (int64_t)s * a.T * a.r_max;
                 const int ntr = (un.cnt + 7) >> 3;
                 int nt;
                 if (rv > 32)
@@ -619,7 +632,7 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
     if (MODE != MODE_SHRINK) {
         const int nb = a.blk_off[S];
         const int total = live * nb;
-        const int need = S * GM + (a.dbg_stall ? 1 : 0);   // the stall test hook waits for one more
+        const int need = S * GM * (MODE == MODE_FUSED && SPLIT ? 2 : 1) + (a.dbg_stall ? 1 : 0);   // the stall test hook waits for one more
         auto claim = [&](int prev) -> int {
             if (MODE == MODE_FUSED) {
                 const int v = lane == 0 ? atomicAdd(a.ctl + GB_T_EXPAND, 1) : 0;
@@ -660,10 +673,10 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
                     const int rows = un.cnt - 32 * rg;
                     if (rows > 16)
                         ok_pass = expand_dispatch<2>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
-                                                        vs, ring, wt);
+                                                        vs, MODE == MODE_FUSED && SPLIT ? a.vpiece : 0, ring, wt);
                     else
                         ok_pass = expand_dispatch<1>(r8, row_l, Bn, a.r_max, r_n, scale, c_lo, c_hi, ys, a.ld_y,
-                                                        vs, ring, wt);
+                                                        vs, MODE == MODE_FUSED && SPLIT ? a.vpiece : 0, ring, wt);
                     wt.done = nullptr;
                 }
                 if (!ok_pass) break;   // the wait ran out: the warp takes no more work
@@ -694,8 +707,9 @@ __global__ void __launch_bounds__(BG_THREADS, 1) bgmv_kernel(const GbArgs a) {
     }
 }
 
-const void *bg_fn(int mode) {
-    return mode == MODE_FUSED ? (const void *)bgmv_kernel<MODE_FUSED>
+const void *bg_fn(int mode, bool split) {
+    return mode == MODE_FUSED ? (split ? (const void *)bgmv_kernel<MODE_FUSED, true>
+                                       : (const void *)bgmv_kernel<MODE_FUSED>)
                               : (mode == MODE_SHRINK ? (const void *)bgmv_kernel<MODE_SHRINK>
                                                      : (const void *)bgmv_kernel<MODE_EXPAND>);
 }
@@ -712,7 +726,7 @@ size_t bgmv_workspace_head(int units) {
 }
 
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max) {
-    const size_t v32 = (size_t)n_slices * (size_t)T * (size_t)r_max * 4;   // this kernel's fp32 v
+    const size_t v32 = (size_t)BG_KSPLIT_MAX * n_slices * (size_t)T * (size_t)r_max * 4;   // this kernel's fp32 v
     const size_t vtc = bgmv_tc_v_bytes(units, n_slices, r_max);            // the tensor-core kernel's v pairs
     return bgmv_workspace_head(units) + (v32 > vtc ? v32 : vtc);
 }
@@ -727,20 +741,25 @@ int launch_bgmv(int mode, const GbArgs &args, int blocks, cudaStream_t st) {
     {
         // the limit is a per-device attribute of the kernel: set once, to the largest ring
         static std::mutex mu;
-        static bool set[64][3] = {};
+        static bool set[64][4] = {};
+        const bool split = mode == MODE_FUSED && a.ks == 2;
+        const int slot = split ? 3 : mode;
         std::lock_guard<std::mutex> lock(mu);
         const int d = dev & 63;
-        if (!set[d][mode]) {
+        if (!set[d][slot]) {
             const cudaError_t e =
-                cudaFuncSetAttribute(bg_fn(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                cudaFuncSetAttribute(bg_fn(mode, split), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return cuda_rc(e);
-            set[d][mode] = true;
+            set[d][slot] = true;
         }
     }
     const int grid = blocks > 0 ? blocks : sms;
-    if (mode == MODE_FUSED)
-        bgmv_kernel<MODE_FUSED><<<grid, BG_THREADS, smem, st>>>(a);
-    else if (mode == MODE_SHRINK)
+    if (mode == MODE_FUSED) {
+        if (a.ks == 2)
+            bgmv_kernel<MODE_FUSED, true><<<grid, BG_THREADS, smem, st>>>(a);
+        else
+            bgmv_kernel<MODE_FUSED><<<grid, BG_THREADS, smem, st>>>(a);
+    } else if (mode == MODE_SHRINK)
         bgmv_kernel<MODE_SHRINK><<<grid, BG_THREADS, smem, st>>>(a);
     else
         bgmv_kernel<MODE_EXPAND><<<grid, BG_THREADS, smem, st>>>(a);

@@ -19,6 +19,9 @@ int tensor_map_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t o
 int tensor_map_chunks(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows,
                       uint64_t row_stride, uint32_t box_rows, uint32_t box_chunks);
 
+// Pieces a shrink item may be split into along d_in (fused mode, small batches).
+constexpr int BG_KSPLIT_MAX = 2;
+
 // Fused-mode workspace head shared by the gathered-tile kernels: GB_CTL_INTS
 // control words (tickets and the exit counter), then one done word per unit.
 constexpr int GB_CTL_INTS = 64;
@@ -44,6 +47,9 @@ struct GbArgs {
     int bc;            // output columns of one expand item (multiple of 32)
     int blk_off[LORA_MAX_SLICES + 1];   // expand items per unit: slice s owns [blk_off[s], blk_off[s+1])
     unsigned wait_limit;   // tries of the bounded wait (WAIT_LIMIT; shorter for the stall test hook)
+    int ks;            // fused mode: pieces a shrink item's d_in is split into (1 or 2); piece p writes
+                       // its partial v at v + p * vpiece, and the expand adds the pieces in order
+    int64_t vpiece;    // floats between the pieces' v (S * T * r_max)
     int dbg_stall;     // test hook: expand items wait for one shrink signal more than exists
 };
 
@@ -132,8 +138,8 @@ int launch_build_segments(const int32_t *ids, const lora_meta *m, void *scratch,
 size_t bgmv_smem_bytes(int mode);
 int launch_bgmv(int mode, const GbArgs &a, int blocks, cudaStream_t st);
 // workspace of the fused mode: control words, then one int per unit (the head),
-// then v: fp32 [S][T][r_max] for this kernel or the v pairs of bgmv_tc.cu,
-// whichever is larger
+// then v: fp32 [BG_KSPLIT_MAX][S][T][r_max] for this kernel or the v pairs of
+// bgmv_tc.cu, whichever is larger
 size_t bgmv_workspace_head(int units);
 size_t bgmv_workspace_bytes(int units, int T, int n_slices, int r_max);
 

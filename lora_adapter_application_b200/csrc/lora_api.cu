@@ -374,6 +374,18 @@ bool bgmv_tc_maps(const Call &c, BtArgs &b) {
     return true;
 }
 
+// Pieces a fused call's shrink items are split into along d_in: two when the
+// batch is so small that twice its expected shrink items still fit one block per
+// SM (decode batches: the items then run on idle SMs, halving the item every
+// expand waits for), else one.  Tuning / test override: LORA_BG_KSPLIT = 1 or 2.
+int bgmv_ksplit(const Call &c, int est_units) {
+    const int e = env_int("LORA_BG_KSPLIT", 0);
+    if (e == 1 || e == 2) return e;
+    const int gm = c.meta->rows_per_tile <= 16 ? 1 : (c.r_max + 31) / 32;
+    const int64_t items = (int64_t)est_units * c.n_slices * gm;
+    return (c.d_in >= 1024 && 2 * items <= device_sms()) ? 2 : 1;
+}
+
 // The gathered tiles (and the contiguous ones unless tc_took) on a gathered-tile
 // kernel, or the general kernel when the data does not suit them, on `stream`.
 int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took, cudaStream_t stream) {
@@ -434,6 +446,11 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
             // a map could not be encoded: the mma.sync kernel takes the call
         }
         set_cols(bgmv_item_cols(c, std::max(1, est)));
+        g.ks = 1;
+        if (mode == MODE_FUSED) {
+            g.ks = bgmv_ksplit(c, std::max(1, est));
+            g.vpiece = (int64_t)c.n_slices * c.meta->T * c.r_max;
+        }
         return launch_bgmv(mode, g, bgmv_blocks(), stream);
     }
     SimtArgs a{};

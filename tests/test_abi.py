@@ -81,8 +81,9 @@ def test_scratch_and_workspace_sizes(lib):
 def test_linear_workspace_size(lib):
     """256-byte head, one int per unit of the meta's tile capacity (rounded up to
     256 bytes), then room for the larger of the two kernels' v: fp32
-    [n_slices][T][r_max], or per unit and slice a bf16 hi + lo pair of 16 rows by
-    r_max rounded up to 16 ranks."""
+    [2][n_slices][T][r_max] (a small batch's shrink items may be split in two), or
+    per unit and slice a bf16 hi + lo pair of 16 rows by r_max rounded up to 16
+    ranks."""
     def r256(b):
         return (b + 255) // 256 * 256
     for T, N, R, min_run, S, r_max in [(1024, 100, 64, 0, 3, 64), (256, 32, 64, 0, 1, 16),
@@ -90,7 +91,7 @@ def test_linear_workspace_size(lib):
         m = _meta(T, N, R, min_run)
         mg, mc = lora.lora_meta_capacity(T, N, R, min_run, 128)
         units = mg + (mc * -(-128 // R) if min_run > 0 else 0)
-        want = 256 + r256(4 * units) + max(S * T * r_max * 4, units * S * 2 * 16 * -(-r_max // 16) * 16 * 2)
+        want = 256 + r256(4 * units) + max(2 * S * T * r_max * 4, units * S * 2 * 16 * -(-r_max // 16) * 16 * 2)
         assert lib.lora_linear_workspace_bytes(ctypes.byref(m), S, r_max) == want, (T, N, R)
     m = _meta()
     assert lib.lora_linear_workspace_bytes(ctypes.byref(m), 0, 16) == 0

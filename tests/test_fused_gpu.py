@@ -208,6 +208,7 @@ def test_eight_slices_rank_64_multi_pass(cuda_lib, blocks, monkeypatch):
     {"LORA_BG_ITEM_COLS": "32"}, {"LORA_BG_ITEM_COLS": "96"}, {"LORA_BG_ITEM_COLS": "192"},
     {"LORA_BG_ITEM_COLS": "4096"}, {"LORA_BG_ITEM_COLS": "8192"},
     {"LORA_BG_BLOCKS": "1"}, {"LORA_BG_BLOCKS": "2"}, {"LORA_BG_BLOCKS": "7"},
+    {"LORA_BG_KSPLIT": "1"}, {"LORA_BG_KSPLIT": "2"}, {"LORA_BG_KSPLIT": "2", "LORA_BG_BLOCKS": "3"},
 ])
 def test_overrides_keep_parity(cuda_lib, env, monkeypatch):
     for k, v in env.items():
