@@ -30,9 +30,11 @@
 // 16-byte pieces per lane, read and written once.
 //
 // In the fused mode v moves between the phases through a caller-provided
-// workspace: an expand item of unit u starts once u's S * ceil(r_max / 32)
-// shrink items have signalled (a per-unit counter, release / acquire at GPU
-// scope).  Shrink items are taken by blocks and expand items by warps from
+// workspace: an expand item of unit u starts once all of u's shrink items have
+// signalled (S slices x rank groups x pieces; a per-unit counter, release /
+// acquire at GPU scope).  A small batch runs a second instantiation whose
+// shrink items are two pieces along d_in, each writing its own partial v, which
+// the expand adds in piece order.  Shrink items are taken by blocks and expand items by warps from
 // atomic tickets, and a block turns to expand items only once every shrink
 // item has been taken, so a warp only ever waits for units that a running
 // block holds: the launch makes progress whatever number of its blocks is
