@@ -28,7 +28,8 @@
 // Warp roles (192 threads):
 //   warp 0     producer: tickets, item records, and every copy.  A boxes
 //              (64 columns x 8 ranks, 128-byte swizzle) and B boxes (8 ranks
-//              x 128 columns) and y rows (128 columns) by TMA tensor copies;
+//              x 128 columns) and y rows (four rows of 128 columns a copy, tile::gather4)
+//              by TMA tensor copies;
 //              x rows by cp.async into the swizzled layout (one 16-byte piece
 //              per lane); s_n v by a bulk copy once the unit is done.
 //   warp 1     tensor-memory allocator and MMA issuer (one thread issues).
@@ -136,6 +137,16 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;\n" :
 // generic-proxy global writes (another block's v pair, seen through an acquire)
 // before this thread's bulk copy reads them
 __device__ __forceinline__ void proxy_fence_global() { asm volatile("fence.proxy.async.global;\n" ::: "memory"); }
+// Four gathered rows of a 2-D tensor (box one row high) in one TMA copy, landing
+// one after the other in shared memory
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int x, int r0, int r1, int r2,
+                                            int r3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3, %4, %5, %6}], [%7];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+        : "memory");
+}
 // K-major operand without swizzle: 8-row x 16-byte core matrices of 128
 // contiguous bytes, the next 8 rows `sbo` bytes on, the next 8 K elements
 // `lbo` bytes on (same field layout as desc_plain)
@@ -418,13 +429,21 @@ __global__ void __launch_bounds__(BT_THREADS, BT_PER_SM) bgmv_tc_kernel(const __
             // tile t's y rows and B boxes; the first tile flies while the unit's shrink may
             // still run, the others follow the v copy (the MMA warp starts on v, so the
             // item's tiles go back one by one and never need the ring all at once)
+            // y rows in groups of four (one gather copy each; a group past the unit's last
+            // row repeats that row, whose copy lands in bytes the epilogue does not read)
+            const int nq = (un.cnt + 3) >> 2;
+            int yr[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) yr[i] = __shfl_sync(FULL, row_l, min(4 * (lane & 3) + i, un.cnt - 1));
             auto issue_tile = [&](int t) {
                 int yi = 0, bi = 0;
-                const uint32_t ya = alloc_y((uint32_t)un.cnt * 256u, &yi);
+                const uint32_t ya = alloc_y((uint32_t)nq * 1024u, &yi);
                 if (failed) return;
-                if (lane == 0) mbar_expect_tx(yfull + 8 * yi, (uint32_t)un.cnt * 256u);
+                if (lane == 0) mbar_expect_tx(yfull + 8 * yi, (uint32_t)nq * 1024u);
                 __syncwarp();
-                if (lane < un.cnt) tma_2d(ya + (uint32_t)lane * 256u, &p.tmY[s], c_lo + 128 * t, row_l, yfull + 8 * yi);
+                if (lane < nq)
+                    tma_gather4(ya + (uint32_t)lane * 1024u, &p.tmY[s], c_lo + 128 * t, yr[0], yr[1], yr[2], yr[3],
+                                yfull + 8 * yi);
                 const uint32_t ba = alloc_b((uint32_t)g8 * 2048u, &bi);
                 if (failed) return;
                 if (lane == 0) mbar_expect_tx(sfull + 8 * bi, (uint32_t)g8 * 2048u);
