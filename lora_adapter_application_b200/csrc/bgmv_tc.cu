@@ -26,12 +26,13 @@
 // without waiting on anything, so every wait on a done word ends.
 //
 // Warp roles (192 threads):
-//   warp 0     producer: tickets, item records, and every copy.  A boxes
-//              (64 columns x 8 ranks, 128-byte swizzle) and B boxes (8 ranks
-//              x 128 columns) and y rows (four rows of 128 columns a copy, tile::gather4)
-//              by TMA tensor copies;
-//              x rows by cp.async into the swizzled layout (one 16-byte piece
-//              per lane); s_n v by a bulk copy once the unit is done.
+//   warp 0     producer: tickets, item records, and every copy.  By TMA tensor
+//              copies: A, one box per 256-column stage (4 chunks of 64 columns x
+//              the item's ranks rounded to 8, 128-byte swizzle; 64 x 8-rank boxes
+//              when d_in is not a multiple of 64), B boxes (8 ranks x 128
+//              columns) and y rows (four rows of 128 columns a copy,
+//              tile::gather4).  x rows by cp.async into the swizzled layout (one
+//              16-byte piece per lane); s_n v by a bulk copy once the unit is done.
 //   warp 1     tensor-memory allocator and MMA issuer (one thread issues).
 //   warps 2-5  epilogue: tensor memory -> registers (lane = rank or output
 //              column), then v to the workspace, or y + D2 rounded once to
