@@ -190,7 +190,7 @@ __device__ __forceinline__ void shrink_warp(const char *A_rows, int64_t lda, int
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[mi][i][e] = 0.f;
 
-#pragma unroll
+#pragma unroll 1   // one copy of the issue code (the instruction cache is a first-order cost)
     for (int j = 0; j < NSL - 1; ++j) {
         if (j < nst) issue(j, j);
         cp_commit();
@@ -402,7 +402,7 @@ __device__ __forceinline__ bool expand_warp(int row_l, const char *Bn, int r_max
     };
     // the first steps fly while the unit's shrink finishes and v is read
     constexpr int PRO = NSL - 1;
-#pragma unroll
+#pragma unroll 1   // one copy of the issue code (the instruction cache is a first-order cost)
     for (int j = 0; j < PRO; ++j) {
         if (j < nst) issue(j, j);
         cp_commit();
