@@ -237,21 +237,59 @@ def step(ds):
                              ds.meta, ds.status)
 
 
-def min_run_of(w):
-    return MIN_RUN.get(w.name, 64)
+WIDE_COLS = 8192
+WIDE_ROWS_PER_TILE = 32
 
 
-def launches_per_step(w):
+def routes_all_gathered(T, d_out, sms):
+    """The library's route for a fused layer call: a batch with fewer 128-row
+    tiles than SMs and a layer of 8192 or more output columns runs every row on
+    the gathered-tile kernel (LORA_TC_ROUTE = 1 / 2 forces the split / the
+    single launch)."""
+    route = os.environ.get("LORA_TC_ROUTE", "")
+    if route in ("1", "2"):
+        return route == "2"
+    return -(-T // 128) < sms and sum(d_out) >= WIDE_COLS
+
+
+def device_sms(sms=None):
+    if sms is not None:
+        return sms
+    return torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+
+
+def segment_params(w, sms=None):
+    """(rows per gathered tile, shortest contiguous run) for one batch's segment
+    build.  When the library routes every row of every layer to the gathered-tile
+    kernel, contiguous runs would only be cut back into gathered tiles, so the
+    build makes none and tiles 32 rows: a tile reads its adapter once for twice
+    the rows, and with thousands of rows the tile count still fills the SMs
+    (measured on B200, the mixed 70B batch: 363 us with 16-row tiles and 64-row
+    runs, 347 us with 32-row tiles and no runs, 350-355 us with 16 or 64)."""
+    min_run = MIN_RUN.get(w.name, 64)
+    sms = device_sms(sms)
+    if min_run > 0 and w.layers and all(routes_all_gathered(w.T, l.d_out, sms) for l in w.layers):
+        return WIDE_ROWS_PER_TILE, 0
+    return ROWS_PER_TILE, min_run
+
+
+def launches_per_step(w, sms=None):
     """Kernels one step launches: the grouping (one block when T <= 2048, or
     T <= 8192 with N <= 1023; else seven passes), then per layer the gathered-tile kernel, plus the tensor-core
     SGMV kernel when contiguous tiles are enabled and the layer qualifies (bf16,
-    r_max a multiple of 16, n_slices * r_max <= 128)."""
+    r_max a multiple of 16, n_slices * r_max <= 128) and pays: not when the batch
+    has fewer 128-row tiles than SMs and the layer is 8192 or more columns wide
+    (then the gathered-tile kernel takes every row; LORA_TC_ROUTE overrides), and
+    not when the batch was built without contiguous runs (segment_params)."""
+    sms = device_sms(sms)
+    _, min_run = segment_params(w, sms)
     builder = 1 if (w.T <= 2048 or (w.T <= 8192 and w.N <= 1023)) else 7
     n = builder
     for l in w.layers:
         n += 1
-        if (min_run_of(w) > 0 and w.dtype == torch.bfloat16 and w.r_max % 16 == 0 and
-                len(l.d_out) * w.r_max <= 128):
+        qualifies = (min_run > 0 and w.dtype == torch.bfloat16 and w.r_max % 16 == 0 and
+                     len(l.d_out) * w.r_max <= 128)
+        if qualifies and not routes_all_gathered(w.T, l.d_out, sms):
             n += 1
     return n
 
@@ -374,7 +412,7 @@ def time_e2e(w, device, K, dist, n_streams=2):
     serving loop; every step still copies its own inputs in and its result out."""
     import lora_adapter_application_b200 as lora
     n_streams = max(1, int(n_streams))
-    sets = [DeviceSet(w, device, ROWS_PER_TILE, min_run_of(w)) for _ in range(n_streams)]
+    sets = [DeviceSet(w, device, *segment_params(w)) for _ in range(n_streams)]
     streams = [torch.cuda.Stream(device) for _ in range(n_streams)]
     host = {"ids": w.ids.pin_memory(),
             "layers": [{"x": l.x.pin_memory(), "y": l.y0.pin_memory()} for l in w.layers]}
@@ -462,7 +500,7 @@ def bench_ours(args, dist):
     sampler.start()
 
     w = workloads.make(args.workload, seed=args.seed + 1000 * dist.rank)
-    sets, per_set = make_sets(w, device, l2, ROWS_PER_TILE, min_run_of(w))
+    sets, per_set = make_sets(w, device, l2, *segment_params(w))
     step_ms_local, t0, t1, graphed = time_device(sets, args.steps, args.warmup, dist,
                                                  not args.no_graph)
     step_ms = dist.max(step_ms_local)
@@ -491,7 +529,7 @@ def bench_ours(args, dist):
                    "launch": ("CUDA graph of the K timed steps" if graphed else "eager") +
                              f"; kernel time from a separate graph of {KERNEL_STEPS} steps of "
                              "the layer calls alone",
-                   "rows_per_tile": ROWS_PER_TILE, "min_run": min_run_of(w),
+                   "rows_per_tile": segment_params(w)[0], "min_run": segment_params(w)[1],
                    "seed": args.seed},
         "roofline": rl,
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -528,7 +566,7 @@ def roofline_entry(w, kern_ms, pk):
     out = {"bound": "hbm", "achieved": None, "peak": peak, "unit": "GB/s", "frac": None,
            "traffic": traffic, "traffic_per_layer": per_layer,
            "kernel": "bgmv_kernel<MODE_FUSED>" + (" + sgmv_tc_kernel<MODE_FUSED>"
-                                                  if min_run_of(w) > 0 else ""),
+                                                  if segment_params(w)[1] > 0 else ""),
            "kernel_ms": kern_ms, "algorithmic_bytes": alg,
            "algorithmic_flops": roofline.workload_flops(w),
            "peak_source": f"{pk.get('source')} hbm_gbs"}
@@ -540,7 +578,7 @@ def roofline_entry(w, kern_ms, pk):
 
 def sweep_one(name, args, device, l2, pk, dist):
     w = workloads.make(name, seed=args.seed)
-    sets, per_set = make_sets(w, device, l2, ROWS_PER_TILE, min_run_of(w), max_sets=4)
+    sets, per_set = make_sets(w, device, l2, *segment_params(w), max_sets=4)
     probe_ms, _, _, _ = time_device(sets, 3, 3, dist, graph=False)
     K = int(min(500, max(20, args.sweep_seconds * 1e3 / probe_ms)))
     step_ms, _, _, _ = time_device(sets, K, 3, dist, graph=not args.no_graph)

@@ -66,6 +66,11 @@
  *                       the gathered-tile kernel instead
  *   LORA_TC_STAGES      2 to 6: depth of the tensor-core kernel's load ring (ignored
  *                       when shared memory cannot hold that many stages)
+ *   LORA_TC_ROUTE       1: lora_add_linear gives contiguous tiles to the tensor-core
+ *                       kernel whenever it qualifies; 2: never (the gathered-tile
+ *                       kernel takes every row).  Default: the tensor-core kernel unless
+ *                       the batch has fewer 128-row tiles than SMs and the layer's
+ *                       slices total 8192 or more output columns
  *   LORA_TC_LOAD_ROWS   8 to 128, a power of two: rows per x / y load box
  *   LORA_TC_STORE_ROWS  8 to 128, a power of two: rows per y store box
  *
@@ -308,7 +313,11 @@ LORA_API int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x,
  * every slice of one linear layer (fused QKV, gate/up, or a single output) to
  * y in place.  Gathered tiles (decode rows) take the fused BGMV kernel;
  * contiguous tiles (prompt runs) take the tensor-core SGMV kernel when the
- * data is bf16; everything else takes the general kernel.  Same result as
+ * data is bf16, except when the batch has fewer 128-row tiles than the GPU has
+ * SMs and the layer's slices total 8192 or more output columns: then the fused
+ * BGMV kernel takes every row in one launch (it spreads a wide layer's columns
+ * over every SM; LORA_TC_ROUTE overrides); everything else takes the general
+ * kernel.  Same result as
  * lora_bgmv_fused; the same workspace contract.  When both kinds of tiles are
  * present the gathered ones run on a library-owned second stream, forked from
  * and joined back into `stream` with events (also under stream capture); each

@@ -470,9 +470,32 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
     return launch_simt(mode, c.dtype == LORA_BF16, a, units, stream);
 }
 
+// A fused call's contiguous tiles take the tensor-core SGMV kernel unless the
+// batch is too small to give every SM a 128-row tile while the layer is wide: a
+// cluster expands its tile over every output column as one long piece, and one
+// round of such tiles leaves SMs idle, where the gathered-tile kernel spreads the
+// same columns over every warp as items and takes all rows in one launch.
+// Measured on B200 (fused calls, 16-row tiles): the mixed 70B batch's
+// 8192 -> 28672 layer 226 -> 208 us and its 28672 -> 8192 layer 152 -> 147 us,
+// each now one launch; prefill batches of 11-77k tokens at 4096 wide keep the
+// tensor-core kernel (71 against 82 us at 11k tokens).  Override: LORA_TC_ROUTE = 1
+// (the tensor-core kernel whenever it qualifies) or 2 (the gathered-tile kernel
+// for every row).
+constexpr int64_t TC_WIDE_COLS = 8192;
+bool tc_pays(int mode, const Call &c) {
+    const int e = env_int("LORA_TC_ROUTE", 0);
+    if (e == 1) return true;
+    if (e == 2) return false;
+    if (mode != MODE_FUSED) return true;
+    int64_t cols = 0;
+    for (int s = 0; s < c.n_slices; ++s) cols += c.slices[s].d_out;
+    const int64_t tiles = ((int64_t)c.meta->T + c.meta->long_tile - 1) / c.meta->long_tile;
+    return !(tiles < device_sms() && cols >= TC_WIDE_COLS);
+}
+
 int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = true) {
     const bool need_x = mode != MODE_EXPAND, need_y = mode != MODE_SHRINK;
-    if (tensor_core && contig && c.meta->T > 0 && tc_ok(c, need_x, need_y)) {
+    if (tensor_core && contig && c.meta->T > 0 && tc_ok(c, need_x, need_y) && tc_pays(mode, c)) {
         // contiguous tiles on the tensor-core kernel (caller's stream), gathered tiles on
         // the side stream: the fork comes first, so the two launches overlap
         return with_side_stream(c.stream, [&](cudaStream_t side) -> int {

@@ -70,8 +70,9 @@ def test_traffic_missing_record(tmp_path, monkeypatch):
     assert bench.measured_traffic("decode_qproj", 1) == (None, None)
 
 
-def _w(name, T, N, r_max, slices_per_layer, dtype=torch.bfloat16):
-    layers = [SimpleNamespace(d_out=[64] * s) for s in slices_per_layer]
+def _w(name, T, N, r_max, slices_per_layer, dtype=torch.bfloat16, d_out=64):
+    widths = d_out if isinstance(d_out, list) else [d_out] * len(slices_per_layer)
+    layers = [SimpleNamespace(d_out=[c] * s) for s, c in zip(slices_per_layer, widths)]
     return SimpleNamespace(name=name, T=T, N=N, r_max=r_max, dtype=dtype, layers=layers)
 
 
@@ -89,6 +90,32 @@ def test_launches_per_step_hand_counted():
     assert bench.launches_per_step(_w("prefill", 2048, 8, 64, [3])) == 1 + 1
     assert bench.launches_per_step(_w("prefill", 2048, 8, 24, [1])) == 1 + 1
     assert bench.launches_per_step(_w("prefill", 2048, 8, 16, [1], torch.float32)) == 1 + 1
+    # a batch with fewer 128-row tiles than SMs and a layer 8192+ columns wide: the
+    # gathered-tile kernel takes every row of that layer (the 70B MLP's two layers)
+    assert bench.launches_per_step(_w("mixed_70b", 8192, 16, 16, [1, 1], d_out=[28672, 8192]), sms=148) == 1 + 1 + 1
+    assert bench.launches_per_step(_w("mixed_70b", 8192, 16, 16, [1, 1], d_out=[28672, 4096]), sms=148) == 1 + 1 + 2
+    assert bench.launches_per_step(_w("mixed_70b", 8192, 16, 16, [1, 1], d_out=[28672, 8192]), sms=40) == 1 + 2 + 2
+    assert bench.launches_per_step(_w("prefill", 77000, 8, 16, [1], d_out=[28672]), sms=148) == 7 + 2
+
+
+def test_segment_params_follow_the_route(monkeypatch):
+    monkeypatch.delenv("LORA_TC_ROUTE", raising=False)
+    # decode-only and narrow prompt batches: the table's runs, 16-row tiles
+    assert bench.segment_params(_w("decode_qproj", 256, 32, 16, [1]), sms=148) == (16, 0)
+    assert bench.segment_params(_w("prefill", 77000, 8, 16, [1], d_out=4096), sms=148) == (16, 64)
+    # every layer 8192+ wide with fewer 128-row tiles than SMs: no runs, 32-row tiles
+    wide = _w("mixed_70b", 8192, 16, 16, [1, 1], d_out=[28672, 8192])
+    assert bench.segment_params(wide, sms=148) == (32, 0)
+    assert bench.segment_params(wide, sms=40) == (16, 64)
+    # one narrow layer keeps the runs for the tensor-core kernel
+    assert bench.segment_params(_w("mixed_70b", 8192, 16, 16, [1, 1], d_out=[28672, 4096]), sms=148) == (16, 64)
+    # a long prefill batch fills the SMs with 128-row tiles: runs kept
+    assert bench.segment_params(_w("prefill", 77000, 8, 16, [1], d_out=[28672]), sms=148) == (16, 64)
+    monkeypatch.setenv("LORA_TC_ROUTE", "1")
+    assert bench.segment_params(wide, sms=148) == (16, 64)
+    assert bench.launches_per_step(wide, sms=148) == 1 + 2 + 2
+    monkeypatch.setenv("LORA_TC_ROUTE", "2")
+    assert bench.segment_params(wide, sms=148) == (32, 0)
 
 
 def test_launches_per_step_grouping_boundaries():
