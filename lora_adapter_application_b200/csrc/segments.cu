@@ -231,10 +231,10 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
     const int wl = min(warp * wpw, W), wh = min(wl + wpw, W);
     bool overflow = false;
 
-    if (o.min_run <= 0) {   // no contiguous tiles: every valid position is gathered
-        for (int w = tid; w < W; w += SEG_THREADS) lngw[w] = 0u;
+    // no contiguous tiles: every valid position is gathered, in position order
+    const bool all_gathered = o.min_run <= 0;
+    if (all_gathered) {
         if (tid == 0) o.counts[2] = 0;
-        __syncthreads();
     } else {
     // 1. pack run starts
     for (int w = warp; w < W; w += NW) {
@@ -394,7 +394,10 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
         return ~lngw[w] & valid;
     };
     int n_short;
-    {
+    if (all_gathered) {   // the gathered rows are perm[0:P]
+        for (int p = tid; p < P; p += SEG_THREADS) o.grow[p] = perm[p];
+        n_short = P;
+    } else {
         int cnt = 0;
         for (int w = wl + lane; w < wh; w += 32) cnt += __popc(short_bits(w));
 #pragma unroll
@@ -406,11 +409,12 @@ __device__ void dev_tiles(const int32_t *ids, const int32_t *perm, const uint8_t
             if (lane == 0) gpre[w] = base;
             base += __popc(bits);
         }
+        __syncthreads();
     }
-    __syncthreads();
 
     // 6. gathered tiles: each id's gathered rows cut every R rows
     auto short_before = [&](int q) -> int {
+        if (all_gathered) return min(q, P);
         if (q >= P) return n_short;
         const int w = q >> 5, b = q & 31;
         return gpre[w] + __popc(short_bits(w) & ((1u << b) - 1u));
