@@ -237,40 +237,26 @@ def step(ds):
                              ds.meta, ds.status)
 
 
-WIDE_COLS = 8192
-WIDE_ROWS_PER_TILE = 32
-
-
-def routes_all_gathered(T, d_out, sms):
-    """The library's route for a fused layer call: a batch with fewer 128-row
-    tiles than SMs and a layer of 8192 or more output columns runs every row on
-    the gathered-tile kernel (LORA_TC_ROUTE = 1 / 2 forces the split / the
-    single launch)."""
-    route = os.environ.get("LORA_TC_ROUTE", "")
-    if route in ("1", "2"):
-        return route == "2"
-    return -(-T // 128) < sms and sum(d_out) >= WIDE_COLS
-
-
 def device_sms(sms=None):
     if sms is not None:
         return sms
     return torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
 
 
+def segment_plan(w, sms=None):
+    """(rows per gathered tile, shortest contiguous run, per-layer all-gathered
+    flags) for one batch's segment build, from the library's lora_segment_plan:
+    when lora_add_linear will run every row of every layer on the gathered-tile
+    kernel, the build makes no contiguous runs and 32-row tiles (the mixed 70B
+    batch on B200: 363 us with 16-row tiles and 64-row runs, 347 us so)."""
+    import lora_adapter_application_b200 as lora
+    return lora.lora_segment_plan(w.T, [sum(l.d_out) for l in w.layers], ROWS_PER_TILE,
+                                  MIN_RUN.get(w.name, 64), sms=device_sms(sms))
+
+
 def segment_params(w, sms=None):
-    """(rows per gathered tile, shortest contiguous run) for one batch's segment
-    build.  When the library routes every row of every layer to the gathered-tile
-    kernel, contiguous runs would only be cut back into gathered tiles, so the
-    build makes none and tiles 32 rows: a tile reads its adapter once for twice
-    the rows, and with thousands of rows the tile count still fills the SMs
-    (measured on B200, the mixed 70B batch: 363 us with 16-row tiles and 64-row
-    runs, 347 us with 32-row tiles and no runs, 350-355 us with 16 or 64)."""
-    min_run = MIN_RUN.get(w.name, 64)
-    sms = device_sms(sms)
-    if min_run > 0 and w.layers and all(routes_all_gathered(w.T, l.d_out, sms) for l in w.layers):
-        return WIDE_ROWS_PER_TILE, 0
-    return ROWS_PER_TILE, min_run
+    rows_per_tile, min_run, _ = segment_plan(w, sms)
+    return rows_per_tile, min_run
 
 
 def launches_per_step(w, sms=None):
@@ -280,16 +266,15 @@ def launches_per_step(w, sms=None):
     r_max a multiple of 16, n_slices * r_max <= 128) and pays: not when the batch
     has fewer 128-row tiles than SMs and the layer is 8192 or more columns wide
     (then the gathered-tile kernel takes every row; LORA_TC_ROUTE overrides), and
-    not when the batch was built without contiguous runs (segment_params)."""
-    sms = device_sms(sms)
-    _, min_run = segment_params(w, sms)
+    not when the batch was built without contiguous runs (segment_plan)."""
+    _, min_run, all_gathered = segment_plan(w, sms)
     builder = 1 if (w.T <= 2048 or (w.T <= 8192 and w.N <= 1023)) else 7
     n = builder
-    for l in w.layers:
+    for l, gathered in zip(w.layers, all_gathered):
         n += 1
         qualifies = (min_run > 0 and w.dtype == torch.bfloat16 and w.r_max % 16 == 0 and
                      len(l.d_out) * w.r_max <= 128)
-        if qualifies and not routes_all_gathered(w.T, l.d_out, sms):
+        if qualifies and not gathered:
             n += 1
     return n
 

@@ -70,7 +70,8 @@
  *                       kernel whenever it qualifies; 2: never (the gathered-tile
  *                       kernel takes every row).  Default: the tensor-core kernel unless
  *                       the batch has fewer 128-row tiles than SMs and the layer's
- *                       slices total 8192 or more output columns
+ *                       slices total 8192 or more output columns (lora_segment_plan
+ *                       follows the same setting)
  *   LORA_TC_LOAD_ROWS   8 to 128, a power of two: rows per x / y load box
  *   LORA_TC_STORE_ROWS  8 to 128, a power of two: rows per y store box
  *
@@ -145,8 +146,11 @@ typedef enum { LORA_BF16 = 0, LORA_FP32 = 1 } lora_dtype;
  * prefill).  Runs of at least min_run rows (min_run > 0) are cut into
  * contiguous tiles of at most long_tile rows; every other row is gathered,
  * and each id's gathered rows are cut into tiles of at most rows_per_tile.
- * The fused kernel reads a tile's adapter once for all of the tile's rows, so
- * decode batches are best grouped with rows_per_tile = LORA_MAX_TILE_ROWS.
+ * The fused kernel reads a tile's adapter once for all of the tile's rows, but
+ * a tile's shrink runs on one SM and its expand waits for it: 16-row tiles
+ * measured best on decode batches (64-row tiles were 8 % slower on a
+ * Llama-3-8B layer set at 1024 rows).  lora_segment_plan gives rows_per_tile
+ * and min_run for a batch whose layers all take the fused kernel for every row.
  */
 typedef struct {
     int32_t T;
@@ -316,8 +320,9 @@ LORA_API int lora_bgmv_fused(void *y, int64_t ld_y, const void *x, int64_t ld_x,
  * data is bf16, except when the batch has fewer 128-row tiles than the GPU has
  * SMs and the layer's slices total 8192 or more output columns: then the fused
  * BGMV kernel takes every row in one launch (it spreads a wide layer's columns
- * over every SM; LORA_TC_ROUTE overrides); everything else takes the general
- * kernel.  Same result as
+ * over every SM; LORA_TC_ROUTE overrides; lora_segment_plan gives the segment
+ * build that suits this route); everything else takes the general kernel.
+ * Same result as
  * lora_bgmv_fused; the same workspace contract.  When both kinds of tiles are
  * present the gathered ones run on a library-owned second stream, forked from
  * and joined back into `stream` with events (also under stream capture); each
@@ -329,6 +334,39 @@ LORA_API int lora_add_linear(void *y, int64_t ld_y, const void *x, int64_t ld_x,
                     const int32_t *ranks, const float *alphas, const lora_meta *meta,
                     void *workspace, size_t workspace_bytes, lora_dtype dtype,
                     int32_t *status, void *stream);
+
+/*
+ * Segment-build plan for one batch that will run through lora_add_linear
+ * (page "Multi-LoRA Serving", section 3.2: SGMV for prompt segments and BGMV
+ * for single rows in one heterogeneous batch; which rows become segments is the
+ * scheduler's choice).  Host only: no device work, no stream.
+ *
+ *   T            rows of the batch, 0..LORA_MAX_ROWS
+ *   layer_cols   host array of n_layers entries: per layer the total output
+ *                columns of its slices (sum of d_out); may be NULL when n_layers
+ *                is 0
+ *   sms          SMs of the device the batch runs on, or 0 for the current device
+ *   long_tile    rows per contiguous tile the meta will use, 1..LORA_LONG_TILE
+ *   rows_per_tile, min_run  in: the caller's choice for this batch (min_run 0 =
+ *                no contiguous tiles); out: the plan
+ *   all_gathered optional host array of n_layers bytes (NULL to skip): 1 where
+ *                lora_add_linear sends every row of that layer to the fused
+ *                BGMV kernel, 0 where the tensor-core kernel may take its
+ *                contiguous tiles
+ *
+ * A layer routes all rows to the fused BGMV kernel when the batch has fewer
+ * long_tile-row tiles than SMs and the layer is 8192 or more columns wide (the
+ * rule lora_add_linear applies; LORA_TC_ROUTE = 1 / 2 forces 0 / 1 for every
+ * layer).  When every layer does and min_run > 0, contiguous runs would only be
+ * cut back into gathered tiles, so the plan is min_run = 0 with 32-row tiles;
+ * otherwise the caller's values come back unchanged.  Returns LORA_ERR_NULL
+ * for a missing pointer, LORA_ERR_SHAPE for T, n_layers (0..4096), sms,
+ * long_tile, rows_per_tile (1..LORA_MAX_TILE_ROWS), min_run (>= 0) or a
+ * layer's columns (>= 1) out of range, with nothing written.
+ */
+LORA_API int lora_segment_plan(int32_t T, const int64_t *layer_cols, int32_t n_layers, int32_t sms,
+                               int32_t long_tile, int32_t *rows_per_tile, int32_t *min_run,
+                               uint8_t *all_gathered);
 
 
 /*

@@ -30,7 +30,7 @@ __all__ = [
     "lora_linear_workspace_bytes", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_bgmv_fused",
     "lora_add_linear", "alphas_full", "lora_load_adapter", "SlotCache", "lora_slot_cache_create",
     "lora_slot_cache_destroy", "lora_slot_cache_acquire", "lora_slot_cache_release",
-    "lora_slot_cache_key", "lora_slot_cache_evict", "lora_merge_adapter",
+    "lora_slot_cache_key", "lora_slot_cache_evict", "lora_merge_adapter", "lora_segment_plan",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -69,6 +69,9 @@ _SIGS = {
     "lora_meta_capacity": (ctypes.c_int, [_I32, _I32, _I32, _I32, _I32, ctypes.POINTER(_I32),
                                           ctypes.POINTER(_I32)]),
     "lora_segments_scratch_bytes": (_SZ, [_I32, _I32]),
+    "lora_segment_plan": (ctypes.c_int, [_I32, ctypes.POINTER(_I64), _I32, _I32, _I32,
+                                         ctypes.POINTER(_I32), ctypes.POINTER(_I32),
+                                         ctypes.POINTER(ctypes.c_uint8)]),
     "lora_build_segments": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _SZ, _P, _P]),
     "lora_build_segments_static": (ctypes.c_int, [_P, ctypes.POINTER(lora_meta), _P, _P]),
     "lora_shrink_workspace_bytes": (_SZ, [_I32, _I32, _I32]),
@@ -170,6 +173,19 @@ def lora_meta_capacity(T, N, rows_per_tile=MAX_TILE_ROWS, min_run=64, long_tile=
 
 def lora_segments_scratch_bytes(T, N):
     return int(load().lora_segments_scratch_bytes(T, N))
+
+
+def lora_segment_plan(T, layer_cols, rows_per_tile, min_run, sms=0, long_tile=LONG_TILE):
+    """(rows_per_tile, min_run, all_gathered) for a batch of T rows that will run
+    through lora_add_linear once per layer, layer_cols[l] being layer l's total
+    output columns (see include/lora_delta.h); host only."""
+    n = len(layer_cols)
+    cols = (_I64 * max(n, 1))(*[int(c) for c in layer_cols])
+    flags = (ctypes.c_uint8 * max(n, 1))()
+    rt, mr = _I32(rows_per_tile), _I32(min_run)
+    _check(load().lora_segment_plan(T, cols, n, sms, long_tile, ctypes.byref(rt), ctypes.byref(mr),
+                                    flags))
+    return rt.value, mr.value, [bool(flags[i]) for i in range(n)]
 
 
 def lora_build_segments_static(ids, meta: Meta, status, stream=None):

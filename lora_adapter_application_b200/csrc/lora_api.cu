@@ -482,15 +482,32 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
 // (the tensor-core kernel whenever it qualifies) or 2 (the gathered-tile kernel
 // for every row).
 constexpr int64_t TC_WIDE_COLS = 8192;
-bool tc_pays(int mode, const Call &c) {
+// Rows per gathered tile when every row of every layer takes the fused kernel:
+// a tile reads its adapter once for twice the rows of a 16-row tile, and a batch
+// of thousands of rows still has tiles for every SM (the mixed 70B pair: 347 us
+// with 32-row tiles, 355 with 16, 351 with 64, all without contiguous runs).
+constexpr int32_t WIDE_ROWS_PER_TILE = 32;
+
+// -1: no override; 0: the tensor-core kernel whenever it qualifies; 1: every row
+// of every fused call on the gathered-tile kernel.
+int route_override() {
     const int e = env_int("LORA_TC_ROUTE", 0);
-    if (e == 1) return true;
-    if (e == 2) return false;
+    return e == 1 ? 0 : e == 2 ? 1 : -1;
+}
+
+// The rule itself: a fused call over T rows and `cols` output columns sends every
+// row to the gathered-tile kernel.
+bool wide_and_few_tiles(int64_t T, int64_t long_tile, int64_t cols, int sms) {
+    return (T + long_tile - 1) / long_tile < sms && cols >= TC_WIDE_COLS;
+}
+
+bool tc_pays(int mode, const Call &c) {
+    const int e = route_override();
+    if (e >= 0) return e == 0;
     if (mode != MODE_FUSED) return true;
     int64_t cols = 0;
     for (int s = 0; s < c.n_slices; ++s) cols += c.slices[s].d_out;
-    const int64_t tiles = ((int64_t)c.meta->T + c.meta->long_tile - 1) / c.meta->long_tile;
-    return !(tiles < device_sms() && cols >= TC_WIDE_COLS);
+    return !wide_and_few_tiles(c.meta->T, c.meta->long_tile, cols, device_sms());
 }
 
 int run(int mode, const Call &c, bool gather, bool contig, bool tensor_core = true) {
@@ -558,6 +575,31 @@ int lora_meta_capacity(int32_t T, int32_t N, int32_t rows_per_tile, int32_t min_
         return LORA_ERR_SHAPE;
     *max_gather = (T + rows_per_tile - 1) / rows_per_tile + (N < T ? N : T);
     *max_contig = min_run > 0 ? (T + long_tile - 1) / long_tile + T / min_run : 0;
+    return LORA_OK;
+}
+
+int lora_segment_plan(int32_t T, const int64_t *layer_cols, int32_t n_layers, int32_t sms,
+                      int32_t long_tile, int32_t *rows_per_tile, int32_t *min_run,
+                      uint8_t *all_gathered) {
+    if (!rows_per_tile || !min_run || (n_layers > 0 && !layer_cols)) return LORA_ERR_NULL;
+    if (T < 0 || T > LORA_MAX_ROWS || n_layers < 0 || n_layers > LORA_MAX_ADAPTERS || sms < 0 ||
+        long_tile < 1 || long_tile > LORA_LONG_TILE || *rows_per_tile < 1 ||
+        *rows_per_tile > LORA_MAX_TILE_ROWS || *min_run < 0)
+        return LORA_ERR_SHAPE;
+    for (int l = 0; l < n_layers; ++l)
+        if (layer_cols[l] < 1) return LORA_ERR_SHAPE;
+    const int n_sms = sms > 0 ? sms : device_sms();
+    const int e = route_override();
+    bool every = n_layers > 0;
+    for (int l = 0; l < n_layers; ++l) {
+        const bool g = e >= 0 ? e == 1 : wide_and_few_tiles(T, long_tile, layer_cols[l], n_sms);
+        if (all_gathered) all_gathered[l] = g ? 1 : 0;
+        every = every && g;
+    }
+    if (every && *min_run > 0) {
+        *rows_per_tile = WIDE_ROWS_PER_TILE;
+        *min_run = 0;
+    }
     return LORA_OK;
 }
 

@@ -55,6 +55,52 @@ def test_capacity_bounds(lib):
     assert lora.lora_meta_capacity(1024, 100, 64, 0, 128) == (16 + 100, 0)
 
 
+def test_segment_plan(lib, monkeypatch):
+    """lora_segment_plan: a layer routes every row to the fused kernel when the
+    batch has fewer long_tile-row tiles than SMs and the layer is 8192+ columns
+    wide; when all layers do and the batch has runs, the plan is 32-row tiles and
+    no runs; otherwise the caller's values come back."""
+    monkeypatch.delenv("LORA_TC_ROUTE", raising=False)
+    plan = lora.lora_segment_plan
+    # 8192 rows = 64 tiles of 128 < 148 SMs; both layers wide
+    assert plan(8192, [28672, 8192], 16, 64, sms=148) == (32, 0, [True, True])
+    # one narrow layer: runs kept; the flags still say which layer routes
+    assert plan(8192, [28672, 8191], 16, 64, sms=148) == (16, 64, [True, False])
+    # as many tiles as SMs: the tensor-core kernel keeps the runs
+    assert plan(148 * 128, [28672], 16, 64, sms=148) == (16, 64, [False])
+    assert plan(147 * 128, [28672], 16, 64, sms=148) == (32, 0, [True])
+    assert plan(147 * 128 + 1, [28672], 16, 64, sms=148) == (16, 64, [False])
+    # a decode batch (no runs) keeps its tile size; no layers: unchanged
+    assert plan(8192, [28672, 8192], 16, 0, sms=148) == (16, 0, [True, True])
+    assert plan(8192, [], 16, 64, sms=148) == (16, 64, [])
+    # the long tile sets the tile count: 8192 rows in 32-row tiles = 256 > 148
+    assert plan(8192, [28672], 16, 64, sms=148, long_tile=32) == (16, 64, [False])
+    # LORA_TC_ROUTE: 1 = never all-gathered, 2 = always
+    monkeypatch.setenv("LORA_TC_ROUTE", "1")
+    assert plan(8192, [28672, 8192], 16, 64, sms=148) == (16, 64, [False, False])
+    monkeypatch.setenv("LORA_TC_ROUTE", "2")
+    assert plan(77000, [4096], 16, 64, sms=148) == (32, 0, [True])
+    monkeypatch.delenv("LORA_TC_ROUTE")
+    # out-of-range arguments: LORA_ERR_SHAPE, nothing written
+    for args, kw in [((-1, [8192], 16, 64), {}), ((lora.MAX_ROWS + 1, [8192], 16, 64), {}),
+                     ((8192, [0], 16, 64), {}), ((8192, [8192], 0, 64), {}),
+                     ((8192, [8192], 65, 64), {}), ((8192, [8192], 16, -1), {}),
+                     ((8192, [8192], 16, 64), {"sms": -1}), ((8192, [8192], 16, 64), {"long_tile": 0}),
+                     ((8192, [8192], 16, 64), {"long_tile": 129})]:
+        with pytest.raises(lora.LoraError):
+            plan(*args, **kw)
+    # NULL pointers through the C ABI
+    rt, mr = ctypes.c_int32(16), ctypes.c_int32(64)
+    cols = (ctypes.c_int64 * 1)(8192)
+    assert lib.lora_segment_plan(8192, None, 1, 148, 128, ctypes.byref(rt), ctypes.byref(mr), None) == -1
+    assert lib.lora_segment_plan(8192, cols, 1, 148, 128, None, ctypes.byref(mr), None) == -1
+    assert lib.lora_segment_plan(8192, cols, 1, 148, 128, ctypes.byref(rt), None, None) == -1
+    assert (rt.value, mr.value) == (16, 64)
+    # the flag array is optional
+    assert lib.lora_segment_plan(8192, cols, 1, 148, 128, ctypes.byref(rt), ctypes.byref(mr), None) == 0
+    assert (rt.value, mr.value) == (32, 0)
+
+
 def test_scratch_and_workspace_sizes(lib):
     assert lora.lora_segments_scratch_bytes(2048, 100) == 0
     # one thread block, no scratch: T <= 2048, or T <= 8192 with N <= 1023

@@ -5,9 +5,20 @@ import json
 import os
 from types import SimpleNamespace
 
+import pytest
 import torch
 
 import bench
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    """segment_params and launches_per_step take the route from the library's
+    host-only lora_segment_plan."""
+    from lora_adapter_application_b200 import build
+    build.build()
+    import lora_adapter_application_b200 as lora
+    lora.load()
 
 CODE = """// fused kernel
 __global__ void k(float* y) {   /* body */
