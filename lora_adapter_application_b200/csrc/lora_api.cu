@@ -473,14 +473,15 @@ int launch_rest(int mode, const Call &c, bool gather, bool contig, bool tc_took,
 // A fused call's contiguous tiles take the tensor-core SGMV kernel unless the
 // batch is too small to give every SM a 128-row tile while the layer is wide: a
 // cluster expands its tile over every output column as one long piece, and one
-// round of such tiles leaves SMs idle, where the gathered-tile kernel spreads the
+// wave of such tiles leaves SMs idle, where the gathered-tile kernel spreads the
 // same columns over every warp as items and takes all rows in one launch.
-// Measured on B200 (fused calls, 16-row tiles): the mixed 70B batch's
-// 8192 -> 28672 layer 226 -> 208 us and its 28672 -> 8192 layer 152 -> 147 us,
-// each now one launch; prefill batches of 11-77k tokens at 4096 wide keep the
-// tensor-core kernel (71 against 82 us at 11k tokens).  Override: LORA_TC_ROUTE = 1
-// (the tensor-core kernel whenever it qualifies) or 2 (the gathered-tile kernel
-// for every row).
+// Measured on B200, the mixed 70B batch (8192 rows, 7892 of them in prompts),
+// 16-row tiles and 64-row runs: 8192 -> 28672 layer 227 -> 211 us, 28672 -> 8192
+// layer 151 -> 152 us (one launch each); built for the single launch (32-row
+// tiles, no runs) 201 and 146 us.  Prefill batches of 11-77k tokens at 4096 wide
+// keep the tensor-core kernel (71 against 82 us at 11k tokens).  Override:
+// LORA_TC_ROUTE = 1 (the tensor-core kernel whenever it qualifies) or 2 (the
+// gathered-tile kernel for every row).
 constexpr int64_t TC_WIDE_COLS = 8192;
 // Rows per gathered tile when every row of every layer takes the fused kernel:
 // a tile reads its adapter once for twice the rows of a 16-row tile, and a batch
