@@ -197,18 +197,36 @@ def test_decode_qproj_full(cuda_lib):
     _check_full(w, R=16, min_run=0)
 
 
-def test_prefill_full(cuda_lib):
+def _launch(w, launch, min_run):
+    """Segment parameters: the ones bench.py times the workload with, or 64-row
+    gathered tiles with the given shortest run."""
+    if launch == "bench":
+        import bench
+        return bench.segment_params(w)
+    return 64, min_run
+
+
+@pytest.mark.parametrize("launch", ["bench", "R64"])
+def test_prefill_full(cuda_lib, launch):
     w = workloads.prefill()
-    _full_size(w, 0)
+    R, min_run = _launch(w, launch, 64)
+    _full_size(w, 0, R=R, min_run=min_run)
 
 
+@pytest.mark.parametrize("launch", ["bench", "R64"])
 @pytest.mark.parametrize("layer_idx", [0, 1, 2, 3])
-def test_multislice_8b_full(cuda_lib, layer_idx):
+def test_multislice_8b_full(cuda_lib, layer_idx, launch):
     w = workloads.multislice_8b()
-    _full_size(w, layer_idx, min_run=0)
+    R, min_run = _launch(w, launch, 0)
+    _full_size(w, layer_idx, R=R, min_run=min_run)
 
 
+@pytest.mark.parametrize("launch", ["bench", "R64"])
 @pytest.mark.parametrize("layer_idx", [0, 1])
-def test_mixed_70b_full(cuda_lib, layer_idx):
+def test_mixed_70b_full(cuda_lib, layer_idx, launch):
+    """bench.py's launch: 32-row tiles without contiguous runs, every row of both
+    layers on the gathered-tile kernel in one launch; R64: 64-row tiles with the
+    prompts as contiguous tiles."""
     w = workloads.mixed_70b()
-    _full_size(w, layer_idx)
+    R, min_run = _launch(w, launch, 64)
+    _full_size(w, layer_idx, R=R, min_run=min_run)
