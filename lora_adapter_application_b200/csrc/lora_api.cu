@@ -549,7 +549,7 @@ int check_meta_args(const lora_meta *m) { return check_meta(m); }
 
 extern "C" {
 
-int lora_version(void) { return 20000; }
+int lora_version(void) { return 20100; }
 
 const char *lora_last_error(void) { return g_last_error; }
 
